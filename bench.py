@@ -1,0 +1,491 @@
+#!/usr/bin/env python
+"""Batch-invariant greedy decode throughput on the Llama-3.1-8B-shaped random-init model.
+
+One step = one bi_decode_step over a batch of B decode tokens (every row of the
+hot path: embed, 32 x [RMSNorm, QKV GEMM + RoPE/KV append, chunked attention +
+merge, O GEMM, RMSNorm, gate/up GEMM + SwiGLU, down GEMM], final RMSNorm, LM
+head + logsumexp/top-2 merge + selective FP32 recompute) plus the greedy
+feedback (next ids, positions) -- replayed as one CUDA graph, inputs resident
+in HBM.  value = B * K / (device time of K steps), max over ranks, summed over
+ranks (replicas: every rank decodes its own batch, no collective on the data
+path).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B] [--impl ours|reference]
+
+--impl reference times the fp64 CPU oracle (the only other implementation of
+this computation here) on the host cores, on a bounded sample of the same
+workload scaled to tok/s.
+"""
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "batch-invariant decode tok/s (8B shape, bs 1-32); % of HBM roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=4)
+    ap.add_argument("--batch", type=int, default=32)
+    ap.add_argument("--prompt", type=int, default=512)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--mode", default="bf16", choices=["bf16", "layercast"])
+    ap.add_argument("--sweep", default="1,4,8,16,32", help="extra batch sizes to report ('' = none)")
+    ap.add_argument("--no-fast", action="store_true", help="skip the non-invariant FAST-variant comparison")
+    ap.add_argument("--no-layercast", action="store_true", help="skip the LayerCast-mode line")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_init(args):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks during the timed region
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.rows, self.proc = index, [], None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+                for n, v in zip(names, r[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                pass
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- roofline bookkeeping
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def step_bytes(cfg, B, ctx_lens, f32_kv=False):
+    """Algorithmic bytes one decode step must move: every weight once, the embedding rows, the KV rows read
+    (positions 0..ctx of every sequence, every layer) and written."""
+    L, H, Hq, Hkv, d, F, V = (cfg["n_layers"], cfg["hidden"], cfg["n_heads"], cfg["n_kv_heads"], cfg["head_dim"],
+                              cfg["ffn"], cfg["vocab"])
+    w = 2 * (L * ((Hq + 2 * Hkv) * d * H + H * Hq * d + 3 * F * H + 2 * H) + V * H + H)
+    kv_row = L * Hkv * d * 2 * (4 if f32_kv else 2)  # k and v of one position, all layers
+    kv = sum((c + 1) * kv_row for c in ctx_lens) + B * kv_row
+    return w + B * H * 2 + kv
+
+
+def gemm_bytes(cfg, B):
+    """Algorithmic bytes of the weight-streaming GEMM launches of one bf16 decode step (weights + inputs + outputs)."""
+    L, H, Hq, Hkv, d, F, V = (cfg["n_layers"], cfg["hidden"], cfg["n_heads"], cfg["n_kv_heads"], cfg["head_dim"],
+                              cfg["ffn"], cfg["vocab"])
+    QKV = (Hq + 2 * Hkv) * d
+    per_layer = [(QKV, H, 4), (H, Hq * d, 2), (2 * F, H, 2), (H, F, 2)]  # (N, K, output bytes per element)
+    tot, n = 0, 0
+    for N, K, ob in per_layer:
+        tot += L * (N * K * 2 + B * K * 2 + B * (N // 2 if N == 2 * F else N) * ob)
+        n += L
+    tot += V * H * 2 + B * H * 2 + B * V * 4
+    n += 1
+    return tot, n
+
+
+# ---------------------------------------------------------------- our arm
+def run_decode(m, B, P, K, W, ws, rank, graph=True):
+    """Prefill B prompts of P tokens (one batched call), then time K greedy decode steps (CUDA graph replay)."""
+    import numpy as np
+    import torch
+
+    import synth
+    from invariant_deterministic_full_b200 import ops
+
+    V = m.cfg["vocab"]
+    prompts = [synth.prompt_tokens(1000 * rank + r, P, V) for r in range(B)]
+    ids = np.concatenate(prompts).astype(np.int32)
+    slots = np.repeat(np.arange(B), P).astype(np.int32)
+    pos = np.tile(np.arange(P), B).astype(np.int32)
+    lm = np.full(B * P, -1, dtype=np.int32)
+    lm[np.arange(B) * P + P - 1] = np.arange(B)
+    o = m.step(ids, slots, pos, lm)
+    dev = m.device
+    ids_d = o["argmax"].clone()
+    pos_d = torch.full((B,), P, dtype=torch.int32, device=dev)
+    slot_d = torch.arange(B, dtype=torch.int32, device=dev)
+    lm_d = torch.arange(B, dtype=torch.int32, device=dev)
+    slots_h = torch.arange(B, dtype=torch.int32)
+    total = W + K + 1
+    pos_plan = torch.full((B,), P + total - 1, dtype=torch.int32)  # positions the replays will reach
+    out = m.alloc_out(B)
+    m.workspace(B, B, P + total)
+
+    def one_step():
+        m.step_dev(B, ids_d, slot_d, pos_d, slots_h, pos_plan, lm_d, B, None, out, max_pos=P + total)
+        ops.greedy_advance(out["argmax"], ids_d, pos_d)
+
+    # one eager step (library one-time set-up happens outside capture), then capture
+    from invariant_deterministic_full_b200._lib import lib
+    c0 = lib.bi_launch_count()
+    one_step()
+    launches = lib.bi_launch_count() - c0
+    torch.cuda.synchronize()
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(g, stream=s):
+            one_step()
+        torch.cuda.current_stream().wait_stream(s)
+        run = g.replay
+    else:
+        run = one_step
+    for _ in range(W):
+        run()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record()
+        for _ in range(K):
+            run()
+        e1.record()
+        e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    torch.cuda.synchronize()
+    err = ops.device_error()
+    if err:
+        raise RuntimeError(f"device error flags 0x{err:x}")
+    ctx_first = P + 1 + W  # position of the first timed step
+    ctx_lens = [ctx_first + i for i in range(K)]
+    rec = dict(ms=ms, launches=launches, clocks=clk.summary(), ctx_lens=ctx_lens,
+               recompute_rate=float(out["recomputed"].float().mean().item()))
+    if graph:
+        del g
+    return rec
+
+
+def time_gemms(m, B, reps=3):
+    """Average duration of the weight-streaming GEMM launches of one decode step, timed alone with CUDA events
+    on the launching stream (all layers' four projections + the LM-head GEMM, B token rows)."""
+    import torch
+    from invariant_deterministic_full_b200 import ops
+    cfg, w, dev = m.cfg, m.w, m.device
+    L, H, F = cfg["n_layers"], cfg["hidden"], cfg["ffn"]
+    QD = cfg["n_heads"] * cfg["head_dim"]
+    x_h, x_q, x_f = (torch.randn(B, n, device=dev).to(torch.bfloat16) for n in (H, QD, F))
+    o_qkv = torch.empty(B, w["w_qkv"].shape[1], dtype=torch.float32, device=dev)
+    o_h = torch.empty(B, H, dtype=torch.bfloat16, device=dev)
+    o_f = torch.empty(B, F, dtype=torch.bfloat16, device=dev)
+    o_lm = torch.empty(B, cfg["vocab"], dtype=torch.float32, device=dev)
+
+    def once():
+        for l in range(L):
+            ops.gemm(x_h, w["w_qkv"][l], out=o_qkv)
+            ops.gemm(x_q, w["w_o"][l], out=o_h)
+            ops.gemm(x_h, w["w_gu"][l], epilogue=1, out=o_f)
+            ops.gemm(x_f, w["w_down"][l], out=o_h)
+        ops.gemm(x_h, w["lm_head"], out=o_lm)
+
+    once()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        once()
+    e1.record()
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def run_e2e(m, B, P, K, rank):
+    """Same metric through the public API with host buffers: per step an H2D copy of the step's inputs from
+    pinned host memory, bi_decode_step, and a D2H read of the step's results; the host feeds the next ids."""
+    import numpy as np
+    import torch
+    import synth
+    V = m.cfg["vocab"]
+    dev = m.device
+    prompts = [synth.prompt_tokens(1000 * rank + 500 + r, P, V) for r in range(B)]
+    ids = np.concatenate(prompts).astype(np.int32)
+    slots = np.repeat(np.arange(B), P).astype(np.int32)
+    pos = np.tile(np.arange(P), B).astype(np.int32)
+    lm = np.full(B * P, -1, dtype=np.int32)
+    lm[np.arange(B) * P + P - 1] = np.arange(B)
+    o = m.step(ids, slots, pos, lm)
+    nxt = o["argmax"].cpu().numpy()
+    h_in = torch.empty(4, B, dtype=torch.int32).pin_memory()  # ids, slot, pos, lm_row
+    h_out_ids = torch.empty(B, dtype=torch.int32).pin_memory()
+    h_out_lp = torch.empty(B, dtype=torch.float32).pin_memory()
+    d_in = torch.empty(4, B, dtype=torch.int32, device=dev)
+    out = m.alloc_out(B)
+    slots_h = torch.arange(B, dtype=torch.int32)
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = P
+    for it in range(K + 1):
+        if it == 1:
+            e0.record()
+        h_in[0].copy_(torch.from_numpy(nxt))
+        h_in[1].copy_(slots_h)
+        h_in[2].fill_(cur)
+        h_in[3].copy_(torch.arange(B, dtype=torch.int32))
+        d_in.copy_(h_in, non_blocking=True)
+        m.step_dev(B, d_in[0], d_in[1], d_in[2], slots_h, h_in[2].clone(), d_in[3], B, None, out)
+        h_out_ids.copy_(out["argmax"], non_blocking=True)
+        h_out_lp.copy_(out["logprob"], non_blocking=True)
+        st.synchronize()
+        nxt = h_out_ids.numpy().copy()
+        cur += 1
+    e1.record()
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    return dict(ms=ms, h2d=4 * B * 4, d2h=B * 4 + B * 4)
+
+
+class CpuSample:
+    """The fp64 oracle as it stands, on the host cores: one decode token through 8B-width models of 1 and 2
+    layers (each with the 128256-row LM head); the per-layer time is scaled to 32 layers -> tok/s."""
+
+    def __init__(self):
+        import oracle
+        import synth
+        from synth import configs
+        self.oracle = oracle
+        self.cfg32 = configs.LLAMA8B
+        self.cfg2 = configs.shrink(self.cfg32, n_layers=2)
+        self.cfg1 = configs.shrink(self.cfg32, n_layers=1)
+        self.w2 = synth.model_weights(self.cfg2)
+        self.w1 = {k: (v[:1] if (v.ndim == 3 or k in ("attn_norm", "ffn_norm")) else v) for k, v in self.w2.items()}
+        self.tok = synth.prompt_tokens(0, 1, self.cfg2["vocab"])
+
+    def once(self):
+        t = time.perf_counter()
+        self.oracle.forward(self.cfg1, self.w1, self.tok)
+        t1 = time.perf_counter() - t
+        t = time.perf_counter()
+        self.oracle.forward(self.cfg2, self.w2, self.tok)
+        t2 = time.perf_counter() - t
+        per_layer = max(t2 - t1, 1e-9)
+        return per_layer * self.cfg32["n_layers"] + (t1 - per_layer), t1, t2
+
+    def describe(self, n, t1, t2):
+        return (f"fp64 oracle forward of 1 decode token through 1- and 2-layer 8B-width models incl. the "
+                f"128256-row LM head; the per-layer time (2-layer minus 1-layer) scaled to 32 layers; "
+                f"{n} repeats ({t1:.2f} s, {t2:.2f} s per forward)")
+
+
+def cores():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def cpu_baseline(seconds):
+    cs = CpuSample()
+    t_end = time.time() + seconds
+    best = None
+    n = 0
+    while n == 0 or time.time() < t_end:
+        r = cs.once()
+        n += 1
+        best = r if best is None or r[0] < best[0] else best
+    return {"value": round(1.0 / best[0], 4), "unit": "tok/s", "cores": cores(), "kind": "oracle",
+            "sample": cs.describe(n, best[1], best[2])}
+
+
+def main_ours(args):
+    import numpy as np
+    import torch
+    from synth import configs
+    from invariant_deterministic_full_b200 import model as mdl
+    ws, rank, local = dist_init(args)
+    cfg = configs.LLAMA8B
+    B, P, K, W = args.batch, args.prompt, args.steps, args.warmup
+    assert W >= 3, "at least 3 warm-up steps"
+    mode = 1 if args.mode == "layercast" else 0
+    sweep = [int(b) for b in args.sweep.split(",") if b.strip()] if args.sweep else []
+    n_slots = max([B] + sweep)
+    cap = P + W + K + 8
+    m = mdl.Model(cfg, mode=mode, n_slots=n_slots, capacity=cap, init="device", device="cuda")
+    r = run_decode(m, B, P, K, W, ws, rank)
+    ms = max_over_ranks(r["ms"], ws)
+    value = B * K * ws / (ms / 1e3)
+    hbm, tf_burst, tf_sus, src = peaks()
+    sb = step_bytes(cfg, B, [0] * B, f32_kv=(mode == 1))  # weights + rows at one position, per step
+    kv_row = cfg["n_layers"] * cfg["n_kv_heads"] * cfg["head_dim"] * 2 * (4 if mode else 2)
+    tot_bytes = sum(step_bytes(cfg, B, [c] * B, f32_kv=(mode == 1)) for c in r["ctx_lens"])
+    step_frac = tot_bytes / (ms / 1e3) / 1e9 / hbm
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "tok/s", "n_gpus": ws, "steps": K, "warmup": W,
+            "ms_per_step": round(ms / K, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if mode == 0 else "f32 (bf16 weights)",
+            "data": "synthetic: random-init bf16 weights N(0,0.02) (seed 20261202), uniform random prompt ids",
+            "config": {"workload": f"llama3.1-8b-shape greedy decode, batch {B} per GPU, prompt {P}, "
+                                   f"{K} timed steps (positions {P + 1 + W}..{P + W + K})",
+                       "model": cfg["name"] + " (random init)", "global_batch": B * ws, "seq_len": P + W + K + 1,
+                       "parallelism": "replicas" if ws > 1 else "single GPU",
+                       "mode": args.mode, "variant": "invariant", "margin_threshold": 0.1,
+                       "l2": "inputs larger than L2: every step streams 16 GB of weights"},
+            "hbm_roofline_frac_step": round(step_frac, 4),
+            "recompute_rate": r["recompute_rate"],
+            "gpu_launches": int(r["launches"] * K),
+            "clocks": r["clocks"]}
+    # dominant kernel: the weight-streaming GEMM (all projections of one step + LM head), timed alone
+    if mode == 0:
+        gms = time_gemms(m, B)
+        gb, gl = gemm_bytes(cfg, B)
+        ach = gb / (gms / 1e3) / 1e9
+        line["roofline"] = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                            "frac": round(ach / hbm, 4), "traffic": None,
+                            "kernel": "gemm_bf16_kernel (weight-streaming mma.sync GEMM)",
+                            "per_launch": f"{gb / gl / 1e6:.1f} MB algorithmic over {gl} launches, "
+                                          f"{gms / gl * 1e3:.1f} us average",
+                            "peak_source": f"{src} hbm_gbs (copy), kernel timed alone"}
+    else:
+        line["roofline"] = {"bound": "alu", "achieved": None, "peak": None, "unit": "TFLOP/s", "frac": None,
+                            "traffic": None}
+    if rank == 0 and not args.no_e2e:
+        e = run_e2e(m, B, P, min(K, 32), rank)
+        line["e2e"] = {"value": round(B * min(K, 32) / (e["ms"] / 1e3) * ws, 2), "unit": "tok/s",
+                       "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"]}
+    # batch sweep and the non-invariant comparison (same weights)
+    extra = {}
+    for b in sweep:
+        if b == B:
+            extra[str(b)] = round(value / ws, 2)
+            continue
+        rb = run_decode(m, b, P, min(K, 32), W, 1, rank)
+        extra[str(b)] = round(b * min(K, 32) / (rb["ms"] / 1e3), 2)
+    if extra:
+        line["sweep_tok_s_per_gpu"] = extra
+    if not args.no_fast:
+        mf = mdl.Model(cfg, mode=mode, variant=1, n_slots=n_slots, capacity=cap, init="device")
+        rf = run_decode(mf, B, P, K, W, 1, rank)
+        line["fast_variant"] = {"value": round(B * K / (rf["ms"] / 1e3), 2), "unit": "tok/s",
+                                "note": "non-invariant split-K / batch-dependent KV split, same weights and batch"}
+        mf.close()
+        del mf
+        torch.cuda.empty_cache()
+    if mode == 0 and not args.no_layercast:
+        ml = mdl.Model(cfg, mode=1, n_slots=max(B, 1), capacity=cap, init="device")
+        rl = run_decode(ml, B, P, min(K, 16), W, 1, rank)
+        line["layercast"] = {"value": round(B * min(K, 16) / (rl["ms"] / 1e3), 2), "unit": "tok/s",
+                             "batch": B, "note": "bf16 weights upcast in registers, fp32 FMA, fp32 activations/KV"}
+        ml.close()
+        del ml
+    if rank == 0 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds) if ws == 1 else None
+    m.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main_reference(args):
+    """Reference arm: the oracle, timed as it stands on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cs = CpuSample()
+    for _ in range(args.warmup):
+        cs.once()
+    t0 = time.perf_counter()
+    ts = [cs.once() for _ in range(args.steps)]
+    wall = time.perf_counter() - t0
+    per_tok = statistics.median(t[0] for t in ts)
+    v = 1.0 / per_tok
+    cb = {"value": round(v, 4), "unit": "tok/s", "cores": cores(), "kind": "oracle",
+          "sample": cs.describe(len(ts), ts[0][1], ts[0][2])}
+    line = {"metric": METRIC, "value": round(v, 4), "unit": "tok/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(per_tok * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
+            "data": "synthetic: same recipe as the GPU arm",
+            "config": {"workload": "llama3.1-8b-shape greedy decode, 1 token per step (bounded CPU sample)",
+                       "model": "llama3.1-8b-shape (random init)", "global_batch": 1, "seq_len": 1,
+                       "parallelism": "host cores"},
+            "cpu_baseline": cb,
+            "e2e": {"value": round(v, 4), "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_s": round(wall, 1)}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        main_reference(a)
+    else:
+        main_ours(a)

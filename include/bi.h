@@ -1,0 +1,263 @@
+/* bi.h -- C ABI of the batch-invariant decoder library (libbi.so, sm_100a).
+ *
+ * Every call computes the same per-row result whatever else is in the batch:
+ * the reduction order of every sum (GEMM K loop, RMSNorm, attention score
+ * sum, softmax denominator, PV accumulation, LM-head logsumexp) is fixed and
+ * depends neither on the number of rows, nor on how prefill is chunked, nor
+ * on prefill vs decode.  This is the method of the page "Meituan bitwise
+ * train/infer consistency" (root-cause list: attention score sums, softmax
+ * denominators, cross-device matrix reductions and logprob accumulation;
+ * scheme: fix the order of every reduce-add and share one reduction path
+ * between training, Prefill and Decode; TP computed over the full K
+ * dimension instead of segmented reduce-scatter).
+ *
+ * Conventions for every function:
+ *  - extern "C", returns int status (bi_status).  On failure nothing has been
+ *    launched and bi_last_error() returns a message (thread-local).
+ *  - Work is enqueued on the given CUDA stream (a cudaStream_t passed as
+ *    void*; NULL = legacy default stream) and runs asynchronously; a fault
+ *    inside a kernel surfaces at the caller's next synchronisation.
+ *  - Ownership: the caller owns EVERY device buffer (weights, KV cache,
+ *    inputs, outputs, workspace).  The library never allocates or frees
+ *    device memory and keeps no pointer after a call returns, except that a
+ *    bi_ctx stores the caller's weight/KV pointers until bi_ctx_destroy.
+ *  - Pointers marked (device) must be device-accessible; (host) are read on
+ *    the host during the call only.  Layouts are row-major, contiguous unless
+ *    a leading dimension is given.
+ *  - bf16 = IEEE bfloat16 bit pattern (uint16); f32 = IEEE binary32.
+ */
+#ifndef BI_H
+#define BI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BI_OK = 0,
+  BI_ERR_INVALID_ARG = 1, /* NULL pointer, negative size, inconsistent batch */
+  BI_ERR_UNSUPPORTED = 2, /* shape or mode the kernels do not implement */
+  BI_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than *_workspace_size */
+  BI_ERR_CAPACITY = 4,    /* position beyond KV capacity or RoPE table */
+  BI_ERR_CUDA = 5         /* a CUDA runtime/driver call failed at launch */
+} bi_status;
+
+enum { BI_MODE_BF16 = 0, BI_MODE_LAYERCAST = 1 };
+/* BI_MODE_BF16: bf16 activations and KV cache, bf16 x bf16 products with fp32
+ *   accumulation on tensor cores, fp32 softmax/norm arithmetic.
+ * BI_MODE_LAYERCAST: the "LayerCast" scheme of "Give Me FP32 or Give Me
+ *   Death?" (LayerCast section): weights stay bf16 in memory and are cast to
+ *   fp32 in registers just before use; every product and sum is fp32 FMA;
+ *   activations and KV cache are fp32. */
+enum { BI_VARIANT_INVARIANT = 0, BI_VARIANT_FAST = 1 };
+/* BI_VARIANT_FAST is the non-invariant comparison baseline: split-K GEMMs
+ * whose split factor is chosen from the row count M and the SM count, and
+ * attention whose KV split is chosen from the batch size.  Its results are
+ * deterministic for a fixed shape but change with batch size.  Not a product
+ * path; it exists so the cost of invariance can be measured. */
+enum { BI_DTYPE_BF16 = 0, BI_DTYPE_F32 = 1 };
+enum { BI_EPI_NONE = 0, BI_EPI_SWIGLU = 1 };
+
+/* Granule of the gate/up interleave used by BI_EPI_SWIGLU: the fused weight
+ * holds 16 gate rows, then the 16 up rows of the same output columns, etc. */
+#define BI_GU_INTERLEAVE 16
+/* Absolute KV chunk size of the attention grid (positions 0..255, 256..511, ...). */
+#define BI_ATTN_CHUNK 256
+/* Vocabulary chunk of the LM-head partial reductions. */
+#define BI_VOCAB_CHUNK 256
+
+const char* bi_last_error(void);
+int bi_version(void);
+/* Device error word: kernels never trap; a bounded wait that runs out, a
+ * position beyond capacity or an out-of-range id sets a bit here instead
+ * (1 = wait timeout, 2 = capacity, 4 = index) and the kernel skips the access.
+ * Synchronous read of the current device's word; reset != 0 clears it. */
+int bi_device_error(unsigned* flags, int reset);
+int bi_num_sms(int device); /* SM count of a device, -1 on error */
+/* Number of kernels the library has launched in this process (host-side
+ * counter, incremented at every launch site; not thread-safe). */
+long long bi_launch_count(void);
+
+/* ------------------------------------------------------------------ GEMM
+ * y[m][n] = sum_k x[m][k] * w[n][k]   (x: [M][K] with leading dim ldx,
+ *   w: bf16 [N][K] contiguous, y: [M][N] with leading dim ldy).
+ * Invariant variant: each output element is accumulated in fp32 over the
+ *   FULL K range in ascending K order, by the same instruction sequence for
+ *   any M (no split-K; the row tile and K loop do not depend on M).
+ *   ("Meituan bitwise train/infer consistency": TP rewritten to full-K
+ *   computation instead of segmented reduce-scatter.)
+ * mode BI_MODE_BF16: x is bf16.  mode BI_MODE_LAYERCAST: x is f32 and w is
+ *   upcast to f32 in registers; products and sums are fp32 FMA.
+ * y_dtype: BI_DTYPE_BF16 (round-to-nearest-even) or BI_DTYPE_F32.
+ * epilogue BI_EPI_SWIGLU: w rows are gate/up interleaved by BI_GU_INTERLEAVE
+ *   and y has N/2 columns: y = silu(gate) * up, silu(g) = g / (1 + exp(-g)).
+ * Requirements: K % 64 == 0, N % 64 == 0, ldx % 8 == 0 (16-byte rows),
+ *   x, w 16-byte aligned; else BI_ERR_UNSUPPORTED.
+ * Workspace: bi_gemm_workspace_size() bytes (0 for the invariant variant). */
+size_t bi_gemm_workspace_size(int M, int N, int K, int mode, int variant);
+int bi_gemm(const void* x, int ldx, const void* w, void* y, int ldy, int y_dtype, int M, int N, int K,
+            int epilogue, int mode, int variant, void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------- RMSNorm
+ * Per row m (fused residual add, as in a pre-norm decoder):
+ *   r'  = x + residual_in          (residual_in NULL: r' = x)
+ *   residual_out = r' (rounded to the activation dtype; may alias residual_in)
+ *   y   = r' / sqrt(mean(r'^2) + eps) * gamma        (activation dtype)
+ *   y_f32 (optional, f32) = the same value before rounding.
+ * The mean of squares is a fixed reduction tree over H (per-thread strided
+ * partials, fixed shuffle tree, ascending cross-warp sum) that does not
+ * depend on M.  Activation dtype: bf16 (BI_MODE_BF16) or f32 (LAYERCAST).
+ * gamma: bf16 [H].  H % 8 == 0 and H <= 16384. */
+int bi_rmsnorm(const void* x, const void* residual_in, void* residual_out, const void* gamma, void* y,
+               float* y_f32, int M, int H, float eps, int mode, void* stream);
+
+/* --------------------------------------------------------------- KV cache
+ * k and v: [n_slots][n_layers][n_kv_heads][capacity][head_dim], dtype bf16
+ * (BI_MODE_BF16) or f32 (BI_MODE_LAYERCAST).  Position p of slot s is row p. */
+typedef struct {
+  void* k;
+  void* v;
+  int n_slots, n_layers, n_kv_heads, capacity, head_dim;
+  int dtype; /* BI_DTYPE_BF16 or BI_DTYPE_F32 */
+} bi_kv_layout;
+
+/* RoPE table: [max_pos][head_dim/2][2] f32 (cos, sin) of pos * theta^(-2i/d),
+ * evaluated in fp64 on the host and rounded to f32.  Rotate-half pairing
+ * (i, i + d/2).  table: device, caller-allocated max_pos*head_dim floats. */
+int bi_rope_table_fill(float* table, int max_pos, int head_dim, double theta, void* stream);
+
+/* Rotary embedding + KV append for T tokens after the QKV projection.
+ * qkv: f32 [T][(Hq + 2*Hkv) * d] (q heads, then k heads, then v heads).
+ * q_out: [T][Hq*d] activation dtype; k and v rows are written to the cache at
+ * (slot[t], layer, head, pos[t]).  slot/pos: device int32 [T]. */
+int bi_rope_kv_append(const float* qkv, const float* rope, int rope_max_pos, void* q_out, const bi_kv_layout* kv,
+                      int layer, const int32_t* slot, const int32_t* pos, int T, int Hq, int mode, void* stream);
+
+/* ------------------------------------------------------------- Attention
+ * For each token t and q head h (kv head h / (Hq/Hkv)): causal softmax
+ * attention of q[t][h] over positions 0..pos[t] of slot[t]'s cache:
+ *   s_j = scale * q . k_j,  out = sum_j softmax(s)_j v_j.
+ * Fixed order ("Meituan bitwise train/infer consistency": the attention score
+ * sum and softmax denominator must reduce in one order for Prefill and Decode):
+ * the keys are cut on the ABSOLUTE grid of BI_ATTN_CHUNK positions; per chunk
+ * the partial (max, sum of exp, sum of p*v) is formed with fixed trees; the
+ * chunk partials are merged in ascending chunk order.  A query's result
+ * depends only on its own q and the cache rows it reads.
+ * q: [T][Hq*d], out: [T][Hq*d] (activation dtype); slot/pos: device int32 [T];
+ * slot_host/pos_host: host copies (validation and work planning).  Tokens of
+ * one slot that are adjacent in the batch must have consecutive positions.
+ * head_dim must be 64 or 128. */
+size_t bi_attention_workspace_size(int T, int Hq, int head_dim, int max_pos);
+int bi_attention(const void* q, const bi_kv_layout* kv, int layer, const int32_t* slot, const int32_t* pos,
+                 const int32_t* slot_host, const int32_t* pos_host, void* out, int T, int Hq, float scale, int mode,
+                 int variant, void* ws, size_t ws_bytes, void* stream);
+
+/* -------------------------------------------------------- LM-head logprob
+ * For each row b of h (f32 [B][H], device):
+ *   z = h . W^T (W bf16 [V][H]).  BI_MODE_BF16: h is rounded to bf16 and
+ *   z is a bf16 x bf16 tensor-core product with fp32 accumulation.
+ *   BI_MODE_LAYERCAST: z = fp32 FMA of h with W upcast to fp32.
+ *   lse = M + ln S over the vocabulary, reduced in BI_VOCAB_CHUNK chunks
+ *   (per chunk: max, sum exp(z - max), top-1 and top-2) merged in ascending
+ *   chunk order; logprob = z[target] - lse (target NULL or < 0: the argmax);
+ *   argmax = lowest id among equal maxima; margin = top-1 minus top-2 logit.
+ * Selective FP32 recompute ("Greedy Decoding Is Not Precision-Invariant",
+ *   method section: recompute the LM head in FP32 only when the top-two logit
+ *   margin falls below a threshold): in BI_MODE_BF16, rows with
+ *   margin < margin_threshold are recomputed as fp32 FMA of the f32 h with the
+ *   upcast W (the same arithmetic as LAYERCAST), and their lse, logprob and
+ *   argmax are replaced; margin keeps the bf16-path value that triggered it;
+ *   recomputed[b] = 1.  margin_threshold <= 0 disables it.  In LAYERCAST the
+ *   main pass is already fp32 and recomputed[b] = 0.
+ * Outputs (device, [B]): logprob f32, lse f32, argmax int32, margin f32,
+ *   recomputed uint8; logits (optional, f32 [B][V]): the main-pass logits
+ *   (bf16-path logits in BI_MODE_BF16; rows are not replaced by the recompute).
+ * Requirements: H % 64 == 0, V % 64 == 0. */
+size_t bi_lmhead_workspace_size(int B, int H, int V, int mode);
+int bi_lmhead_logprob(const float* h, const void* W, const int32_t* target, int B, int H, int V,
+                      float margin_threshold, int mode, float* logprob, float* lse, int32_t* argmax, float* margin,
+                      uint8_t* recomputed, float* logits, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------ Decode step
+ * A whole decoder forward for a batch of tokens (any mix of prefill chunks and
+ * decode tokens of many slots: continuous batching), followed by the LM-head
+ * logprob above for the tokens that ask for it.  Weights: bf16, caller-owned,
+ * device pointers; layouts below.  Architecture: pre-norm Llama-style decoder
+ * (RMSNorm, GQA attention with rotate-half RoPE, SwiGLU MLP, untied LM head,
+ * no biases). */
+typedef struct {
+  int n_layers, hidden, n_heads, n_kv_heads, head_dim, ffn, vocab;
+  float eps;
+  int mode;    /* BI_MODE_BF16 or BI_MODE_LAYERCAST */
+  int variant; /* BI_VARIANT_INVARIANT or BI_VARIANT_FAST */
+  float margin_threshold;
+} bi_model_desc;
+
+typedef struct {
+  const void* embed;      /* bf16 [V][H] */
+  const void* lm_head;    /* bf16 [V][H] */
+  const void* final_norm; /* bf16 [H] */
+  const void* attn_norm;  /* bf16 [L][H] */
+  const void* ffn_norm;   /* bf16 [L][H] */
+  const void* w_qkv;      /* bf16 [L][(Hq + 2 Hkv) d][H]: q rows, k rows, v rows */
+  const void* w_o;        /* bf16 [L][H][Hq d] */
+  const void* w_gu;       /* bf16 [L][2F][H], gate/up interleaved by BI_GU_INTERLEAVE */
+  const void* w_down;     /* bf16 [L][H][F] */
+  const float* rope;      /* f32 table from bi_rope_table_fill */
+  int rope_max_pos;
+} bi_weights;
+
+typedef struct bi_ctx bi_ctx;
+int bi_ctx_create(const bi_model_desc* desc, const bi_weights* w, const bi_kv_layout* kv, bi_ctx** out);
+int bi_ctx_destroy(bi_ctx* ctx);
+
+typedef struct {
+  int n_tokens;
+  const int32_t* ids;       /* device [n_tokens] token ids */
+  const int32_t* slot;      /* device [n_tokens] KV slot of each token */
+  const int32_t* pos;       /* device [n_tokens] position of each token in its slot */
+  const int32_t* slot_host; /* host copies of slot and pos (validation, planning) */
+  const int32_t* pos_host;
+  const int32_t* lm_row;    /* device [n_tokens]: output row of the token, or -1 */
+  int n_lm;                 /* number of output rows (tokens with lm_row >= 0) */
+  const int32_t* target;    /* device [n_lm]: token whose logprob is wanted; NULL or -1 = greedy */
+} bi_batch;
+
+typedef struct {
+  float* logprob;      /* device [n_lm] */
+  float* lse;          /* device [n_lm] */
+  int32_t* argmax;     /* device [n_lm]  (greedy next token) */
+  float* margin;       /* device [n_lm] */
+  uint8_t* recomputed; /* device [n_lm] */
+  float* logits;       /* optional device [n_lm][V] */
+  float* h;            /* optional device [n_lm][H]: final norm output, f32 */
+} bi_step_out;
+
+size_t bi_decode_workspace_size(const bi_ctx* ctx, int max_tokens, int max_lm_rows, int max_pos);
+int bi_decode_step(bi_ctx* ctx, const bi_batch* batch, const bi_step_out* out, void* ws, size_t ws_bytes,
+                   void* stream);
+
+/* Greedy feedback for a device-resident decode loop: for b < B,
+ * ids[b] = argmax[b] and pos[b] += 1 (device int32 arrays). */
+int bi_greedy_advance(const int32_t* argmax, int32_t* ids, int32_t* pos, int B, void* stream);
+
+/* ----------------------------------------------------------- Synthetic init
+ * Device twin of the seeded generator used for the synthetic workloads:
+ * SplitMix64 counters -> Irwin-Hall(12) normal -> bf16(f32(z * std)).
+ * Writes logical element i (row i / cols, column i % cols) of a [rows][cols]
+ * tensor of stream `key`, starting at logical element 0, to
+ *   dst[dst_row(i / cols) * cols + i % cols], where
+ *   dst_row(r) = r                                   if interleave == 0,
+ *   dst_row(r) = (r / g) * 2g + phase * g + r % g    if interleave == g > 0
+ * (phase 0 = gate rows, 1 = up rows of a BI_GU_INTERLEAVE fused weight).
+ * Not part of the method: it only produces inputs without a host round trip. */
+int bi_synth_fill_bf16(uint16_t* dst, int64_t rows, int64_t cols, uint64_t key, double std, int interleave,
+                       int phase, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BI_H */

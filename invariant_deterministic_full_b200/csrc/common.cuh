@@ -1,0 +1,163 @@
+// Shared helpers of libbi: status/error state, tensor-map encoding, and the
+// inline-PTX primitives the kernels use (mbarrier, TMA, ldmatrix, mma.sync).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/bi.h"
+
+namespace bi {
+
+// ------------------------------------------------------------------ errors
+int set_error(int status, const char* fmt, ...);
+void clear_error();
+
+#define BI_CHECK_CUDA(call)                                                                   \
+  do {                                                                                        \
+    cudaError_t e_ = (call);                                                                  \
+    if (e_ != cudaSuccess) return ::bi::set_error(BI_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+extern long long g_launches;  // host-side count of kernels launched by the library
+#define BI_CHECK_LAUNCH()            \
+  do {                               \
+    ++::bi::g_launches;              \
+    BI_CHECK_CUDA(cudaGetLastError()); \
+  } while (0)
+#define BI_REQUIRE(cond, status, ...)                 \
+  do {                                                \
+    if (!(cond)) return ::bi::set_error(status, __VA_ARGS__); \
+  } while (0)
+#define BI_TRY(expr)             \
+  do {                           \
+    int s_ = (expr);             \
+    if (s_ != BI_OK) return s_;  \
+  } while (0)
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+int num_sms();  // of the current device (cached per device)
+
+// Device-side error word: kernels set bits here instead of trapping when a
+// bounded wait runs out or an index fails its check.
+enum : unsigned { DEVERR_TIMEOUT = 1u, DEVERR_CAPACITY = 2u, DEVERR_INDEX = 4u };
+__device__ unsigned g_dev_error = 0;  // one translation unit: defined here
+__device__ __forceinline__ void dev_flag(unsigned bit) { atomicOr(&g_dev_error, bit); }
+
+// Tensor maps (TMA descriptors), encoded through the driver entry point.
+int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,
+                   uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                   CUtensorMapSwizzle swizzle);
+
+// ------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: returns false (and flags the device error word) if the phase
+// does not complete within the iteration limit (each try_wait suspends for a
+// hardware-chosen interval, so the limit is seconds, never forever).
+constexpr uint32_t kWaitLimit = 1u << 22;
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  dev_flag(DEVERR_TIMEOUT);
+  return false;
+}
+
+// 2D tiled TMA load into shared memory, completion counted on an mbarrier.
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int c_inner, int c_outer,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c_inner), "r"(c_outer), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+// D = A(16x16 bf16, row) * B(16x8 bf16, col) + D, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Address of the 16-byte chunk `chunk` of row `row` inside a TMA tile written
+// with CU_TENSOR_MAP_SWIZZLE_128B (128-byte rows, tile base 1024-byte aligned):
+// chunk c of row r lives at chunk position c ^ (r & 7).
+__device__ __forceinline__ uint32_t swz128(uint32_t tile_base, int row, int chunk) {
+  return tile_base + row * 128 + ((chunk ^ (row & 7)) << 4);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+// Store one activation value in the mode's dtype (bf16: round to nearest even).
+__device__ __forceinline__ void store_act(void* base, size_t idx, float v, bool f32) {
+  if (f32)
+    reinterpret_cast<float*>(base)[idx] = v;
+  else
+    reinterpret_cast<uint16_t*>(base)[idx] = f32_to_bf16_bits(v);
+}
+__device__ __forceinline__ float load_act(const void* base, size_t idx, bool f32) {
+  return f32 ? reinterpret_cast<const float*>(base)[idx]
+             : bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(base)[idx]);
+}
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+
+// Fixed butterfly sum over the 32 lanes: every lane ends with the same value
+// (each level adds the same two operands, only their order differs, and fp
+// addition is commutative).
+__device__ __forceinline__ float warp_sum_fixed(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+}  // namespace bi

@@ -1,0 +1,396 @@
+// bi_gemm kernels.
+//
+// Invariance ("Meituan bitwise train/infer consistency": full-K computation in
+// place of segmented reductions, one accumulation order for Prefill and
+// Decode): every output element y[m][n] is accumulated in fp32 over the full K
+// range, in ascending K, by the same instruction sequence whatever M is.
+//
+// bf16 path (gemm_bf16_kernel): mma.sync m16n8k16 (bf16 x bf16 -> fp32) with
+// the weight on the 16-row side and the tokens on the 8-column side.  Each
+// instruction adds 16 products of one (n, m) pair into that pair's fp32
+// accumulator; the products of one element never meet another element's, so
+// neither the number of token columns in a tile nor the tile a token lands in
+// can change an element's bits.  K advances 16 at a time in ascending order.
+// Weight tiles (BN rows x 64 k) and token tiles (32 rows x 64 k) stream by TMA
+// (128-byte swizzle) into a multi-stage shared-memory ring filled by one
+// producer warp; four consumer warps read them with ldmatrix.  The grid is
+// persistent (at most one CTA per SM), each CTA walking its work items
+// (row group x token tile) so the ring never drains between items.
+//
+// LayerCast path (gemm_f32_kernel): the weight is upcast from bf16 to fp32 in
+// registers and every product/sum is an fp32 FMA ("Give Me FP32 or Give Me
+// Death?", LayerCast section).  Element order: lane l of a warp owns the
+// k-slices [256 i + 8 l, 256 i + 8 l + 8) for i = 0, 1, ...; it accumulates
+// them with sequential FMAs in ascending k, and the 32 lane partials are then
+// combined by a fixed xor-butterfly.  This is the same for every M and every
+// row/token tiling.
+#pragma once
+#include "common.cuh"
+
+namespace bi {
+
+constexpr int GEMM_BM = 32;  // token rows per tile (fixed; never depends on M)
+constexpr int GEMM_BK = 64;  // k per TMA box (128 bytes of bf16)
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int STAGES = BN == 32 ? 16 : (BN == 64 ? 12 : 8);
+  static constexpr int W_BYTES = BN * 128;
+  static constexpr int X_BYTES = GEMM_BM * 128;
+  static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;
+  static constexpr int RW = BN / 32;      // warps along the weight rows (32 rows each)
+  static constexpr int TW = 4 / RW;       // warps along the token columns
+  static constexpr int NT = GEMM_BM / TW / 8;  // n8 token tiles per warp
+};
+
+// Work item -> (split, row group, token tile).  Splits > 1 only in the
+// non-invariant FAST variant, which then writes fp32 partials per split.
+template <int BN, int EPI>
+__global__ void __launch_bounds__(160, 1)
+    gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                     void* __restrict__ y, int ldy, int y_f32, int M, int N, int K, int m_tiles, int n_groups,
+                     int splits, float* __restrict__ partial) {
+  using C = GemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[C::STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kblocks_total = K / GEMM_BK;
+  const int kb_per_split = (kblocks_total + splits - 1) / splits;
+  const int n_items = splits * n_groups * m_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 4);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == 4) {  // ---------------- producer: one elected lane issues TMA
+    if (lane == 0) {
+      prefetch_tmap(&tmW);
+      prefetch_tmap(&tmX);
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int mt = item % m_tiles;
+        const int g = (item / m_tiles) % n_groups;
+        const int sp = item / (m_tiles * n_groups);
+        const int kb0 = sp * kb_per_split;
+        const int kb1 = min(kblocks_total, kb0 + kb_per_split);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1)) return;
+          uint8_t* sb = smem + stage * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+          tma_load_2d(sb, &tmW, kb * GEMM_BK, g * BN, &full_bar[stage]);
+          tma_load_2d(sb + C::W_BYTES, &tmX, kb * GEMM_BK, mt * GEMM_BM, &full_bar[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers
+  const int rw = warp % C::RW, tw = warp / C::RW;
+  const int row0 = rw * 32;                      // weight rows [row0, row0+32) of the tile
+  const int tok0 = tw * (GEMM_BM / C::TW);       // token columns [tok0, tok0 + 8*NT)
+  const int g8 = lane >> 2, t4 = lane & 3;
+  int stage = 0;
+  uint32_t phase = 0;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int mt = item % m_tiles;
+    const int g = (item / m_tiles) % n_groups;
+    const int sp = item / (m_tiles * n_groups);
+    const int kb0 = sp * kb_per_split;
+    const int kb1 = min(kblocks_total, kb0 + kb_per_split);
+    const bool active = mt * GEMM_BM + tok0 < M;
+    float acc[2][C::NT][4];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int b = 0; b < C::NT; ++b)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[a][b][c] = 0.f;
+
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(&full_bar[stage], phase)) return;
+      if (active) {
+        const uint32_t wb = smem_u32(smem + stage * C::STAGE_BYTES);
+        const uint32_t xb = wb + C::W_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          uint32_t a[2][4];
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int row = row0 + r * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            ldsm_x4(swz128(wb, row, 2 * kk + (lane >> 4)), a[r][0], a[r][1], a[r][2], a[r][3]);
+          }
+          uint32_t b[C::NT][2];
+          if constexpr (C::NT >= 2) {
+#pragma unroll
+            for (int p = 0; p < C::NT / 2; ++p) {
+              const int tok = tok0 + p * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+              ldsm_x4(swz128(xb, tok, 2 * kk + ((lane >> 3) & 1)), b[2 * p][0], b[2 * p][1], b[2 * p + 1][0],
+                      b[2 * p + 1][1]);
+            }
+          } else {
+            const int tok = tok0 + (lane & 7);
+            ldsm_x2(swz128(xb, tok, 2 * kk + ((lane >> 3) & 1)), b[0][0], b[0][1]);
+          }
+#pragma unroll
+          for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int nt = 0; nt < C::NT; ++nt) mma_bf16_16816(acc[r][nt], a[r], b[nt][0], b[nt][1]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[stage]);
+      if (++stage == C::STAGES) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+    if (!active) continue;
+
+    // ---------------- epilogue: fragment (row g8 (+8), cols 2*t4 (+1)) of each m16n8 tile
+    const int nbase = g * BN + row0;
+#pragma unroll
+    for (int nt = 0; nt < C::NT; ++nt) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int m = mt * GEMM_BM + tok0 + nt * 8 + 2 * t4 + (i & 1);
+        if (m >= M) continue;
+        const int rin = g8 + (i >> 1) * 8;
+        if (splits > 1) {  // FAST variant: raw fp32 partial of this split
+#pragma unroll
+          for (int r = 0; r < 2; ++r)
+            partial[((size_t)sp * M + m) * N + nbase + r * 16 + rin] = acc[r][nt][i];
+        } else if constexpr (EPI == BI_EPI_SWIGLU) {
+          const int col = (nbase >> 1) + rin;  // 32-row block -> 16 output columns
+          store_act(y, (size_t)m * ldy + col, silu(acc[0][nt][i]) * acc[1][nt][i], y_f32);
+        } else {
+#pragma unroll
+          for (int r = 0; r < 2; ++r) store_act(y, (size_t)m * ldy + nbase + r * 16 + rin, acc[r][nt][i], y_f32);
+        }
+      }
+    }
+  }
+}
+
+// FAST variant: y = sum over splits (ascending) of the fp32 partials, then the epilogue.
+template <int EPI>
+__global__ void splitk_reduce_kernel(const float* __restrict__ partial, void* __restrict__ y, int ldy, int y_f32, int M,
+                                     int N, int splits) {
+  const int n_out = EPI == BI_EPI_SWIGLU ? N / 2 : N;
+  const size_t total = (size_t)M * n_out;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total; idx += (size_t)gridDim.x * blockDim.x) {
+    const int m = (int)(idx / n_out), c = (int)(idx % n_out);
+    if constexpr (EPI == BI_EPI_SWIGLU) {
+      const int blk = c / 16, r = c % 16;
+      const int ng = blk * 32 + r, nu = ng + 16;
+      float sg = 0.f, su = 0.f;
+      for (int s = 0; s < splits; ++s) {
+        sg += partial[((size_t)s * M + m) * N + ng];
+        su += partial[((size_t)s * M + m) * N + nu];
+      }
+      store_act(y, (size_t)m * ldy + c, silu(sg) * su, y_f32);
+    } else {
+      float s0 = 0.f;
+      for (int s = 0; s < splits; ++s) s0 += partial[((size_t)s * M + m) * N + c];
+      store_act(y, (size_t)m * ldy + c, s0, y_f32);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- LayerCast (fp32 FMA)
+constexpr int F32_ROWS = 32;  // weight rows per CTA (8 warps x 4 rows)
+constexpr int F32_TOK = 8;    // token columns per CTA
+
+// x: f32 [M][ldx]; w: bf16 [N][K]; y: [M][ldy].  Optional device row count
+// (count != nullptr): only token rows < *count are computed (used by the
+// selective recompute, whose row count is known only on the device).
+template <int EPI>
+__global__ void __launch_bounds__(256)
+    gemm_f32_kernel(const float* __restrict__ x, int ldx, const uint16_t* __restrict__ w, void* __restrict__ y,
+                    int ldy, int y_f32, int M, int N, int K, const int* __restrict__ count) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * F32_TOK;
+  int Meff = M;
+  if (count) Meff = min(M, *count);
+  if (m0 >= Meff) return;
+  const int ntok = min(F32_TOK, Meff - m0);
+  const int grp = blockIdx.y;
+  int rows[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    if constexpr (EPI == BI_EPI_SWIGLU)
+      rows[r] = grp * F32_ROWS + (r >> 1) * 16 + 2 * warp + (r & 1);  // 2 gate rows, then the 2 matching up rows
+    else
+      rows[r] = grp * F32_ROWS + 4 * warp + r;
+  }
+  float acc[4][F32_TOK];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int t = 0; t < F32_TOK; ++t) acc[r][t] = 0.f;
+
+  for (int kbase = 0; kbase < K; kbase += 256) {
+    const int k = kbase + 8 * lane;
+    if (k < K) {
+      float wf[4][8];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(w + (size_t)rows[r] * K + k));
+        wf[r][0] = bf16lo(u.x); wf[r][1] = bf16hi(u.x); wf[r][2] = bf16lo(u.y); wf[r][3] = bf16hi(u.y);
+        wf[r][4] = bf16lo(u.z); wf[r][5] = bf16hi(u.z); wf[r][6] = bf16lo(u.w); wf[r][7] = bf16hi(u.w);
+      }
+#pragma unroll
+      for (int t = 0; t < F32_TOK; ++t) {
+        if (t < ntok) {
+          const float4* xp = reinterpret_cast<const float4*>(x + (size_t)(m0 + t) * ldx + k);
+          const float4 x0 = __ldg(xp), x1 = __ldg(xp + 1);
+          const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) acc[r][t] = fmaf(wf[r][j], xv[j], acc[r][t]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < F32_TOK; ++t) {
+    if (t >= ntok) break;
+    float s[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) s[r] = warp_sum_fixed(acc[r][t]);
+    const int m = m0 + t;
+    if constexpr (EPI == BI_EPI_SWIGLU) {
+      if (lane < 2) {
+        const float gv = lane == 0 ? s[0] : s[1];
+        const float uv = lane == 0 ? s[2] : s[3];
+        const int col = grp * 16 + 2 * warp + lane;
+        store_act(y, (size_t)m * ldy + col, silu(gv) * uv, y_f32);
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        if (lane == r) store_act(y, (size_t)m * ldy + rows[r], s[r], y_f32);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- host side
+static int gemm_pick_bn(int N) {
+  if (N <= 8192 && N % 32 == 0) return 32;
+  if (N % 128 == 0) return 128;
+  return 64;
+}
+
+// Split factor of the FAST variant: more K splits for small M so that the
+// grid fills the SMs (the usual library heuristic) -- which is exactly what
+// makes the result depend on the batch size.
+static int gemm_fast_splits(int M, int n_items, int kblocks) {
+  const int sms = num_sms();
+  if (M > 16) return 1;
+  int s = (2 * sms + n_items - 1) / n_items;
+  if (M <= 4) s *= 2;
+  s = s < 1 ? 1 : (s > 8 ? 8 : s);
+  while (s > 1 && kblocks / s < 4) --s;
+  return s;
+}
+
+size_t gemm_ws_bytes(int M, int N, int K, int mode, int variant) {
+  if (variant != BI_VARIANT_FAST || mode != BI_MODE_BF16) return 0;
+  const int bn = gemm_pick_bn(N);
+  const int items = (N / bn) * ((M + GEMM_BM - 1) / GEMM_BM);
+  const int s = gemm_fast_splits(M, items, K / GEMM_BK);
+  return s > 1 ? (size_t)s * M * N * sizeof(float) : 0;
+}
+
+template <int BN, int EPI>
+static int launch_gemm_bf16_t(const CUtensorMap& tw, const CUtensorMap& tx, void* y, int ldy, int y_f32, int M, int N,
+                              int K, int splits, float* partial, cudaStream_t st) {
+  using C = GemmCfg<BN>;
+  static bool attr_done = false;  // per instantiation; set once per process
+  if (!attr_done) {
+    BI_CHECK_CUDA(cudaFuncSetAttribute(gemm_bf16_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    attr_done = true;
+  }
+  const int m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
+  const int n_groups = N / BN;
+  const int items = splits * n_groups * m_tiles;
+  const int grid = items < num_sms() ? items : num_sms();
+  gemm_bf16_kernel<BN, EPI><<<grid, 160, C::SMEM, st>>>(tw, tx, y, ldy, y_f32, M, N, K, m_tiles, n_groups, splits,
+                                                         partial);
+  BI_CHECK_LAUNCH();
+  return BI_OK;
+}
+
+int gemm_bf16(const void* x, int ldx, const void* w, void* y, int ldy, int y_f32, int M, int N, int K, int epi,
+              int variant, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const int bn = gemm_pick_bn(N);
+  CUtensorMap tw, tx;
+  BI_TRY(encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, K, N, (uint64_t)K * 2, GEMM_BK, bn,
+                        CU_TENSOR_MAP_SWIZZLE_128B));
+  BI_TRY(encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, K, M, (uint64_t)ldx * 2, GEMM_BK, GEMM_BM,
+                        CU_TENSOR_MAP_SWIZZLE_128B));
+  int splits = 1;
+  if (variant == BI_VARIANT_FAST) {
+    const int items = (N / bn) * ((M + GEMM_BM - 1) / GEMM_BM);
+    splits = gemm_fast_splits(M, items, K / GEMM_BK);
+  }
+  float* partial = nullptr;
+  if (splits > 1) {
+    const size_t need = (size_t)splits * M * N * sizeof(float);
+    BI_REQUIRE(ws && ws_bytes >= need, BI_ERR_WORKSPACE, "bi_gemm FAST: workspace %zu < %zu", ws_bytes, need);
+    partial = reinterpret_cast<float*>(ws);
+  }
+#define BI_GEMM_CASE(BNV)                                                                                          \
+  if (bn == BNV) {                                                                                                 \
+    if (epi == BI_EPI_SWIGLU)                                                                                      \
+      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_SWIGLU>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, st)));     \
+    else                                                                                                           \
+      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_NONE>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, st)));       \
+  }
+  BI_GEMM_CASE(32)
+  BI_GEMM_CASE(64)
+  BI_GEMM_CASE(128)
+#undef BI_GEMM_CASE
+  if (splits > 1) {
+    const int n_out = epi == BI_EPI_SWIGLU ? N / 2 : N;
+    const size_t total = (size_t)M * n_out;
+    int blocks = (int)((total + 255) / 256);
+    if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
+    if (epi == BI_EPI_SWIGLU)
+      splitk_reduce_kernel<BI_EPI_SWIGLU><<<blocks, 256, 0, st>>>(partial, y, ldy, y_f32, M, N, splits);
+    else
+      splitk_reduce_kernel<BI_EPI_NONE><<<blocks, 256, 0, st>>>(partial, y, ldy, y_f32, M, N, splits);
+    BI_CHECK_LAUNCH();
+  }
+  return BI_OK;
+}
+
+int gemm_f32(const float* x, int ldx, const void* w, void* y, int ldy, int y_f32, int M, int N, int K, int epi,
+             const int* count, cudaStream_t st) {
+  dim3 grid((M + F32_TOK - 1) / F32_TOK, N / F32_ROWS);
+  if (epi == BI_EPI_SWIGLU)
+    gemm_f32_kernel<BI_EPI_SWIGLU><<<grid, 256, 0, st>>>(x, ldx, reinterpret_cast<const uint16_t*>(w), y, ldy, y_f32,
+                                                         M, N, K, count);
+  else
+    gemm_f32_kernel<BI_EPI_NONE><<<grid, 256, 0, st>>>(x, ldx, reinterpret_cast<const uint16_t*>(w), y, ldy, y_f32, M,
+                                                       N, K, count);
+  BI_CHECK_LAUNCH();
+  return BI_OK;
+}
+
+}  // namespace bi

@@ -1,0 +1,547 @@
+// libbi: batch-invariant decoder forward + LM-head logprob for sm_100a.
+// One translation unit: the kernels live in the included .cuh files; this
+// file holds the C ABI declared in include/bi.h (argument checks, workspace
+// carving, launches) and the decode-step orchestration.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "host_common.cuh"
+#include "gemm.cuh"
+#include "norm_rope.cuh"
+#include "attention.cuh"
+#include "lmhead.cuh"
+#include "synth_fill.cuh"
+
+namespace bi {
+
+// Workspace carving: 256-byte aligned sub-buffers.  With base == nullptr it
+// only measures.
+struct Carver {
+  uint8_t* base;
+  size_t used = 0;
+  explicit Carver(void* b) : base(reinterpret_cast<uint8_t*>(b)) {}
+  template <typename T>
+  T* take(size_t count) {
+    used = (used + 255) & ~size_t(255);
+    T* p = base ? reinterpret_cast<T*>(base + used) : nullptr;
+    used += count * sizeof(T);
+    return p;
+  }
+};
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// ------------------------------------------------------------------ GEMM
+static int gemm_run(const void* x, int ldx, const void* w, void* y, int ldy, int y_dtype, int M, int N, int K, int epi,
+                    int mode, int variant, void* ws, size_t ws_bytes, cudaStream_t st) {
+  BI_REQUIRE(x && w && y, BI_ERR_INVALID_ARG, "bi_gemm: NULL pointer");
+  BI_REQUIRE(M >= 0 && N > 0 && K > 0, BI_ERR_INVALID_ARG, "bi_gemm: bad sizes M=%d N=%d K=%d", M, N, K);
+  BI_REQUIRE(K % 64 == 0 && N % 64 == 0, BI_ERR_UNSUPPORTED, "bi_gemm: need K %% 64 == 0 and N %% 64 == 0 (N=%d K=%d)",
+             N, K);
+  BI_REQUIRE(ldx >= K && ldx % 8 == 0, BI_ERR_UNSUPPORTED, "bi_gemm: ldx=%d must be >= K and a multiple of 8", ldx);
+  const int n_out = epi == BI_EPI_SWIGLU ? N / 2 : N;
+  BI_REQUIRE(ldy >= n_out, BI_ERR_INVALID_ARG, "bi_gemm: ldy=%d < output columns %d", ldy, n_out);
+  BI_REQUIRE(aligned16(x) && aligned16(w), BI_ERR_UNSUPPORTED, "bi_gemm: x and w must be 16-byte aligned");
+  BI_REQUIRE(epi == BI_EPI_NONE || epi == BI_EPI_SWIGLU, BI_ERR_INVALID_ARG, "bi_gemm: bad epilogue %d", epi);
+  BI_REQUIRE(mode == BI_MODE_BF16 || mode == BI_MODE_LAYERCAST, BI_ERR_INVALID_ARG, "bi_gemm: bad mode %d", mode);
+  BI_REQUIRE(y_dtype == BI_DTYPE_BF16 || y_dtype == BI_DTYPE_F32, BI_ERR_INVALID_ARG, "bi_gemm: bad y dtype");
+  if (M == 0) return BI_OK;
+  const int y_f32 = y_dtype == BI_DTYPE_F32;
+  if (mode == BI_MODE_LAYERCAST)
+    return gemm_f32(reinterpret_cast<const float*>(x), ldx, w, y, ldy, y_f32, M, N, K, epi, nullptr, st);
+  return gemm_bf16(x, ldx, w, y, ldy, y_f32, M, N, K, epi, variant, ws, ws_bytes, st);
+}
+
+// ------------------------------------------------------------------ attention
+static int attn_chunk_for(int T, int variant) {
+  if (variant != BI_VARIANT_FAST) return ATT_CHUNK;
+  // FAST: KV split chosen from the batch size (more, smaller chunks for small batches).
+  return T <= 4 ? 64 : (T <= 16 ? 128 : 256);
+}
+
+static size_t attn_ws_bytes(int T, int Hq, int d, int max_pos, int chunk) {
+  const int tg = std::min(T, ATT_TOKEN_GROUP);
+  const int max_chunks = max_pos / chunk + 1;
+  return (size_t)tg * Hq * max_chunks * (d + 4) * sizeof(float) + 256;
+}
+
+static int attn_smem_bytes(int d, int f32) {
+  const size_t kv_region = (size_t)ATT_CHUNK * d * (f32 ? 4 : 2);
+  return (int)((f32 ? kv_region : 2 * kv_region) + (size_t)ATT_MAX_PAIRS * d * 4 + (size_t)ATT_MAX_PAIRS * ATT_CHUNK * 4 +
+               1024);
+}
+
+static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const int32_t* slot, const int32_t* pos,
+                         const int32_t* slot_h, const int32_t* pos_h, void* out, int T, int Hq, float scale, int mode,
+                         int variant, void* ws, size_t ws_bytes, cudaStream_t st) {
+  BI_REQUIRE(q && kv && slot && pos && slot_h && pos_h && out, BI_ERR_INVALID_ARG, "bi_attention: NULL pointer");
+  BI_REQUIRE(kv->k && kv->v, BI_ERR_INVALID_ARG, "bi_attention: NULL KV cache");
+  const int d = kv->head_dim, Hkv = kv->n_kv_heads;
+  BI_REQUIRE(d == 64 || d == 128, BI_ERR_UNSUPPORTED, "bi_attention: head_dim %d (need 64 or 128)", d);
+  BI_REQUIRE(Hkv > 0 && Hq > 0 && Hq % Hkv == 0, BI_ERR_INVALID_ARG, "bi_attention: Hq=%d Hkv=%d", Hq, Hkv);
+  BI_REQUIRE(layer >= 0 && layer < kv->n_layers, BI_ERR_INVALID_ARG, "bi_attention: layer %d", layer);
+  const int f32 = mode == BI_MODE_LAYERCAST;
+  BI_REQUIRE(kv->dtype == (f32 ? BI_DTYPE_F32 : BI_DTYPE_BF16), BI_ERR_INVALID_ARG,
+             "bi_attention: KV dtype does not match the mode");
+  if (T == 0) return BI_OK;
+  const int G = Hq / Hkv;
+  BI_REQUIRE(G <= ATT_MAX_PAIRS, BI_ERR_UNSUPPORTED, "bi_attention: %d q heads per kv head (max %d)", G, ATT_MAX_PAIRS);
+  const int chunk = attn_chunk_for(T, variant);
+  const int QB = std::max(1, ATT_MAX_PAIRS / G);
+
+  // validation + plan: blocks of <= QB adjacent tokens of one slot at consecutive positions
+  int max_pos = 0;
+  std::vector<int2> blocks;
+  blocks.reserve(T);
+  for (int t = 0; t < T; ++t) {
+    const int s = slot_h[t], p = pos_h[t];
+    BI_REQUIRE(s >= 0 && s < kv->n_slots, BI_ERR_INVALID_ARG, "bi_attention: token %d slot %d out of range", t, s);
+    BI_REQUIRE(p >= 0 && p < kv->capacity, BI_ERR_CAPACITY, "bi_attention: token %d position %d >= capacity %d", t, p,
+               kv->capacity);
+    max_pos = std::max(max_pos, p);
+    const bool extend = !blocks.empty() && slot_h[t - 1] == s && pos_h[t - 1] + 1 == p &&
+                        blocks.back().y < QB && (t - blocks.back().x) == blocks.back().y;
+    if (extend)
+      blocks.back().y++;
+    else
+      blocks.push_back(make_int2(t, 1));
+  }
+  const int max_chunks = max_pos / chunk + 1;
+  const size_t need = attn_ws_bytes(T, Hq, d, max_pos, chunk);
+  BI_REQUIRE(ws && ws_bytes >= need, BI_ERR_WORKSPACE, "bi_attention: workspace %zu < %zu", ws_bytes, need);
+
+  const int esz = f32 ? 4 : 2;
+  const uint64_t rows = (uint64_t)kv->n_slots * kv->n_layers * Hkv * kv->capacity;
+  CUtensorMap tk, tv;
+  const CUtensorMapDataType dt = f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  BI_TRY(encode_tmap_2d(&tk, dt, esz, kv->k, d, rows, (uint64_t)d * esz, 128 / esz, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+  BI_TRY(encode_tmap_2d(&tv, dt, esz, kv->v, d, rows, (uint64_t)d * esz, 128 / esz, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+
+  const int smem = attn_smem_bytes(d, f32);
+  static bool attr_done = false;
+  if (!attr_done) {
+    BI_CHECK_CUDA(cudaFuncSetAttribute(attn_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       attn_smem_bytes(128, 0) > attn_smem_bytes(128, 1) ? attn_smem_bytes(128, 0)
+                                                                                          : attn_smem_bytes(128, 1)));
+    attr_done = true;
+  }
+  float* part = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
+
+  // token groups bound the partials workspace; blocks never straddle a group
+  // boundary because a block is cut whenever it would cross one.
+  size_t bi0 = 0;
+  while (bi0 < blocks.size()) {
+    const int t_base = blocks[bi0].x;
+    size_t bi1 = bi0;
+    AttnPlan plan;
+    plan.n = 0;
+    while (bi1 < blocks.size() && plan.n < ATT_MAX_BLOCKS &&
+           blocks[bi1].x + blocks[bi1].y - t_base <= ATT_TOKEN_GROUP) {
+      plan.blk[plan.n++] = blocks[bi1++];
+    }
+    if (plan.n == 0) return set_error(BI_ERR_UNSUPPORTED, "bi_attention: planning failed");
+    const int t_end = blocks[bi1 - 1].x + blocks[bi1 - 1].y;
+    AttnArgs a;
+    a.q = q; a.slot = slot; a.pos = pos; a.part = part; a.t_base = t_base;
+    a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.d = d; a.chunk = chunk; a.max_chunks = max_chunks;
+    a.layer = layer; a.n_layers = kv->n_layers; a.cap = kv->capacity; a.f32 = f32; a.scale = scale;
+    dim3 grid(plan.n, max_chunks, Hkv);
+    attn_partial_kernel<<<grid, ATT_THREADS, smem, st>>>(tk, tv, plan, a);
+    BI_CHECK_LAUNCH();
+    const int nw = (t_end - t_base) * Hq;
+    attn_merge_kernel<<<(nw * 32 + 255) / 256, 256, 0, st>>>(part, pos, out, t_base, t_end - t_base, Hq, d, chunk,
+                                                              max_chunks, f32);
+    BI_CHECK_LAUNCH();
+    bi0 = bi1;
+  }
+  return BI_OK;
+}
+
+// ------------------------------------------------------------------ LM head
+struct LmWs {
+  uint16_t* h16;
+  float* logits;
+  LmPart* part;
+  uint8_t* flag;
+  int32_t* list;
+  int* count;
+  float* hc;
+  float* logits_c;
+};
+static LmWs lm_carve(Carver& cv, int B, int H, int V, int mode, bool own_logits) {
+  const int nch = (V + LM_CHUNK - 1) / LM_CHUNK;
+  LmWs w{};
+  w.h16 = mode == BI_MODE_BF16 ? cv.take<uint16_t>((size_t)B * H) : nullptr;
+  w.logits = own_logits ? cv.take<float>((size_t)B * V) : nullptr;
+  w.part = cv.take<LmPart>((size_t)B * nch);
+  w.flag = cv.take<uint8_t>(B);
+  w.list = cv.take<int32_t>(B);
+  w.count = cv.take<int>(1);
+  if (mode == BI_MODE_BF16) {
+    w.hc = cv.take<float>((size_t)B * H);
+    w.logits_c = cv.take<float>((size_t)B * V);
+  }
+  return w;
+}
+
+static int lmhead_run(const float* h, const void* W, const int32_t* target, int B, int H, int V, float thresh, int mode,
+                      float* logprob, float* lse, int32_t* argmax, float* margin, uint8_t* recomputed, float* logits,
+                      void* ws, size_t ws_bytes, cudaStream_t st) {
+  BI_REQUIRE(h && W && logprob && lse && argmax && margin && recomputed, BI_ERR_INVALID_ARG,
+             "bi_lmhead_logprob: NULL pointer");
+  BI_REQUIRE(B >= 0 && H > 0 && V > 0, BI_ERR_INVALID_ARG, "bi_lmhead_logprob: bad sizes");
+  BI_REQUIRE(H % 64 == 0 && V % 64 == 0, BI_ERR_UNSUPPORTED, "bi_lmhead_logprob: need H, V multiples of 64");
+  BI_REQUIRE(mode == BI_MODE_BF16 || mode == BI_MODE_LAYERCAST, BI_ERR_INVALID_ARG, "bi_lmhead_logprob: bad mode");
+  BI_REQUIRE(aligned16(h) && aligned16(W), BI_ERR_UNSUPPORTED, "bi_lmhead_logprob: h and W must be 16-byte aligned");
+  if (B == 0) return BI_OK;
+  Carver probe(nullptr);
+  lm_carve(probe, B, H, V, mode, logits == nullptr);
+  BI_REQUIRE(ws && ws_bytes >= probe.used + 256, BI_ERR_WORKSPACE, "bi_lmhead_logprob: workspace %zu < %zu", ws_bytes,
+             probe.used + 256);
+  Carver cv(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255)));
+  LmWs w = lm_carve(cv, B, H, V, mode, logits == nullptr);
+  float* z = logits ? logits : w.logits;
+  const int nch = (V + LM_CHUNK - 1) / LM_CHUNK;
+
+  if (mode == BI_MODE_BF16) {
+    const size_t n = (size_t)B * H;
+    f32_to_bf16_kernel<<<(int)std::min<size_t>((n + 255) / 256, 4096), 256, 0, st>>>(h, w.h16, n);
+    BI_CHECK_LAUNCH();
+    BI_TRY(gemm_bf16(w.h16, H, W, z, V, 1, B, V, H, BI_EPI_NONE, BI_VARIANT_INVARIANT, nullptr, 0, st));
+  } else {
+    BI_TRY(gemm_f32(h, H, W, z, V, 1, B, V, H, BI_EPI_NONE, nullptr, st));
+  }
+  lm_partial_kernel<<<dim3(nch, B), LM_CHUNK, 0, st>>>(z, V, V, target, nullptr, nullptr, w.part, nch);
+  BI_CHECK_LAUNCH();
+  const float th = mode == BI_MODE_BF16 ? thresh : 0.f;
+  lm_merge_kernel<<<(B * 32 + 127) / 128, 128, 0, st>>>(w.part, nch, B, nullptr, nullptr, target, th, 0, logprob, lse,
+                                                        argmax, margin, recomputed, w.flag);
+  BI_CHECK_LAUNCH();
+  if (mode == BI_MODE_BF16 && th > 0.f) {
+    lm_compact_kernel<<<1, 256, 0, st>>>(w.flag, B, h, H, w.list, w.count, w.hc);
+    BI_CHECK_LAUNCH();
+    BI_TRY(gemm_f32(w.hc, H, W, w.logits_c, V, 1, B, V, H, BI_EPI_NONE, w.count, st));
+    lm_partial_kernel<<<dim3(nch, B), LM_CHUNK, 0, st>>>(w.logits_c, V, V, target, w.list, w.count, w.part, nch);
+    BI_CHECK_LAUNCH();
+    lm_merge_kernel<<<(B * 32 + 127) / 128, 128, 0, st>>>(w.part, nch, B, w.count, w.list, target, th, 1, logprob,
+                                                          lse, argmax, margin, recomputed, nullptr);
+    BI_CHECK_LAUNCH();
+  }
+  return BI_OK;
+}
+
+}  // namespace bi
+
+// ====================================================================== C ABI
+using namespace bi;
+
+struct bi_ctx {
+  bi_model_desc desc;
+  bi_weights w;
+  bi_kv_layout kv;
+};
+
+extern "C" {
+
+const char* bi_last_error(void) { return t_last_error.c_str(); }
+int bi_version(void) { return 1; }
+long long bi_launch_count(void) { return g_launches; }
+int bi_num_sms(int device) {
+  int n = -1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return -1;
+  return n;
+}
+
+int bi_device_error(unsigned* flags, int reset) {
+  unsigned v = 0;
+  BI_CHECK_CUDA(cudaMemcpyFromSymbol(&v, g_dev_error, sizeof(v)));
+  if (flags) *flags = v;
+  if (reset) {
+    unsigned z = 0;
+    BI_CHECK_CUDA(cudaMemcpyToSymbol(g_dev_error, &z, sizeof(z)));
+  }
+  return BI_OK;
+}
+
+size_t bi_gemm_workspace_size(int M, int N, int K, int mode, int variant) {
+  if (M <= 0 || N <= 0 || K <= 0 || N % 64 || K % 64) return 0;
+  return gemm_ws_bytes(M, N, K, mode, variant);
+}
+
+int bi_gemm(const void* x, int ldx, const void* w, void* y, int ldy, int y_dtype, int M, int N, int K, int epilogue,
+            int mode, int variant, void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  return gemm_run(x, ldx, w, y, ldy, y_dtype, M, N, K, epilogue, mode, variant, ws, ws_bytes, as_stream(stream));
+}
+
+int bi_rmsnorm(const void* x, const void* residual_in, void* residual_out, const void* gamma, void* y, float* y_f32,
+               int M, int H, float eps, int mode, void* stream) {
+  clear_error();
+  BI_REQUIRE(x && gamma && y, BI_ERR_INVALID_ARG, "bi_rmsnorm: NULL pointer");
+  BI_REQUIRE(M >= 0 && H > 0 && H % 8 == 0 && H <= NORM_THREADS * NORM_MAX_CHUNKS * 8, BI_ERR_UNSUPPORTED,
+             "bi_rmsnorm: H=%d (need H %% 8 == 0, H <= 16384)", H);
+  BI_REQUIRE(mode == BI_MODE_BF16 || mode == BI_MODE_LAYERCAST, BI_ERR_INVALID_ARG, "bi_rmsnorm: bad mode");
+  BI_REQUIRE(aligned16(x) && aligned16(gamma) && aligned16(y) && (!residual_in || aligned16(residual_in)) &&
+                 (!residual_out || aligned16(residual_out)) && (!y_f32 || aligned16(y_f32)),
+             BI_ERR_UNSUPPORTED, "bi_rmsnorm: buffers must be 16-byte aligned");
+  if (M == 0) return BI_OK;
+  rmsnorm_kernel<<<M, NORM_THREADS, 0, as_stream(stream)>>>(x, residual_in, residual_out,
+                                                            reinterpret_cast<const uint16_t*>(gamma), y, y_f32, H, eps,
+                                                            mode == BI_MODE_LAYERCAST);
+  BI_CHECK_LAUNCH();
+  return BI_OK;
+}
+
+int bi_rope_table_fill(float* table, int max_pos, int head_dim, double theta, void* stream) {
+  clear_error();
+  BI_REQUIRE(table && max_pos > 0 && head_dim > 0 && head_dim % 2 == 0 && theta > 0, BI_ERR_INVALID_ARG,
+             "bi_rope_table_fill: bad arguments");
+  const int half = head_dim / 2;
+  std::vector<float> host((size_t)max_pos * head_dim);
+  for (int p = 0; p < max_pos; ++p)
+    for (int i = 0; i < half; ++i) {
+      const double ang = (double)p * std::pow(theta, -2.0 * i / head_dim);
+      host[((size_t)p * half + i) * 2] = (float)std::cos(ang);
+      host[((size_t)p * half + i) * 2 + 1] = (float)std::sin(ang);
+    }
+  // synchronous copy: the host buffer dies with this call
+  BI_CHECK_CUDA(cudaStreamSynchronize(as_stream(stream)));
+  BI_CHECK_CUDA(cudaMemcpy(table, host.data(), host.size() * sizeof(float), cudaMemcpyHostToDevice));
+  return BI_OK;
+}
+
+int bi_rope_kv_append(const float* qkv, const float* rope, int rope_max_pos, void* q_out, const bi_kv_layout* kv,
+                      int layer, const int32_t* slot, const int32_t* pos, int T, int Hq, int mode, void* stream) {
+  clear_error();
+  BI_REQUIRE(qkv && rope && q_out && kv && kv->k && kv->v && slot && pos, BI_ERR_INVALID_ARG,
+             "bi_rope_kv_append: NULL pointer");
+  BI_REQUIRE(layer >= 0 && layer < kv->n_layers && T >= 0 && Hq > 0, BI_ERR_INVALID_ARG, "bi_rope_kv_append: bad args");
+  BI_REQUIRE(kv->dtype == (mode == BI_MODE_LAYERCAST ? BI_DTYPE_F32 : BI_DTYPE_BF16), BI_ERR_INVALID_ARG,
+             "bi_rope_kv_append: KV dtype does not match the mode");
+  if (T == 0) return BI_OK;
+  rope_append_kernel<<<T, 256, 0, as_stream(stream)>>>(qkv, rope, rope_max_pos, q_out, kv->k, kv->v, slot, pos, Hq,
+                                                       kv->n_kv_heads, kv->head_dim, layer, kv->n_layers, kv->n_slots,
+                                                       kv->capacity, mode == BI_MODE_LAYERCAST);
+  BI_CHECK_LAUNCH();
+  return BI_OK;
+}
+
+size_t bi_attention_workspace_size(int T, int Hq, int head_dim, int max_pos) {
+  if (T <= 0 || Hq <= 0 || head_dim <= 0 || max_pos < 0) return 0;
+  // the largest of the invariant and FAST chunkings
+  return attn_ws_bytes(T, Hq, head_dim, max_pos, 64);
+}
+
+int bi_attention(const void* q, const bi_kv_layout* kv, int layer, const int32_t* slot, const int32_t* pos,
+                 const int32_t* slot_host, const int32_t* pos_host, void* out, int T, int Hq, float scale, int mode,
+                 int variant, void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  return attention_run(q, kv, layer, slot, pos, slot_host, pos_host, out, T, Hq, scale, mode, variant, ws, ws_bytes,
+                       as_stream(stream));
+}
+
+size_t bi_lmhead_workspace_size(int B, int H, int V, int mode) {
+  if (B <= 0 || H <= 0 || V <= 0) return 0;
+  Carver cv(nullptr);
+  lm_carve(cv, B, H, V, mode, true);
+  return cv.used + 256;
+}
+
+int bi_lmhead_logprob(const float* h, const void* W, const int32_t* target, int B, int H, int V,
+                      float margin_threshold, int mode, float* logprob, float* lse, int32_t* argmax, float* margin,
+                      uint8_t* recomputed, float* logits, void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  return lmhead_run(h, W, target, B, H, V, margin_threshold, mode, logprob, lse, argmax, margin, recomputed, logits,
+                    ws, ws_bytes, as_stream(stream));
+}
+
+int bi_ctx_create(const bi_model_desc* desc, const bi_weights* w, const bi_kv_layout* kv, bi_ctx** out) {
+  clear_error();
+  BI_REQUIRE(desc && w && kv && out, BI_ERR_INVALID_ARG, "bi_ctx_create: NULL pointer");
+  const bi_model_desc& d = *desc;
+  BI_REQUIRE(d.n_layers > 0 && d.hidden > 0 && d.n_heads > 0 && d.n_kv_heads > 0 && d.head_dim > 0 && d.ffn > 0 &&
+                 d.vocab > 0,
+             BI_ERR_INVALID_ARG, "bi_ctx_create: bad model sizes");
+  BI_REQUIRE(d.n_heads % d.n_kv_heads == 0, BI_ERR_INVALID_ARG, "bi_ctx_create: n_heads %% n_kv_heads != 0");
+  BI_REQUIRE(d.mode == BI_MODE_BF16 || d.mode == BI_MODE_LAYERCAST, BI_ERR_INVALID_ARG, "bi_ctx_create: bad mode");
+  BI_REQUIRE(d.variant == BI_VARIANT_INVARIANT || d.variant == BI_VARIANT_FAST, BI_ERR_INVALID_ARG,
+             "bi_ctx_create: bad variant");
+  const int QKV = (d.n_heads + 2 * d.n_kv_heads) * d.head_dim;
+  BI_REQUIRE(d.hidden % 64 == 0 && d.ffn % 64 == 0 && d.vocab % 64 == 0 && QKV % 64 == 0 &&
+                 (d.n_heads * d.head_dim) % 64 == 0 && d.ffn % BI_GU_INTERLEAVE == 0,
+             BI_ERR_UNSUPPORTED, "bi_ctx_create: hidden/ffn/vocab/projection sizes must be multiples of 64");
+  BI_REQUIRE(d.head_dim == 64 || d.head_dim == 128, BI_ERR_UNSUPPORTED, "bi_ctx_create: head_dim must be 64 or 128");
+  BI_REQUIRE(d.hidden <= 16384, BI_ERR_UNSUPPORTED, "bi_ctx_create: hidden > 16384");
+  BI_REQUIRE(w->embed && w->lm_head && w->final_norm && w->attn_norm && w->ffn_norm && w->w_qkv && w->w_o &&
+                 w->w_gu && w->w_down && w->rope && w->rope_max_pos > 0,
+             BI_ERR_INVALID_ARG, "bi_ctx_create: NULL weight pointer");
+  BI_REQUIRE(kv->k && kv->v && kv->n_layers == d.n_layers && kv->n_kv_heads == d.n_kv_heads &&
+                 kv->head_dim == d.head_dim && kv->n_slots > 0 && kv->capacity > 0,
+             BI_ERR_INVALID_ARG, "bi_ctx_create: KV layout does not match the model");
+  BI_REQUIRE(kv->dtype == (d.mode == BI_MODE_LAYERCAST ? BI_DTYPE_F32 : BI_DTYPE_BF16), BI_ERR_INVALID_ARG,
+             "bi_ctx_create: KV dtype does not match the mode");
+  bi_ctx* c = new (std::nothrow) bi_ctx;
+  BI_REQUIRE(c, BI_ERR_INVALID_ARG, "bi_ctx_create: out of host memory");
+  c->desc = d;
+  c->w = *w;
+  c->kv = *kv;
+  *out = c;
+  return BI_OK;
+}
+
+int bi_ctx_destroy(bi_ctx* ctx) {
+  delete ctx;
+  return BI_OK;
+}
+
+struct StepWs {
+  void *res, *u, *y, *q, *o, *a;
+  float* qkv;
+  float* h32;
+  float* hl;
+  uint8_t* attn;
+  size_t attn_bytes;
+  uint8_t* lm;
+  size_t lm_bytes;
+  uint8_t* gemm;  // split-K partials of the FAST variant
+  size_t gemm_bytes;
+};
+
+static StepWs step_carve(Carver& cv, const bi_model_desc& d, int T, int n_lm, int max_pos) {
+  const size_t es = d.mode == BI_MODE_LAYERCAST ? 4 : 2;
+  const int QD = d.n_heads * d.head_dim, KD = d.n_kv_heads * d.head_dim;
+  StepWs s{};
+  s.res = cv.take<uint8_t>((size_t)T * d.hidden * es);
+  s.u = cv.take<uint8_t>((size_t)T * d.hidden * es);
+  s.y = cv.take<uint8_t>((size_t)T * d.hidden * es);
+  s.q = cv.take<uint8_t>((size_t)T * QD * es);
+  s.o = cv.take<uint8_t>((size_t)T * QD * es);
+  s.a = cv.take<uint8_t>((size_t)T * d.ffn * es);
+  s.qkv = cv.take<float>((size_t)T * (QD + 2 * KD));
+  s.h32 = cv.take<float>((size_t)T * d.hidden);
+  s.hl = cv.take<float>((size_t)std::max(n_lm, 1) * d.hidden);
+  s.attn_bytes = bi_attention_workspace_size(T, d.n_heads, d.head_dim, max_pos);
+  s.attn = cv.take<uint8_t>(s.attn_bytes);
+  s.lm_bytes = bi_lmhead_workspace_size(std::max(n_lm, 1), d.hidden, d.vocab, d.mode);
+  s.lm = cv.take<uint8_t>(s.lm_bytes);
+  const int QKV = QD + 2 * KD;
+  s.gemm_bytes = std::max(std::max(gemm_ws_bytes(T, QKV, d.hidden, d.mode, d.variant),
+                                   gemm_ws_bytes(T, d.hidden, QD, d.mode, d.variant)),
+                          std::max(gemm_ws_bytes(T, 2 * d.ffn, d.hidden, d.mode, d.variant),
+                                   gemm_ws_bytes(T, d.hidden, d.ffn, d.mode, d.variant)));
+  s.gemm = s.gemm_bytes ? cv.take<uint8_t>(s.gemm_bytes) : nullptr;
+  return s;
+}
+
+size_t bi_decode_workspace_size(const bi_ctx* ctx, int max_tokens, int max_lm_rows, int max_pos) {
+  if (!ctx || max_tokens <= 0 || max_lm_rows < 0 || max_pos < 0) return 0;
+  Carver cv(nullptr);
+  step_carve(cv, ctx->desc, max_tokens, max_lm_rows, max_pos);
+  return cv.used + 256;
+}
+
+__global__ void gather_lm_rows_kernel(const int32_t* __restrict__ lm_row, const float* __restrict__ h32, int T, int H,
+                                      int n_lm, float* __restrict__ hl, float* __restrict__ h_out) {
+  const int t = blockIdx.x;
+  const int r = lm_row[t];
+  if (r < 0) return;
+  if (r >= n_lm) {
+    if (threadIdx.x == 0) dev_flag(DEVERR_INDEX);
+    return;
+  }
+  for (int i = threadIdx.x; i < H; i += blockDim.x) {
+    const float v = h32[(size_t)t * H + i];
+    hl[(size_t)r * H + i] = v;
+    if (h_out) h_out[(size_t)r * H + i] = v;
+  }
+}
+
+int bi_decode_step(bi_ctx* ctx, const bi_batch* batch, const bi_step_out* out, void* ws, size_t ws_bytes,
+                   void* stream) {
+  clear_error();
+  BI_REQUIRE(ctx && batch && out, BI_ERR_INVALID_ARG, "bi_decode_step: NULL pointer");
+  const bi_model_desc& d = ctx->desc;
+  const bi_weights& w = ctx->w;
+  const int T = batch->n_tokens, n_lm = batch->n_lm;
+  BI_REQUIRE(T >= 0 && n_lm >= 0 && n_lm <= T, BI_ERR_INVALID_ARG, "bi_decode_step: n_tokens=%d n_lm=%d", T, n_lm);
+  if (T == 0) return BI_OK;
+  BI_REQUIRE(batch->ids && batch->slot && batch->pos && batch->slot_host && batch->pos_host && batch->lm_row,
+             BI_ERR_INVALID_ARG, "bi_decode_step: NULL batch array");
+  BI_REQUIRE(n_lm == 0 || (out->logprob && out->lse && out->argmax && out->margin && out->recomputed),
+             BI_ERR_INVALID_ARG, "bi_decode_step: NULL output array");
+  int max_pos = 0;
+  for (int t = 0; t < T; ++t) {
+    const int p = batch->pos_host[t];
+    BI_REQUIRE(p >= 0 && p < ctx->kv.capacity && p < w.rope_max_pos, BI_ERR_CAPACITY,
+               "bi_decode_step: token %d position %d beyond KV capacity %d / RoPE table %d", t, p, ctx->kv.capacity,
+               w.rope_max_pos);
+    max_pos = std::max(max_pos, p);
+  }
+  const size_t need = bi_decode_workspace_size(ctx, T, n_lm, max_pos);
+  BI_REQUIRE(ws && ws_bytes >= need, BI_ERR_WORKSPACE, "bi_decode_step: workspace %zu < %zu", ws_bytes, need);
+  Carver cv(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255)));
+  StepWs s = step_carve(cv, d, T, n_lm, max_pos);
+  cudaStream_t st = as_stream(stream);
+  const int H = d.hidden, Hq = d.n_heads, Hkv = d.n_kv_heads, hd = d.head_dim, F = d.ffn;
+  const int QD = Hq * hd, KD = Hkv * hd, QKV = QD + 2 * KD;
+  const int f32 = d.mode == BI_MODE_LAYERCAST;
+  const int act_dtype = f32 ? BI_DTYPE_F32 : BI_DTYPE_BF16;
+  const size_t wbytes = 2;
+  const float scale = 1.0f / std::sqrt((float)hd);
+  auto lw = [&](const void* base, size_t per_layer, int l) {
+    return reinterpret_cast<const void*>(reinterpret_cast<const uint8_t*>(base) + per_layer * l * wbytes);
+  };
+
+  embed_kernel<<<T, 256, 0, st>>>(batch->ids, reinterpret_cast<const uint16_t*>(w.embed), s.y, H, d.vocab, f32);
+  BI_CHECK_LAUNCH();
+  for (int l = 0; l < d.n_layers; ++l) {
+    const void* g_attn = lw(w.attn_norm, H, l);
+    const void* g_ffn = lw(w.ffn_norm, H, l);
+    BI_TRY(bi_rmsnorm(s.y, l == 0 ? nullptr : s.res, s.res, g_attn, s.u, nullptr, T, H, d.eps, d.mode, stream));
+    BI_TRY(gemm_run(s.u, H, lw(w.w_qkv, (size_t)QKV * H, l), s.qkv, QKV, BI_DTYPE_F32, T, QKV, H, BI_EPI_NONE, d.mode,
+                    d.variant, s.gemm, s.gemm_bytes, st));
+    BI_TRY(bi_rope_kv_append(s.qkv, w.rope, w.rope_max_pos, s.q, &ctx->kv, l, batch->slot, batch->pos, T, Hq, d.mode,
+                             stream));
+    BI_TRY(attention_run(s.q, &ctx->kv, l, batch->slot, batch->pos, batch->slot_host, batch->pos_host, s.o, T, Hq,
+                         scale, d.mode, d.variant, s.gemm, s.gemm_bytes, st));
+    BI_TRY(gemm_run(s.o, QD, lw(w.w_o, (size_t)H * QD, l), s.y, H, act_dtype, T, H, QD, BI_EPI_NONE, d.mode,
+                    d.variant, s.gemm, s.gemm_bytes, st));
+    BI_TRY(bi_rmsnorm(s.y, s.res, s.res, g_ffn, s.u, nullptr, T, H, d.eps, d.mode, stream));
+    BI_TRY(gemm_run(s.u, H, lw(w.w_gu, (size_t)2 * F * H, l), s.a, F, act_dtype, T, 2 * F, H, BI_EPI_SWIGLU, d.mode,
+                    d.variant, s.gemm, s.gemm_bytes, st));
+    BI_TRY(gemm_run(s.a, F, lw(w.w_down, (size_t)H * F, l), s.y, H, act_dtype, T, H, F, BI_EPI_NONE, d.mode,
+                    d.variant, s.gemm, s.gemm_bytes, st));
+  }
+  BI_TRY(bi_rmsnorm(s.y, s.res, s.res, w.final_norm, s.u, s.h32, T, H, d.eps, d.mode, stream));
+  if (n_lm == 0) return BI_OK;
+  gather_lm_rows_kernel<<<T, 256, 0, st>>>(batch->lm_row, s.h32, T, H, n_lm, s.hl, out->h);
+  BI_CHECK_LAUNCH();
+  return lmhead_run(s.hl, w.lm_head, batch->target, n_lm, H, d.vocab, d.margin_threshold, d.mode, out->logprob,
+                    out->lse, out->argmax, out->margin, out->recomputed, out->logits, s.lm, s.lm_bytes, st);
+}
+
+int bi_greedy_advance(const int32_t* argmax, int32_t* ids, int32_t* pos, int B, void* stream) {
+  clear_error();
+  BI_REQUIRE(argmax && ids && pos && B >= 0, BI_ERR_INVALID_ARG, "bi_greedy_advance: bad arguments");
+  if (B == 0) return BI_OK;
+  greedy_advance_kernel<<<(B + 127) / 128, 128, 0, as_stream(stream)>>>(argmax, ids, pos, B);
+  BI_CHECK_LAUNCH();
+  return BI_OK;
+}
+
+int bi_synth_fill_bf16(uint16_t* dst, int64_t rows, int64_t cols, uint64_t key, double std, int interleave, int phase,
+                       void* stream) {
+  clear_error();
+  BI_REQUIRE(dst && rows >= 0 && cols > 0 && interleave >= 0 && (phase == 0 || phase == 1), BI_ERR_INVALID_ARG,
+             "bi_synth_fill_bf16: bad arguments");
+  BI_REQUIRE(interleave == 0 || rows % interleave == 0, BI_ERR_INVALID_ARG,
+             "bi_synth_fill_bf16: rows must be a multiple of the interleave");
+  if (rows == 0) return BI_OK;
+  synth_fill_kernel<<<4 * num_sms(), 256, 0, as_stream(stream)>>>(dst, rows, cols, key, std, interleave, phase);
+  BI_CHECK_LAUNCH();
+  return BI_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,186 @@
+// bi_lmhead_logprob kernels: vocabulary-chunk partials, fixed-order merge,
+// and the selective FP32 recompute bookkeeping.
+//
+// ("Meituan bitwise train/infer consistency": logprob accumulation is one of
+// the reductions whose order is fixed; "Greedy Decoding Is Not
+// Precision-Invariant", method section: top-two logit margin, FP32 LM-head
+// recompute only when it falls below a threshold.)
+//
+// Per row and per chunk of BI_VOCAB_CHUNK = 256 logits (thread j <-> logit j):
+//   max (exact), sum exp(z - max) with a fixed tree (xor-butterfly per warp,
+//   then the 8 warp sums in ascending order), top-1 and top-2 as (value, id)
+//   under the total order "larger value, then lower id" (exact, order-free),
+//   and the target logit if the target falls in the chunk.
+// Merge per row: M = max over chunks (exact); S = sum_c s_c exp(m_c - M):
+//   lane i of one warp sums chunks i, i+32, ... in ascending order, then a
+//   fixed xor-butterfly; lse = M + ln S; top-2 merged exactly.
+#pragma once
+#include "common.cuh"
+
+namespace bi {
+
+constexpr int LM_CHUNK = BI_VOCAB_CHUNK;  // 256
+struct LmPart {
+  float mx, sum, v1, v2, zt;
+  int i1, i2, has_t;
+};
+
+// (v, i) beats (w, j) if v > w, or v == w and i < j.
+__device__ __forceinline__ bool lm_better(float v, int i, float w, int j) { return v > w || (v == w && i < j); }
+__device__ __forceinline__ void lm_top2_insert(float& v1, int& i1, float& v2, int& i2, float v, int i) {
+  if (lm_better(v, i, v1, i1)) {
+    v2 = v1; i2 = i1; v1 = v; i1 = i;
+  } else if (lm_better(v, i, v2, i2)) {
+    v2 = v; i2 = i;
+  }
+}
+__device__ __forceinline__ void lm_top2_warp(float& v1, int& i1, float& v2, int& i2) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov1 = __shfl_xor_sync(0xffffffffu, v1, o), ov2 = __shfl_xor_sync(0xffffffffu, v2, o);
+    const int oi1 = __shfl_xor_sync(0xffffffffu, i1, o), oi2 = __shfl_xor_sync(0xffffffffu, i2, o);
+    lm_top2_insert(v1, i1, v2, i2, ov1, oi1);
+    lm_top2_insert(v1, i1, v2, i2, ov2, oi2);
+  }
+}
+
+// Grid (n_chunks, B).  logits: [rows][ldz] f32.  Row r of the grid is
+// logits row r; rows >= *count (when count != nullptr) are skipped.
+// target: per-row target id (nullptr: none); rows_map maps grid row -> target
+// row (nullptr: identity).
+__global__ void __launch_bounds__(LM_CHUNK)
+    lm_partial_kernel(const float* __restrict__ logits, size_t ldz, int V, const int32_t* __restrict__ target,
+                      const int32_t* __restrict__ rows_map, const int* __restrict__ count, LmPart* __restrict__ part,
+                      int n_chunks) {
+  const int c = blockIdx.x, r = blockIdx.y;
+  if (count && r >= *count) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int v = c * LM_CHUNK + tid;
+  const bool ok = v < V;
+  const float z = ok ? logits[(size_t)r * ldz + v] : -INFINITY;
+  __shared__ float wm[LM_CHUNK / 32], ws[LM_CHUNK / 32], wv1[LM_CHUNK / 32], wv2[LM_CHUNK / 32];
+  __shared__ int wi1[LM_CHUNK / 32], wi2[LM_CHUNK / 32];
+  __shared__ float zt_s;
+  __shared__ int has_s;
+  if (tid == 0) has_s = 0;
+  float mx = warp_max(z);
+  if (lane == 0) wm[warp] = mx;
+  float v1 = z, v2 = -INFINITY;
+  int i1 = ok ? v : 0x7fffffff, i2 = 0x7fffffff;
+  lm_top2_warp(v1, i1, v2, i2);
+  if (lane == 0) {
+    wv1[warp] = v1; wi1[warp] = i1; wv2[warp] = v2; wi2[warp] = i2;
+  }
+  __syncthreads();
+  float M = wm[0];
+#pragma unroll
+  for (int w = 1; w < LM_CHUNK / 32; ++w) M = fmaxf(M, wm[w]);
+  float e = ok ? expf(z - M) : 0.f;
+  e = warp_sum_fixed(e);
+  if (lane == 0) ws[warp] = e;
+  if (target) {
+    const int tr = rows_map ? rows_map[r] : r;
+    const int tg = target[tr];
+    if (ok && v == tg) {
+      zt_s = z;
+      has_s = 1;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float S = 0.f;
+    for (int w = 0; w < LM_CHUNK / 32; ++w) S += ws[w];
+    float a1 = wv1[0], a2 = wv2[0];
+    int j1 = wi1[0], j2 = wi2[0];
+    for (int w = 1; w < LM_CHUNK / 32; ++w) {
+      lm_top2_insert(a1, j1, a2, j2, wv1[w], wi1[w]);
+      lm_top2_insert(a1, j1, a2, j2, wv2[w], wi2[w]);
+    }
+    LmPart pr;
+    pr.mx = M; pr.sum = S; pr.v1 = a1; pr.i1 = j1; pr.v2 = a2; pr.i2 = j2;
+    pr.has_t = has_s; pr.zt = has_s ? zt_s : 0.f;
+    part[(size_t)r * n_chunks + c] = pr;
+  }
+}
+
+// One warp per row.  mode_recompute = 0: main pass (writes every output and
+// sets the flag); 1: recompute pass (rows given by rows_map, writes lse,
+// logprob, argmax and recomputed = 1; margin keeps the main-pass value).
+__global__ void lm_merge_kernel(const LmPart* __restrict__ part, int n_chunks, int B, const int* __restrict__ count,
+                                const int32_t* __restrict__ rows_map, const int32_t* __restrict__ target,
+                                float thresh, int mode_recompute, float* __restrict__ logprob, float* __restrict__ lse,
+                                int32_t* __restrict__ argmax, float* __restrict__ margin,
+                                uint8_t* __restrict__ recomputed, uint8_t* __restrict__ flag) {
+  const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nrows = count ? min(B, *count) : B;
+  if (r >= nrows) return;
+  const LmPart* pr = part + (size_t)r * n_chunks;
+  float M = -INFINITY;
+  for (int c = lane; c < n_chunks; c += 32) M = fmaxf(M, pr[c].mx);
+  M = warp_max(M);
+  float S = 0.f, zt = 0.f;
+  int has = 0;
+  float v1 = -INFINITY, v2 = -INFINITY;
+  int i1 = 0x7fffffff, i2 = 0x7fffffff;
+  for (int c = lane; c < n_chunks; c += 32) {
+    const LmPart q = pr[c];
+    S = fmaf(q.sum, expf(q.mx - M), S);
+    lm_top2_insert(v1, i1, v2, i2, q.v1, q.i1);
+    lm_top2_insert(v1, i1, v2, i2, q.v2, q.i2);
+    if (q.has_t) {
+      has = 1;
+      zt = q.zt;
+    }
+  }
+  S = warp_sum_fixed(S);
+  lm_top2_warp(v1, i1, v2, i2);
+  const unsigned hb = __ballot_sync(0xffffffffu, has);
+  const int src = hb ? __ffs(hb) - 1 : 0;
+  zt = __shfl_sync(0xffffffffu, zt, src);
+  if (lane != 0) return;
+  const float L = M + logf(S);
+  const int orow = rows_map ? rows_map[r] : r;
+  const int tg = target ? target[orow] : -1;
+  const float lp = (tg >= 0 && hb) ? zt - L : v1 - L;
+  lse[orow] = L;
+  logprob[orow] = lp;
+  argmax[orow] = i1;
+  if (!mode_recompute) {
+    const float mg = v1 - v2;
+    margin[orow] = mg;
+    const bool f = thresh > 0.f && mg < thresh;
+    if (flag) flag[orow] = f;
+    recomputed[orow] = 0;
+  } else {
+    recomputed[orow] = 1;
+  }
+}
+
+// Ascending compaction of the flagged rows: list[k] = k-th flagged row, and
+// the f32 hidden rows gathered in that order.  One CTA.
+__global__ void lm_compact_kernel(const uint8_t* __restrict__ flag, int B, const float* __restrict__ h, int H,
+                                  int32_t* __restrict__ list, int* __restrict__ count, float* __restrict__ hc) {
+  __shared__ int n_s;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int b = 0; b < B; ++b)
+      if (flag[b]) list[n++] = b;
+    n_s = n;
+    *count = n;
+  }
+  __syncthreads();
+  const int n = n_s;
+  for (int k = 0; k < n; ++k) {
+    const int b = list[k];
+    for (int i = threadIdx.x; i < H; i += blockDim.x) hc[(size_t)k * H + i] = h[(size_t)b * H + i];
+  }
+}
+
+// h (f32) -> bf16 (round to nearest even), the main-pass LM-head input.
+__global__ void f32_to_bf16_kernel(const float* __restrict__ in, uint16_t* __restrict__ out, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    out[i] = f32_to_bf16_bits(in[i]);
+}
+
+}  // namespace bi

@@ -1,0 +1,143 @@
+"""The C-ABI library loads, exports every symbol include/bi.h declares, and
+rejects invalid arguments on the host with status codes (no GPU needed: every
+case here fails validation before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from invariant_deterministic_full_b200 import build
+    build.build()
+    from invariant_deterministic_full_b200 import _lib
+    return _lib
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "bi.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bi_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_symbols_exported(L):
+    names = _declared()
+    assert len(names) >= 19
+    so = ctypes.CDLL(L.LIB_PATH)
+    for n in names:
+        assert hasattr(so, n), f"{n} declared in bi.h but not exported"
+    assert set(names) == set(L.SIGNATURES), "binding and header disagree"
+
+
+def test_version_and_status_codes(L):
+    assert L.lib.bi_version() == 1
+    assert (L.BI_ERR_INVALID_ARG, L.BI_ERR_UNSUPPORTED, L.BI_ERR_WORKSPACE, L.BI_ERR_CAPACITY, L.BI_ERR_CUDA) == \
+        (1, 2, 3, 4, 5)
+
+
+def test_gemm_validation(L):
+    lib = L.lib
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    assert lib.bi_gemm(None, 64, fake, fake, 64, 0, 4, 64, 64, 0, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
+    assert lib.bi_gemm(fake, 96, fake, fake, 64, 0, 4, 64, 96, 0, 0, 0, None, 0, None) == L.BI_ERR_UNSUPPORTED
+    assert b"K % 64" in lib.bi_last_error()
+    assert lib.bi_gemm(fake, 64, fake, fake, 64, 0, 4, 96, 64, 0, 0, 0, None, 0, None) == L.BI_ERR_UNSUPPORTED
+    assert lib.bi_gemm(fake, 60, fake, fake, 64, 0, 4, 64, 64, 0, 0, 0, None, 0, None) == L.BI_ERR_UNSUPPORTED
+    assert lib.bi_gemm(fake, 64, fake, fake, 16, 0, 4, 64, 64, 0, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
+    assert lib.bi_gemm(fake, 64, fake, fake, 64, 0, 4, 64, 64, 7, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
+    assert lib.bi_gemm(fake, 64, ctypes.c_void_p((1 << 20) + 2), fake, 64, 0, 4, 64, 64, 0, 0, 0, None, 0,
+                       None) == L.BI_ERR_UNSUPPORTED
+    assert lib.bi_gemm(fake, 64, fake, fake, 64, 0, 0, 64, 64, 0, 0, 0, None, 0, None) == L.BI_OK  # M = 0: no work
+    assert lib.bi_gemm_workspace_size(4, 64, 64, 0, 0) == 0
+
+
+def test_rmsnorm_lmhead_validation(L):
+    lib = L.lib
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.bi_rmsnorm(None, None, None, fake, fake, None, 2, 64, 1e-5, 0, None) == L.BI_ERR_INVALID_ARG
+    assert lib.bi_rmsnorm(fake, None, None, fake, fake, None, 2, 60, 1e-5, 0, None) == L.BI_ERR_UNSUPPORTED
+    assert lib.bi_rmsnorm(fake, None, None, fake, fake, None, 2, 32768, 1e-5, 0, None) == L.BI_ERR_UNSUPPORTED
+    args = [fake] * 6
+    assert lib.bi_lmhead_logprob(None, fake, None, 2, 64, 128, 0.1, 0, *args[:5], None, fake, 1 << 30,
+                                 None) == L.BI_ERR_INVALID_ARG
+    assert lib.bi_lmhead_logprob(fake, fake, None, 2, 64, 100, 0.1, 0, *args[:5], None, fake, 1 << 30,
+                                 None) == L.BI_ERR_UNSUPPORTED
+    need = lib.bi_lmhead_workspace_size(2, 64, 128, 0)
+    assert need > 0
+    assert lib.bi_lmhead_logprob(fake, fake, None, 2, 64, 128, 0.1, 0, *args[:5], None, fake, need - 512,
+                                 None) == L.BI_ERR_WORKSPACE
+
+
+def _tiny_ctx(L, capacity=64, mode=0):
+    fake = 1 << 20
+    desc = L.ModelDesc(1, 256, 4, 4, 64, 1024, 4096, 1e-5, mode, 0, 0.1)
+    w = L.Weights(*([fake] * 10), capacity)
+    kv = L.KvLayout(fake, fake, 2, 1, 4, capacity, 64, 1 if mode else 0)
+    ctx = ctypes.c_void_p()
+    rc = L.lib.bi_ctx_create(ctypes.byref(desc), ctypes.byref(w), ctypes.byref(kv), ctypes.byref(ctx))
+    return rc, ctx, kv
+
+
+def test_ctx_validation(L):
+    lib = L.lib
+    rc, ctx, kv = _tiny_ctx(L)
+    assert rc == L.BI_OK and ctx.value
+    assert lib.bi_decode_workspace_size(ctx, 8, 8, 63) > 0
+    # KV dtype must follow the mode
+    desc = L.ModelDesc(1, 256, 4, 4, 64, 1024, 4096, 1e-5, 1, 0, 0.1)
+    w = L.Weights(*([1 << 20] * 10), 64)
+    c2 = ctypes.c_void_p()
+    assert lib.bi_ctx_create(ctypes.byref(desc), ctypes.byref(w), ctypes.byref(kv), ctypes.byref(c2)) == \
+        L.BI_ERR_INVALID_ARG
+    bad = L.ModelDesc(1, 250, 4, 4, 64, 1024, 4096, 1e-5, 0, 0, 0.1)
+    assert lib.bi_ctx_create(ctypes.byref(bad), ctypes.byref(w), ctypes.byref(kv), ctypes.byref(c2)) == \
+        L.BI_ERR_UNSUPPORTED
+    bad = L.ModelDesc(1, 256, 6, 4, 64, 1024, 4096, 1e-5, 0, 0, 0.1)
+    assert lib.bi_ctx_create(ctypes.byref(bad), ctypes.byref(w), ctypes.byref(kv), ctypes.byref(c2)) == \
+        L.BI_ERR_INVALID_ARG
+    lib.bi_ctx_destroy(ctx)
+
+
+def test_decode_step_capacity_and_workspace_rejected_on_host(L):
+    lib = L.lib
+    rc, ctx, _ = _tiny_ctx(L, capacity=64)
+    assert rc == L.BI_OK
+    slot = np.zeros(3, dtype=np.int32)
+    pos = np.array([10, 11, 64], dtype=np.int32)  # 64 == capacity
+    fake = 1 << 20
+    b = L.Batch(3, fake, fake, fake, slot.ctypes.data, pos.ctypes.data, fake, 3, 0)
+    o = L.StepOut(fake, fake, fake, fake, fake, 0, 0)
+    assert lib.bi_decode_step(ctx, ctypes.byref(b), ctypes.byref(o), ctypes.c_void_p(fake), 1 << 40, None) == \
+        L.BI_ERR_CAPACITY
+    assert b"capacity" in lib.bi_last_error()
+    pos[2] = 12
+    need = lib.bi_decode_workspace_size(ctx, 3, 3, 12)
+    assert lib.bi_decode_step(ctx, ctypes.byref(b), ctypes.byref(o), ctypes.c_void_p(fake), need - 1024, None) == \
+        L.BI_ERR_WORKSPACE
+    b.n_lm = 4  # more output rows than tokens
+    assert lib.bi_decode_step(ctx, ctypes.byref(b), ctypes.byref(o), ctypes.c_void_p(fake), need, None) == \
+        L.BI_ERR_INVALID_ARG
+    lib.bi_ctx_destroy(ctx)
+
+
+def test_attention_validation(L):
+    lib = L.lib
+    fake = 1 << 20
+    kv = L.KvLayout(fake, fake, 2, 1, 4, 64, 64, 0)
+    slot = np.array([0, 2], dtype=np.int32)
+    pos = np.array([0, 1], dtype=np.int32)
+    args = lambda s, p: (ctypes.c_void_p(fake), ctypes.byref(kv), 0, ctypes.c_void_p(fake), ctypes.c_void_p(fake),
+                         s.ctypes.data, p.ctypes.data, ctypes.c_void_p(fake), 2, 4, 0.125, 0, 0,
+                         ctypes.c_void_p(fake), 1 << 30, None)
+    assert lib.bi_attention(*args(slot, pos)) == L.BI_ERR_INVALID_ARG  # slot 2 of 2
+    slot[1] = 1
+    pos[1] = 70
+    assert lib.bi_attention(*args(slot, pos)) == L.BI_ERR_CAPACITY
+    kv.head_dim = 96
+    pos[1] = 1
+    assert lib.bi_attention(*args(slot, pos)) == L.BI_ERR_UNSUPPORTED

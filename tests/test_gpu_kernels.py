@@ -1,0 +1,323 @@
+"""Kernel-level GPU tests through the C ABI: oracle parity and bitwise batch invariance.
+
+Tolerances (floating point), derived from the arithmetic:
+  * fp32-accumulated dot products of length K vs the fp64 oracle:
+    |err| <= K * 2^-24 * sum_k |x_k w_k| (worst-case recursive-summation bound);
+    index or layout mistakes give errors ~ sum|xw| / sqrt(K), far above it.
+  * bf16-rounded outputs add one half-ulp of the result: 2^-8 |y|.
+Integer-valued inputs make every product and partial sum exact in fp32, so
+there the GPU must match exactly (pins layout and indexing with no rounding).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bi():
+    import invariant_deterministic_full_b200 as pkg
+    from invariant_deterministic_full_b200 import ops
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    ops.device_error(reset=True)
+    return ops
+
+
+def _bf16_dev(a):
+    return torch.from_numpy(np.ascontiguousarray(synth.f32_to_bf16_bits(np.asarray(a, np.float32))).view(np.int16)) \
+        .cuda().view(torch.bfloat16)
+
+
+def _f(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def _after(bi):
+    torch.cuda.synchronize()
+    assert bi.device_error(reset=True) == 0
+
+
+# ------------------------------------------------------------------ synthetic generator
+def test_device_generator_matches_host(bi):
+    k = synth.key(synth.WEIGHT_SEED, 12345)
+    rows, cols = 64, 96
+    d = torch.empty(rows, cols, dtype=torch.bfloat16, device="cuda")
+    bi.synth_fill_bf16(d, rows, cols, k, 0.02)
+    host = synth.normal_bf16(k, rows * cols, 0.02).reshape(rows, cols)
+    assert np.array_equal(d.view(torch.int16).cpu().numpy().view(np.uint16), host)
+    # gate/up interleave: logical row r -> fused row (r//16)*32 + phase*16 + r%16
+    gu = torch.zeros(2 * rows, cols, dtype=torch.bfloat16, device="cuda")
+    kg, ku = synth.key(1, 2), synth.key(1, 3)
+    bi.synth_fill_bf16(gu, rows, cols, kg, 0.02, interleave=16, phase=0)
+    bi.synth_fill_bf16(gu, rows, cols, ku, 0.02, interleave=16, phase=1)
+    from invariant_deterministic_full_b200.model import interleave_gu
+    ref = interleave_gu(synth.normal_bf16(kg, rows * cols).reshape(rows, cols),
+                        synth.normal_bf16(ku, rows * cols).reshape(rows, cols))
+    assert np.array_equal(gu.view(torch.int16).cpu().numpy().view(np.uint16), ref)
+    _after(bi)
+
+
+# ------------------------------------------------------------------ GEMM
+GEMM_SHAPES = [(1, 64, 64), (5, 192, 128), (32, 256, 320), (33, 4096, 256), (77, 8256, 128), (40, 16384, 64)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_gemm_integer_exact(bi, M, N, K):
+    rng = np.random.default_rng(M * 1000 + N + K)
+    x = rng.integers(-4, 5, size=(M, K)).astype(np.float32)
+    w = rng.integers(-4, 5, size=(N, K)).astype(np.float32)
+    exact = (x.astype(np.int64) @ w.T.astype(np.int64)).astype(np.float64)
+    xd, wd = _bf16_dev(x), _bf16_dev(w)
+    y = bi.gemm(xd, wd, out_dtype=torch.float32)
+    assert np.array_equal(_f(y), exact)
+    yb = bi.gemm(xd, wd, out_dtype=torch.bfloat16)
+    assert np.array_equal(yb.view(torch.int16).cpu().numpy().view(np.uint16),
+                          synth.f32_to_bf16_bits(exact.astype(np.float32)))
+    # LayerCast: f32 activations, bf16 weights upcast in registers
+    y32 = bi.gemm(torch.from_numpy(x).cuda(), wd, mode=1, out_dtype=torch.float32)
+    assert np.array_equal(_f(y32), exact)
+    _after(bi)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_gemm_swiglu_epilogue(bi, mode):
+    rng = np.random.default_rng(7 + mode)
+    M, F, K = 9, 256, 128
+    x = rng.integers(-2, 3, size=(M, K)).astype(np.float32)
+    wg = rng.integers(-2, 3, size=(F, K)).astype(np.float32) * 0.125
+    wu = rng.integers(-2, 3, size=(F, K)).astype(np.float32) * 0.125
+    from invariant_deterministic_full_b200.model import interleave_gu
+    wgu = interleave_gu(wg, wu)
+    g = x.astype(np.float64) @ wg.T
+    u = x.astype(np.float64) @ wu.T
+    ref = g / (1 + np.exp(-g)) * u
+    xd = _bf16_dev(x) if mode == 0 else torch.from_numpy(x).cuda()
+    y = bi.gemm(xd, _bf16_dev(wgu), epilogue=1, mode=mode, out_dtype=torch.float32)
+    assert np.allclose(_f(y), ref, rtol=1e-6, atol=1e-6)
+    _after(bi)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("M,N,K", [(3, 128, 4096), (45, 6144, 512), (8, 4096, 14336)])
+def test_gemm_random_vs_oracle(bi, mode, M, N, K):
+    rng = np.random.default_rng(11)
+    xb = synth.f32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    wb = synth.f32_to_bf16_bits((0.02 * rng.standard_normal((N, K))).astype(np.float32))
+    x = synth.bf16_to_f32(xb)
+    ref = oracle.gemm(x.astype(np.float64), wb)
+    bound = K * 2.0 ** -24 * (np.abs(x).astype(np.float64) @ np.abs(synth.bf16_to_f32(wb)).astype(np.float64).T)
+    xd = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16) if mode == 0 else torch.from_numpy(x).cuda()
+    y = _f(bi.gemm(xd, torch.from_numpy(wb.view(np.int16)).cuda().view(torch.bfloat16), mode=mode,
+                   out_dtype=torch.float32))
+    assert (np.abs(y - ref) <= bound + 1e-30).all()
+    _after(bi)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_gemm_batch_invariance(bi, mode):
+    """Row r of x.W^T is bitwise the same whatever the number of rows and the row's position."""
+    rng = np.random.default_rng(5)
+    N, K = 4096, 1024
+    xs = rng.standard_normal((100, K)).astype(np.float32)
+    if mode == 0:
+        xs = synth.bf16_to_f32(synth.f32_to_bf16_bits(xs))
+    w = _bf16_dev(0.02 * rng.standard_normal((N, K)))
+    dev = lambda a: (_bf16_dev(a) if mode == 0 else torch.from_numpy(np.ascontiguousarray(a)).cuda())
+    full = bi.gemm(dev(xs), w, mode=mode, out_dtype=torch.float32).cpu()
+    for M, off in [(1, 0), (1, 57), (4, 30), (31, 2), (32, 40), (33, 17), (64, 36)]:
+        part = bi.gemm(dev(xs[off:off + M]), w, mode=mode, out_dtype=torch.float32).cpu()
+        assert torch.equal(part, full[off:off + M]), (M, off)
+    _after(bi)
+
+
+def test_gemm_fast_variant_is_not_invariant_but_close(bi):
+    rng = np.random.default_rng(6)
+    N, K = 4096, 4096
+    xs = synth.bf16_to_f32(synth.f32_to_bf16_bits(rng.standard_normal((32, K)).astype(np.float32)))
+    w = _bf16_dev(0.02 * rng.standard_normal((N, K)))
+    inv = bi.gemm(_bf16_dev(xs), w, out_dtype=torch.float32).cpu()
+    f1 = bi.gemm(_bf16_dev(xs[:1]), w, variant=1, out_dtype=torch.float32).cpu()
+    f32 = bi.gemm(_bf16_dev(xs), w, variant=1, out_dtype=torch.float32).cpu()
+    assert torch.allclose(f1[0], inv[0], rtol=1e-4, atol=1e-4)
+    assert not torch.equal(f1[0], f32[0])  # split-K chosen from M changes the bits
+    _after(bi)
+
+
+# ------------------------------------------------------------------ RMSNorm
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("H", [256, 3584, 4096])
+def test_rmsnorm_vs_oracle_and_invariance(bi, mode, H):
+    rng = np.random.default_rng(H + mode)
+    M = 19
+    x = rng.standard_normal((M, H)).astype(np.float32) * 3
+    r = rng.standard_normal((M, H)).astype(np.float32)
+    gamma = synth.f32_to_bf16_bits((1 + 0.1 * rng.standard_normal(H)).astype(np.float32))
+    dt = torch.float32 if mode else torch.bfloat16
+    xd = torch.from_numpy(x).cuda().to(dt)
+    rd = torch.from_numpy(r).cuda().to(dt)
+    gd = torch.from_numpy(gamma.view(np.int16)).cuda().view(torch.bfloat16)
+    rout = torch.empty_like(rd)
+    y, y32 = bi.rmsnorm(xd, gd, 1e-5, residual_in=rd, residual_out=rout, want_f32=True, mode=mode)
+    rsum = _f(xd) + _f(rd)
+    if mode == 0:
+        rsum = oracle.round_bf16(rsum)
+        assert np.array_equal(_f(rout), rsum)
+    else:
+        assert np.allclose(_f(rout), rsum, rtol=2 ** -23, atol=0)
+    ref = oracle.rmsnorm(_f(rout), gamma, 1e-5)
+    assert np.allclose(_f(y32), ref, rtol=3e-6, atol=1e-7)
+    if mode == 0:
+        assert np.allclose(_f(y), ref, rtol=2 ** -8 + 3e-6, atol=1e-7)
+    # invariance: each row alone equals the batched row
+    for i in (0, 7, 18):
+        ro = torch.empty_like(rd[i:i + 1])
+        yi, y32i = bi.rmsnorm(xd[i:i + 1].contiguous(), gd, 1e-5, residual_in=rd[i:i + 1].contiguous(),
+                              residual_out=ro, want_f32=True, mode=mode)
+        assert torch.equal(yi, y[i:i + 1]) and torch.equal(y32i, y32[i:i + 1]) and torch.equal(ro, rout[i:i + 1])
+    _after(bi)
+
+
+# ------------------------------------------------------------------ attention
+def _make_cache(bi, mode, n_slots, Hkv, cap, d, fill_upto, seed):
+    rng = np.random.default_rng(seed)
+    kv = bi.KVCache(n_slots, 1, Hkv, cap, d, mode=mode)
+    k = rng.standard_normal((n_slots, 1, Hkv, cap, d)).astype(np.float32)
+    v = rng.standard_normal((n_slots, 1, Hkv, cap, d)).astype(np.float32)
+    if mode == 0:
+        k = synth.bf16_to_f32(synth.f32_to_bf16_bits(k))
+        v = synth.bf16_to_f32(synth.f32_to_bf16_bits(v))
+    kv.k.copy_(torch.from_numpy(k))
+    kv.v.copy_(torch.from_numpy(v))
+    return kv, k, v
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("Hq,Hkv,d", [(32, 8, 128), (4, 4, 64), (28, 4, 128)])
+def test_attention_vs_oracle(bi, mode, Hq, Hkv, d):
+    cap = 1200
+    kv, k, v = _make_cache(bi, mode, 3, Hkv, cap, d, cap, seed=Hq + d + mode)
+    rng = np.random.default_rng(3)
+    # a mixed batch: decode tokens of slots 0 and 2, and a 5-token prefill block of slot 1
+    slots = np.array([0, 1, 1, 1, 1, 1, 2], dtype=np.int32)
+    pos = np.array([700, 250, 251, 252, 253, 254, 1100], dtype=np.int32)
+    T = len(slots)
+    q = rng.standard_normal((T, Hq * d)).astype(np.float32)
+    dt = torch.float32 if mode else torch.bfloat16
+    qd = torch.from_numpy(q).cuda().to(dt)
+    scale = 1.0 / math.sqrt(d)
+    out = _f(bi.attention(qd, kv, 0, torch.from_numpy(slots).cuda(), torch.from_numpy(pos).cuda(), slots, pos, Hq,
+                          np.float32(scale), mode=mode))
+    qf = _f(qd)
+    G = Hq // Hkv
+    for t in range(T):
+        for h in (0, Hq // 2 + 1, Hq - 1):
+            hk = h // G
+            ref = oracle.attention_query(qf[t, h * d:(h + 1) * d], k[slots[t], 0, hk, :pos[t] + 1],
+                                         v[slots[t], 0, hk, :pos[t] + 1], float(np.float32(scale)))
+            got = out[t, h * d:(h + 1) * d]
+            tol = 2e-5 * np.abs(v[slots[t], 0, hk]).max() + (2 ** -8 * np.abs(ref) if mode == 0 else 0)
+            assert (np.abs(got - ref) <= tol).all(), (t, h, np.abs(got - ref).max())
+    _after(bi)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_attention_invariance_decode_vs_prefill(bi, mode):
+    """A query's output is bitwise the same alone, inside a prefill block, and beside other slots."""
+    Hq, Hkv, d, cap = 32, 8, 128, 800
+    kv, _, _ = _make_cache(bi, mode, 4, Hkv, cap, d, cap, seed=9 + mode)
+    rng = np.random.default_rng(4)
+    n = 40
+    base = 230  # block crosses the chunk boundary at 256
+    q = rng.standard_normal((n, Hq * d)).astype(np.float32)
+    dt = torch.float32 if mode else torch.bfloat16
+    qd = torch.from_numpy(q).cuda().to(dt)
+    run = lambda qq, s, p: bi.attention(qq, kv, 0, torch.from_numpy(s).cuda(), torch.from_numpy(p).cuda(), s, p, Hq,
+                                        0.08838834764831845, mode=mode).cpu()
+    slots = np.full(n, 2, dtype=np.int32)
+    pos = np.arange(base, base + n, dtype=np.int32)
+    block = run(qd, slots, pos)
+    for i in (0, 5, 25, 26, 39):
+        alone = run(qd[i:i + 1].contiguous(), slots[i:i + 1], pos[i:i + 1])
+        assert torch.equal(alone[0], block[i]), i
+    # beside decode tokens of other slots
+    s2 = np.array([0, 2, 3], dtype=np.int32)
+    p2 = np.array([17, base + 25, 790], dtype=np.int32)
+    q2 = torch.stack([qd[0], qd[25], qd[1]])
+    mixed = run(q2, s2, p2)
+    assert torch.equal(mixed[1], block[25])
+    _after(bi)
+
+
+# ------------------------------------------------------------------ LM head
+def _h_rows(B, H, seed=7):
+    return synth.hidden_states(seed, B, H)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_lmhead_vs_oracle_small_vocab(bi, mode):
+    H, V, B = 512, 4096, 24
+    rng = np.random.default_rng(8)
+    Wb = synth.f32_to_bf16_bits((0.02 * rng.standard_normal((V, H))).astype(np.float32))
+    # scale logits up so both flagged and unflagged rows occur
+    h = _h_rows(B, H) * 4
+    hd = torch.from_numpy(h).cuda()
+    Wd = torch.from_numpy(Wb.view(np.int16)).cuda().view(torch.bfloat16)
+    tgt = rng.integers(0, V, size=B).astype(np.int32)
+    tgt[::3] = -1
+    o = bi.lmhead_logprob(hd, Wd, torch.from_numpy(tgt).cuda(), threshold=0.1, mode=mode, want_logits=True)
+    o = {k: v.cpu().numpy() for k, v in o.items()}
+    hb = synth.bf16_to_f32(synth.f32_to_bf16_bits(h)).astype(np.float64) if mode == 0 else h.astype(np.float64)
+    res_main, z_main = oracle.lmhead(hb, Wb, target=tgt, want_logits=True)
+    res_exact, _ = oracle.lmhead(h.astype(np.float64), Wb, target=tgt)
+    bound = H * 2.0 ** -24 * (np.abs(hb) @ np.abs(synth.bf16_to_f32(Wb)).astype(np.float64).T)
+    assert (np.abs(o["logits"] - z_main) <= bound + 1e-30).all()
+    # margin and the flag come from the main pass
+    assert np.allclose(o["margin"], res_main[:, 3], atol=2e-5)
+    if mode == 0:
+        assert np.array_equal(o["recomputed"], (o["margin"] < 0.1).astype(np.uint8))
+        assert 0 < o["recomputed"].sum() < B
+    else:
+        assert (o["recomputed"] == 0).all()
+    for b in range(B):
+        ref = res_exact[b] if (mode == 1 or o["recomputed"][b]) else res_main[b]
+        assert abs(o["logprob"][b] - ref[1]) <= 1e-5 * abs(ref[1]) + 1e-6, b
+        assert abs(o["lse"][b] - ref[0]) <= 1e-5 * abs(ref[0]) + 1e-6, b
+        if ref[3] > 1e-4:
+            assert o["argmax"][b] == int(ref[2]), b
+    _after(bi)
+
+
+def test_lmhead_full_size_invariance_and_samples(bi):
+    """LM head alone at hidden 4096, vocab 128256: each row bitwise equal across batch 1..256."""
+    H, V = 4096, 128256
+    W = torch.empty(V, H, dtype=torch.bfloat16, device="cuda")
+    kW = synth.key(synth.WEIGHT_SEED, synth.S_LMHEAD)
+    bi.synth_fill_bf16(W, V, H, kW, 0.02)
+    h = _h_rows(256, H)
+    hd = torch.from_numpy(h).cuda()
+    ref = {k: v.cpu() for k, v in bi.lmhead_logprob(hd, W, None, 0.1).items()}
+    for B in (1, 2, 4, 8, 16, 32, 64, 128):
+        for off in (0, 256 - B):
+            o = bi.lmhead_logprob(hd[off:off + B].contiguous(), W, None, 0.1)
+            for k in ("logprob", "lse", "argmax", "margin", "recomputed"):
+                assert torch.equal(o[k].cpu(), ref[k][off:off + B]), (B, off, k)
+    # sampled oracle parity on 3 rows (host weights regenerated from the same seed)
+    Wb = synth.normal_bf16(kW, V * H).reshape(V, H)
+    rows = [0, 100, 255]
+    recomputed = ref["recomputed"].numpy()
+    hb = synth.bf16_to_f32(synth.f32_to_bf16_bits(h[rows])).astype(np.float64)
+    res_main, _ = oracle.lmhead(hb, Wb)
+    res_exact, _ = oracle.lmhead(h[rows].astype(np.float64), Wb)
+    for i, r in enumerate(rows):
+        rr = res_exact[i] if recomputed[r] else res_main[i]
+        assert abs(ref["logprob"][r].item() - rr[1]) <= 1e-5 * abs(rr[1]) + 1e-6
+        assert abs(ref["margin"][r].item() - res_main[i][3]) <= 1e-4
+    rate = recomputed.mean()
+    assert 0.0 < rate < 1.0
+    _after(bi)
