@@ -505,7 +505,7 @@ int bi_decode_step(bi_ctx* ctx, const bi_batch* batch, const bi_step_out* out, v
     BI_TRY(bi_rope_kv_append(s.qkv, w.rope, w.rope_max_pos, s.q, &ctx->kv, l, batch->slot, batch->pos, T, Hq, d.mode,
                              stream));
     BI_TRY(attention_run(s.q, &ctx->kv, l, batch->slot, batch->pos, batch->slot_host, batch->pos_host, s.o, T, Hq,
-                         scale, d.mode, d.variant, s.gemm, s.gemm_bytes, st));
+                         scale, d.mode, d.variant, s.attn, s.attn_bytes, st));
     BI_TRY(gemm_run(s.o, QD, lw(w.w_o, (size_t)H * QD, l), s.y, H, act_dtype, T, H, QD, BI_EPI_NONE, d.mode,
                     d.variant, s.gemm, s.gemm_bytes, st));
     BI_TRY(bi_rmsnorm(s.y, s.res, s.res, g_ffn, s.u, nullptr, T, H, d.eps, d.mode, stream));
