@@ -86,7 +86,9 @@ long long bi_launch_count(void);
  *   w: bf16 [N][K] contiguous, y: [M][N] with leading dim ldy).
  * Invariant variant: each output element is accumulated in fp32 over the
  *   FULL K range in ascending K order, by the same instruction sequence for
- *   any M (no split-K; the row tile and K loop do not depend on M).
+ *   any M (no split-K; the row tile and K loop do not depend on M).  The
+ *   16-wide K steps go round-robin into a fixed number of accumulators (1, 2
+ *   or 4, set by N alone) that are added in a fixed tree at the end.
  *   ("Meituan bitwise train/infer consistency": TP rewritten to full-K
  *   computation instead of segmented reduce-scatter.)
  * mode BI_MODE_BF16: x is bf16.  mode BI_MODE_LAYERCAST: x is f32 and w is

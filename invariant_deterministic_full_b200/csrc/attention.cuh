@@ -45,13 +45,30 @@ struct AttnArgs {
 
 __host__ __device__ inline int att_ninner(int d, int f32) { return d * (f32 ? 4 : 2) / 128; }
 
-// Grid: (block, chunk, kv head).  Dynamic smem: K tile, V tile (the same
-// buffer in f32 mode), q pairs (fp32), scores/probabilities [pairs][CH].
+constexpr int ATT_SUB = 64;  // keys per TMA sub-tile
+constexpr int ATT_RING = 2;  // sub-tile buffers
+
+__host__ __device__ inline size_t att_sub_bytes(int d, int f32) { return (size_t)ATT_SUB * d * (f32 ? 4 : 2); }
+__host__ __device__ inline size_t att_smem_bytes(int np, int d, int f32) {
+  return ATT_RING * att_sub_bytes(d, f32) + (size_t)np * d * 4 + (size_t)np * ATT_CHUNK * 4 + 1024;
+}
+
+// Grid: (block, chunk, kv head).  The chunk's K rows, then its V rows, stream
+// through a ring of two 64-key sub-tiles (TMA, 128-byte swizzle).  A block's
+// (query, head) pairs p = i*G + g (head hk*G + g) are processed NP at a time;
+// each group re-streams the chunk (an L2 hit after the first).  Work layout:
+//   scores  thread t: key 64*st + (t % 64), pairs (t / 64) + 4k
+//   softmax warp w: pairs w, w + 8, ...; lane i: keys i + 32k
+//   PV      thread t: element t % d, pairs t / d + (256/d) k
+// None of it changes a pair's arithmetic, which is fixed as described above.
+template <int NP>
 __global__ void __launch_bounds__(ATT_THREADS)
     attn_partial_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ AttnPlan plan, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ __align__(8) uint64_t bar[ATT_RING];
+  __shared__ float m_s[NP], l_s[NP];
+  __shared__ int live_s[NP];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int b = blockIdx.x, c = blockIdx.y, hk = blockIdx.z;
   if (b >= plan.n) return;
@@ -61,172 +78,185 @@ __global__ void __launch_bounds__(ATT_THREADS)
   const int key0 = c * a.chunk;
   if (key0 > pmax) return;  // chunk beyond every query of the block
   const int nvalid = min(a.chunk, pmax - key0 + 1);
-  const int nsub = (nvalid + 63) / 64;
+  const int nsub = (nvalid + ATT_SUB - 1) / ATT_SUB;
   const int ninner = att_ninner(a.d, a.f32);
   const int esz = a.f32 ? 4 : 2;
   const int boxe = 128 / esz;
-  const size_t kv_region = (size_t)ATT_CHUNK * a.d * esz;
-  uint8_t* kbuf = smem;
-  uint8_t* vbuf = a.f32 ? smem : smem + kv_region;
-  float* qs = reinterpret_cast<float*>(smem + (a.f32 ? kv_region : 2 * kv_region));
-  float* S = qs + ATT_MAX_PAIRS * a.d;
+  const size_t sub_bytes = att_sub_bytes(a.d, a.f32);
+  float* qs = reinterpret_cast<float*>(smem + ATT_RING * sub_bytes);
+  float* S = qs + NP * a.d;
   const int npairs = nq * a.G;
   const int row_base = ((s * a.n_layers + a.layer) * a.Hkv + hk) * a.cap + key0;
-  const uint32_t bytes = nsub * ninner * 64 * 128;
-
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nloads = 2 * nsub;  // K sub-tiles then V sub-tiles, per pair group
+
   if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
+    for (int r = 0; r < ATT_RING; ++r) mbar_init(&bar[r], 1);
     fence_mbar_init();
   }
   __syncthreads();
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bar[0], bytes);
-    for (int sb = 0; sb < nsub; ++sb)
-      for (int ib = 0; ib < ninner; ++ib)
-        tma_load_2d(kbuf + ib * (ATT_CHUNK * 128) + sb * 64 * 128, &tmK, ib * boxe, row_base + sb * 64, &bar[0]);
-    if (!a.f32) {
-      mbar_arrive_expect_tx(&bar[1], bytes);
-      for (int sb = 0; sb < nsub; ++sb)
-        for (int ib = 0; ib < ninner; ++ib)
-          tma_load_2d(vbuf + ib * (ATT_CHUNK * 128) + sb * 64 * 128, &tmV, ib * boxe, row_base + sb * 64, &bar[1]);
-    }
-  }
-  // q of the block's (query, head) pairs -> fp32 smem; pair p = i*G + g, head hk*G + g
-  for (int idx = tid; idx < npairs * a.d; idx += ATT_THREADS) {
-    const int p = idx / a.d, e = idx % a.d;
-    const int i = p / a.G, g = p % a.G;
-    const int hq = hk * a.G + g;
-    qs[p * a.d + e] = load_act(a.q, (size_t)(t0 + i) * a.Hq * a.d + hq * a.d + e, a.f32);
-  }
-  __syncthreads();
-  if (!mbar_wait(&bar[0], 0)) return;
+  // load number L (counted over the whole CTA): sub-tile L % nloads of the
+  // sequence K0..K(nsub-1), V0..V(nsub-1), into ring buffer L % ATT_RING.
+  auto issue = [&](int L) {
+    const int li = L % nloads;
+    const bool isv = li >= nsub;
+    const int st = isv ? li - nsub : li;
+    uint8_t* buf = smem + (L % ATT_RING) * sub_bytes;
+    uint64_t* br = &bar[L % ATT_RING];
+    mbar_arrive_expect_tx(br, (uint32_t)(ninner * ATT_SUB * 128));
+    for (int ib = 0; ib < ninner; ++ib)
+      tma_load_2d(buf + ib * (ATT_SUB * 128), isv ? &tmV : &tmK, ib * boxe, row_base + st * ATT_SUB, br);
+  };
+  const int ngroups = (npairs + NP - 1) / NP;
+  const int total_loads = ngroups * nloads;
+  if (tid == 0)
+    for (int L = 0; L < ATT_RING && L < total_loads; ++L) issue(L);
+  int L = 0;  // next load to consume
+  auto consume_wait = [&]() -> bool { return mbar_wait(&bar[L % ATT_RING], (uint32_t)((L / ATT_RING) & 1)); };
+  auto release = [&]() {  // every thread is done with load L: refill its buffer
+    __syncthreads();
+    if (tid == 0 && L + ATT_RING < total_loads) issue(L + ATT_RING);
+    ++L;
+  };
 
-  // ---- scores: thread j = key j of the chunk
-  {
-    const int j = tid;
-    if (j < nvalid) {
-      float acc[ATT_MAX_PAIRS];
+  for (int pg0 = 0; pg0 < npairs; pg0 += NP) {
+    const int gp = min(NP, npairs - pg0);
+    for (int idx = tid; idx < gp * a.d; idx += ATT_THREADS) {
+      const int pl = idx / a.d, e = idx % a.d;
+      const int p = pg0 + pl;
+      const int i = p / a.G, g = p % a.G;
+      qs[pl * a.d + e] = load_act(a.q, (size_t)(t0 + i) * a.Hq * a.d + (hk * a.G + g) * a.d + e, a.f32);
+    }
+    __syncthreads();
+
+    // ---- scores: s = scale * (q . k_j), a sequential fp32 FMA chain over e ascending
+    const int pq = tid >> 6;
+    for (int st = 0; st < nsub; ++st) {
+      if (!consume_wait()) return;
+      const int jl = tid & 63;
+      const int j = st * ATT_SUB + jl;
+      if (j < nvalid) {
+        const uint8_t* kb = smem + (L % ATT_RING) * sub_bytes;
+        float acc[NP / 4];
 #pragma unroll
-      for (int p = 0; p < ATT_MAX_PAIRS; ++p) acc[p] = 0.f;
-      const int nch = a.d * esz / 16;  // 16-byte chunks per key row
-      for (int ch = 0; ch < nch; ++ch) {
-        const int ib = ch >> 3, cc = ch & 7;
-        const uint8_t* rowp = kbuf + ib * (ATT_CHUNK * 128) + j * 128;
-        const uint4 u = *reinterpret_cast<const uint4*>(rowp + ((cc ^ (j & 7)) << 4));
-        float kv[8];
-        int ne;
-        if (a.f32) {
-          kv[0] = __uint_as_float(u.x); kv[1] = __uint_as_float(u.y);
-          kv[2] = __uint_as_float(u.z); kv[3] = __uint_as_float(u.w);
-          ne = 4;
-        } else {
-          kv[0] = bf16lo(u.x); kv[1] = bf16hi(u.x); kv[2] = bf16lo(u.y); kv[3] = bf16hi(u.y);
-          kv[4] = bf16lo(u.z); kv[5] = bf16hi(u.z); kv[6] = bf16lo(u.w); kv[7] = bf16hi(u.w);
-          ne = 8;
-        }
-        const int e0 = ch * ne;
+        for (int k = 0; k < NP / 4; ++k) acc[k] = 0.f;
+        const int nch = a.d * esz / 16;
+        for (int ch = 0; ch < nch; ++ch) {
+          const int ib = ch >> 3, cc = ch & 7;
+          const uint4 u = *reinterpret_cast<const uint4*>(kb + ib * (ATT_SUB * 128) + jl * 128 + ((cc ^ (jl & 7)) << 4));
+          if (a.f32) {
+            const float kv[4] = {__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z),
+                                 __uint_as_float(u.w)};
 #pragma unroll
-        for (int p = 0; p < ATT_MAX_PAIRS; ++p) {
-          if (p < npairs) {
-            const float* qp = qs + p * a.d + e0;
-            if (ne == 8) {
-              const float4 q0 = *reinterpret_cast<const float4*>(qp);
-              const float4 q1 = *reinterpret_cast<const float4*>(qp + 4);
-              float x = acc[p];
-              x = fmaf(q0.x, kv[0], x); x = fmaf(q0.y, kv[1], x); x = fmaf(q0.z, kv[2], x); x = fmaf(q0.w, kv[3], x);
-              x = fmaf(q1.x, kv[4], x); x = fmaf(q1.y, kv[5], x); x = fmaf(q1.z, kv[6], x); x = fmaf(q1.w, kv[7], x);
-              acc[p] = x;
-            } else {
-              const float4 q0 = *reinterpret_cast<const float4*>(qp);
-              float x = acc[p];
-              x = fmaf(q0.x, kv[0], x); x = fmaf(q0.y, kv[1], x); x = fmaf(q0.z, kv[2], x); x = fmaf(q0.w, kv[3], x);
-              acc[p] = x;
+            for (int k = 0; k < NP / 4; ++k) {
+              const int p = pq + 4 * k;
+              if (p < gp) {
+                const float4 q0 = *reinterpret_cast<const float4*>(qs + p * a.d + ch * 4);
+                float x = acc[k];
+                x = fmaf(q0.x, kv[0], x); x = fmaf(q0.y, kv[1], x); x = fmaf(q0.z, kv[2], x); x = fmaf(q0.w, kv[3], x);
+                acc[k] = x;
+              }
+            }
+          } else {
+            const float kv[8] = {bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y),
+                                 bf16lo(u.z), bf16hi(u.z), bf16lo(u.w), bf16hi(u.w)};
+#pragma unroll
+            for (int k = 0; k < NP / 4; ++k) {
+              const int p = pq + 4 * k;
+              if (p < gp) {
+                const float* qp = qs + p * a.d + ch * 8;
+                const float4 q0 = *reinterpret_cast<const float4*>(qp);
+                const float4 q1 = *reinterpret_cast<const float4*>(qp + 4);
+                float x = acc[k];
+                x = fmaf(q0.x, kv[0], x); x = fmaf(q0.y, kv[1], x); x = fmaf(q0.z, kv[2], x); x = fmaf(q0.w, kv[3], x);
+                x = fmaf(q1.x, kv[4], x); x = fmaf(q1.y, kv[5], x); x = fmaf(q1.z, kv[6], x); x = fmaf(q1.w, kv[7], x);
+                acc[k] = x;
+              }
             }
           }
         }
+#pragma unroll
+        for (int k = 0; k < NP / 4; ++k) {
+          const int p = pq + 4 * k;
+          if (p < gp) S[p * ATT_CHUNK + j] = acc[k] * a.scale;
+        }
       }
-#pragma unroll
-      for (int p = 0; p < ATT_MAX_PAIRS; ++p)
-        if (p < npairs) S[p * ATT_CHUNK + j] = acc[p] * a.scale;
+      release();
     }
-  }
-  __syncthreads();
-  if (a.f32 && tid == 0) {  // f32: V reuses the K buffer, load it now
-    mbar_arrive_expect_tx(&bar[1], bytes);
-    for (int sb = 0; sb < nsub; ++sb)
-      for (int ib = 0; ib < ninner; ++ib)
-        tma_load_2d(vbuf + ib * (ATT_CHUNK * 128) + sb * 64 * 128, &tmV, ib * boxe, row_base + sb * 64, &bar[1]);
-  }
 
-  // ---- softmax per pair: warp w handles pairs w, w+8, ...; lane i keys i + 32k
-  __shared__ float m_s[ATT_MAX_PAIRS], l_s[ATT_MAX_PAIRS];
-  __shared__ int live_s[ATT_MAX_PAIRS];
-  for (int p = warp; p < npairs; p += ATT_THREADS / 32) {
-    const int i = p / a.G;
-    const int lim = a.pos[t0 + i] - key0;  // keys j <= lim are visible to this query
-    float mx = -INFINITY;
+    // ---- softmax per pair: max (exact), exp, l = per-lane ascending sums then fixed butterfly
+    for (int pl = warp; pl < gp; pl += ATT_THREADS / 32) {
+      const int i = (pg0 + pl) / a.G;
+      const int lim = a.pos[t0 + i] - key0;  // keys j <= lim are visible to this query
+      float mx = -INFINITY;
 #pragma unroll
-    for (int k = 0; k < ATT_CHUNK / 32; ++k) {
-      const int j = lane + 32 * k;
-      if (j <= lim && j < nvalid) mx = fmaxf(mx, S[p * ATT_CHUNK + j]);
-    }
-    mx = warp_max(mx);
-    float sum = 0.f;
+      for (int k = 0; k < ATT_CHUNK / 32; ++k) {
+        const int j = lane + 32 * k;
+        if (j <= lim && j < nvalid) mx = fmaxf(mx, S[pl * ATT_CHUNK + j]);
+      }
+      mx = warp_max(mx);
+      float sum = 0.f;
 #pragma unroll
-    for (int k = 0; k < ATT_CHUNK / 32; ++k) {
-      const int j = lane + 32 * k;
-      float pj = 0.f;
-      if (j <= lim && j < nvalid) pj = expf(S[p * ATT_CHUNK + j] - mx);
-      if (j < nvalid) S[p * ATT_CHUNK + j] = pj;
-      sum += pj;
+      for (int k = 0; k < ATT_CHUNK / 32; ++k) {
+        const int j = lane + 32 * k;
+        float pj = 0.f;
+        if (j <= lim && j < nvalid) pj = expf(S[pl * ATT_CHUNK + j] - mx);
+        if (j < nvalid) S[pl * ATT_CHUNK + j] = pj;
+        sum += pj;
+      }
+      sum = warp_sum_fixed(sum);
+      if (lane == 0) {
+        m_s[pl] = mx;
+        l_s[pl] = sum;
+        live_s[pl] = lim >= 0;
+      }
     }
-    sum = warp_sum_fixed(sum);
-    if (lane == 0) {
-      m_s[p] = mx;
-      l_s[p] = sum;
-      live_s[p] = lim >= 0;
-    }
-  }
-  __syncthreads();
-  if (!mbar_wait(&bar[1], 0)) return;
+    __syncthreads();
 
-  // ---- PV: thread -> (e = tid % d, pairs p = tid / d + k * (256 / d))
-  {
+    // ---- PV: acc[e] = sum_j p_j v_j[e], sequential FMA over the valid keys ascending
+    constexpr int PPT = NP >= 2 ? NP / 2 : 1;  // pairs per thread upper bound (d >= 64: at most 4 pair lanes)
     const int e = tid % a.d;
     const int pstep = ATT_THREADS / a.d;
     const int p0 = tid / a.d;
-    const int ib = (e * esz) >> 7;            // inner box of element e
-    const int cc = ((e * esz) & 127) >> 4;    // 16-byte chunk within the 128-byte row
+    const int ib_e = (e * esz) >> 7;
+    const int cc_e = ((e * esz) & 127) >> 4;
     const int within = (e * esz) & 15;
-    float acc[ATT_MAX_PAIRS / 2];
+    float pacc[PPT];
 #pragma unroll
-    for (int k = 0; k < ATT_MAX_PAIRS / 2; ++k) acc[k] = 0.f;
-    const uint8_t* vb = vbuf + ib * (ATT_CHUNK * 128) + within;
-    for (int j = 0; j < nvalid; ++j) {
-      const uint8_t* vp = vb + j * 128 + ((cc ^ (j & 7)) << 4);
-      const float v = a.f32 ? *reinterpret_cast<const float*>(vp) : bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(vp));
+    for (int k = 0; k < PPT; ++k) pacc[k] = 0.f;
+    for (int st = 0; st < nsub; ++st) {
+      if (!consume_wait()) return;
+      const uint8_t* vb = smem + (L % ATT_RING) * sub_bytes + ib_e * (ATT_SUB * 128) + within;
+      const int jend = min(ATT_SUB, nvalid - st * ATT_SUB);
+      for (int jl = 0; jl < jend; ++jl) {
+        const uint8_t* vp = vb + jl * 128 + ((cc_e ^ (jl & 7)) << 4);
+        const float v = a.f32 ? *reinterpret_cast<const float*>(vp)
+                              : bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(vp));
+        const int j = st * ATT_SUB + jl;
 #pragma unroll
-      for (int k = 0; k < ATT_MAX_PAIRS / 2; ++k) {
-        const int p = p0 + k * pstep;
-        if (p < npairs) acc[k] = fmaf(S[p * ATT_CHUNK + j], v, acc[k]);
+        for (int k = 0; k < PPT; ++k) {
+          const int pl = p0 + k * pstep;
+          if (pl < gp) pacc[k] = fmaf(S[pl * ATT_CHUNK + j], v, pacc[k]);
+        }
       }
+      release();
     }
 #pragma unroll
-    for (int k = 0; k < ATT_MAX_PAIRS / 2; ++k) {
-      const int p = p0 + k * pstep;
-      if (p < npairs && live_s[p]) {
+    for (int k = 0; k < PPT; ++k) {
+      const int pl = p0 + k * pstep;
+      if (pl < gp && live_s[pl]) {
+        const int p = pg0 + pl;
         const int i = p / a.G, g = p % a.G;
         const int hq = hk * a.G + g;
         float* rec = a.part + (((size_t)(t0 + i - a.t_base) * a.Hq + hq) * a.max_chunks + c) * (a.d + 4);
-        rec[e] = acc[k];
+        rec[e] = pacc[k];
         if (e == 0) {
-          rec[a.d] = m_s[p];
-          rec[a.d + 1] = l_s[p];
+          rec[a.d] = m_s[pl];
+          rec[a.d + 1] = l_s[pl];
         }
       }
     }
+    __syncthreads();  // the next group overwrites q, S and the pair statistics
   }
 }
 

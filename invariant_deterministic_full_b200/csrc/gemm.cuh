@@ -10,7 +10,12 @@
 // instruction adds 16 products of one (n, m) pair into that pair's fp32
 // accumulator; the products of one element never meet another element's, so
 // neither the number of token columns in a tile nor the tile a token lands in
-// can change an element's bits.  K advances 16 at a time in ascending order.
+// can change an element's bits.  K advances 16 at a time in ascending order;
+// step s (k = 16s .. 16s+15) goes into accumulator set s % KS, and the KS sets
+// are combined as ((a0 + a1) + (a2 + a3)) (KS = 4), a0 + a1 (KS = 2) or a0,
+// where KS follows from the weight-row tile BN, itself chosen from N alone.
+// The fixed interleave keeps several independent mma chains per warp so the
+// tensor-pipe latency is covered even when M is small.
 // Weight tiles (BN rows x 64 k) and token tiles (32 rows x 64 k) stream by TMA
 // (128-byte swizzle) into a multi-stage shared-memory ring filled by one
 // producer warp; four consumer warps read them with ldmatrix.  The grid is
@@ -42,6 +47,10 @@ struct GemmCfg {
   static constexpr int RW = BN / 32;      // warps along the weight rows (32 rows each)
   static constexpr int TW = 4 / RW;       // warps along the token columns
   static constexpr int NT = GEMM_BM / TW / 8;  // n8 token tiles per warp
+  // Interleaved accumulator sets per output element (a property of the matrix
+  // shape through BN, never of M): enough independent mma chains per warp
+  // (2 row tiles x NT x KS = 8) to cover the tensor-pipe latency.
+  static constexpr int KS = NT >= 4 ? 1 : 4 / NT;
 };
 
 // Work item -> (split, row group, token tile).  Splits > 1 only in the
@@ -113,13 +122,17 @@ __global__ void __launch_bounds__(160, 1)
     const int kb0 = sp * kb_per_split;
     const int kb1 = min(kblocks_total, kb0 + kb_per_split);
     const bool active = mt * GEMM_BM + tok0 < M;
-    float acc[2][C::NT][4];
+    // KS interleaved accumulator sets: k16 step s (counted from k = 0) adds into
+    // set s % KS; the sets are combined in a fixed tree after the K loop.
+    float accs[C::KS][2][C::NT][4];
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
+    for (int q = 0; q < C::KS; ++q)
 #pragma unroll
-      for (int b = 0; b < C::NT; ++b)
+      for (int a = 0; a < 2; ++a)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[a][b][c] = 0.f;
+        for (int b = 0; b < C::NT; ++b)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) accs[q][a][b][c] = 0.f;
 
     for (int kb = kb0; kb < kb1; ++kb) {
       if (!mbar_wait(&full_bar[stage], phase)) return;
@@ -149,7 +162,7 @@ __global__ void __launch_bounds__(160, 1)
 #pragma unroll
           for (int r = 0; r < 2; ++r)
 #pragma unroll
-            for (int nt = 0; nt < C::NT; ++nt) mma_bf16_16816(acc[r][nt], a[r], b[nt][0], b[nt][1]);
+            for (int nt = 0; nt < C::NT; ++nt) mma_bf16_16816(accs[kk % C::KS][r][nt], a[r], b[nt][0], b[nt][1]);
         }
       }
       __syncwarp();
@@ -160,6 +173,20 @@ __global__ void __launch_bounds__(160, 1)
       }
     }
     if (!active) continue;
+    float acc[2][C::NT][4];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int b = 0; b < C::NT; ++b)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if constexpr (C::KS == 4)
+            acc[a][b][c] = (accs[0][a][b][c] + accs[1][a][b][c]) + (accs[2][a][b][c] + accs[3][a][b][c]);
+          else if constexpr (C::KS == 2)
+            acc[a][b][c] = accs[0][a][b][c] + accs[1][a][b][c];
+          else
+            acc[a][b][c] = accs[0][a][b][c];
+        }
 
     // ---------------- epilogue: fragment (row g8 (+8), cols 2*t4 (+1)) of each m16n8 tile
     const int nbase = g * BN + row0;

@@ -67,10 +67,33 @@ static size_t attn_ws_bytes(int T, int Hq, int d, int max_pos, int chunk) {
   return (size_t)tg * Hq * max_chunks * (d + 4) * sizeof(float) + 256;
 }
 
-static int attn_smem_bytes(int d, int f32) {
-  const size_t kv_region = (size_t)ATT_CHUNK * d * (f32 ? 4 : 2);
-  return (int)((f32 ? kv_region : 2 * kv_region) + (size_t)ATT_MAX_PAIRS * d * 4 + (size_t)ATT_MAX_PAIRS * ATT_CHUNK * 4 +
-               1024);
+static int attn_set_smem_attrs() {
+  static bool done = false;
+  if (done) return BI_OK;
+  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_partial_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)att_smem_bytes(4, 128, 1)));
+  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_partial_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)att_smem_bytes(8, 128, 1)));
+  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_partial_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)att_smem_bytes(16, 128, 1)));
+  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_partial_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)att_smem_bytes(32, 128, 1)));
+  done = true;
+  return BI_OK;
+}
+
+static int attn_launch(int np, const CUtensorMap& tk, const CUtensorMap& tv, const AttnPlan& plan, const AttnArgs& a,
+                       cudaStream_t st) {
+  const dim3 grid(plan.n, a.max_chunks, a.Hkv);
+  const size_t smem = att_smem_bytes(np, a.d, a.f32);
+  switch (np) {
+    case 4: attn_partial_kernel<4><<<grid, ATT_THREADS, smem, st>>>(tk, tv, plan, a); break;
+    case 8: attn_partial_kernel<8><<<grid, ATT_THREADS, smem, st>>>(tk, tv, plan, a); break;
+    case 16: attn_partial_kernel<16><<<grid, ATT_THREADS, smem, st>>>(tk, tv, plan, a); break;
+    default: attn_partial_kernel<32><<<grid, ATT_THREADS, smem, st>>>(tk, tv, plan, a); break;
+  }
+  BI_CHECK_LAUNCH();
+  return BI_OK;
 }
 
 static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const int32_t* slot, const int32_t* pos,
@@ -89,7 +112,9 @@ static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const
   const int G = Hq / Hkv;
   BI_REQUIRE(G <= ATT_MAX_PAIRS, BI_ERR_UNSUPPORTED, "bi_attention: %d q heads per kv head (max %d)", G, ATT_MAX_PAIRS);
   const int chunk = attn_chunk_for(T, variant);
-  const int QB = std::max(1, ATT_MAX_PAIRS / G);
+  // query-block size (work assignment only): a CTA streams one KV chunk and loops over
+  // the block's (query, head) pairs 32 at a time; blocks hold up to 256 pairs.
+  const int QB = std::max(1, std::min(64, 256 / G));
 
   // validation + plan: blocks of <= QB adjacent tokens of one slot at consecutive positions
   int max_pos = 0;
@@ -119,37 +144,38 @@ static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const
   BI_TRY(encode_tmap_2d(&tk, dt, esz, kv->k, d, rows, (uint64_t)d * esz, 128 / esz, 64, CU_TENSOR_MAP_SWIZZLE_128B));
   BI_TRY(encode_tmap_2d(&tv, dt, esz, kv->v, d, rows, (uint64_t)d * esz, 128 / esz, 64, CU_TENSOR_MAP_SWIZZLE_128B));
 
-  const int smem = attn_smem_bytes(d, f32);
-  static bool attr_done = false;
-  if (!attr_done) {
-    BI_CHECK_CUDA(cudaFuncSetAttribute(attn_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       attn_smem_bytes(128, 0) > attn_smem_bytes(128, 1) ? attn_smem_bytes(128, 0)
-                                                                                          : attn_smem_bytes(128, 1)));
-    attr_done = true;
-  }
+  BI_TRY(attn_set_smem_attrs());
   float* part = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
+  // pairs per group for single-token (decode) blocks: G rounded up to a power of two
+  int np1 = 4;
+  while (np1 < G) np1 *= 2;
 
-  // token groups bound the partials workspace; blocks never straddle a group
-  // boundary because a block is cut whenever it would cross one.
+  // Token groups of at most ATT_TOKEN_GROUP tokens bound the partials
+  // workspace; a group is made of whole blocks.  Within a group, single-token
+  // blocks and multi-token blocks go to two launches with different pair-group
+  // sizes (work assignment only).
   size_t bi0 = 0;
   while (bi0 < blocks.size()) {
     const int t_base = blocks[bi0].x;
     size_t bi1 = bi0;
-    AttnPlan plan;
-    plan.n = 0;
-    while (bi1 < blocks.size() && plan.n < ATT_MAX_BLOCKS &&
+    AttnPlan p1, pm;
+    p1.n = 0;
+    pm.n = 0;
+    while (bi1 < blocks.size() && p1.n < ATT_MAX_BLOCKS && pm.n < ATT_MAX_BLOCKS &&
            blocks[bi1].x + blocks[bi1].y - t_base <= ATT_TOKEN_GROUP) {
-      plan.blk[plan.n++] = blocks[bi1++];
+      if (blocks[bi1].y == 1)
+        p1.blk[p1.n++] = blocks[bi1++];
+      else
+        pm.blk[pm.n++] = blocks[bi1++];
     }
-    if (plan.n == 0) return set_error(BI_ERR_UNSUPPORTED, "bi_attention: planning failed");
+    if (bi1 == bi0) return set_error(BI_ERR_UNSUPPORTED, "bi_attention: planning failed");
     const int t_end = blocks[bi1 - 1].x + blocks[bi1 - 1].y;
     AttnArgs a;
     a.q = q; a.slot = slot; a.pos = pos; a.part = part; a.t_base = t_base;
     a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.d = d; a.chunk = chunk; a.max_chunks = max_chunks;
     a.layer = layer; a.n_layers = kv->n_layers; a.cap = kv->capacity; a.f32 = f32; a.scale = scale;
-    dim3 grid(plan.n, max_chunks, Hkv);
-    attn_partial_kernel<<<grid, ATT_THREADS, smem, st>>>(tk, tv, plan, a);
-    BI_CHECK_LAUNCH();
+    if (p1.n) BI_TRY(attn_launch(np1, tk, tv, p1, a, st));
+    if (pm.n) BI_TRY(attn_launch(ATT_MAX_PAIRS, tk, tv, pm, a, st));
     const int nw = (t_end - t_base) * Hq;
     attn_merge_kernel<<<(nw * 32 + 255) / 256, 256, 0, st>>>(part, pos, out, t_base, t_end - t_base, Hq, d, chunk,
                                                               max_chunks, f32);
