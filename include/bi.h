@@ -183,6 +183,31 @@ int bi_lmhead_logprob(const float* h, const void* W, const int32_t* target, int 
                       float margin_threshold, int mode, float* logprob, float* lse, int32_t* argmax, float* margin,
                       uint8_t* recomputed, float* logits, void* ws, size_t ws_bytes, void* stream);
 
+/* LM-head logprob for callers that cannot allocate device memory.  (No
+ * counterpart on the pages: this is an interface convenience, not part of
+ * the method.)  Some callers cannot call cudaMalloc -- code running while a
+ * caching allocator owns all device memory, plug-ins handed only their inputs
+ * and outputs, request paths where allocation is forbidden -- so this variant
+ * takes no workspace: its scratch is a fixed array of BI_NOALLOC_SCRATCH_BYTES
+ * inside the library, which every GPU that loads the library keeps until the
+ * process exits.  Arguments and results are those of bi_lmhead_logprob, and
+ * so is the arithmetic (the results are bit-identical).
+ *  - Calls whose scratch need (bi_lmhead_workspace_size, less the logits when
+ *    `logits` is given) exceeds BI_NOALLOC_SCRATCH_BYTES are rejected with
+ *    BI_ERR_WORKSPACE and a message; at hidden 4096 / vocab 128256 that
+ *    allows up to 32 rows in BI_MODE_BF16.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any
+ *    stream capture.
+ *  - All calls share the one array: calls whose GPU work overlaps (different
+ *    streams, or host threads racing) corrupt each other's scratch.  Issue
+ *    them in one stream order.  Nothing in the array needs to start zeroed.
+ *  - It allocates nothing: no cudaMalloc/cudaFree, no allocating library call. */
+#define BI_NOALLOC_SCRATCH_BYTES (40 << 20)
+int bi_lmhead_logprob_noalloc(const float* h, const void* W, const int32_t* target, int B, int H, int V,
+                              float margin_threshold, int mode, float* logprob, float* lse, int32_t* argmax,
+                              float* margin, uint8_t* recomputed, float* logits, void* stream);
+
 /* ------------------------------------------------------------ Decode step
  * A whole decoder forward for a batch of tokens (any mix of prefill chunks and
  * decode tokens of many slots: continuous batching), followed by the LM-head

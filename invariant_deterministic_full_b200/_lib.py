@@ -78,6 +78,7 @@ SIGNATURES = {
     "bi_attention": (I, [P, ctypes.POINTER(KvLayout), I, P, P, P, P, P, I, I, F, I, I, P, SZ, P]),
     "bi_lmhead_workspace_size": (SZ, [I, I, I, I]),
     "bi_lmhead_logprob": (I, [P, P, P, I, I, I, F, I, P, P, P, P, P, P, P, SZ, P]),
+    "bi_lmhead_logprob_noalloc": (I, [P, P, P, I, I, I, F, I, P, P, P, P, P, P, P]),
     "bi_ctx_create": (I, [ctypes.POINTER(ModelDesc), ctypes.POINTER(Weights), ctypes.POINTER(KvLayout),
                           ctypes.POINTER(P)]),
     "bi_ctx_destroy": (I, [P]),

@@ -548,6 +548,56 @@ int bi_decode_step(bi_ctx* ctx, const bi_batch* batch, const bi_step_out* out, v
                     out->lse, out->argmax, out->margin, out->recomputed, out->logits, s.lm, s.lm_bytes, st);
 }
 
+// ------------------------------------------------ LM head without caller-supplied scratch
+// Some callers cannot call cudaMalloc: code that runs while a caching
+// allocator owns all device memory, plug-ins that are handed only their
+// inputs and outputs, or hosts that forbid allocation on the request path.
+// For them bi_lmhead_logprob_noalloc takes its scratch from this fixed
+// file-scope array instead of a workspace argument.  The array is part of
+// the library image: every GPU that loads the library holds it until the
+// process exits.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[BI_NOALLOC_SCRATCH_BYTES];
+
+// Device address of the array on each device.  Host code cannot use the
+// symbol itself (on the host it names a stand-in, not device memory), so the
+// address is looked up once per device, with that device current.
+static int noalloc_scratch_ptr(void** out) {
+  static std::mutex mu;
+  static std::vector<void*> addr;
+  int dev = 0;
+  BI_CHECK_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> g(mu);
+  if ((int)addr.size() <= dev) addr.resize(dev + 1, nullptr);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    BI_CHECK_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return BI_OK;
+}
+
+int bi_lmhead_logprob_noalloc(const float* h, const void* W, const int32_t* target, int B, int H, int V,
+                              float margin_threshold, int mode, float* logprob, float* lse, int32_t* argmax,
+                              float* margin, uint8_t* recomputed, float* logits, void* stream) {
+  clear_error();
+  BI_REQUIRE(B >= 0 && H > 0 && V > 0, BI_ERR_INVALID_ARG, "bi_lmhead_logprob_noalloc: bad sizes");
+  if (B == 0) return BI_OK;
+  Carver probe(nullptr);
+  lm_carve(probe, B, H, V, mode, logits == nullptr);
+  const size_t need = probe.used + 256;
+  BI_REQUIRE(need <= (size_t)BI_NOALLOC_SCRATCH_BYTES, BI_ERR_WORKSPACE,
+             "bi_lmhead_logprob_noalloc: B=%d H=%d V=%d needs %zu bytes of scratch, more than the fixed %d; "
+             "use bi_lmhead_logprob with a workspace or fewer rows",
+             B, H, V, need, BI_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  BI_TRY(noalloc_scratch_ptr(&scratch));
+  // Every scratch byte the kernels read is written earlier in the same call,
+  // so nothing needs clearing between calls.
+  return lmhead_run(h, W, target, B, H, V, margin_threshold, mode, logprob, lse, argmax, margin, recomputed, logits,
+                    scratch, BI_NOALLOC_SCRATCH_BYTES, as_stream(stream));
+}
+
 int bi_greedy_advance(const int32_t* argmax, int32_t* ids, int32_t* pos, int B, void* stream) {
   clear_error();
   BI_REQUIRE(argmax && ids && pos && B >= 0, BI_ERR_INVALID_ARG, "bi_greedy_advance: bad arguments");
