@@ -65,6 +65,8 @@ template <int NP>
 __global__ void __launch_bounds__(ATT_THREADS)
     attn_partial_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ AttnPlan plan, const AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar[ATT_RING];
   __shared__ float m_s[NP], l_s[NP];
@@ -263,6 +265,8 @@ __global__ void __launch_bounds__(ATT_THREADS)
 // One warp per (token, q head): fixed ascending merge of the chunk partials.
 __global__ void attn_merge_kernel(const float* __restrict__ part, const int32_t* __restrict__ pos, void* __restrict__ out,
                                   int t_base, int T, int Hq, int d, int chunk, int max_chunks, int f32) {
+  pdl_wait();
+  pdl_trigger();
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= T * Hq) return;

@@ -8,7 +8,9 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <string>
+#include <utility>
 
 #include "../../include/bi.h"
 
@@ -41,6 +43,26 @@ extern long long g_launches;  // host-side count of kernels launched by the libr
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 int num_sms();  // of the current device (cached per device)
+bool pdl_enabled();  // programmatic dependent launch (env BI_PDL=0 turns it off)
+
+// Launch a library kernel on `st`, with programmatic stream serialisation
+// allowed (see pdl_wait / pdl_trigger), counting it in g_launches.
+template <typename... KArgs, typename... Args>
+int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  BI_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...));
+  BI_CHECK_LAUNCH();
+  return BI_OK;
+}
 
 // Device-side error word: kernels set bits here instead of trapping when a
 // bounded wait runs out or an index fails its check.
@@ -52,8 +74,20 @@ __device__ __forceinline__ void dev_flag(unsigned bit) { atomicOr(&g_dev_error, 
 int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,
                    uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                    CUtensorMapSwizzle swizzle);
+// 3-D view: dims[0] contiguous elements; strides in bytes of dims 1 and 2.
+int encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, const uint64_t dims[3],
+                   const uint64_t strides[2], const uint32_t box[3], CUtensorMapSwizzle swizzle);
 
 // ------------------------------------------------------------------ PTX helpers
+// Programmatic dependent launch.  Every kernel of the library calls pdl_wait()
+// before it reads anything an earlier kernel wrote and before it writes
+// anything (so the chain of completions stays transitive), then pdl_trigger()
+// so the next kernel may be scheduled and run its independent prologue
+// (barrier set-up, weight prefetch) while this one finishes.  Both are no-ops
+// for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -95,6 +129,15 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
           "r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c_inner), "r"(c_outer), "r"(smem_u32(bar))
+      : "memory");
+}
+// 3D tiled TMA load (coordinates innermost first).
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {

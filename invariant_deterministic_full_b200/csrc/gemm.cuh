@@ -35,14 +35,21 @@
 namespace bi {
 
 constexpr int GEMM_BM = 32;  // token rows per tile (fixed; never depends on M)
-constexpr int GEMM_BK = 64;  // k per TMA box (128 bytes of bf16)
+constexpr int GEMM_BK = 64;  // k per k-block (128 bytes of bf16: one swizzled smem line)
 
+// One ring stage holds KBS consecutive k-blocks of the weight tile (BN rows)
+// and of the token tile (32 rows), each fetched by ONE 3-D TMA operation whose
+// box is {64 k, rows, KBS k-blocks}: the k-block dimension is the outermost of
+// the box, so in shared memory every k-block is a [rows][128 B] slab with the
+// 128-byte swizzle -- the layout ldmatrix reads without bank conflicts.  Few,
+// large TMA operations per stage keep each SM streaming near its peak rate.
 template <int BN>
 struct GemmCfg {
-  static constexpr int STAGES = BN == 32 ? 16 : (BN == 64 ? 12 : 8);
-  static constexpr int W_BYTES = BN * 128;
-  static constexpr int X_BYTES = GEMM_BM * 128;
+  static constexpr int KBS = BN == 128 ? 2 : 4;
+  static constexpr int W_BYTES = KBS * BN * 128;
+  static constexpr int X_BYTES = KBS * GEMM_BM * 128;
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;
   static constexpr int RW = BN / 32;      // warps along the weight rows (32 rows each)
   static constexpr int TW = 4 / RW;       // warps along the token columns
@@ -67,8 +74,10 @@ __global__ void __launch_bounds__(160, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kblocks_total = K / GEMM_BK;
-  const int kb_per_split = (kblocks_total + splits - 1) / splits;
+  // stages of KBS k-blocks; a final partial stage reads zeros past K (TMA fill),
+  // which add exact zeros to the accumulators
+  const int kstages_total = (K / GEMM_BK + C::KBS - 1) / C::KBS;
+  const int ks_per_split = (kstages_total + splits - 1) / splits;
   const int n_items = splits * n_groups * m_tiles;
 
   if (threadIdx.x == 0) {
@@ -84,29 +93,51 @@ __global__ void __launch_bounds__(160, 1)
     if (lane == 0) {
       prefetch_tmap(&tmW);
       prefetch_tmap(&tmX);
+      // Prologue: the first ring stages of weight tiles depend on no earlier
+      // kernel, so they are requested before waiting for the previous launch.
+      int pre = 0;
+      if ((int)blockIdx.x < n_items) {
+        const int item = blockIdx.x;
+        const int g = (item / m_tiles) % n_groups;
+        const int ks0 = (item / (m_tiles * n_groups)) * ks_per_split;
+        const int ks1 = min(kstages_total, ks0 + ks_per_split);
+        pre = max(0, min(C::STAGES, ks1 - ks0));
+        for (int s = 0; s < pre; ++s) {
+          mbar_arrive_expect_tx(&full_bar[s], C::STAGE_BYTES);
+          tma_load_3d(smem + s * C::STAGE_BYTES, &tmW, 0, g * BN, (ks0 + s) * C::KBS, &full_bar[s]);
+        }
+      }
+      pdl_wait();
+      pdl_trigger();
       int stage = 0;
       uint32_t phase = 0;
+      bool first = true;
       for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
         const int mt = item % m_tiles;
         const int g = (item / m_tiles) % n_groups;
         const int sp = item / (m_tiles * n_groups);
-        const int kb0 = sp * kb_per_split;
-        const int kb1 = min(kblocks_total, kb0 + kb_per_split);
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1)) return;
+        const int ks0 = sp * ks_per_split;
+        const int ks1 = min(kstages_total, ks0 + ks_per_split);
+        for (int ks = ks0; ks < ks1; ++ks) {
           uint8_t* sb = smem + stage * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
-          tma_load_2d(sb, &tmW, kb * GEMM_BK, g * BN, &full_bar[stage]);
-          tma_load_2d(sb + C::W_BYTES, &tmX, kb * GEMM_BK, mt * GEMM_BM, &full_bar[stage]);
+          if (!(first && ks - ks0 < pre)) {
+            if (!mbar_wait(&empty_bar[stage], phase ^ 1)) return;
+            mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+            tma_load_3d(sb, &tmW, 0, g * BN, ks * C::KBS, &full_bar[stage]);
+          }
+          tma_load_3d(sb + C::W_BYTES, &tmX, 0, mt * GEMM_BM, ks * C::KBS, &full_bar[stage]);
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
+        first = false;
       }
     }
     return;
   }
+  pdl_wait();
+  pdl_trigger();
 
   // ---------------- consumers
   const int rw = warp % C::RW, tw = warp / C::RW;
@@ -119,8 +150,8 @@ __global__ void __launch_bounds__(160, 1)
     const int mt = item % m_tiles;
     const int g = (item / m_tiles) % n_groups;
     const int sp = item / (m_tiles * n_groups);
-    const int kb0 = sp * kb_per_split;
-    const int kb1 = min(kblocks_total, kb0 + kb_per_split);
+    const int ks0 = sp * ks_per_split;
+    const int ks1 = min(kstages_total, ks0 + ks_per_split);
     const bool active = mt * GEMM_BM + tok0 < M;
     // KS interleaved accumulator sets: k16 step s (counted from k = 0) adds into
     // set s % KS; the sets are combined in a fixed tree after the K loop.
@@ -134,35 +165,40 @@ __global__ void __launch_bounds__(160, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c) accs[q][a][b][c] = 0.f;
 
-    for (int kb = kb0; kb < kb1; ++kb) {
+    for (int ks = ks0; ks < ks1; ++ks) {
       if (!mbar_wait(&full_bar[stage], phase)) return;
       if (active) {
-        const uint32_t wb = smem_u32(smem + stage * C::STAGE_BYTES);
-        const uint32_t xb = wb + C::W_BYTES;
+        const uint32_t sbase = smem_u32(smem + stage * C::STAGE_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          uint32_t a[2][4];
+        for (int kb = 0; kb < C::KBS; ++kb) {
+          const uint32_t wb = sbase + kb * (BN * 128);
+          const uint32_t xb = sbase + C::W_BYTES + kb * (GEMM_BM * 128);
 #pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const int row = row0 + r * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            ldsm_x4(swz128(wb, row, 2 * kk + (lane >> 4)), a[r][0], a[r][1], a[r][2], a[r][3]);
-          }
-          uint32_t b[C::NT][2];
-          if constexpr (C::NT >= 2) {
+          for (int kk = 0; kk < 4; ++kk) {
+            uint32_t a[2][4];
 #pragma unroll
-            for (int p = 0; p < C::NT / 2; ++p) {
-              const int tok = tok0 + p * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-              ldsm_x4(swz128(xb, tok, 2 * kk + ((lane >> 3) & 1)), b[2 * p][0], b[2 * p][1], b[2 * p + 1][0],
-                      b[2 * p + 1][1]);
+            for (int r = 0; r < 2; ++r) {
+              const int row = row0 + r * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+              ldsm_x4(swz128(wb, row, 2 * kk + (lane >> 4)), a[r][0], a[r][1], a[r][2], a[r][3]);
             }
-          } else {
-            const int tok = tok0 + (lane & 7);
-            ldsm_x2(swz128(xb, tok, 2 * kk + ((lane >> 3) & 1)), b[0][0], b[0][1]);
+            uint32_t b[C::NT][2];
+            if constexpr (C::NT >= 2) {
+#pragma unroll
+              for (int p = 0; p < C::NT / 2; ++p) {
+                const int tok = tok0 + p * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+                ldsm_x4(swz128(xb, tok, 2 * kk + ((lane >> 3) & 1)), b[2 * p][0], b[2 * p][1], b[2 * p + 1][0],
+                        b[2 * p + 1][1]);
+              }
+            } else {
+              const int tok = tok0 + (lane & 7);
+              ldsm_x2(swz128(xb, tok, 2 * kk + ((lane >> 3) & 1)), b[0][0], b[0][1]);
+            }
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+              for (int nt = 0; nt < C::NT; ++nt)
+                mma_bf16_16816(accs[kk % C::KS][r][nt], a[r], b[nt][0], b[nt][1]);
           }
-#pragma unroll
-          for (int r = 0; r < 2; ++r)
-#pragma unroll
-            for (int nt = 0; nt < C::NT; ++nt) mma_bf16_16816(accs[kk % C::KS][r][nt], a[r], b[nt][0], b[nt][1]);
         }
       }
       __syncwarp();
@@ -217,6 +253,8 @@ __global__ void __launch_bounds__(160, 1)
 template <int EPI>
 __global__ void splitk_reduce_kernel(const float* __restrict__ partial, void* __restrict__ y, int ldy, int y_f32, int M,
                                      int N, int splits) {
+  pdl_wait();
+  pdl_trigger();
   const int n_out = EPI == BI_EPI_SWIGLU ? N / 2 : N;
   const size_t total = (size_t)M * n_out;
   for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total; idx += (size_t)gridDim.x * blockDim.x) {
@@ -240,7 +278,7 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, void* __
 
 // ---------------------------------------------------------------- LayerCast (fp32 FMA)
 constexpr int F32_ROWS = 32;  // weight rows per CTA (8 warps x 4 rows)
-constexpr int F32_TOK = 8;    // token columns per CTA
+constexpr int F32_TOK = 16;   // token columns per CTA
 
 // x: f32 [M][ldx]; w: bf16 [N][K]; y: [M][ldy].  Optional device row count
 // (count != nullptr): only token rows < *count are computed (used by the
@@ -249,6 +287,8 @@ template <int EPI>
 __global__ void __launch_bounds__(256)
     gemm_f32_kernel(const float* __restrict__ x, int ldx, const uint16_t* __restrict__ w, void* __restrict__ y,
                     int ldy, int y_f32, int M, int N, int K, const int* __restrict__ count) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * F32_TOK;
   int Meff = M;
@@ -326,13 +366,15 @@ static int gemm_pick_bn(int N) {
 // Split factor of the FAST variant: more K splits for small M so that the
 // grid fills the SMs (the usual library heuristic) -- which is exactly what
 // makes the result depend on the batch size.
-static int gemm_fast_splits(int M, int n_items, int kblocks) {
+static int gemm_kbs(int bn) { return bn == 128 ? GemmCfg<128>::KBS : (bn == 64 ? GemmCfg<64>::KBS : GemmCfg<32>::KBS); }
+
+static int gemm_fast_splits(int M, int n_items, int kstages) {
   const int sms = num_sms();
   if (M > 16) return 1;
   int s = (2 * sms + n_items - 1) / n_items;
   if (M <= 4) s *= 2;
   s = s < 1 ? 1 : (s > 8 ? 8 : s);
-  while (s > 1 && kblocks / s < 4) --s;
+  while (s > 1 && kstages / s < 2) --s;
   return s;
 }
 
@@ -340,7 +382,8 @@ size_t gemm_ws_bytes(int M, int N, int K, int mode, int variant) {
   if (variant != BI_VARIANT_FAST || mode != BI_MODE_BF16) return 0;
   const int bn = gemm_pick_bn(N);
   const int items = (N / bn) * ((M + GEMM_BM - 1) / GEMM_BM);
-  const int s = gemm_fast_splits(M, items, K / GEMM_BK);
+  const int kbs = gemm_kbs(bn);
+  const int s = gemm_fast_splits(M, items, (K / GEMM_BK + kbs - 1) / kbs);
   return s > 1 ? (size_t)s * M * N * sizeof(float) : 0;
 }
 
@@ -357,24 +400,30 @@ static int launch_gemm_bf16_t(const CUtensorMap& tw, const CUtensorMap& tx, void
   const int n_groups = N / BN;
   const int items = splits * n_groups * m_tiles;
   const int grid = items < num_sms() ? items : num_sms();
-  gemm_bf16_kernel<BN, EPI><<<grid, 160, C::SMEM, st>>>(tw, tx, y, ldy, y_f32, M, N, K, m_tiles, n_groups, splits,
-                                                         partial);
-  BI_CHECK_LAUNCH();
+  BI_TRY(launch(gemm_bf16_kernel<BN, EPI>, dim3(grid), dim3(160), C::SMEM, st, tw, tx, y, ldy, y_f32, M, N, K, m_tiles, n_groups, splits,
+                                                         partial));
   return BI_OK;
 }
 
 int gemm_bf16(const void* x, int ldx, const void* w, void* y, int ldy, int y_f32, int M, int N, int K, int epi,
               int variant, void* ws, size_t ws_bytes, cudaStream_t st) {
   const int bn = gemm_pick_bn(N);
+  const int kbs = gemm_kbs(bn);
+  // 3-D views {64 k, rows, k-block}: the k-block dimension (stride 128 B) is the
+  // outermost of the box, so a box lands as kbs swizzled [rows][128 B] slabs.
   CUtensorMap tw, tx;
-  BI_TRY(encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, K, N, (uint64_t)K * 2, GEMM_BK, bn,
-                        CU_TENSOR_MAP_SWIZZLE_128B));
-  BI_TRY(encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, K, M, (uint64_t)ldx * 2, GEMM_BK, GEMM_BM,
-                        CU_TENSOR_MAP_SWIZZLE_128B));
+  const uint64_t dw[3] = {(uint64_t)GEMM_BK, (uint64_t)N, (uint64_t)(K / GEMM_BK)};
+  const uint64_t sw[2] = {(uint64_t)K * 2, (uint64_t)GEMM_BK * 2};
+  const uint32_t bw[3] = {(uint32_t)GEMM_BK, (uint32_t)bn, (uint32_t)kbs};
+  BI_TRY(encode_tmap_3d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, dw, sw, bw, CU_TENSOR_MAP_SWIZZLE_128B));
+  const uint64_t dx[3] = {(uint64_t)GEMM_BK, (uint64_t)M, (uint64_t)(K / GEMM_BK)};
+  const uint64_t sx[2] = {(uint64_t)ldx * 2, (uint64_t)GEMM_BK * 2};
+  const uint32_t bx[3] = {(uint32_t)GEMM_BK, (uint32_t)GEMM_BM, (uint32_t)kbs};
+  BI_TRY(encode_tmap_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_128B));
   int splits = 1;
   if (variant == BI_VARIANT_FAST) {
     const int items = (N / bn) * ((M + GEMM_BM - 1) / GEMM_BM);
-    splits = gemm_fast_splits(M, items, K / GEMM_BK);
+    splits = gemm_fast_splits(M, items, (K / GEMM_BK + kbs - 1) / kbs);
   }
   float* partial = nullptr;
   if (splits > 1) {
@@ -399,10 +448,9 @@ int gemm_bf16(const void* x, int ldx, const void* w, void* y, int ldy, int y_f32
     int blocks = (int)((total + 255) / 256);
     if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
     if (epi == BI_EPI_SWIGLU)
-      splitk_reduce_kernel<BI_EPI_SWIGLU><<<blocks, 256, 0, st>>>(partial, y, ldy, y_f32, M, N, splits);
+      BI_TRY(launch(splitk_reduce_kernel<BI_EPI_SWIGLU>, dim3(blocks), dim3(256), 0, st, partial, y, ldy, y_f32, M, N, splits));
     else
-      splitk_reduce_kernel<BI_EPI_NONE><<<blocks, 256, 0, st>>>(partial, y, ldy, y_f32, M, N, splits);
-    BI_CHECK_LAUNCH();
+      BI_TRY(launch(splitk_reduce_kernel<BI_EPI_NONE>, dim3(blocks), dim3(256), 0, st, partial, y, ldy, y_f32, M, N, splits));
   }
   return BI_OK;
 }
@@ -411,12 +459,11 @@ int gemm_f32(const float* x, int ldx, const void* w, void* y, int ldy, int y_f32
              const int* count, cudaStream_t st) {
   dim3 grid((M + F32_TOK - 1) / F32_TOK, N / F32_ROWS);
   if (epi == BI_EPI_SWIGLU)
-    gemm_f32_kernel<BI_EPI_SWIGLU><<<grid, 256, 0, st>>>(x, ldx, reinterpret_cast<const uint16_t*>(w), y, ldy, y_f32,
-                                                         M, N, K, count);
+    BI_TRY(launch(gemm_f32_kernel<BI_EPI_SWIGLU>, dim3(grid), dim3(256), 0, st, x, ldx, reinterpret_cast<const uint16_t*>(w), y, ldy, y_f32,
+                                                         M, N, K, count));
   else
-    gemm_f32_kernel<BI_EPI_NONE><<<grid, 256, 0, st>>>(x, ldx, reinterpret_cast<const uint16_t*>(w), y, ldy, y_f32, M,
-                                                       N, K, count);
-  BI_CHECK_LAUNCH();
+    BI_TRY(launch(gemm_f32_kernel<BI_EPI_NONE>, dim3(grid), dim3(256), 0, st, x, ldx, reinterpret_cast<const uint16_t*>(w), y, ldy, y_f32, M,
+                                                       N, K, count));
   return BI_OK;
 }
 

@@ -87,12 +87,11 @@ static int attn_launch(int np, const CUtensorMap& tk, const CUtensorMap& tv, con
   const dim3 grid(plan.n, a.max_chunks, a.Hkv);
   const size_t smem = att_smem_bytes(np, a.d, a.f32);
   switch (np) {
-    case 4: attn_partial_kernel<4><<<grid, ATT_THREADS, smem, st>>>(tk, tv, plan, a); break;
-    case 8: attn_partial_kernel<8><<<grid, ATT_THREADS, smem, st>>>(tk, tv, plan, a); break;
-    case 16: attn_partial_kernel<16><<<grid, ATT_THREADS, smem, st>>>(tk, tv, plan, a); break;
-    default: attn_partial_kernel<32><<<grid, ATT_THREADS, smem, st>>>(tk, tv, plan, a); break;
+    case 4: BI_TRY(launch(attn_partial_kernel<4>, dim3(grid), dim3(ATT_THREADS), smem, st, tk, tv, plan, a)); break;
+    case 8: BI_TRY(launch(attn_partial_kernel<8>, dim3(grid), dim3(ATT_THREADS), smem, st, tk, tv, plan, a)); break;
+    case 16: BI_TRY(launch(attn_partial_kernel<16>, dim3(grid), dim3(ATT_THREADS), smem, st, tk, tv, plan, a)); break;
+    default: BI_TRY(launch(attn_partial_kernel<32>, dim3(grid), dim3(ATT_THREADS), smem, st, tk, tv, plan, a)); break;
   }
-  BI_CHECK_LAUNCH();
   return BI_OK;
 }
 
@@ -177,9 +176,8 @@ static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const
     if (p1.n) BI_TRY(attn_launch(np1, tk, tv, p1, a, st));
     if (pm.n) BI_TRY(attn_launch(ATT_MAX_PAIRS, tk, tv, pm, a, st));
     const int nw = (t_end - t_base) * Hq;
-    attn_merge_kernel<<<(nw * 32 + 255) / 256, 256, 0, st>>>(part, pos, out, t_base, t_end - t_base, Hq, d, chunk,
-                                                              max_chunks, f32);
-    BI_CHECK_LAUNCH();
+    BI_TRY(launch(attn_merge_kernel, dim3((nw * 32 + 255) / 256), dim3(256), 0, st, part, pos, out, t_base, t_end - t_base, Hq, d, chunk,
+                                                              max_chunks, f32));
     bi0 = bi1;
   }
   return BI_OK;
@@ -233,27 +231,21 @@ static int lmhead_run(const float* h, const void* W, const int32_t* target, int 
 
   if (mode == BI_MODE_BF16) {
     const size_t n = (size_t)B * H;
-    f32_to_bf16_kernel<<<(int)std::min<size_t>((n + 255) / 256, 4096), 256, 0, st>>>(h, w.h16, n);
-    BI_CHECK_LAUNCH();
+    BI_TRY(launch(f32_to_bf16_kernel, dim3((int)std::min<size_t>((n + 255) / 256, 4096)), dim3(256), 0, st, h, w.h16, n));
     BI_TRY(gemm_bf16(w.h16, H, W, z, V, 1, B, V, H, BI_EPI_NONE, BI_VARIANT_INVARIANT, nullptr, 0, st));
   } else {
     BI_TRY(gemm_f32(h, H, W, z, V, 1, B, V, H, BI_EPI_NONE, nullptr, st));
   }
-  lm_partial_kernel<<<dim3(nch, B), LM_CHUNK, 0, st>>>(z, V, V, target, nullptr, nullptr, w.part, nch);
-  BI_CHECK_LAUNCH();
+  BI_TRY(launch(lm_partial_kernel, dim3(dim3(nch, B)), dim3(LM_CHUNK), 0, st, z, V, V, target, nullptr, nullptr, w.part, nch));
   const float th = mode == BI_MODE_BF16 ? thresh : 0.f;
-  lm_merge_kernel<<<(B * 32 + 127) / 128, 128, 0, st>>>(w.part, nch, B, nullptr, nullptr, target, th, 0, logprob, lse,
-                                                        argmax, margin, recomputed, w.flag);
-  BI_CHECK_LAUNCH();
+  BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, nullptr, nullptr, target, th, 0, logprob, lse,
+                                                        argmax, margin, recomputed, w.flag));
   if (mode == BI_MODE_BF16 && th > 0.f) {
-    lm_compact_kernel<<<1, 256, 0, st>>>(w.flag, B, h, H, w.list, w.count, w.hc);
-    BI_CHECK_LAUNCH();
+    BI_TRY(launch(lm_compact_kernel, dim3(B), dim3(256), 0, st, w.flag, B, h, H, w.list, w.count, w.hc));
     BI_TRY(gemm_f32(w.hc, H, W, w.logits_c, V, 1, B, V, H, BI_EPI_NONE, w.count, st));
-    lm_partial_kernel<<<dim3(nch, B), LM_CHUNK, 0, st>>>(w.logits_c, V, V, target, w.list, w.count, w.part, nch);
-    BI_CHECK_LAUNCH();
-    lm_merge_kernel<<<(B * 32 + 127) / 128, 128, 0, st>>>(w.part, nch, B, w.count, w.list, target, th, 1, logprob,
-                                                          lse, argmax, margin, recomputed, nullptr);
-    BI_CHECK_LAUNCH();
+    BI_TRY(launch(lm_partial_kernel, dim3(dim3(nch, B)), dim3(LM_CHUNK), 0, st, w.logits_c, V, V, target, w.list, w.count, w.part, nch));
+    BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, w.count, w.list, target, th, 1, logprob,
+                                                          lse, argmax, margin, recomputed, nullptr));
   }
   return BI_OK;
 }
@@ -313,10 +305,9 @@ int bi_rmsnorm(const void* x, const void* residual_in, void* residual_out, const
                  (!residual_out || aligned16(residual_out)) && (!y_f32 || aligned16(y_f32)),
              BI_ERR_UNSUPPORTED, "bi_rmsnorm: buffers must be 16-byte aligned");
   if (M == 0) return BI_OK;
-  rmsnorm_kernel<<<M, NORM_THREADS, 0, as_stream(stream)>>>(x, residual_in, residual_out,
+  BI_TRY(launch(rmsnorm_kernel, dim3(M), dim3(NORM_THREADS), 0, as_stream(stream), x, residual_in, residual_out,
                                                             reinterpret_cast<const uint16_t*>(gamma), y, y_f32, H, eps,
-                                                            mode == BI_MODE_LAYERCAST);
-  BI_CHECK_LAUNCH();
+                                                            mode == BI_MODE_LAYERCAST));
   return BI_OK;
 }
 
@@ -347,10 +338,9 @@ int bi_rope_kv_append(const float* qkv, const float* rope, int rope_max_pos, voi
   BI_REQUIRE(kv->dtype == (mode == BI_MODE_LAYERCAST ? BI_DTYPE_F32 : BI_DTYPE_BF16), BI_ERR_INVALID_ARG,
              "bi_rope_kv_append: KV dtype does not match the mode");
   if (T == 0) return BI_OK;
-  rope_append_kernel<<<T, 256, 0, as_stream(stream)>>>(qkv, rope, rope_max_pos, q_out, kv->k, kv->v, slot, pos, Hq,
+  BI_TRY(launch(rope_append_kernel, dim3(T), dim3(256), 0, as_stream(stream), qkv, rope, rope_max_pos, q_out, kv->k, kv->v, slot, pos, Hq,
                                                        kv->n_kv_heads, kv->head_dim, layer, kv->n_layers, kv->n_slots,
-                                                       kv->capacity, mode == BI_MODE_LAYERCAST);
-  BI_CHECK_LAUNCH();
+                                                       kv->capacity, mode == BI_MODE_LAYERCAST));
   return BI_OK;
 }
 
@@ -470,6 +460,8 @@ size_t bi_decode_workspace_size(const bi_ctx* ctx, int max_tokens, int max_lm_ro
 
 __global__ void gather_lm_rows_kernel(const int32_t* __restrict__ lm_row, const float* __restrict__ h32, int T, int H,
                                       int n_lm, float* __restrict__ hl, float* __restrict__ h_out) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   const int r = lm_row[t];
   if (r < 0) return;
@@ -520,8 +512,7 @@ int bi_decode_step(bi_ctx* ctx, const bi_batch* batch, const bi_step_out* out, v
     return reinterpret_cast<const void*>(reinterpret_cast<const uint8_t*>(base) + per_layer * l * wbytes);
   };
 
-  embed_kernel<<<T, 256, 0, st>>>(batch->ids, reinterpret_cast<const uint16_t*>(w.embed), s.y, H, d.vocab, f32);
-  BI_CHECK_LAUNCH();
+  BI_TRY(launch(embed_kernel, dim3(T), dim3(256), 0, st, batch->ids, reinterpret_cast<const uint16_t*>(w.embed), s.y, H, d.vocab, f32));
   for (int l = 0; l < d.n_layers; ++l) {
     const void* g_attn = lw(w.attn_norm, H, l);
     const void* g_ffn = lw(w.ffn_norm, H, l);
@@ -542,8 +533,7 @@ int bi_decode_step(bi_ctx* ctx, const bi_batch* batch, const bi_step_out* out, v
   }
   BI_TRY(bi_rmsnorm(s.y, s.res, s.res, w.final_norm, s.u, s.h32, T, H, d.eps, d.mode, stream));
   if (n_lm == 0) return BI_OK;
-  gather_lm_rows_kernel<<<T, 256, 0, st>>>(batch->lm_row, s.h32, T, H, n_lm, s.hl, out->h);
-  BI_CHECK_LAUNCH();
+  BI_TRY(launch(gather_lm_rows_kernel, dim3(T), dim3(256), 0, st, batch->lm_row, s.h32, T, H, n_lm, s.hl, out->h));
   return lmhead_run(s.hl, w.lm_head, batch->target, n_lm, H, d.vocab, d.margin_threshold, d.mode, out->logprob,
                     out->lse, out->argmax, out->margin, out->recomputed, out->logits, s.lm, s.lm_bytes, st);
 }
@@ -602,8 +592,7 @@ int bi_greedy_advance(const int32_t* argmax, int32_t* ids, int32_t* pos, int B, 
   clear_error();
   BI_REQUIRE(argmax && ids && pos && B >= 0, BI_ERR_INVALID_ARG, "bi_greedy_advance: bad arguments");
   if (B == 0) return BI_OK;
-  greedy_advance_kernel<<<(B + 127) / 128, 128, 0, as_stream(stream)>>>(argmax, ids, pos, B);
-  BI_CHECK_LAUNCH();
+  BI_TRY(launch(greedy_advance_kernel, dim3((B + 127) / 128), dim3(128), 0, as_stream(stream), argmax, ids, pos, B));
   return BI_OK;
 }
 
@@ -615,8 +604,7 @@ int bi_synth_fill_bf16(uint16_t* dst, int64_t rows, int64_t cols, uint64_t key, 
   BI_REQUIRE(interleave == 0 || rows % interleave == 0, BI_ERR_INVALID_ARG,
              "bi_synth_fill_bf16: rows must be a multiple of the interleave");
   if (rows == 0) return BI_OK;
-  synth_fill_kernel<<<4 * num_sms(), 256, 0, as_stream(stream)>>>(dst, rows, cols, key, std, interleave, phase);
-  BI_CHECK_LAUNCH();
+  BI_TRY(launch(synth_fill_kernel, dim3(4 * num_sms()), dim3(256), 0, as_stream(stream), dst, rows, cols, key, std, interleave, phase));
   return BI_OK;
 }
 

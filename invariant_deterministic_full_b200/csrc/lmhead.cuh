@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(LM_CHUNK)
     lm_partial_kernel(const float* __restrict__ logits, size_t ldz, int V, const int32_t* __restrict__ target,
                       const int32_t* __restrict__ rows_map, const int* __restrict__ count, LmPart* __restrict__ part,
                       int n_chunks) {
+  pdl_wait();
+  pdl_trigger();
   const int c = blockIdx.x, r = blockIdx.y;
   if (count && r >= *count) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -111,6 +113,8 @@ __global__ void lm_merge_kernel(const LmPart* __restrict__ part, int n_chunks, i
                                 float thresh, int mode_recompute, float* __restrict__ logprob, float* __restrict__ lse,
                                 int32_t* __restrict__ argmax, float* __restrict__ margin,
                                 uint8_t* __restrict__ recomputed, uint8_t* __restrict__ flag) {
+  pdl_wait();
+  pdl_trigger();
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int nrows = count ? min(B, *count) : B;
@@ -158,27 +162,43 @@ __global__ void lm_merge_kernel(const LmPart* __restrict__ part, int n_chunks, i
 }
 
 // Ascending compaction of the flagged rows: list[k] = k-th flagged row, and
-// the f32 hidden rows gathered in that order.  One CTA.
+// the f32 hidden rows gathered in that order.  CTA b handles row b: its rank
+// is the number of flagged rows before it; CTA 0 also writes the count.
 __global__ void lm_compact_kernel(const uint8_t* __restrict__ flag, int B, const float* __restrict__ h, int H,
                                   int32_t* __restrict__ list, int* __restrict__ count, float* __restrict__ hc) {
-  __shared__ int n_s;
-  if (threadIdx.x == 0) {
-    int n = 0;
-    for (int b = 0; b < B; ++b)
-      if (flag[b]) list[n++] = b;
-    n_s = n;
-    *count = n;
+  pdl_wait();
+  pdl_trigger();
+  const int b = blockIdx.x;
+  __shared__ int rank_s, total_s;
+  if (threadIdx.x < 32) {
+    int before = 0, total = 0;
+    for (int i = threadIdx.x; i < B; i += 32) {
+      const int f = flag[i] != 0;
+      before += (i < b) ? f : 0;
+      total += f;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      before += __shfl_xor_sync(0xffffffffu, before, o);
+      total += __shfl_xor_sync(0xffffffffu, total, o);
+    }
+    if (threadIdx.x == 0) {
+      rank_s = before;
+      total_s = total;
+    }
   }
   __syncthreads();
-  const int n = n_s;
-  for (int k = 0; k < n; ++k) {
-    const int b = list[k];
-    for (int i = threadIdx.x; i < H; i += blockDim.x) hc[(size_t)k * H + i] = h[(size_t)b * H + i];
-  }
+  if (b == 0 && threadIdx.x == 0) *count = total_s;
+  if (!flag[b]) return;
+  const int k = rank_s;
+  if (threadIdx.x == 0) list[k] = b;
+  for (int i = threadIdx.x; i < H; i += blockDim.x) hc[(size_t)k * H + i] = h[(size_t)b * H + i];
 }
 
 // h (f32) -> bf16 (round to nearest even), the main-pass LM-head input.
 __global__ void f32_to_bf16_kernel(const float* __restrict__ in, uint16_t* __restrict__ out, size_t n) {
+  pdl_wait();
+  pdl_trigger();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
     out[i] = f32_to_bf16_bits(in[i]);
 }

@@ -45,6 +45,8 @@ __global__ void __launch_bounds__(NORM_THREADS)
     rmsnorm_kernel(const void* __restrict__ x, const void* __restrict__ res_in, void* __restrict__ res_out,
                    const uint16_t* __restrict__ gamma, void* __restrict__ y, float* __restrict__ y32, int H, float eps,
                    int f32) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float wsum[NORM_THREADS / 32];
   const int row = blockIdx.x;
   const int nch = H / 8;
@@ -100,6 +102,8 @@ __global__ void rope_append_kernel(const float* __restrict__ qkv, const float* _
                                    void* __restrict__ q_out, void* __restrict__ kc, void* __restrict__ vc,
                                    const int32_t* __restrict__ slot, const int32_t* __restrict__ pos, int Hq, int Hkv,
                                    int d, int layer, int n_layers, int n_slots, int cap, int f32) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   const int half = d / 2;
   const int p = pos[t], s = slot[t];
@@ -139,6 +143,8 @@ __global__ void rope_append_kernel(const float* __restrict__ qkv, const float* _
 // x[t][:] = E[ids[t]][:] in the activation dtype.
 __global__ void embed_kernel(const int32_t* __restrict__ ids, const uint16_t* __restrict__ E, void* __restrict__ x,
                              int H, int V, int f32) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   const int id = ids[t];
   if (id < 0 || id >= V) {
@@ -152,6 +158,8 @@ __global__ void embed_kernel(const int32_t* __restrict__ ids, const uint16_t* __
 
 __global__ void greedy_advance_kernel(const int32_t* __restrict__ argmax, int32_t* __restrict__ ids,
                                       int32_t* __restrict__ pos, int B) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) {
     ids[b] = argmax[b];

@@ -16,6 +16,8 @@ __device__ __forceinline__ uint64_t sm64_mix(uint64_t z) {
 
 __global__ void synth_fill_kernel(uint16_t* __restrict__ dst, int64_t rows, int64_t cols, uint64_t key, double std,
                                   int interleave, int phase) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t n = rows * cols;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     int64_t s = 0;
