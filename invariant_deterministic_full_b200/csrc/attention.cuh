@@ -11,9 +11,11 @@
 //   * chunk denominator l = sum_j exp(s_j - m): lane i of a warp sums keys
 //     i, i+32, ..., i+224 in ascending order (masked keys add exactly 0), then
 //     a fixed xor-butterfly over the 32 lanes;
-//   * chunk numerator acc[e] = sum_j p_j v_j[e]: sequential FMA over the valid
-//     keys in ascending order (keys past the query add exact zeros, so it is
-//     the same sum whether later queries share the tile or not);
+//   * chunk numerator acc[e] = sum_j p_j v_j[e]: the keys form 4 interleaved
+//     groups (j % 4); each group is a sequential FMA chain over its valid keys
+//     in ascending order, and the group sums are added as ((g0+g1)+(g2+g3))
+//     (keys past the query add exact zeros, so the sums are the same whether
+//     later queries share the tile or not);
 //   * merge over chunks 0..pos/CH: M = max m_c, L = sum_c l_c exp(m_c - M),
 //     o = sum_c acc_c exp(m_c - M), all in ascending chunk order; out = o / L.
 // A query's result depends only on its q and the cache rows 0..pos it reads.
@@ -50,7 +52,7 @@ constexpr int ATT_RING = 2;  // sub-tile buffers
 
 __host__ __device__ inline size_t att_sub_bytes(int d, int f32) { return (size_t)ATT_SUB * d * (f32 ? 4 : 2); }
 __host__ __device__ inline size_t att_smem_bytes(int np, int d, int f32) {
-  return ATT_RING * att_sub_bytes(d, f32) + (size_t)np * d * 4 + (size_t)np * ATT_CHUNK * 4 + 1024;
+  return ATT_RING * att_sub_bytes(d, f32) + (size_t)np * d * 4 + 2 * (size_t)np * ATT_CHUNK * 4 + 1024;
 }
 
 // Grid: (block, chunk, kv head).  The chunk's K rows, then its V rows, stream
@@ -86,7 +88,8 @@ __global__ void __launch_bounds__(ATT_THREADS)
   const int boxe = 128 / esz;
   const size_t sub_bytes = att_sub_bytes(a.d, a.f32);
   float* qs = reinterpret_cast<float*>(smem + ATT_RING * sub_bytes);
-  float* S = qs + NP * a.d;
+  float* S = qs + NP * a.d;       // scores [NP][256]
+  float* PT = S + NP * ATT_CHUNK;  // probabilities, key-major [256][NP] (S and PT also host the PV combine)
   const int npairs = nq * a.G;
   const int row_base = ((s * a.n_layers + a.layer) * a.Hkv + hk) * a.cap + key0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -203,7 +206,7 @@ __global__ void __launch_bounds__(ATT_THREADS)
         const int j = lane + 32 * k;
         float pj = 0.f;
         if (j <= lim && j < nvalid) pj = expf(S[pl * ATT_CHUNK + j] - mx);
-        if (j < nvalid) S[pl * ATT_CHUNK + j] = pj;
+        if (j < nvalid) PT[j * NP + pl] = pj;
         sum += pj;
       }
       sum = warp_sum_fixed(sum);
@@ -215,47 +218,80 @@ __global__ void __launch_bounds__(ATT_THREADS)
     }
     __syncthreads();
 
-    // ---- PV: acc[e] = sum_j p_j v_j[e], sequential FMA over the valid keys ascending
-    constexpr int PPT = NP >= 2 ? NP / 2 : 1;  // pairs per thread upper bound (d >= 64: at most 4 pair lanes)
-    const int e = tid % a.d;
-    const int pstep = ATT_THREADS / a.d;
-    const int p0 = tid / a.d;
-    const int ib_e = (e * esz) >> 7;
-    const int cc_e = ((e * esz) & 127) >> 4;
-    const int within = (e * esz) & 15;
-    float pacc[PPT];
+    // ---- PV: acc[e] = sum_j p_j v_j[e].  The keys of the chunk fall into 4
+    // interleaved groups (j % 4); each group is summed with sequential FMAs in
+    // ascending j, and the group sums are combined as ((g0 + g1) + (g2 + g3)).
+    // Thread t: key group t / 64, element pair ep, all pairs of its phase.
+    const int kg = tid >> 6;
+    const int r64 = tid & 63;
+    const int nep = a.d / 2;           // element pairs per row (64 or 32)
+    const int ep = r64 % nep;
+    const int ph = r64 / nep;          // pair phase (d = 64: pairs ph, ph + 2, ...)
+    const int pst = 64 / nep;          // pair stride: 1 (d = 128) or 2 (d = 64)
+    const int ebyte = ep * 2 * esz;
+    const int ib_e = ebyte >> 7, cc_e = (ebyte & 127) >> 4, within = ebyte & 15;
+    float pacc[NP][2];
 #pragma unroll
-    for (int k = 0; k < PPT; ++k) pacc[k] = 0.f;
+    for (int k = 0; k < NP; ++k) pacc[k][0] = pacc[k][1] = 0.f;
     for (int st = 0; st < nsub; ++st) {
       if (!consume_wait()) return;
       const uint8_t* vb = smem + (L % ATT_RING) * sub_bytes + ib_e * (ATT_SUB * 128) + within;
       const int jend = min(ATT_SUB, nvalid - st * ATT_SUB);
-      for (int jl = 0; jl < jend; ++jl) {
+      for (int jl = kg; jl < jend; jl += 4) {
         const uint8_t* vp = vb + jl * 128 + ((cc_e ^ (jl & 7)) << 4);
-        const float v = a.f32 ? *reinterpret_cast<const float*>(vp)
-                              : bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(vp));
-        const int j = st * ATT_SUB + jl;
+        float v0, v1;
+        if (a.f32) {
+          const float2 vv = *reinterpret_cast<const float2*>(vp);
+          v0 = vv.x;
+          v1 = vv.y;
+        } else {
+          const uint32_t vv = *reinterpret_cast<const uint32_t*>(vp);
+          v0 = bf16lo(vv);
+          v1 = bf16hi(vv);
+        }
+        const float* pr = PT + (st * ATT_SUB + jl) * NP;
+        if (pst == 1) {
 #pragma unroll
-        for (int k = 0; k < PPT; ++k) {
-          const int pl = p0 + k * pstep;
-          if (pl < gp) pacc[k] = fmaf(S[pl * ATT_CHUNK + j], v, pacc[k]);
+          for (int k = 0; k < NP; ++k) {
+            const float pv = pr[k];
+            pacc[k][0] = fmaf(pv, v0, pacc[k][0]);
+            pacc[k][1] = fmaf(pv, v1, pacc[k][1]);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < NP / 2; ++k) {
+            const float pv = pr[ph + 2 * k];
+            pacc[k][0] = fmaf(pv, v0, pacc[k][0]);
+            pacc[k][1] = fmaf(pv, v1, pacc[k][1]);
+          }
         }
       }
       release();
     }
+    // combine the 4 key groups in a fixed tree (S and PT are free: reuse them)
+    float* red = S;  // [4][NP][d]
 #pragma unroll
-    for (int k = 0; k < PPT; ++k) {
-      const int pl = p0 + k * pstep;
-      if (pl < gp && live_s[pl]) {
-        const int p = pg0 + pl;
-        const int i = p / a.G, g = p % a.G;
-        const int hq = hk * a.G + g;
-        float* rec = a.part + (((size_t)(t0 + i - a.t_base) * a.Hq + hq) * a.max_chunks + c) * (a.d + 4);
-        rec[e] = pacc[k];
-        if (e == 0) {
-          rec[a.d] = m_s[pl];
-          rec[a.d + 1] = l_s[pl];
-        }
+    for (int k = 0; k < NP; ++k) {
+      const int pl = ph + k * pst;
+      if (k < NP / pst) {
+        red[(kg * NP + pl) * a.d + 2 * ep] = pacc[k][0];
+        red[(kg * NP + pl) * a.d + 2 * ep + 1] = pacc[k][1];
+      }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < gp * a.d; idx += ATT_THREADS) {
+      const int pl = idx / a.d, e = idx % a.d;
+      if (!live_s[pl]) continue;
+      const float o = (red[(0 * NP + pl) * a.d + e] + red[(1 * NP + pl) * a.d + e]) +
+                      (red[(2 * NP + pl) * a.d + e] + red[(3 * NP + pl) * a.d + e]);
+      const int p = pg0 + pl;
+      const int i = p / a.G, g = p % a.G;
+      const int hq = hk * a.G + g;
+      float* rec = a.part + (((size_t)(t0 + i - a.t_base) * a.Hq + hq) * a.max_chunks + c) * (a.d + 4);
+      rec[e] = o;
+      if (e == 0) {
+        rec[a.d] = m_s[pl];
+        rec[a.d + 1] = l_s[pl];
       }
     }
     __syncthreads();  // the next group overwrites q, S and the pair statistics

@@ -279,16 +279,20 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, void* __
 // ---------------------------------------------------------------- LayerCast (fp32 FMA)
 constexpr int F32_ROWS = 32;  // weight rows per CTA (8 warps x 4 rows)
 constexpr int F32_TOK = 16;   // token columns per CTA
+constexpr int F32_KC = 256;   // k per chunk (32 lanes x 8)
 
 // x: f32 [M][ldx]; w: bf16 [N][K]; y: [M][ldy].  Optional device row count
 // (count != nullptr): only token rows < *count are computed (used by the
 // selective recompute, whose row count is known only on the device).
+// The CTA's 16 token rows are staged chunk by chunk (256 k) in shared memory,
+// double-buffered, and read by all 8 warps; each warp streams 4 weight rows.
 template <int EPI>
 __global__ void __launch_bounds__(256)
     gemm_f32_kernel(const float* __restrict__ x, int ldx, const uint16_t* __restrict__ w, void* __restrict__ y,
                     int ldy, int y_f32, int M, int N, int K, const int* __restrict__ count) {
   pdl_wait();
   pdl_trigger();
+  __shared__ __align__(16) float xs[2][F32_TOK][F32_KC];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * F32_TOK;
   int Meff = M;
@@ -304,54 +308,81 @@ __global__ void __launch_bounds__(256)
     else
       rows[r] = grp * F32_ROWS + 4 * warp + r;
   }
+  // staging: thread t copies 16 consecutive floats of token t / 16 at offset (t % 16) * 16
+  const int st_tok = threadIdx.x >> 4, st_off = (threadIdx.x & 15) * 16;
+  auto fetch = [&](int kc, float4* v) {
+    const int k = kc * F32_KC + st_off;
+    const bool ok = st_tok < ntok && k < K;
+    const float4* src = reinterpret_cast<const float4*>(x + (size_t)(m0 + st_tok) * ldx + k);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] = ok ? __ldg(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  auto stash = [&](int buf, const float4* v) {
+    float4* dst = reinterpret_cast<float4*>(&xs[buf][st_tok][st_off]);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = v[q];
+  };
   float acc[4][F32_TOK];
 #pragma unroll
   for (int r = 0; r < 4; ++r)
 #pragma unroll
     for (int t = 0; t < F32_TOK; ++t) acc[r][t] = 0.f;
 
-  for (int kbase = 0; kbase < K; kbase += 256) {
-    const int k = kbase + 8 * lane;
+  const int nk = (K + F32_KC - 1) / F32_KC;
+  {
+    float4 v[4];
+    fetch(0, v);
+    stash(0, v);
+  }
+  __syncthreads();
+  for (int kc = 0; kc < nk; ++kc) {
+    const int buf = kc & 1;
+    float4 nxt[4];
+    if (kc + 1 < nk) fetch(kc + 1, nxt);
+    const int k = kc * F32_KC + 8 * lane;
     if (k < K) {
-      float wf[4][8];
+      uint4 u[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(w + (size_t)rows[r] * K + k));
-        wf[r][0] = bf16lo(u.x); wf[r][1] = bf16hi(u.x); wf[r][2] = bf16lo(u.y); wf[r][3] = bf16hi(u.y);
-        wf[r][4] = bf16lo(u.z); wf[r][5] = bf16hi(u.z); wf[r][6] = bf16lo(u.w); wf[r][7] = bf16hi(u.w);
-      }
+      for (int r = 0; r < 4; ++r) u[r] = __ldg(reinterpret_cast<const uint4*>(w + (size_t)rows[r] * K + k));
 #pragma unroll
       for (int t = 0; t < F32_TOK; ++t) {
         if (t < ntok) {
-          const float4* xp = reinterpret_cast<const float4*>(x + (size_t)(m0 + t) * ldx + k);
-          const float4 x0 = __ldg(xp), x1 = __ldg(xp + 1);
+          const float4 x0 = *reinterpret_cast<const float4*>(&xs[buf][t][8 * lane]);
+          const float4 x1 = *reinterpret_cast<const float4*>(&xs[buf][t][8 * lane + 4]);
           const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
+          for (int j = 0; j < 8; ++j) {
 #pragma unroll
-            for (int r = 0; r < 4; ++r) acc[r][t] = fmaf(wf[r][j], xv[j], acc[r][t]);
+            for (int r = 0; r < 4; ++r) {
+              const uint32_t word = j < 2 ? u[r].x : j < 4 ? u[r].y : j < 6 ? u[r].z : u[r].w;
+              const float wv = (j & 1) ? bf16hi(word) : bf16lo(word);
+              acc[r][t] = fmaf(wv, xv[j], acc[r][t]);
+            }
+          }
         }
       }
     }
+    if (kc + 1 < nk) stash(buf ^ 1, nxt);
+    __syncthreads();
   }
 #pragma unroll
   for (int t = 0; t < F32_TOK; ++t) {
     if (t >= ntok) break;
-    float s[4];
+    float sr[4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) s[r] = warp_sum_fixed(acc[r][t]);
+    for (int r = 0; r < 4; ++r) sr[r] = warp_sum_fixed(acc[r][t]);
     const int m = m0 + t;
     if constexpr (EPI == BI_EPI_SWIGLU) {
       if (lane < 2) {
-        const float gv = lane == 0 ? s[0] : s[1];
-        const float uv = lane == 0 ? s[2] : s[3];
+        const float gv = lane == 0 ? sr[0] : sr[1];
+        const float uv = lane == 0 ? sr[2] : sr[3];
         const int col = grp * 16 + 2 * warp + lane;
         store_act(y, (size_t)m * ldy + col, silu(gv) * uv, y_f32);
       }
     } else {
 #pragma unroll
       for (int r = 0; r < 4; ++r)
-        if (lane == r) store_act(y, (size_t)m * ldy + rows[r], s[r], y_f32);
+        if (lane == r) store_act(y, (size_t)m * ldy + rows[r], sr[r], y_f32);
     }
   }
 }
