@@ -169,9 +169,12 @@ int bi_attention(const void* q, const bi_kv_layout* kv, int layer, const int32_t
  * Selective FP32 recompute ("Greedy Decoding Is Not Precision-Invariant",
  *   method section: recompute the LM head in FP32 only when the top-two logit
  *   margin falls below a threshold): in BI_MODE_BF16, rows with
- *   margin < margin_threshold are recomputed as fp32 FMA of the f32 h with the
- *   upcast W (the same arithmetic as LAYERCAST), and their lse, logprob and
- *   argmax are replaced; margin keeps the bf16-path value that triggered it;
+ *   margin < margin_threshold are recomputed from the f32 h at FP32 accuracy:
+ *   h is split exactly into three bf16 parts (h = p0 + p1 + p2; 8+8+8
+ *   significant bits), each product with W is exact, the three products are
+ *   accumulated in fp32 on the tensor cores and added as (z0 + z1) + z2.
+ *   Their lse, logprob and argmax are replaced; margin keeps the bf16-path
+ *   value that triggered the recompute;
  *   recomputed[b] = 1.  margin_threshold <= 0 disables it.  In LAYERCAST the
  *   main pass is already fp32 and recomputed[b] = 0.
  * Outputs (device, [B]): logprob f32, lse f32, argmax int32, margin f32,
@@ -203,7 +206,7 @@ int bi_lmhead_logprob(const float* h, const void* W, const int32_t* target, int 
  *    streams, or host threads racing) corrupt each other's scratch.  Issue
  *    them in one stream order.  Nothing in the array needs to start zeroed.
  *  - It allocates nothing: no cudaMalloc/cudaFree, no allocating library call. */
-#define BI_NOALLOC_SCRATCH_BYTES (40 << 20)
+#define BI_NOALLOC_SCRATCH_BYTES (80 << 20)
 int bi_lmhead_logprob_noalloc(const float* h, const void* W, const int32_t* target, int B, int H, int V,
                               float margin_threshold, int mode, float* logprob, float* lse, int32_t* argmax,
                               float* margin, uint8_t* recomputed, float* logits, void* stream);

@@ -48,11 +48,13 @@ struct AttnArgs {
 __host__ __device__ inline int att_ninner(int d, int f32) { return d * (f32 ? 4 : 2) / 128; }
 
 constexpr int ATT_SUB = 64;  // keys per TMA sub-tile
-constexpr int ATT_RING = 2;  // sub-tile buffers
+// sub-tile ring depth: deeper for the small pair groups of decode, whose
+// CTAs are short and latency-bound; 2 for the large groups of prefill.
+__host__ __device__ constexpr int att_ring(int np) { return np <= 8 ? 4 : 2; }
 
 __host__ __device__ inline size_t att_sub_bytes(int d, int f32) { return (size_t)ATT_SUB * d * (f32 ? 4 : 2); }
 __host__ __device__ inline size_t att_smem_bytes(int np, int d, int f32) {
-  return ATT_RING * att_sub_bytes(d, f32) + (size_t)np * d * 4 + 2 * (size_t)np * ATT_CHUNK * 4 + 1024;
+  return att_ring(np) * att_sub_bytes(d, f32) + (size_t)np * d * 4 + 2 * (size_t)np * ATT_CHUNK * 4 + 1024;
 }
 
 // Grid: (block, chunk, kv head).  The chunk's K rows, then its V rows, stream
@@ -70,6 +72,7 @@ __global__ void __launch_bounds__(ATT_THREADS)
   pdl_wait();
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
+  constexpr int ATT_RING = att_ring(NP);
   __shared__ __align__(8) uint64_t bar[ATT_RING];
   __shared__ float m_s[NP], l_s[NP];
   __shared__ int live_s[NP];
@@ -85,7 +88,6 @@ __global__ void __launch_bounds__(ATT_THREADS)
   const int nsub = (nvalid + ATT_SUB - 1) / ATT_SUB;
   const int ninner = att_ninner(a.d, a.f32);
   const int esz = a.f32 ? 4 : 2;
-  const int boxe = 128 / esz;
   const size_t sub_bytes = att_sub_bytes(a.d, a.f32);
   float* qs = reinterpret_cast<float*>(smem + ATT_RING * sub_bytes);
   float* S = qs + NP * a.d;       // scores [NP][256]
@@ -109,8 +111,8 @@ __global__ void __launch_bounds__(ATT_THREADS)
     uint8_t* buf = smem + (L % ATT_RING) * sub_bytes;
     uint64_t* br = &bar[L % ATT_RING];
     mbar_arrive_expect_tx(br, (uint32_t)(ninner * ATT_SUB * 128));
-    for (int ib = 0; ib < ninner; ++ib)
-      tma_load_2d(buf + ib * (ATT_SUB * 128), isv ? &tmV : &tmK, ib * boxe, row_base + st * ATT_SUB, br);
+    // one 3-D box {128 bytes, 64 rows, ninner}: lands as ninner swizzled [64][128 B] slabs
+    tma_load_3d(buf, isv ? &tmV : &tmK, 0, row_base + st * ATT_SUB, 0, br);
   };
   const int ngroups = (npairs + NP - 1) / NP;
   const int total_loads = ngroups * nloads;

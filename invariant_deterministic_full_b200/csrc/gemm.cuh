@@ -66,7 +66,7 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(160, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                      void* __restrict__ y, int ldy, int y_f32, int M, int N, int K, int m_tiles, int n_groups,
-                     int splits, float* __restrict__ partial) {
+                     int splits, float* __restrict__ partial, const int* __restrict__ mcount, int mmult) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::STAGES];
@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(160, 1)
       // Prologue: the first ring stages of weight tiles depend on no earlier
       // kernel, so they are requested before waiting for the previous launch.
       int pre = 0;
-      if ((int)blockIdx.x < n_items) {
+      if (mcount == nullptr && (int)blockIdx.x < n_items) {
         const int item = blockIdx.x;
         const int g = (item / m_tiles) % n_groups;
         const int ks0 = (item / (m_tiles * n_groups)) * ks_per_split;
@@ -109,11 +109,14 @@ __global__ void __launch_bounds__(160, 1)
       }
       pdl_wait();
       pdl_trigger();
+      // rows beyond a device-side count (selective recompute) are not computed
+      const int Me = mcount ? min(M, *mcount * mmult) : M;
       int stage = 0;
       uint32_t phase = 0;
       bool first = true;
       for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
         const int mt = item % m_tiles;
+        if (mt * GEMM_BM >= Me) continue;
         const int g = (item / m_tiles) % n_groups;
         const int sp = item / (m_tiles * n_groups);
         const int ks0 = sp * ks_per_split;
@@ -146,13 +149,15 @@ __global__ void __launch_bounds__(160, 1)
   const int g8 = lane >> 2, t4 = lane & 3;
   int stage = 0;
   uint32_t phase = 0;
+  const int Me = mcount ? min(M, *mcount * mmult) : M;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const int mt = item % m_tiles;
+    if (mt * GEMM_BM >= Me) continue;
     const int g = (item / m_tiles) % n_groups;
     const int sp = item / (m_tiles * n_groups);
     const int ks0 = sp * ks_per_split;
     const int ks1 = min(kstages_total, ks0 + ks_per_split);
-    const bool active = mt * GEMM_BM + tok0 < M;
+    const bool active = mt * GEMM_BM + tok0 < Me;
     // KS interleaved accumulator sets: k16 step s (counted from k = 0) adds into
     // set s % KS; the sets are combined in a fixed tree after the K loop.
     float accs[C::KS][2][C::NT][4];
@@ -231,7 +236,7 @@ __global__ void __launch_bounds__(160, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int m = mt * GEMM_BM + tok0 + nt * 8 + 2 * t4 + (i & 1);
-        if (m >= M) continue;
+        if (m >= Me) continue;
         const int rin = g8 + (i >> 1) * 8;
         if (splits > 1) {  // FAST variant: raw fp32 partial of this split
 #pragma unroll
@@ -420,7 +425,7 @@ size_t gemm_ws_bytes(int M, int N, int K, int mode, int variant) {
 
 template <int BN, int EPI>
 static int launch_gemm_bf16_t(const CUtensorMap& tw, const CUtensorMap& tx, void* y, int ldy, int y_f32, int M, int N,
-                              int K, int splits, float* partial, cudaStream_t st) {
+                              int K, int splits, float* partial, const int* mcount, int mmult, cudaStream_t st) {
   using C = GemmCfg<BN>;
   static bool attr_done = false;  // per instantiation; set once per process
   if (!attr_done) {
@@ -432,12 +437,13 @@ static int launch_gemm_bf16_t(const CUtensorMap& tw, const CUtensorMap& tx, void
   const int items = splits * n_groups * m_tiles;
   const int grid = items < num_sms() ? items : num_sms();
   BI_TRY(launch(gemm_bf16_kernel<BN, EPI>, dim3(grid), dim3(160), C::SMEM, st, tw, tx, y, ldy, y_f32, M, N, K, m_tiles, n_groups, splits,
-                                                         partial));
+                                                         partial, mcount, mmult));
   return BI_OK;
 }
 
+// mcount (optional, device int): only rows < *mcount * mmult of x are computed.
 int gemm_bf16(const void* x, int ldx, const void* w, void* y, int ldy, int y_f32, int M, int N, int K, int epi,
-              int variant, void* ws, size_t ws_bytes, cudaStream_t st) {
+              int variant, void* ws, size_t ws_bytes, cudaStream_t st, const int* mcount = nullptr, int mmult = 1) {
   const int bn = gemm_pick_bn(N);
   const int kbs = gemm_kbs(bn);
   // 3-D views {64 k, rows, k-block}: the k-block dimension (stride 128 B) is the
@@ -465,9 +471,9 @@ int gemm_bf16(const void* x, int ldx, const void* w, void* y, int ldy, int y_f32
 #define BI_GEMM_CASE(BNV)                                                                                          \
   if (bn == BNV) {                                                                                                 \
     if (epi == BI_EPI_SWIGLU)                                                                                      \
-      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_SWIGLU>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, st)));     \
+      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_SWIGLU>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, mcount, mmult, st)));     \
     else                                                                                                           \
-      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_NONE>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, st)));       \
+      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_NONE>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, mcount, mmult, st)));       \
   }
   BI_GEMM_CASE(32)
   BI_GEMM_CASE(64)

@@ -140,8 +140,14 @@ static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const
   const uint64_t rows = (uint64_t)kv->n_slots * kv->n_layers * Hkv * kv->capacity;
   CUtensorMap tk, tv;
   const CUtensorMapDataType dt = f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  BI_TRY(encode_tmap_2d(&tk, dt, esz, kv->k, d, rows, (uint64_t)d * esz, 128 / esz, 64, CU_TENSOR_MAP_SWIZZLE_128B));
-  BI_TRY(encode_tmap_2d(&tv, dt, esz, kv->v, d, rows, (uint64_t)d * esz, 128 / esz, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+  // 3-D views {128-byte piece of a row, row, piece}: a 64-row box of all pieces is
+  // one TMA operation landing as [piece][64 rows][128 B] swizzled slabs.
+  const uint32_t ninner = (uint32_t)(d * esz / 128);
+  const uint64_t kdims[3] = {(uint64_t)(128 / esz), rows, ninner};
+  const uint64_t kstr[2] = {(uint64_t)d * esz, 128};
+  const uint32_t kbox[3] = {(uint32_t)(128 / esz), 64, ninner};
+  BI_TRY(encode_tmap_3d(&tk, dt, kv->k, kdims, kstr, kbox, CU_TENSOR_MAP_SWIZZLE_128B));
+  BI_TRY(encode_tmap_3d(&tv, dt, kv->v, kdims, kstr, kbox, CU_TENSOR_MAP_SWIZZLE_128B));
 
   BI_TRY(attn_set_smem_attrs());
   float* part = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
@@ -191,8 +197,8 @@ struct LmWs {
   uint8_t* flag;
   int32_t* list;
   int* count;
-  float* hc;
-  float* logits_c;
+  uint16_t* hc3;   // [3B][H] exact bf16 parts of the flagged rows
+  float* logits_c;  // [3B][V] partial logits of the parts
 };
 static LmWs lm_carve(Carver& cv, int B, int H, int V, int mode, bool own_logits) {
   const int nch = (V + LM_CHUNK - 1) / LM_CHUNK;
@@ -204,8 +210,8 @@ static LmWs lm_carve(Carver& cv, int B, int H, int V, int mode, bool own_logits)
   w.list = cv.take<int32_t>(B);
   w.count = cv.take<int>(1);
   if (mode == BI_MODE_BF16) {
-    w.hc = cv.take<float>((size_t)B * H);
-    w.logits_c = cv.take<float>((size_t)B * V);
+    w.hc3 = cv.take<uint16_t>((size_t)3 * B * H);
+    w.logits_c = cv.take<float>((size_t)3 * B * V);
   }
   return w;
 }
@@ -236,14 +242,20 @@ static int lmhead_run(const float* h, const void* W, const int32_t* target, int 
   } else {
     BI_TRY(gemm_f32(h, H, W, z, V, 1, B, V, H, BI_EPI_NONE, nullptr, st));
   }
-  BI_TRY(launch(lm_partial_kernel, dim3(dim3(nch, B)), dim3(LM_CHUNK), 0, st, z, V, V, target, nullptr, nullptr, w.part, nch));
+  BI_TRY(launch(lm_partial_kernel, dim3(dim3(nch, B)), dim3(LM_CHUNK), 0, st, z, V, V, target, nullptr, nullptr, w.part, nch,
+                1));
   const float th = mode == BI_MODE_BF16 ? thresh : 0.f;
   BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, nullptr, nullptr, target, th, 0, logprob, lse,
                                                         argmax, margin, recomputed, w.flag));
   if (mode == BI_MODE_BF16 && th > 0.f) {
-    BI_TRY(launch(lm_compact_kernel, dim3(B), dim3(256), 0, st, w.flag, B, h, H, w.list, w.count, w.hc));
-    BI_TRY(gemm_f32(w.hc, H, W, w.logits_c, V, 1, B, V, H, BI_EPI_NONE, w.count, st));
-    BI_TRY(launch(lm_partial_kernel, dim3(dim3(nch, B)), dim3(LM_CHUNK), 0, st, w.logits_c, V, V, target, w.list, w.count, w.part, nch));
+    // FP32 recompute of the flagged rows: h = p0 + p1 + p2 exactly (bf16 parts), so
+    // h.W^T = ((p0.W^T + p1.W^T) + p2.W^T) with exact products and fp32 accumulation
+    // on the tensor cores; one pass over W serves every flagged row.
+    BI_TRY(launch(lm_compact_kernel, dim3(B), dim3(256), 0, st, w.flag, B, h, H, w.list, w.count, w.hc3));
+    BI_TRY(gemm_bf16(w.hc3, H, W, w.logits_c, V, 1, 3 * B, V, H, BI_EPI_NONE, BI_VARIANT_INVARIANT, nullptr, 0, st,
+                     w.count, 3));
+    BI_TRY(launch(lm_partial_kernel, dim3(dim3(nch, B)), dim3(LM_CHUNK), 0, st, w.logits_c, V, V, target, w.list,
+                  w.count, w.part, nch, 3));
     BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, w.count, w.list, target, th, 1, logprob,
                                                           lse, argmax, margin, recomputed, nullptr));
   }

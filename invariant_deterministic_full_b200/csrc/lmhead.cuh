@@ -48,10 +48,12 @@ __device__ __forceinline__ void lm_top2_warp(float& v1, int& i1, float& v2, int&
 // logits row r; rows >= *count (when count != nullptr) are skipped.
 // target: per-row target id (nullptr: none); rows_map maps grid row -> target
 // row (nullptr: identity).
+// parts == 3: the logit of row r is (z[3r] + z[3r+1]) + z[3r+2], the three
+// partial products of the exact bf16 split of an f32 hidden row.
 __global__ void __launch_bounds__(LM_CHUNK)
     lm_partial_kernel(const float* __restrict__ logits, size_t ldz, int V, const int32_t* __restrict__ target,
                       const int32_t* __restrict__ rows_map, const int* __restrict__ count, LmPart* __restrict__ part,
-                      int n_chunks) {
+                      int n_chunks, int parts) {
   pdl_wait();
   pdl_trigger();
   const int c = blockIdx.x, r = blockIdx.y;
@@ -59,7 +61,14 @@ __global__ void __launch_bounds__(LM_CHUNK)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int v = c * LM_CHUNK + tid;
   const bool ok = v < V;
-  const float z = ok ? logits[(size_t)r * ldz + v] : -INFINITY;
+  float z = -INFINITY;
+  if (ok) {
+    if (parts == 3)
+      z = (logits[(size_t)(3 * r) * ldz + v] + logits[(size_t)(3 * r + 1) * ldz + v]) +
+          logits[(size_t)(3 * r + 2) * ldz + v];
+    else
+      z = logits[(size_t)r * ldz + v];
+  }
   __shared__ float wm[LM_CHUNK / 32], ws[LM_CHUNK / 32], wv1[LM_CHUNK / 32], wv2[LM_CHUNK / 32];
   __shared__ int wi1[LM_CHUNK / 32], wi2[LM_CHUNK / 32];
   __shared__ float zt_s;
@@ -162,10 +171,13 @@ __global__ void lm_merge_kernel(const LmPart* __restrict__ part, int n_chunks, i
 }
 
 // Ascending compaction of the flagged rows: list[k] = k-th flagged row, and
-// the f32 hidden rows gathered in that order.  CTA b handles row b: its rank
-// is the number of flagged rows before it; CTA 0 also writes the count.
+// that row's f32 hidden vector split exactly into three bf16 parts
+// h = p0 + p1 + p2 (p0 = bf16(h), p1 = bf16(h - p0), p2 = h - p0 - p1; 8 + 8 + 8
+// significant bits cover the 24 of an f32), stored as rows 3k, 3k+1, 3k+2 of
+// hc3.  CTA b handles row b: its rank is the number of flagged rows before it;
+// CTA 0 also writes the count.
 __global__ void lm_compact_kernel(const uint8_t* __restrict__ flag, int B, const float* __restrict__ h, int H,
-                                  int32_t* __restrict__ list, int* __restrict__ count, float* __restrict__ hc) {
+                                  int32_t* __restrict__ list, int* __restrict__ count, uint16_t* __restrict__ hc3) {
   pdl_wait();
   pdl_trigger();
   const int b = blockIdx.x;
@@ -192,7 +204,16 @@ __global__ void lm_compact_kernel(const uint8_t* __restrict__ flag, int B, const
   if (!flag[b]) return;
   const int k = rank_s;
   if (threadIdx.x == 0) list[k] = b;
-  for (int i = threadIdx.x; i < H; i += blockDim.x) hc[(size_t)k * H + i] = h[(size_t)b * H + i];
+  for (int i = threadIdx.x; i < H; i += blockDim.x) {
+    const float v = h[(size_t)b * H + i];
+    const uint16_t p0 = f32_to_bf16_bits(v);
+    const float r0 = v - bf16_bits_to_f32(p0);  // exact
+    const uint16_t p1 = f32_to_bf16_bits(r0);
+    const float r1 = r0 - bf16_bits_to_f32(p1);  // exact, at most 8 significant bits
+    hc3[(size_t)(3 * k) * H + i] = p0;
+    hc3[(size_t)(3 * k + 1) * H + i] = p1;
+    hc3[(size_t)(3 * k + 2) * H + i] = f32_to_bf16_bits(r1);
+  }
 }
 
 // h (f32) -> bf16 (round to nearest even), the main-pass LM-head input.
