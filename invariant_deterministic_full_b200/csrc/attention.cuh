@@ -300,6 +300,257 @@ __global__ void __launch_bounds__(ATT_THREADS)
   }
 }
 
+// ---------------------------------------------------------------------------
+// bf16 mode on tensor cores (mma.sync m16n8k16, fp32 accumulate).  The same
+// chunk grid, masks, max and lane-strided denominator as above; the two
+// contractions are tensor-core products:
+//   * score(p, j) = scale * (q_p . k_j): 8 ascending k16 steps over the head
+//     dimension into one fp32 accumulator (bf16 x bf16 products are exact);
+//   * numerator(p, e) = sum_j P(p, j) v_j[e]: the fp32 probabilities are split
+//     exactly into three bf16 parts P = P0 + P1 + P2 (8+8+8 significant bits),
+//     each part's product with V accumulated over ascending k16 steps of keys
+//     in its own fp32 accumulator, and the three added as (a0 + a1) + a2.
+// Row p of an MMA tile depends only on row p of its A operand, so the result
+// of a (query, head) pair does not depend on how many pairs share the tile --
+// decode (one 16-row tile) and prefill (32-row tiles) give the same bits.
+// Keys past a query have P = 0 and add exact zeros; V rows past the last
+// valid key are zeroed in shared memory before use.
+constexpr int ATC_SST = 264;  // padded row stride of the fp32 score tile
+
+__host__ __device__ inline size_t atc_smem_bytes(int pt, int ring) {
+  const size_t rows = 16 * pt;
+  return (size_t)ring * 16384           // K/V sub-tiles: [2 halves][64 keys][128 B]
+         + rows * 256                   // q tile: [2 halves][rows][128 B]
+         + rows * ATC_SST * 4           // scores
+         + 3 * 4 * rows * 128           // probability parts: [3][4 key blocks][rows][128 B]
+         + 1024;
+}
+
+template <int PT, int RING>
+__global__ void __launch_bounds__(ATT_THREADS)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                   const __grid_constant__ AttnPlan plan, const AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int NR = 16 * PT;  // pair rows per group
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar[RING];
+  __shared__ float m_s[NR], l_s[NR];
+  __shared__ int live_s[NR];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int b = blockIdx.x, c = blockIdx.y, hk = blockIdx.z;
+  if (b >= plan.n) return;
+  const int t0 = plan.blk[b].x, nq = plan.blk[b].y;
+  const int s = a.slot[t0];
+  const int pmax = a.pos[t0 + nq - 1];
+  const int key0 = c * a.chunk;
+  if (key0 > pmax) return;
+  const int nvalid = min(a.chunk, pmax - key0 + 1);
+  const int nsub = (nvalid + ATT_SUB - 1) / ATT_SUB;
+  const int npairs = nq * a.G;
+  const int row_base = ((s * a.n_layers + a.layer) * a.Hkv + hk) * a.cap + key0;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g8 = lane >> 2, t4 = lane & 3;
+  constexpr uint32_t SUB = 16384;
+  uint8_t* qt = smem + RING * SUB;                         // [2][NR][128 B]
+  float* S = reinterpret_cast<float*>(qt + NR * 256);      // [NR][ATC_SST]
+  uint8_t* Pp = reinterpret_cast<uint8_t*>(S + NR * ATC_SST);  // [3][4][NR][128 B]
+  const uint32_t qt_s = smem_u32(qt), pp_s = smem_u32(Pp);
+  const int nloads = 2 * nsub;
+
+  if (tid == 0) {
+    for (int r = 0; r < RING; ++r) mbar_init(&bar[r], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](int L) {
+    const int li = L % nloads;
+    const bool isv = li >= nsub;
+    const int st = isv ? li - nsub : li;
+    mbar_arrive_expect_tx(&bar[L % RING], SUB);
+    tma_load_3d(smem + (L % RING) * SUB, isv ? &tmV : &tmK, 0, row_base + st * ATT_SUB, 0, &bar[L % RING]);
+  };
+  const int ngroups = (npairs + NR - 1) / NR;
+  const int total_loads = ngroups * nloads;
+  if (tid == 0)
+    for (int L = 0; L < RING && L < total_loads; ++L) issue(L);
+  int L = 0;
+  auto consume_wait = [&]() -> bool { return mbar_wait(&bar[L % RING], (uint32_t)((L / RING) & 1)); };
+  auto release = [&]() {
+    __syncthreads();
+    if (tid == 0 && L + RING < total_loads) issue(L + RING);
+    ++L;
+  };
+
+  for (int pg0 = 0; pg0 < npairs; pg0 += NR) {
+    const int gp = min(NR, npairs - pg0);
+    // q tile (bf16, 128-byte swizzle per half); padded rows are zero
+    for (int idx = tid; idx < NR * 16; idx += ATT_THREADS) {  // 16 chunks of 8 elements per row
+      const int row = idx >> 4, ch = idx & 15;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (row < gp) {
+        const int p = pg0 + row;
+        const int i = p / a.G, g = p % a.G;
+        v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.q) +
+                                            (size_t)(t0 + i) * a.Hq * 128 + (hk * a.G + g) * 128 + ch * 8);
+      }
+      const int half = ch >> 3, cc = ch & 7;
+      *reinterpret_cast<uint4*>(qt + half * (NR * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
+    }
+    __syncthreads();
+    // q fragments stay in registers for the whole chunk
+    uint32_t qa[PT][8][4];
+#pragma unroll
+    for (int mt = 0; mt < PT; ++mt)
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int half = kk >> 2, ch = 2 * (kk & 3) + (lane >> 4);
+        ldsm_x4(qt_s + half * (NR * 128) + row * 128 + ((ch ^ (row & 7)) << 4), qa[mt][kk][0], qa[mt][kk][1],
+                qa[mt][kk][2], qa[mt][kk][3]);
+      }
+
+    // ---- scores: warp w owns keys 8w..8w+7 of each 64-key sub-tile
+    for (int st = 0; st < nsub; ++st) {
+      if (!consume_wait()) return;
+      const uint32_t kb = smem_u32(smem + (L % RING) * SUB);
+      float acc[PT][4];
+#pragma unroll
+      for (int mt = 0; mt < PT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const int krow = warp * 8 + (lane & 7);
+        const int half = kk >> 2, ch = 2 * (kk & 3) + ((lane >> 3) & 1);
+        uint32_t b0, b1;
+        ldsm_x2(kb + half * 8192 + krow * 128 + ((ch ^ (krow & 7)) << 4), b0, b1);
+#pragma unroll
+        for (int mt = 0; mt < PT; ++mt) mma_bf16_16816(acc[mt], qa[mt][kk], b0, b1);
+      }
+#pragma unroll
+      for (int mt = 0; mt < PT; ++mt) {
+        const int j = st * ATT_SUB + warp * 8 + 2 * t4;
+        float* r0 = S + (mt * 16 + g8) * ATC_SST + j;
+        float* r1 = S + (mt * 16 + g8 + 8) * ATC_SST + j;
+        *reinterpret_cast<float2*>(r0) = make_float2(acc[mt][0] * a.scale, acc[mt][1] * a.scale);
+        *reinterpret_cast<float2*>(r1) = make_float2(acc[mt][2] * a.scale, acc[mt][3] * a.scale);
+      }
+      release();
+    }
+
+    // ---- softmax per pair row: max (exact), exp, l = lane-strided ascending sums then butterfly;
+    // the probabilities go out as three exact bf16 parts (zeros past the valid keys)
+    for (int pl = warp; pl < NR; pl += ATT_THREADS / 32) {
+      float mx = -INFINITY, sum = 0.f;
+      int lim = -1;
+      if (pl < gp) {
+        const int i = (pg0 + pl) / a.G;
+        lim = a.pos[t0 + i] - key0;
+#pragma unroll
+        for (int k = 0; k < ATT_CHUNK / 32; ++k) {
+          const int j = lane + 32 * k;
+          if (j <= lim && j < nvalid) mx = fmaxf(mx, S[pl * ATC_SST + j]);
+        }
+        mx = warp_max(mx);
+      }
+#pragma unroll
+      for (int k = 0; k < ATT_CHUNK / 32; ++k) {
+        const int j = lane + 32 * k;
+        float pj = 0.f;
+        if (pl < gp && j <= lim && j < nvalid) pj = expf(S[pl * ATC_SST + j] - mx);
+        sum += pj;
+        const uint16_t p0 = f32_to_bf16_bits(pj);
+        const float r0 = pj - bf16_bits_to_f32(p0);
+        const uint16_t p1 = f32_to_bf16_bits(r0);
+        const uint16_t p2 = f32_to_bf16_bits(r0 - bf16_bits_to_f32(p1));
+        const int kbk = j >> 6, ch = (j & 63) >> 3;
+        const int off = kbk * (NR * 128) + pl * 128 + ((ch ^ (pl & 7)) << 4) + (j & 7) * 2;
+        *reinterpret_cast<uint16_t*>(Pp + 0 * (4 * NR * 128) + off) = p0;
+        *reinterpret_cast<uint16_t*>(Pp + 1 * (4 * NR * 128) + off) = p1;
+        *reinterpret_cast<uint16_t*>(Pp + 2 * (4 * NR * 128) + off) = p2;
+      }
+      if (pl < gp) {
+        sum = warp_sum_fixed(sum);
+        if (lane == 0) {
+          m_s[pl] = mx;
+          l_s[pl] = sum;
+          live_s[pl] = lim >= 0;
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- PV: warp w owns head elements 16w..16w+15 (two n8 tiles)
+    float pacc[3][PT][2][4];
+#pragma unroll
+    for (int q = 0; q < 3; ++q)
+#pragma unroll
+      for (int mt = 0; mt < PT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) pacc[q][mt][nt][0] = pacc[q][mt][nt][1] = pacc[q][mt][nt][2] = pacc[q][mt][nt][3] = 0.f;
+    for (int st = 0; st < nsub; ++st) {
+      if (!consume_wait()) return;
+      uint8_t* vbuf = smem + (L % RING) * SUB;
+      const int vrows = nvalid - st * ATT_SUB;  // valid rows of this sub-tile
+      if (vrows < ATT_SUB) {  // zero the rows past the last valid key
+        for (int idx = tid; idx < (ATT_SUB - vrows) * 16; idx += ATT_THREADS) {
+          const int r = vrows + (idx >> 4), ch = idx & 15;
+          *reinterpret_cast<uint4*>(vbuf + (ch >> 3) * 8192 + r * 128 + ((ch & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncthreads();
+      }
+      const uint32_t vb = smem_u32(vbuf);
+      const int nk16 = min(4, (vrows + 15) / 16);
+      for (int kk = 0; kk < nk16; ++kk) {
+        // B fragments: V rows = keys 16kk..16kk+15 of the sub-tile, elements 16w..16w+15
+        uint32_t vb0[2], vb1[2];
+        {
+          const int krow = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int e0 = warp * 16 + (lane >> 4) * 8;
+          const int half = e0 >> 6, ch = (e0 & 63) >> 3;
+          ldsm_x4_trans(vb + half * 8192 + krow * 128 + ((ch ^ (krow & 7)) << 4), vb0[0], vb1[0], vb0[1], vb1[1]);
+        }
+        const int kblk = st;  // 64 keys per probability block
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
+#pragma unroll
+          for (int mt = 0; mt < PT; ++mt) {
+            uint32_t pa[4];
+            const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            const int ch = 2 * kk + (lane >> 4);
+            ldsm_x4(pp_s + q * (4 * NR * 128) + kblk * (NR * 128) + row * 128 + ((ch ^ (row & 7)) << 4), pa[0], pa[1],
+                    pa[2], pa[3]);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) mma_bf16_16816(pacc[q][mt][nt], pa, vb0[nt], vb1[nt]);
+          }
+        }
+      }
+      release();
+    }
+#pragma unroll
+    for (int mt = 0; mt < PT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int pl = mt * 16 + g8 + hr * 8;
+          if (pl >= gp || !live_s[pl]) continue;
+          const int p = pg0 + pl;
+          const int i = p / a.G, g = p % a.G;
+          const int hq = hk * a.G + g;
+          float* rec = a.part + (((size_t)(t0 + i - a.t_base) * a.Hq + hq) * a.max_chunks + c) * (128 + 4);
+          const int e = warp * 16 + nt * 8 + 2 * t4;
+          const float o0 = (pacc[0][mt][nt][2 * hr] + pacc[1][mt][nt][2 * hr]) + pacc[2][mt][nt][2 * hr];
+          const float o1 = (pacc[0][mt][nt][2 * hr + 1] + pacc[1][mt][nt][2 * hr + 1]) + pacc[2][mt][nt][2 * hr + 1];
+          *reinterpret_cast<float2*>(rec + e) = make_float2(o0, o1);
+          if (e == 0) {
+            rec[128] = m_s[pl];
+            rec[129] = l_s[pl];
+          }
+        }
+    __syncthreads();  // the next group overwrites q, S, the probability parts and the statistics
+  }
+}
+
 // One warp per (token, q head): fixed ascending merge of the chunk partials.
 __global__ void attn_merge_kernel(const float* __restrict__ part, const int32_t* __restrict__ pos, void* __restrict__ out,
                                   int t_base, int T, int Hq, int d, int chunk, int max_chunks, int f32) {

@@ -78,13 +78,31 @@ static int attn_set_smem_attrs() {
                                      (int)att_smem_bytes(16, 128, 1)));
   BI_CHECK_CUDA(cudaFuncSetAttribute(attn_partial_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)att_smem_bytes(32, 128, 1)));
+  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<1, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)atc_smem_bytes(1, 4)));
+  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)atc_smem_bytes(2, 4)));
+  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)atc_smem_bytes(2, 2)));
   done = true;
   return BI_OK;
 }
 
+// np: pairs per group of the CUDA-core kernel (LayerCast, or head_dim 64); the
+// bf16 head_dim-128 path runs on tensor cores with 16-row pair tiles.
 static int attn_launch(int np, const CUtensorMap& tk, const CUtensorMap& tv, const AttnPlan& plan, const AttnArgs& a,
                        cudaStream_t st) {
   const dim3 grid(plan.n, a.max_chunks, a.Hkv);
+  if (!a.f32 && a.d == 128) {
+    const bool single = np <= 16;  // decode blocks: one token, G pairs
+    if (single && a.G <= 16)
+      BI_TRY(launch(attn_tc_kernel<1, 4>, grid, dim3(ATT_THREADS), atc_smem_bytes(1, 4), st, tk, tv, plan, a));
+    else if (single)
+      BI_TRY(launch(attn_tc_kernel<2, 4>, grid, dim3(ATT_THREADS), atc_smem_bytes(2, 4), st, tk, tv, plan, a));
+    else
+      BI_TRY(launch(attn_tc_kernel<2, 2>, grid, dim3(ATT_THREADS), atc_smem_bytes(2, 2), st, tk, tv, plan, a));
+    return BI_OK;
+  }
   const size_t smem = att_smem_bytes(np, a.d, a.f32);
   switch (np) {
     case 4: BI_TRY(launch(attn_partial_kernel<4>, dim3(grid), dim3(ATT_THREADS), smem, st, tk, tv, plan, a)); break;
