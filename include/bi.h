@@ -134,9 +134,12 @@ int bi_rope_table_fill(float* table, int max_pos, int head_dim, double theta, vo
 /* Rotary embedding + KV append for T tokens after the QKV projection.
  * qkv: f32 [T][(Hq + 2*Hkv) * d] (q heads, then k heads, then v heads).
  * q_out: [T][Hq*d] activation dtype; k and v rows are written to the cache at
- * (slot[t], layer, head, pos[t]).  slot/pos: device int32 [T]. */
+ * (slot[t], layer, head, pos[t]).  slot/pos: device int32 [T].
+ * qk_paired != 0: each q and k head of qkv is in the paired row order of
+ * bi_weights.w_qkv (below); q_out and the cache are always in natural order. */
 int bi_rope_kv_append(const float* qkv, const float* rope, int rope_max_pos, void* q_out, const bi_kv_layout* kv,
-                      int layer, const int32_t* slot, const int32_t* pos, int T, int Hq, int mode, void* stream);
+                      int layer, const int32_t* slot, const int32_t* pos, int T, int Hq, int qk_paired, int mode,
+                      void* stream);
 
 /* ------------------------------------------------------------- Attention
  * For each token t and q head h (kv head h / (Hq/Hkv)): causal softmax
@@ -232,7 +235,11 @@ typedef struct {
   const void* final_norm; /* bf16 [H] */
   const void* attn_norm;  /* bf16 [L][H] */
   const void* ffn_norm;   /* bf16 [L][H] */
-  const void* w_qkv;      /* bf16 [L][(Hq + 2 Hkv) d][H]: q rows, k rows, v rows */
+  const void* w_qkv;      /* bf16 [L][(Hq + 2 Hkv) d][H]: q rows, k rows, v rows; each q and k head in
+                             the PAIRED row order: in every 32-row block b of a head, rows 0..15 are
+                             elements 16b..16b+15 and rows 16..31 their rotate-half partners
+                             d/2+16b..d/2+16b+15 (so RoPE can run in the projection's epilogue);
+                             v heads in natural order */
   const void* w_o;        /* bf16 [L][H][Hq d] */
   const void* w_gu;       /* bf16 [L][2F][H], gate/up interleaved by BI_GU_INTERLEAVE */
   const void* w_down;     /* bf16 [L][H][F] */
@@ -282,7 +289,9 @@ int bi_greedy_advance(const int32_t* argmax, int32_t* ids, int32_t* pos, int B, 
  *   dst[dst_row(i / cols) * cols + i % cols], where
  *   dst_row(r) = r                                   if interleave == 0,
  *   dst_row(r) = (r / g) * 2g + phase * g + r % g    if interleave == g > 0
- * (phase 0 = gate rows, 1 = up rows of a BI_GU_INTERLEAVE fused weight).
+ * (phase 0 = gate rows, 1 = up rows of a BI_GU_INTERLEAVE fused weight),
+ *   dst_row(r) = (r / d) * d + paired(r % d)         if interleave == -d
+ * (d = 64 or 128: the paired row order of q/k heads in bi_weights.w_qkv).
  * Not part of the method: it only produces inputs without a host round trip. */
 int bi_synth_fill_bf16(uint16_t* dst, int64_t rows, int64_t cols, uint64_t key, double std, int interleave,
                        int phase, void* stream);

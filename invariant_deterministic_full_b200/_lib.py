@@ -73,7 +73,7 @@ SIGNATURES = {
     "bi_gemm": (I, [P, I, P, P, I, I, I, I, I, I, I, I, P, SZ, P]),
     "bi_rmsnorm": (I, [P, P, P, P, P, P, I, I, F, I, P]),
     "bi_rope_table_fill": (I, [P, I, I, D, P]),
-    "bi_rope_kv_append": (I, [P, P, I, P, ctypes.POINTER(KvLayout), I, P, P, I, I, I, P]),
+    "bi_rope_kv_append": (I, [P, P, I, P, ctypes.POINTER(KvLayout), I, P, P, I, I, I, I, P]),
     "bi_attention_workspace_size": (SZ, [I, I, I, I]),
     "bi_attention": (I, [P, ctypes.POINTER(KvLayout), I, P, P, P, P, P, I, I, F, I, I, P, SZ, P]),
     "bi_lmhead_workspace_size": (SZ, [I, I, I, I]),

@@ -60,13 +60,34 @@ struct GemmCfg {
   static constexpr int KS = NT >= 4 ? 1 : 4 / NT;
 };
 
+// Fused RoPE + KV-append epilogue of the QKV projection (bf16 mode).  The
+// fused QKV weight stores each q/k head in the "paired" row order: in every
+// 32-row block b of a head, rows 0..15 are elements 16b..16b+15 and rows
+// 16..31 their rotate-half partners d/2 + 16b .. d/2 + 16b + 15 (v rows keep
+// their natural order).  A warp's two 16-row tiles then hold both members of
+// each rotation pair for its tokens, so the epilogue rotates in registers
+// (x' = x c - y s, y' = y c + x s, (c, s) from the f32 table at the token's
+// position), writes q in the activation dtype and appends k and v to the cache.
+constexpr int EPI_ROPE = 2;
+struct RopeEpi {
+  const float* table;
+  int table_max_pos;
+  void* q_out;
+  void* kc;
+  void* vc;
+  const int32_t* slot;
+  const int32_t* pos;
+  int Hq, Hkv, d, layer, n_layers, n_slots, cap;
+};
+
 // Work item -> (split, row group, token tile).  Splits > 1 only in the
 // non-invariant FAST variant, which then writes fp32 partials per split.
 template <int BN, int EPI>
 __global__ void __launch_bounds__(160, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                      void* __restrict__ y, int ldy, int y_f32, int M, int N, int K, int m_tiles, int n_groups,
-                     int splits, float* __restrict__ partial, const int* __restrict__ mcount, int mmult) {
+                     int splits, float* __restrict__ partial, const int* __restrict__ mcount, int mmult,
+                     const RopeEpi re) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::STAGES];
@@ -245,6 +266,37 @@ __global__ void __launch_bounds__(160, 1)
         } else if constexpr (EPI == BI_EPI_SWIGLU) {
           const int col = (nbase >> 1) + rin;  // 32-row block -> 16 output columns
           store_act(y, (size_t)m * ldy + col, silu(acc[0][nt][i]) * acc[1][nt][i], y_f32);
+        } else if constexpr (EPI == EPI_ROPE) {
+          const int p = re.pos[m], sl = re.slot[m];
+          if (p < 0 || p >= re.cap || p >= re.table_max_pos || sl < 0 || sl >= re.n_slots) {
+            dev_flag(DEVERR_CAPACITY);
+            continue;
+          }
+          const int QD = re.Hq * re.d, KD = re.Hkv * re.d, half = re.d >> 1;
+          if (nbase < QD + KD) {
+            const bool isq = nbase < QD;
+            const int rel = isq ? nbase : nbase - QD;
+            const int head = rel / re.d, ei = ((rel % re.d) >> 1) + rin;  // first-half element 16b + rin
+            const float xa = acc[0][nt][i], xb = acc[1][nt][i];
+            const float cs = re.table[(size_t)p * re.d + 2 * ei], sn = re.table[(size_t)p * re.d + 2 * ei + 1];
+            const float ra = xa * cs - xb * sn;
+            const float rb = xb * cs + xa * sn;
+            if (isq) {
+              store_act(re.q_out, (size_t)m * QD + head * re.d + ei, ra, false);
+              store_act(re.q_out, (size_t)m * QD + head * re.d + ei + half, rb, false);
+            } else {
+              const size_t crow = (((size_t)sl * re.n_layers + re.layer) * re.Hkv + head) * re.cap + p;
+              store_act(re.kc, crow * re.d + ei, ra, false);
+              store_act(re.kc, crow * re.d + ei + half, rb, false);
+            }
+          } else {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const int ev = nbase - QD - KD + r * 16 + rin;
+              const size_t crow = (((size_t)sl * re.n_layers + re.layer) * re.Hkv + ev / re.d) * re.cap + p;
+              store_act(re.vc, crow * re.d + ev % re.d, acc[r][nt][i], false);
+            }
+          }
         } else {
 #pragma unroll
           for (int r = 0; r < 2; ++r) store_act(y, (size_t)m * ldy + nbase + r * 16 + rin, acc[r][nt][i], y_f32);
@@ -425,7 +477,8 @@ size_t gemm_ws_bytes(int M, int N, int K, int mode, int variant) {
 
 template <int BN, int EPI>
 static int launch_gemm_bf16_t(const CUtensorMap& tw, const CUtensorMap& tx, void* y, int ldy, int y_f32, int M, int N,
-                              int K, int splits, float* partial, const int* mcount, int mmult, cudaStream_t st) {
+                              int K, int splits, float* partial, const int* mcount, int mmult, const RopeEpi& re,
+                              cudaStream_t st) {
   using C = GemmCfg<BN>;
   static bool attr_done = false;  // per instantiation; set once per process
   if (!attr_done) {
@@ -437,13 +490,15 @@ static int launch_gemm_bf16_t(const CUtensorMap& tw, const CUtensorMap& tx, void
   const int items = splits * n_groups * m_tiles;
   const int grid = items < num_sms() ? items : num_sms();
   BI_TRY(launch(gemm_bf16_kernel<BN, EPI>, dim3(grid), dim3(160), C::SMEM, st, tw, tx, y, ldy, y_f32, M, N, K, m_tiles, n_groups, splits,
-                                                         partial, mcount, mmult));
+                                                         partial, mcount, mmult, re));
   return BI_OK;
 }
 
 // mcount (optional, device int): only rows < *mcount * mmult of x are computed.
 int gemm_bf16(const void* x, int ldx, const void* w, void* y, int ldy, int y_f32, int M, int N, int K, int epi,
-              int variant, void* ws, size_t ws_bytes, cudaStream_t st, const int* mcount = nullptr, int mmult = 1) {
+              int variant, void* ws, size_t ws_bytes, cudaStream_t st, const int* mcount = nullptr, int mmult = 1,
+              const RopeEpi* rope = nullptr) {
+  const RopeEpi re = rope ? *rope : RopeEpi{};
   const int bn = gemm_pick_bn(N);
   const int kbs = gemm_kbs(bn);
   // 3-D views {64 k, rows, k-block}: the k-block dimension (stride 128 B) is the
@@ -468,12 +523,20 @@ int gemm_bf16(const void* x, int ldx, const void* w, void* y, int ldy, int y_f32
     BI_REQUIRE(ws && ws_bytes >= need, BI_ERR_WORKSPACE, "bi_gemm FAST: workspace %zu < %zu", ws_bytes, need);
     partial = reinterpret_cast<float*>(ws);
   }
-#define BI_GEMM_CASE(BNV)                                                                                          \
-  if (bn == BNV) {                                                                                                 \
-    if (epi == BI_EPI_SWIGLU)                                                                                      \
-      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_SWIGLU>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, mcount, mmult, st)));     \
-    else                                                                                                           \
-      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_NONE>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, mcount, mmult, st)));       \
+  if (epi == EPI_ROPE) {
+    if (bn != 32 || splits > 1 || !rope)
+      return set_error(BI_ERR_UNSUPPORTED, "fused RoPE epilogue needs the 32-row tile and no split");
+    BI_TRY((launch_gemm_bf16_t<32, EPI_ROPE>(tw, tx, y, ldy, y_f32, M, N, K, 1, nullptr, mcount, mmult, re, st)));
+    return BI_OK;
+  }
+#define BI_GEMM_CASE(BNV)                                                                                      \
+  if (bn == BNV) {                                                                                             \
+    if (epi == BI_EPI_SWIGLU)                                                                                  \
+      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_SWIGLU>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, mcount,  \
+                                                     mmult, re, st)));                                         \
+    else                                                                                                       \
+      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_NONE>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, mcount,    \
+                                                   mmult, re, st)));                                           \
   }
   BI_GEMM_CASE(32)
   BI_GEMM_CASE(64)

@@ -360,7 +360,8 @@ int bi_rope_table_fill(float* table, int max_pos, int head_dim, double theta, vo
 }
 
 int bi_rope_kv_append(const float* qkv, const float* rope, int rope_max_pos, void* q_out, const bi_kv_layout* kv,
-                      int layer, const int32_t* slot, const int32_t* pos, int T, int Hq, int mode, void* stream) {
+                      int layer, const int32_t* slot, const int32_t* pos, int T, int Hq, int qk_paired, int mode,
+                      void* stream) {
   clear_error();
   BI_REQUIRE(qkv && rope && q_out && kv && kv->k && kv->v && slot && pos, BI_ERR_INVALID_ARG,
              "bi_rope_kv_append: NULL pointer");
@@ -370,7 +371,7 @@ int bi_rope_kv_append(const float* qkv, const float* rope, int rope_max_pos, voi
   if (T == 0) return BI_OK;
   BI_TRY(launch(rope_append_kernel, dim3(T), dim3(256), 0, as_stream(stream), qkv, rope, rope_max_pos, q_out, kv->k, kv->v, slot, pos, Hq,
                                                        kv->n_kv_heads, kv->head_dim, layer, kv->n_layers, kv->n_slots,
-                                                       kv->capacity, mode == BI_MODE_LAYERCAST));
+                                                       kv->capacity, mode == BI_MODE_LAYERCAST, qk_paired ? 1 : 0));
   return BI_OK;
 }
 
@@ -547,10 +548,17 @@ int bi_decode_step(bi_ctx* ctx, const bi_batch* batch, const bi_step_out* out, v
     const void* g_attn = lw(w.attn_norm, H, l);
     const void* g_ffn = lw(w.ffn_norm, H, l);
     BI_TRY(bi_rmsnorm(s.y, l == 0 ? nullptr : s.res, s.res, g_attn, s.u, nullptr, T, H, d.eps, d.mode, stream));
-    BI_TRY(gemm_run(s.u, H, lw(w.w_qkv, (size_t)QKV * H, l), s.qkv, QKV, BI_DTYPE_F32, T, QKV, H, BI_EPI_NONE, d.mode,
-                    d.variant, s.gemm, s.gemm_bytes, st));
-    BI_TRY(bi_rope_kv_append(s.qkv, w.rope, w.rope_max_pos, s.q, &ctx->kv, l, batch->slot, batch->pos, T, Hq, d.mode,
-                             stream));
+    if (f32 || d.variant == BI_VARIANT_FAST) {  // projection, then RoPE + KV append as a kernel
+      BI_TRY(gemm_run(s.u, H, lw(w.w_qkv, (size_t)QKV * H, l), s.qkv, QKV, BI_DTYPE_F32, T, QKV, H, BI_EPI_NONE,
+                      d.mode, d.variant, s.gemm, s.gemm_bytes, st));
+      BI_TRY(bi_rope_kv_append(s.qkv, w.rope, w.rope_max_pos, s.q, &ctx->kv, l, batch->slot, batch->pos, T, Hq, 1,
+                               d.mode, stream));
+    } else {  // RoPE + KV append in the projection's epilogue
+      RopeEpi re{w.rope, w.rope_max_pos, s.q, ctx->kv.k, ctx->kv.v, batch->slot, batch->pos,
+                 Hq, Hkv, hd, l, ctx->kv.n_layers, ctx->kv.n_slots, ctx->kv.capacity};
+      BI_TRY(gemm_bf16(s.u, H, lw(w.w_qkv, (size_t)QKV * H, l), s.qkv, QKV, 1, T, QKV, H, EPI_ROPE,
+                       BI_VARIANT_INVARIANT, nullptr, 0, st, nullptr, 1, &re));
+    }
     BI_TRY(attention_run(s.q, &ctx->kv, l, batch->slot, batch->pos, batch->slot_host, batch->pos_host, s.o, T, Hq,
                          scale, d.mode, d.variant, s.attn, s.attn_bytes, st));
     BI_TRY(gemm_run(s.o, QD, lw(w.w_o, (size_t)H * QD, l), s.y, H, act_dtype, T, H, QD, BI_EPI_NONE, d.mode,
@@ -629,9 +637,11 @@ int bi_greedy_advance(const int32_t* argmax, int32_t* ids, int32_t* pos, int B, 
 int bi_synth_fill_bf16(uint16_t* dst, int64_t rows, int64_t cols, uint64_t key, double std, int interleave, int phase,
                        void* stream) {
   clear_error();
-  BI_REQUIRE(dst && rows >= 0 && cols > 0 && interleave >= 0 && (phase == 0 || phase == 1), BI_ERR_INVALID_ARG,
+  BI_REQUIRE(dst && rows >= 0 && cols > 0 && (phase == 0 || phase == 1), BI_ERR_INVALID_ARG,
              "bi_synth_fill_bf16: bad arguments");
-  BI_REQUIRE(interleave == 0 || rows % interleave == 0, BI_ERR_INVALID_ARG,
+  BI_REQUIRE(interleave >= 0 || interleave == -64 || interleave == -128, BI_ERR_INVALID_ARG,
+             "bi_synth_fill_bf16: paired order needs head_dim 64 or 128");
+  BI_REQUIRE(interleave == 0 || rows % (interleave > 0 ? interleave : -interleave) == 0, BI_ERR_INVALID_ARG,
              "bi_synth_fill_bf16: rows must be a multiple of the interleave");
   if (rows == 0) return BI_OK;
   BI_TRY(launch(synth_fill_kernel, dim3(4 * num_sms()), dim3(256), 0, as_stream(stream), dst, rows, cols, key, std, interleave, phase));

@@ -96,12 +96,21 @@ __global__ void __launch_bounds__(NORM_THREADS)
   }
 }
 
+// Row of element i of a head (size d) in the "paired" QKV layout: within every
+// 32-row block b, rows 0..15 hold elements 16b.. and rows 16..31 their
+// rotate-half partners d/2 + 16b ...
+__host__ __device__ inline int paired_row(int i, int d) {
+  const int half = d >> 1;
+  return i < half ? 32 * (i >> 4) + (i & 15) : 32 * ((i - half) >> 4) + 16 + ((i - half) & 15);
+}
+
 // Rotate-half RoPE of q and k heads, then q -> q_out and k, v -> cache row
 // (slot, layer, head, pos).  One CTA per token.  table: [max_pos][d/2][2].
+// paired != 0: the q and k heads of qkv are in the paired row order.
 __global__ void rope_append_kernel(const float* __restrict__ qkv, const float* __restrict__ table, int table_max_pos,
                                    void* __restrict__ q_out, void* __restrict__ kc, void* __restrict__ vc,
                                    const int32_t* __restrict__ slot, const int32_t* __restrict__ pos, int Hq, int Hkv,
-                                   int d, int layer, int n_layers, int n_slots, int cap, int f32) {
+                                   int d, int layer, int n_layers, int n_slots, int cap, int f32, int paired) {
   pdl_wait();
   pdl_trigger();
   const int t = blockIdx.x;
@@ -120,7 +129,8 @@ __global__ void rope_append_kernel(const float* __restrict__ qkv, const float* _
   for (int idx = threadIdx.x; idx < npairs; idx += blockDim.x) {
     const int h = idx / half, i = idx % half;
     const float c = cs[2 * i], sn = cs[2 * i + 1];
-    const float a = row[h * d + i], b = row[h * d + i + half];
+    const int ia = paired ? paired_row(i, d) : i, ib = paired ? paired_row(i + half, d) : i + half;
+    const float a = row[h * d + ia], b = row[h * d + ib];
     const float ra = a * c - b * sn;
     const float rb = b * c + a * sn;
     if (h < Hq) {

@@ -5,6 +5,7 @@
 // bit-identical to any IEEE host implementation of the same definition.
 #pragma once
 #include "common.cuh"
+#include "norm_rope.cuh"
 
 namespace bi {
 
@@ -31,6 +32,10 @@ __global__ void synth_fill_kernel(uint16_t* __restrict__ dst, int64_t rows, int6
     const int64_t r = i / cols, c = i % cols;
     int64_t dr = r;
     if (interleave > 0) dr = (r / interleave) * 2 * interleave + (int64_t)phase * interleave + r % interleave;
+    if (interleave < 0) {  // paired RoPE row order of heads of size -interleave
+      const int hd = -interleave;
+      dr = (r / hd) * hd + paired_row((int)(r % hd), hd);
+    }
     dst[dr * cols + c] = f32_to_bf16_bits(f);
   }
 }

@@ -22,6 +22,21 @@ def _to_dev_bf16(bits, device):
     return torch.from_numpy(a).to(device).view(torch.bfloat16)
 
 
+def paired_rows(d):
+    """Fused row of each element of a head of size d in the paired q/k order (see bi_weights.w_qkv)."""
+    i = np.arange(d)
+    half = d // 2
+    return np.where(i < half, 32 * (i // 16) + i % 16, 32 * ((i - half) // 16) + 16 + (i - half) % 16)
+
+
+def pair_heads(w, d):
+    """[rows, H] q or k weight with rows in natural head order -> paired order."""
+    out = np.empty_like(w)
+    rows = np.arange(w.shape[0])
+    out[(rows // d) * d + paired_rows(d)[rows % d]] = w
+    return out
+
+
 def interleave_gu(wg, wu, g=GU_INTERLEAVE):
     """[F,H] gate and up -> [2F,H]: g gate rows, then the g up rows of the same outputs, ..."""
     F, H = wg.shape
@@ -49,7 +64,8 @@ class Model:
         if init == "host":
             w = host_weights if host_weights is not None else synth.model_weights(cfg, seed=seed)
             self.host_weights = w
-            qkv = np.concatenate([w["wq"], w["wk"], w["wv"]], axis=1)
+            qkv = np.concatenate([np.stack([pair_heads(w["wq"][l], d) for l in range(L)]),
+                                  np.stack([pair_heads(w["wk"][l], d) for l in range(L)]), w["wv"]], axis=1)
             gu = np.stack([interleave_gu(w["wg"][l], w["wu"][l]) for l in range(L)])
             t = {"embed": w["embed"], "lm_head": w["lm_head"], "final_norm": w["final_norm"],
                  "attn_norm": w["attn_norm"], "ffn_norm": w["ffn_norm"], "w_qkv": qkv, "w_o": w["wo"],
@@ -89,8 +105,8 @@ class Model:
         for l in range(L):
             ls = lambda s: synth.key(seed, synth.layer_stream(l, s))
             q = w["w_qkv"][l]
-            ops.synth_fill_bf16(q[:QD], QD, H, ls(synth.S_WQ), std)
-            ops.synth_fill_bf16(q[QD:QD + KD], KD, H, ls(synth.S_WK), std)
+            ops.synth_fill_bf16(q[:QD], QD, H, ls(synth.S_WQ), std, interleave=-d)
+            ops.synth_fill_bf16(q[QD:QD + KD], KD, H, ls(synth.S_WK), std, interleave=-d)
             ops.synth_fill_bf16(q[QD + KD:], KD, H, ls(synth.S_WV), std)
             ops.synth_fill_bf16(w["w_o"][l], H, QD, ls(synth.S_WO), std)
             ops.synth_fill_bf16(w["w_gu"][l], F, H, ls(synth.S_WG), std, interleave=GU_INTERLEAVE, phase=0)

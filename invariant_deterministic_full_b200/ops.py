@@ -66,12 +66,13 @@ class KVCache:
                                head_dim, DTYPE_F32 if mode == MODE_LAYERCAST else DTYPE_BF16)
 
 
-def rope_kv_append(qkv, rope, rope_max_pos, kv, layer, slot, pos, Hq, mode=MODE_BF16):
+def rope_kv_append(qkv, rope, rope_max_pos, kv, layer, slot, pos, Hq, mode=MODE_BF16, qk_paired=False):
     T = qkv.shape[0]
     d = kv.layout.head_dim
     q = torch.empty(T, Hq * d, dtype=act_dtype(mode), device=qkv.device)
     check(lib.bi_rope_kv_append(_ptr(qkv), _ptr(rope), rope_max_pos, _ptr(q), ctypes.byref(kv.layout), layer,
-                                _ptr(slot), _ptr(pos), T, Hq, mode, _stream()), "bi_rope_kv_append")
+                                _ptr(slot), _ptr(pos), T, Hq, 1 if qk_paired else 0, mode, _stream()),
+          "bi_rope_kv_append")
     return q
 
 

@@ -60,6 +60,13 @@ def test_device_generator_matches_host(bi):
     ref = interleave_gu(synth.normal_bf16(kg, rows * cols).reshape(rows, cols),
                         synth.normal_bf16(ku, rows * cols).reshape(rows, cols))
     assert np.array_equal(gu.view(torch.int16).cpu().numpy().view(np.uint16), ref)
+    # paired q/k head order (RoPE partners in one 32-row block), head_dim 128 and 64
+    from invariant_deterministic_full_b200.model import pair_heads
+    for hd in (128, 64):
+        pq = torch.empty(2 * hd, cols, dtype=torch.bfloat16, device="cuda")
+        bi.synth_fill_bf16(pq, 2 * hd, cols, kg, 0.02, interleave=-hd)
+        ref = pair_heads(synth.normal_bf16(kg, 2 * hd * cols).reshape(2 * hd, cols), hd)
+        assert np.array_equal(pq.view(torch.int16).cpu().numpy().view(np.uint16), ref)
     _after(bi)
 
 
