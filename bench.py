@@ -156,7 +156,7 @@ def gemm_bytes(cfg, B):
     L, H, Hq, Hkv, d, F, V = (cfg["n_layers"], cfg["hidden"], cfg["n_heads"], cfg["n_kv_heads"], cfg["head_dim"],
                               cfg["ffn"], cfg["vocab"])
     QKV = (Hq + 2 * Hkv) * d
-    per_layer = [(QKV, H, 4), (H, Hq * d, 2), (2 * F, H, 2), (H, F, 2)]  # (N, K, output bytes per element)
+    per_layer = [(QKV, H, 2), (H, Hq * d, 2), (2 * F, H, 2), (H, F, 2)]  # (N, K, output bytes per element)
     tot, n = 0, 0
     for N, K, ob in per_layer:
         tot += L * (N * K * 2 + B * K * 2 + B * (N // 2 if N == 2 * F else N) * ob)
@@ -318,8 +318,10 @@ def run_e2e(m, B, P, K, rank):
 
 
 class CpuSample:
-    """The fp64 oracle as it stands, on the host cores: one decode token through 8B-width models of 1 and 2
-    layers (each with the 128256-row LM head); the per-layer time is scaled to 32 layers -> tok/s."""
+    """The fp64 oracle as it stands, on the host cores: one decode token through 8B-width models of 0 and 4
+    layers (both with the 128256-row LM head); the per-layer time is scaled to 32 layers -> tok/s."""
+
+    LAYERS = 4
 
     def __init__(self):
         import oracle
@@ -327,26 +329,26 @@ class CpuSample:
         from synth import configs
         self.oracle = oracle
         self.cfg32 = configs.LLAMA8B
-        self.cfg2 = configs.shrink(self.cfg32, n_layers=2)
-        self.cfg1 = configs.shrink(self.cfg32, n_layers=1)
-        self.w2 = synth.model_weights(self.cfg2)
-        self.w1 = {k: (v[:1] if (v.ndim == 3 or k in ("attn_norm", "ffn_norm")) else v) for k, v in self.w2.items()}
-        self.tok = synth.prompt_tokens(0, 1, self.cfg2["vocab"])
+        self.cfgL = configs.shrink(self.cfg32, n_layers=self.LAYERS)
+        self.cfg0 = configs.shrink(self.cfg32, n_layers=0)
+        self.wL = synth.model_weights(self.cfgL)
+        self.w0 = {k: (v[:0] if (v.ndim == 3 or k in ("attn_norm", "ffn_norm")) else v) for k, v in self.wL.items()}
+        self.tok = synth.prompt_tokens(0, 1, self.cfgL["vocab"])
 
     def once(self):
         t = time.perf_counter()
-        self.oracle.forward(self.cfg1, self.w1, self.tok)
-        t1 = time.perf_counter() - t
+        self.oracle.forward(self.cfg0, self.w0, self.tok)
+        t0 = time.perf_counter() - t
         t = time.perf_counter()
-        self.oracle.forward(self.cfg2, self.w2, self.tok)
-        t2 = time.perf_counter() - t
-        per_layer = max(t2 - t1, 1e-9)
-        return per_layer * self.cfg32["n_layers"] + (t1 - per_layer), t1, t2
+        self.oracle.forward(self.cfgL, self.wL, self.tok)
+        tL = time.perf_counter() - t
+        per_layer = max(tL - t0, 1e-9) / self.LAYERS
+        return t0 + per_layer * self.cfg32["n_layers"], t0, tL
 
-    def describe(self, n, t1, t2):
-        return (f"fp64 oracle forward of 1 decode token through 1- and 2-layer 8B-width models incl. the "
-                f"128256-row LM head; the per-layer time (2-layer minus 1-layer) scaled to 32 layers; "
-                f"{n} repeats ({t1:.2f} s, {t2:.2f} s per forward)")
+    def describe(self, n, t0, tL):
+        return (f"fp64 oracle forward of 1 decode token through 0- and {self.LAYERS}-layer 8B-width models (both with "
+                f"the 128256-row LM head); per-layer time scaled to 32 layers; median of {n} repeats "
+                f"({t0:.3f} s, {tL:.3f} s per forward)")
 
 
 def cores():
@@ -356,14 +358,12 @@ def cores():
 def cpu_baseline(seconds):
     cs = CpuSample()
     t_end = time.time() + seconds
-    best = None
-    n = 0
-    while n == 0 or time.time() < t_end:
-        r = cs.once()
-        n += 1
-        best = r if best is None or r[0] < best[0] else best
-    return {"value": round(1.0 / best[0], 4), "unit": "tok/s", "cores": cores(), "kind": "oracle",
-            "sample": cs.describe(n, best[1], best[2])}
+    runs = []
+    while not runs or time.time() < t_end:
+        runs.append(cs.once())
+    med = sorted(runs)[len(runs) // 2]
+    return {"value": round(1.0 / med[0], 4), "unit": "tok/s", "cores": cores(), "kind": "oracle",
+            "sample": cs.describe(len(runs), med[1], med[2])}
 
 
 def main_ours(args):
@@ -466,10 +466,11 @@ def main_reference(args):
     t0 = time.perf_counter()
     ts = [cs.once() for _ in range(args.steps)]
     wall = time.perf_counter() - t0
-    per_tok = statistics.median(t[0] for t in ts)
+    med = sorted(ts)[len(ts) // 2]
+    per_tok = med[0]
     v = 1.0 / per_tok
     cb = {"value": round(v, 4), "unit": "tok/s", "cores": cores(), "kind": "oracle",
-          "sample": cs.describe(len(ts), ts[0][1], ts[0][2])}
+          "sample": cs.describe(len(ts), med[1], med[2])}
     line = {"metric": METRIC, "value": round(v, 4), "unit": "tok/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(per_tok * 1e3, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
