@@ -1,0 +1,139 @@
+"""Full-size workload tests (GPU): continuous batching on the Llama-3.1-8B shape and a 32K-token context
+on the Qwen2.5-7B shape.  Both check the GPU path bitwise against itself -- a property that holds at any
+size -- under the batch compositions and prefill chunkings of the two workloads.
+
+Continuous batching: 64 requests with prompt lengths uniform in [16, 4096] (seed 99) join a running batch
+at random steps, are prefilled in chunks of up to 512 tokens mixed with the decode tokens of the others,
+decode 128 greedy tokens and leave; every request's greedy tokens and logprobs equal those of its solo
+batch-1 run.
+
+32K context: one 32768-token sequence prefilled in chunks of 512, of 2048, and in one call gives the same
+logprobs at every sampled position; the last 16 positions decoded token by token (after a 2048-chunked
+prefill of the rest) give the same logprobs as the prefills.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from synth import configs
+
+pytestmark = pytest.mark.gpu
+
+
+def _draw_uniform(key, i, lo, hi):
+    return lo + synth.draw(key, i) % (hi - lo + 1)
+
+
+@pytest.fixture(scope="module")
+def pkg():
+    from invariant_deterministic_full_b200 import model, ops
+    assert torch.cuda.is_available()
+    ops.device_error(reset=True)
+    return model, ops
+
+
+def test_continuous_batching_matches_solo_runs(pkg):
+    model, ops = pkg
+    cfg = configs.LLAMA8B
+    V = cfg["vocab"]
+    n_req, n_dec, max_prompt, chunk = 64, 128, 4096, 512
+    k = synth.key(99, 5)
+    lens = [_draw_uniform(k, 2 * r, 16, max_prompt) for r in range(n_req)]
+    arrive = [_draw_uniform(k, 2 * r + 1, 0, 255) for r in range(n_req)]
+    prompts = [synth.prompt_tokens(r, lens[r], V) for r in range(n_req)]
+    cap = max_prompt + n_dec + 1
+    m = model.Model(cfg, mode=0, n_slots=n_req + 1, capacity=cap, init="device")
+
+    # ---- mixed run: slot r holds request r
+    done_prompt = [0] * n_req           # prompt tokens already prefilled
+    gen = [[] for _ in range(n_req)]    # generated tokens
+    lps = [[] for _ in range(n_req)]    # logprob of each generated token
+    step = 0
+    while any(len(g) < n_dec + 1 for g in gen):
+        ids, slots, pos, owner = [], [], [], []
+        budget = chunk
+        for r in range(n_req):          # prefill chunks of joined requests (FIFO), up to the token budget
+            if arrive[r] <= step and done_prompt[r] < lens[r] and budget > 0:
+                n = min(budget, lens[r] - done_prompt[r])
+                for t in range(done_prompt[r], done_prompt[r] + n):
+                    ids.append(int(prompts[r][t])); slots.append(r); pos.append(t)
+                    owner.append((r, t == lens[r] - 1))
+                done_prompt[r] += n
+                budget -= n
+        for r in range(n_req):          # one decode token for every request whose prompt is in the cache
+            if done_prompt[r] == lens[r] and 0 < len(gen[r]) <= n_dec and not any(o[0] == r for o in owner):
+                ids.append(gen[r][-1]); slots.append(r); pos.append(lens[r] + len(gen[r]) - 1)
+                owner.append((r, True))
+        if not ids:
+            step += 1
+            continue
+        lm = np.array([i if o[1] else -1 for i, o in enumerate(owner)], dtype=np.int32)
+        rows = np.cumsum(lm >= 0) - 1
+        lm = np.where(lm >= 0, rows, -1).astype(np.int32)
+        o = model.to_host(m.step(ids, slots, pos, lm))
+        for i, (r, wants) in enumerate(owner):
+            if wants:
+                row = lm[i]
+                gen[r].append(int(o["argmax"][row]))
+                lps[r].append(o["logprob"][row])
+        step += 1
+    torch.cuda.synchronize()
+    assert ops.device_error() == 0
+
+    # ---- solo batch-1 runs in a spare slot
+    solo = n_req
+    for r in range(n_req):
+        o = model.prefill(m, solo, prompts[r], lm_every=lens[r])
+        g = [int(o["argmax"][-1])]
+        lp = [o["logprob"][-1]]
+        for j in range(n_dec):
+            od = model.to_host(m.step([g[-1]], [solo], [lens[r] + j]))
+            g.append(int(od["argmax"][0]))
+            lp.append(od["logprob"][0])
+        assert g == gen[r][:n_dec + 1], r
+        assert np.array_equal(np.array(lp, dtype=np.float32), np.array(lps[r][:n_dec + 1], dtype=np.float32)), r
+    torch.cuda.synchronize()
+    assert ops.device_error() == 0
+    m.close()
+
+
+def test_qwen_32k_chunked_prefill_and_decode_agree(pkg):
+    model, ops = pkg
+    cfg = configs.QWEN7B
+    n = 32768
+    tail = 16
+    V = cfg["vocab"]
+    tok = synth.prompt_tokens(7, n + 1, V)
+    m = model.Model(cfg, mode=0, n_slots=4, capacity=n + 8, init="device")
+    sample = np.unique(np.concatenate([np.arange(0, n, 509), np.arange(n - 64, n)]))
+    want = np.zeros(n, dtype=bool)
+    want[sample] = True
+
+    def prefill(slot, length, chunk):
+        res = {}
+        for c0 in range(0, length, chunk):
+            c1 = min(length, c0 + chunk)
+            idx = np.arange(c0, c1)
+            w = want[idx]
+            lm = np.where(w, np.cumsum(w) - 1, -1).astype(np.int32)
+            if not w.any():
+                lm[-1] = 0  # keep one output row so the call shape stays simple
+            o = model.to_host(m.step(tok[c0:c1], [slot] * (c1 - c0), idx, lm, tok[c0 + 1:c1 + 1][lm >= 0]))
+            for row, p in zip(range(int((lm >= 0).sum())), idx[lm >= 0]):
+                res[int(p)] = (o["logprob"][row], o["lse"][row])
+        return res
+
+    ref = prefill(0, n, 2048)
+    for slot, ch in ((1, 512), (2, n)):
+        got = prefill(slot, n, ch)
+        for p in sample:
+            assert got[int(p)] == ref[int(p)], (ch, int(p))
+    # token-by-token decode of the last positions after a 2048-chunked prefill of the rest
+    prefill(3, n - tail, 2048)
+    for p in range(n - tail, n):
+        o = model.to_host(m.step([int(tok[p])], [3], [p], [0], [int(tok[p + 1])]))
+        assert (o["logprob"][0], o["lse"][0]) == ref[p], p
+    torch.cuda.synchronize()
+    assert ops.device_error() == 0
+    m.close()
