@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling case: the 8B shape with this many layers (0 = all 32; not the headline workload)")
     return ap.parse_args()
 
 
@@ -372,7 +374,9 @@ def main_ours(args):
     from synth import configs
     from invariant_deterministic_full_b200 import model as mdl
     ws, rank, local = dist_init(args)
-    cfg = configs.LLAMA8B
+    cfg = dict(configs.LLAMA8B)
+    if args.layers:
+        cfg["n_layers"] = args.layers
     B, P, K, W = args.batch, args.prompt, args.steps, args.warmup
     assert W >= 3, "at least 3 warm-up steps"
     mode = 1 if args.mode == "layercast" else 0
@@ -392,12 +396,14 @@ def main_ours(args):
             "ms_per_step": round(ms / K, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if mode == 0 else "f32 (bf16 weights)",
             "data": "synthetic: random-init bf16 weights N(0,0.02) (seed 20261202), uniform random prompt ids",
-            "config": {"workload": f"llama3.1-8b-shape greedy decode, batch {B} per GPU, prompt {P}, "
+            "config": {"workload": f"llama3.1-8b-shape{' (%d layers)' % args.layers if args.layers else ''} "
+                                   f"greedy decode, batch {B} per GPU, prompt {P}, "
                                    f"{K} timed steps (positions {P + 1 + W}..{P + W + K})",
                        "model": cfg["name"] + " (random init)", "global_batch": B * ws, "seq_len": P + W + K + 1,
                        "parallelism": "replicas" if ws > 1 else "single GPU",
                        "mode": args.mode, "variant": "invariant", "margin_threshold": 0.1,
-                       "l2": "inputs larger than L2: every step streams 16 GB of weights"},
+                       "l2": "inputs larger than L2: every step streams 16 GB of weights"
+                             if not args.layers else "profiling case (reduced layer count)"},
             "hbm_roofline_frac_step": round(step_frac, 4),
             "recompute_rate": r["recompute_rate"],
             "gpu_launches": int(r["launches"] * K),

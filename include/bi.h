@@ -176,6 +176,10 @@ int bi_attention(const void* q, const bi_kv_layout* kv, int layer, const int32_t
  *   h is split exactly into three bf16 parts (h = p0 + p1 + p2; 8+8+8
  *   significant bits), each product with W is exact, the three products are
  *   accumulated in fp32 on the tensor cores and added as (z0 + z1) + z2.
+ *   p0 = bf16(h) is the main-pass input.  For B <= 10 one GEMM pass over W
+ *   computes the main logits and the parts of every row (3B token rows in
+ *   one 32-row token tile, W read once); for larger B a second pass over W
+ *   computes p1.W^T and p2.W^T of the flagged rows only, when there are any.
  *   Their lse, logprob and argmax are replaced; margin keeps the bf16-path
  *   value that triggered the recompute;
  *   recomputed[b] = 1.  margin_threshold <= 0 disables it.  In LAYERCAST the
@@ -198,10 +202,10 @@ int bi_lmhead_logprob(const float* h, const void* W, const int32_t* target, int 
  * inside the library, which every GPU that loads the library keeps until the
  * process exits.  Arguments and results are those of bi_lmhead_logprob, and
  * so is the arithmetic (the results are bit-identical).
- *  - Calls whose scratch need (bi_lmhead_workspace_size, less the logits when
- *    `logits` is given) exceeds BI_NOALLOC_SCRATCH_BYTES are rejected with
- *    BI_ERR_WORKSPACE and a message; at hidden 4096 / vocab 128256 that
- *    allows up to 32 rows in BI_MODE_BF16.
+ *  - Calls whose scratch need exceeds BI_NOALLOC_SCRATCH_BYTES are rejected
+ *    with BI_ERR_WORKSPACE and a message; at hidden 4096 / vocab 128256 that
+ *    allows up to 53 rows in BI_MODE_BF16 (bi_lmhead_workspace_size gives
+ *    the need of the recompute-enabled case).
  *  - The first call on a device looks up the array's device address (once per
  *    device, with that device current); make that first call before any
  *    stream capture.

@@ -43,7 +43,34 @@ struct AttnArgs {
   int t_base;               // first token of this group
   int Hq, Hkv, G, d, chunk, max_chunks, layer, n_layers, cap, f32;
   float scale;
+  int seg_len;              // chunks per CTA (tensor-core kernel; the CUDA-core kernel takes one)
+  int merge_in_cta;         // 1: one segment spans every chunk, the CTA merges and writes out
+  void* out;                // [T][Hq*d] attention output (activation dtype)
 };
+
+// Fixed ascending merge of one (query, q head)'s chunk partials 0..nc-1; lane
+// l owns head elements l, l+32, ...  The same code serves the merge kernel
+// and the attention CTAs that computed all chunks of their queries, so the
+// two routes give the same bits.
+__device__ __forceinline__ void merge_pair(const float* __restrict__ base, int nc, int d, int lane,
+                                           void* __restrict__ out, size_t off, int f32) {
+  float M = -INFINITY;
+  for (int c = 0; c < nc; ++c) M = fmaxf(M, base[(size_t)c * (d + 4) + d]);
+  float L = 0.f;
+  float o[4] = {0.f, 0.f, 0.f, 0.f};
+  const int ne = d / 32;
+  for (int c = 0; c < nc; ++c) {
+    const float* rec = base + (size_t)c * (d + 4);
+    const float w = expf(rec[d] - M);
+    L = fmaf(rec[d + 1], w, L);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k < ne) o[k] = fmaf(rec[lane + 32 * k], w, o[k]);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    if (k < ne) store_act(out, off + lane + 32 * k, o[k] / L, f32);
+}
 
 __host__ __device__ inline int att_ninner(int d, int f32) { return d * (f32 ? 4 : 2) / 128; }
 
@@ -302,173 +329,211 @@ __global__ void __launch_bounds__(ATT_THREADS)
 
 // ---------------------------------------------------------------------------
 // bf16 mode on tensor cores (mma.sync m16n8k16, fp32 accumulate).  The same
-// chunk grid, masks, max and lane-strided denominator as above; the two
-// contractions are tensor-core products:
-//   * score(p, j) = scale * (q_p . k_j): 8 ascending k16 steps over the head
-//     dimension into one fp32 accumulator (bf16 x bf16 products are exact);
-//   * numerator(p, e) = sum_j P(p, j) v_j[e]: the fp32 probabilities are split
-//     exactly into three bf16 parts P = P0 + P1 + P2 (8+8+8 significant bits),
-//     each part's product with V accumulated over ascending k16 steps of keys
-//     in its own fp32 accumulator, and the three added as (a0 + a1) + a2.
-// Row p of an MMA tile depends only on row p of its A operand, so the result
-// of a (query, head) pair does not depend on how many pairs share the tile --
-// decode (one 16-row tile) and prefill (32-row tiles) give the same bits.
-// Keys past a query have P = 0 and add exact zeros; V rows past the last
-// valid key are zeroed in shared memory before use.
-constexpr int ATC_SST = 264;  // padded row stride of the fp32 score tile
+// chunk grid, masks, max and lane-strided denominator as above.  The
+// (query, q head) pairs are the 8-column side of every mma, so a decode group
+// of G <= 8 pairs fills at least half a tile:
+//   * scores  S^T[key][pair] = scale * sum_d K[key][d] q[pair][d]
+//     (A = K tile, B = q^T): one chain of 8 ascending k16 steps over the head
+//     dimension per element (bf16 x bf16 products are exact);
+//   * output  O^T[e][pair] = sum_key V[key][e] P[pair][key]
+//     (A = V^T tile, B = P^T): the fp32 probabilities are split exactly into
+//     three bf16 parts P = P0 + P1 + P2 (8+8+8 significant bits), each part's
+//     product accumulated over ascending k16 steps of keys in its own fp32
+//     accumulator, and the three added as (o0 + o1) + o2.
+// Column p of an mma result depends only on column p of its B operand, so a
+// pair's result does not depend on how many pairs share the tile -- decode
+// (8- or 16-pair groups) and prefill (32-pair groups) give the same bits.
+// Pair rows past the group are never computed or stored.  Keys past a query
+// have P = 0 and add exact zeros; V rows past the last valid key are zeroed in
+// shared memory before use.
+constexpr int ATC_SST = 260;  // row stride of the fp32 score tile (floats): conflict-free fragment stores
 
-__host__ __device__ inline size_t atc_smem_bytes(int pt, int ring) {
-  const size_t rows = 16 * pt;
-  return (size_t)ring * 16384           // K/V sub-tiles: [2 halves][64 keys][128 B]
-         + rows * 256                   // q tile: [2 halves][rows][128 B]
-         + rows * ATC_SST * 4           // scores
-         + 3 * 4 * rows * 128           // probability parts: [3][4 key blocks][rows][128 B]
+__host__ __device__ inline size_t atc_smem_bytes(int npt, int ring) {
+  const size_t np = 8 * npt;
+  return (size_t)ring * 16384      // K/V sub-tiles: [2 halves][64 keys][128 B]
+         + np * 256                // q tile: [2 halves][np][128 B]
+         + np * ATC_SST * 4        // scores [np][ATC_SST]
+         + 3 * np * 512            // probability parts [3][np][256 keys] bf16, 16-byte chunks swizzled
          + 1024;
 }
 
-template <int PT, int RING>
+// byte offset of key j of pair row r in a probability part
+__device__ __forceinline__ uint32_t atc_poff(int r, int j) {
+  const int c = j >> 3;
+  return (uint32_t)(r * 512 + (((c & ~7) | ((c ^ r) & 7)) << 4) + (j & 7) * 2);
+}
+
+template <int NPT, int RING>
 __global__ void __launch_bounds__(ATT_THREADS)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ AttnPlan plan, const AttnArgs a) {
   pdl_wait();
   pdl_trigger();
-  constexpr int NR = 16 * PT;  // pair rows per group
+  constexpr int NP = 8 * NPT;  // pairs per group
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar[RING];
-  __shared__ float m_s[NR], l_s[NR];
-  __shared__ int live_s[NR];
+  __shared__ float m_s[NP], l_s[NP];
+  __shared__ int live_s[NP];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int b = blockIdx.x, c = blockIdx.y, hk = blockIdx.z;
+  const int b = blockIdx.x, sg = blockIdx.y, hk = blockIdx.z;
   if (b >= plan.n) return;
   const int t0 = plan.blk[b].x, nq = plan.blk[b].y;
   const int s = a.slot[t0];
   const int pmax = a.pos[t0 + nq - 1];
-  const int key0 = c * a.chunk;
-  if (key0 > pmax) return;
-  const int nvalid = min(a.chunk, pmax - key0 + 1);
-  const int nsub = (nvalid + ATT_SUB - 1) / ATT_SUB;
+  // this CTA's segment of the absolute chunk grid, walked in ascending order
+  const int c_lo = sg * a.seg_len;
+  int c_hi = min(pmax / a.chunk + 1, c_lo + a.seg_len);
+  if (c_hi > a.max_chunks) {  // device position beyond what the launch was planned for
+    if (threadIdx.x == 0) dev_flag(DEVERR_CAPACITY);
+    c_hi = a.max_chunks;
+  }
+  if (c_lo >= c_hi) return;
   const int npairs = nq * a.G;
-  const int row_base = ((s * a.n_layers + a.layer) * a.Hkv + hk) * a.cap + key0;
+  const int cache_base = ((s * a.n_layers + a.layer) * a.Hkv + hk) * a.cap;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, t4 = lane & 3;
   constexpr uint32_t SUB = 16384;
-  uint8_t* qt = smem + RING * SUB;                         // [2][NR][128 B]
-  float* S = reinterpret_cast<float*>(qt + NR * 256);      // [NR][ATC_SST]
-  uint8_t* Pp = reinterpret_cast<uint8_t*>(S + NR * ATC_SST);  // [3][4][NR][128 B]
+  uint8_t* qt = smem + RING * SUB;                             // [2][NP][128 B]
+  float* S = reinterpret_cast<float*>(qt + NP * 256);          // [NP][ATC_SST]
+  uint8_t* Pp = reinterpret_cast<uint8_t*>(S + NP * ATC_SST);  // [3][NP][512 B]
   const uint32_t qt_s = smem_u32(qt), pp_s = smem_u32(Pp);
-  const int nloads = 2 * nsub;
+  const int ngroups = (npairs + NP - 1) / NP;
+  auto nsub_of = [&](int c) { return (min(a.chunk, pmax - c * a.chunk + 1) + ATT_SUB - 1) / ATT_SUB; };
 
   if (tid == 0) {
     for (int r = 0; r < RING; ++r) mbar_init(&bar[r], 1);
     fence_mbar_init();
   }
   __syncthreads();
-  auto issue = [&](int L) {
-    const int li = L % nloads;
-    const bool isv = li >= nsub;
-    const int st = isv ? li - nsub : li;
-    mbar_arrive_expect_tx(&bar[L % RING], SUB);
-    tma_load_3d(smem + (L % RING) * SUB, isv ? &tmV : &tmK, 0, row_base + st * ATT_SUB, 0, &bar[L % RING]);
+  // Load stream (thread 0): for each chunk of the segment, for each pair
+  // group, the chunk's K sub-tiles then its V sub-tiles.  The ring runs
+  // across chunk boundaries, so the next chunk's keys arrive while this
+  // chunk's values are consumed.
+  int lp = 0, pc = c_lo, pg = 0, pli = 0, pns = nsub_of(c_lo);
+  auto issue_next = [&]() {
+    if (pc >= c_hi) return;
+    const bool isv = pli >= pns;
+    const int st = isv ? pli - pns : pli;
+    mbar_arrive_expect_tx(&bar[lp % RING], SUB);
+    tma_load_3d(smem + (lp % RING) * SUB, isv ? &tmV : &tmK, 0, cache_base + pc * a.chunk + st * ATT_SUB, 0,
+                &bar[lp % RING]);
+    ++lp;
+    if (++pli == 2 * pns) {
+      pli = 0;
+      if (++pg == ngroups) {
+        pg = 0;
+        if (++pc < c_hi) pns = nsub_of(pc);
+      }
+    }
   };
-  const int ngroups = (npairs + NR - 1) / NR;
-  const int total_loads = ngroups * nloads;
   if (tid == 0)
-    for (int L = 0; L < RING && L < total_loads; ++L) issue(L);
+    for (int r = 0; r < RING; ++r) issue_next();
   int L = 0;
   auto consume_wait = [&]() -> bool { return mbar_wait(&bar[L % RING], (uint32_t)((L / RING) & 1)); };
   auto release = [&]() {
     __syncthreads();
-    if (tid == 0 && L + RING < total_loads) issue(L + RING);
+    if (tid == 0) issue_next();
     ++L;
   };
 
-  for (int pg0 = 0; pg0 < npairs; pg0 += NR) {
-    const int gp = min(NR, npairs - pg0);
-    // q tile (bf16, 128-byte swizzle per half); padded rows are zero
-    for (int idx = tid; idx < NR * 16; idx += ATT_THREADS) {  // 16 chunks of 8 elements per row
-      const int row = idx >> 4, ch = idx & 15;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (row < gp) {
-        const int p = pg0 + row;
-        const int i = p / a.G, g = p % a.G;
-        v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.q) +
-                                            (size_t)(t0 + i) * a.Hq * 128 + (hk * a.G + g) * 128 + ch * 8);
+  // score work of a warp: key tile kt of each 64-key sub-tile, pair tiles pt = spt, spt + 2, ...
+  constexpr int SPT = NPT == 1 ? 1 : NPT / 2;  // pair tiles per warp in the score phase
+  const int kt = warp & 3;
+  const int spt0 = NPT == 1 ? 0 : (warp >> 2);
+  const bool score_warp = NPT > 1 || warp < 4;
+
+  for (int c = c_lo; c < c_hi; ++c) {
+    const int key0 = c * a.chunk;
+    const int nvalid = min(a.chunk, pmax - key0 + 1);
+    const int nsub = (nvalid + ATT_SUB - 1) / ATT_SUB;
+    for (int pg0 = 0; pg0 < npairs; pg0 += NP) {
+      const int gp = min(NP, npairs - pg0);
+      // q tile (bf16, 128-byte swizzle per half); padded rows are zero
+      for (int idx = tid; idx < NP * 16; idx += ATT_THREADS) {  // 16 chunks of 8 elements per row
+        const int row = idx >> 4, ch = idx & 15;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (row < gp) {
+          const int p = pg0 + row;
+          const int i = p / a.G, g = p % a.G;
+          v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.q) +
+                                              (size_t)(t0 + i) * a.Hq * 128 + (hk * a.G + g) * 128 + ch * 8);
+        }
+        const int half = ch >> 3, cc = ch & 7;
+        *reinterpret_cast<uint4*>(qt + half * (NP * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
       }
-      const int half = ch >> 3, cc = ch & 7;
-      *reinterpret_cast<uint4*>(qt + half * (NR * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
-    }
-    __syncthreads();
-    // q fragments stay in registers for the whole chunk
-    uint32_t qa[PT][8][4];
+      __syncthreads();
+      // q^T fragments (B operand) of this warp's pair tiles, kept for the whole chunk
+      uint32_t qb[SPT][8][2];
+      if (score_warp) {
 #pragma unroll
-    for (int mt = 0; mt < PT; ++mt)
+        for (int u = 0; u < SPT; ++u)
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int half = kk >> 2, ch = 2 * (kk & 3) + (lane >> 4);
-        ldsm_x4(qt_s + half * (NR * 128) + row * 128 + ((ch ^ (row & 7)) << 4), qa[mt][kk][0], qa[mt][kk][1],
-                qa[mt][kk][2], qa[mt][kk][3]);
+          for (int kk = 0; kk < 8; ++kk) {
+            const int row = (spt0 + 2 * u) * 8 + (lane & 7);
+            const int half = kk >> 2, ch = 2 * (kk & 3) + ((lane >> 3) & 1);
+            ldsm_x2(qt_s + half * (NP * 128) + row * 128 + ((ch ^ (row & 7)) << 4), qb[u][kk][0], qb[u][kk][1]);
+          }
       }
 
-    // ---- scores: warp w owns keys 8w..8w+7 of each 64-key sub-tile
-    for (int st = 0; st < nsub; ++st) {
-      if (!consume_wait()) return;
-      const uint32_t kb = smem_u32(smem + (L % RING) * SUB);
-      float acc[PT][4];
+      // ---- scores: S[pair][key] = scale * (K[key] . q[pair])
+      for (int st = 0; st < nsub; ++st) {
+        if (!consume_wait()) return;
+        if (score_warp) {
+          const uint32_t kb = smem_u32(smem + (L % RING) * SUB);
+          float acc[SPT][4];
 #pragma unroll
-      for (int mt = 0; mt < PT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+          for (int u = 0; u < SPT; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int krow = warp * 8 + (lane & 7);
-        const int half = kk >> 2, ch = 2 * (kk & 3) + ((lane >> 3) & 1);
-        uint32_t b0, b1;
-        ldsm_x2(kb + half * 8192 + krow * 128 + ((ch ^ (krow & 7)) << 4), b0, b1);
+          for (int kk = 0; kk < 8; ++kk) {
+            const int krow = kt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            const int half = kk >> 2, ch = 2 * (kk & 3) + (lane >> 4);
+            uint32_t ka[4];
+            ldsm_x4(kb + half * 8192 + krow * 128 + ((ch ^ (krow & 7)) << 4), ka[0], ka[1], ka[2], ka[3]);
 #pragma unroll
-        for (int mt = 0; mt < PT; ++mt) mma_bf16_16816(acc[mt], qa[mt][kk], b0, b1);
+            for (int u = 0; u < SPT; ++u) mma_bf16_16816(acc[u], ka, qb[u][kk][0], qb[u][kk][1]);
+          }
+#pragma unroll
+          for (int u = 0; u < SPT; ++u) {
+            const int pr = (spt0 + 2 * u) * 8 + 2 * t4;
+            const int j = st * ATT_SUB + kt * 16 + g8;
+            S[pr * ATC_SST + j] = acc[u][0] * a.scale;
+            S[(pr + 1) * ATC_SST + j] = acc[u][1] * a.scale;
+            S[pr * ATC_SST + j + 8] = acc[u][2] * a.scale;
+            S[(pr + 1) * ATC_SST + j + 8] = acc[u][3] * a.scale;
+          }
+        }
+        release();
       }
-#pragma unroll
-      for (int mt = 0; mt < PT; ++mt) {
-        const int j = st * ATT_SUB + warp * 8 + 2 * t4;
-        float* r0 = S + (mt * 16 + g8) * ATC_SST + j;
-        float* r1 = S + (mt * 16 + g8 + 8) * ATC_SST + j;
-        *reinterpret_cast<float2*>(r0) = make_float2(acc[mt][0] * a.scale, acc[mt][1] * a.scale);
-        *reinterpret_cast<float2*>(r1) = make_float2(acc[mt][2] * a.scale, acc[mt][3] * a.scale);
-      }
-      release();
-    }
 
-    // ---- softmax per pair row: max (exact), exp, l = lane-strided ascending sums then butterfly;
-    // the probabilities go out as three exact bf16 parts (zeros past the valid keys)
-    for (int pl = warp; pl < NR; pl += ATT_THREADS / 32) {
-      float mx = -INFINITY, sum = 0.f;
-      int lim = -1;
-      if (pl < gp) {
+      // ---- softmax of the live pair rows: max (exact), exp, l = lane-strided ascending sums then
+      // butterfly; the probabilities go out as three exact bf16 parts (zeros past the valid keys).
+      // Rows past the group's pairs are not computed: they only reach output columns never stored.
+      for (int pl = warp; pl < gp; pl += ATT_THREADS / 32) {
         const int i = (pg0 + pl) / a.G;
-        lim = a.pos[t0 + i] - key0;
+        const int lim = a.pos[t0 + i] - key0;
+        float mx = -INFINITY;
 #pragma unroll
         for (int k = 0; k < ATT_CHUNK / 32; ++k) {
           const int j = lane + 32 * k;
           if (j <= lim && j < nvalid) mx = fmaxf(mx, S[pl * ATC_SST + j]);
         }
         mx = warp_max(mx);
-      }
+        float sum = 0.f;
 #pragma unroll
-      for (int k = 0; k < ATT_CHUNK / 32; ++k) {
-        const int j = lane + 32 * k;
-        float pj = 0.f;
-        if (pl < gp && j <= lim && j < nvalid) pj = expf(S[pl * ATC_SST + j] - mx);
-        sum += pj;
-        const uint16_t p0 = f32_to_bf16_bits(pj);
-        const float r0 = pj - bf16_bits_to_f32(p0);
-        const uint16_t p1 = f32_to_bf16_bits(r0);
-        const uint16_t p2 = f32_to_bf16_bits(r0 - bf16_bits_to_f32(p1));
-        const int kbk = j >> 6, ch = (j & 63) >> 3;
-        const int off = kbk * (NR * 128) + pl * 128 + ((ch ^ (pl & 7)) << 4) + (j & 7) * 2;
-        *reinterpret_cast<uint16_t*>(Pp + 0 * (4 * NR * 128) + off) = p0;
-        *reinterpret_cast<uint16_t*>(Pp + 1 * (4 * NR * 128) + off) = p1;
-        *reinterpret_cast<uint16_t*>(Pp + 2 * (4 * NR * 128) + off) = p2;
-      }
-      if (pl < gp) {
+        for (int k = 0; k < ATT_CHUNK / 32; ++k) {
+          const int j = lane + 32 * k;
+          float pj = 0.f;
+          if (j <= lim && j < nvalid) pj = expf(S[pl * ATC_SST + j] - mx);
+          sum += pj;
+          const uint16_t p0 = f32_to_bf16_bits(pj);
+          const float r0 = pj - bf16_bits_to_f32(p0);
+          const uint16_t p1 = f32_to_bf16_bits(r0);
+          const uint16_t p2 = f32_to_bf16_bits(r0 - bf16_bits_to_f32(p1));
+          const uint32_t off = atc_poff(pl, j);
+          *reinterpret_cast<uint16_t*>(Pp + 0 * (NP * 512) + off) = p0;
+          *reinterpret_cast<uint16_t*>(Pp + 1 * (NP * 512) + off) = p1;
+          *reinterpret_cast<uint16_t*>(Pp + 2 * (NP * 512) + off) = p2;
+        }
         sum = warp_sum_fixed(sum);
         if (lane == 0) {
           m_s[pl] = mx;
@@ -476,78 +541,81 @@ __global__ void __launch_bounds__(ATT_THREADS)
           live_s[pl] = lim >= 0;
         }
       }
-    }
-    __syncthreads();
+      __syncthreads();
 
-    // ---- PV: warp w owns head elements 16w..16w+15 (two n8 tiles)
-    float pacc[3][PT][2][4];
+      // ---- P.V: warp w owns head elements 16w..16w+15 (one m16 tile of V^T)
+      float pacc[3][NPT][4];
 #pragma unroll
-    for (int q = 0; q < 3; ++q)
+      for (int q = 0; q < 3; ++q)
 #pragma unroll
-      for (int mt = 0; mt < PT; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) pacc[q][mt][nt][0] = pacc[q][mt][nt][1] = pacc[q][mt][nt][2] = pacc[q][mt][nt][3] = 0.f;
-    for (int st = 0; st < nsub; ++st) {
-      if (!consume_wait()) return;
-      uint8_t* vbuf = smem + (L % RING) * SUB;
-      const int vrows = nvalid - st * ATT_SUB;  // valid rows of this sub-tile
-      if (vrows < ATT_SUB) {  // zero the rows past the last valid key
-        for (int idx = tid; idx < (ATT_SUB - vrows) * 16; idx += ATT_THREADS) {
-          const int r = vrows + (idx >> 4), ch = idx & 15;
-          *reinterpret_cast<uint4*>(vbuf + (ch >> 3) * 8192 + r * 128 + ((ch & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        for (int u = 0; u < NPT; ++u) pacc[q][u][0] = pacc[q][u][1] = pacc[q][u][2] = pacc[q][u][3] = 0.f;
+      for (int st = 0; st < nsub; ++st) {
+        if (!consume_wait()) return;
+        uint8_t* vbuf = smem + (L % RING) * SUB;
+        const int vrows = nvalid - st * ATT_SUB;  // valid rows of this sub-tile
+        if (vrows < ATT_SUB) {  // zero the rows past the last valid key
+          for (int idx = tid; idx < (ATT_SUB - vrows) * 16; idx += ATT_THREADS) {
+            const int r = vrows + (idx >> 4), ch = idx & 15;
+            *reinterpret_cast<uint4*>(vbuf + (ch >> 3) * 8192 + r * 128 + ((ch & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          __syncthreads();
         }
-        __syncthreads();
-      }
-      const uint32_t vb = smem_u32(vbuf);
-      const int nk16 = min(4, (vrows + 15) / 16);
-      for (int kk = 0; kk < nk16; ++kk) {
-        // B fragments: V rows = keys 16kk..16kk+15 of the sub-tile, elements 16w..16w+15
-        uint32_t vb0[2], vb1[2];
-        {
-          const int krow = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-          const int e0 = warp * 16 + (lane >> 4) * 8;
-          const int half = e0 >> 6, ch = (e0 & 63) >> 3;
-          ldsm_x4_trans(vb + half * 8192 + krow * 128 + ((ch ^ (krow & 7)) << 4), vb0[0], vb1[0], vb0[1], vb1[1]);
-        }
-        const int kblk = st;  // 64 keys per probability block
+        const uint32_t vb = smem_u32(vbuf);
+        const int nk16 = min(4, (vrows + 15) / 16);
+        for (int kk = 0; kk < nk16; ++kk) {
+          // A fragment: V^T rows = head elements 16w.., columns = keys 16kk.. of the sub-tile
+          uint32_t va[4];
+          {
+            const int krow = kk * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+            const int e0 = warp * 16 + ((lane >> 3) & 1) * 8;
+            const int half = e0 >> 6, ch = (e0 & 63) >> 3;
+            ldsm_x4_trans(vb + half * 8192 + krow * 128 + ((ch ^ (krow & 7)) << 4), va[0], va[1], va[2], va[3]);
+          }
+          const int j0 = st * ATT_SUB + kk * 16;  // first key of this k16 step within the chunk
 #pragma unroll
-        for (int q = 0; q < 3; ++q) {
+          for (int q = 0; q < 3; ++q) {
 #pragma unroll
-          for (int mt = 0; mt < PT; ++mt) {
-            uint32_t pa[4];
-            const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            const int ch = 2 * kk + (lane >> 4);
-            ldsm_x4(pp_s + q * (4 * NR * 128) + kblk * (NR * 128) + row * 128 + ((ch ^ (row & 7)) << 4), pa[0], pa[1],
-                    pa[2], pa[3]);
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) mma_bf16_16816(pacc[q][mt][nt], pa, vb0[nt], vb1[nt]);
+            for (int u = 0; u < NPT; ++u) {
+              uint32_t pb0, pb1;
+              const int row = u * 8 + (lane & 7);
+              ldsm_x2(pp_s + q * (NP * 512) + atc_poff(row, j0 + ((lane >> 3) & 1) * 8), pb0, pb1);
+              mma_bf16_16816(pacc[q][u], va, pb0, pb1);
+            }
           }
         }
+        release();
       }
-      release();
-    }
+      // partial record of each live pair: acc[e] = (o0 + o1) + o2, then m and l
 #pragma unroll
-    for (int mt = 0; mt < PT; ++mt)
+      for (int u = 0; u < NPT; ++u)
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          const int pl = mt * 16 + g8 + hr * 8;
+        for (int cc = 0; cc < 2; ++cc) {
+          const int pl = u * 8 + 2 * t4 + cc;
           if (pl >= gp || !live_s[pl]) continue;
           const int p = pg0 + pl;
           const int i = p / a.G, g = p % a.G;
           const int hq = hk * a.G + g;
           float* rec = a.part + (((size_t)(t0 + i - a.t_base) * a.Hq + hq) * a.max_chunks + c) * (128 + 4);
-          const int e = warp * 16 + nt * 8 + 2 * t4;
-          const float o0 = (pacc[0][mt][nt][2 * hr] + pacc[1][mt][nt][2 * hr]) + pacc[2][mt][nt][2 * hr];
-          const float o1 = (pacc[0][mt][nt][2 * hr + 1] + pacc[1][mt][nt][2 * hr + 1]) + pacc[2][mt][nt][2 * hr + 1];
-          *reinterpret_cast<float2*>(rec + e) = make_float2(o0, o1);
-          if (e == 0) {
+          const int e = warp * 16 + g8;
+          rec[e] = (pacc[0][u][cc] + pacc[1][u][cc]) + pacc[2][u][cc];
+          rec[e + 8] = (pacc[0][u][2 + cc] + pacc[1][u][2 + cc]) + pacc[2][u][2 + cc];
+          if (warp == 0 && g8 == 0) {
             rec[128] = m_s[pl];
             rec[129] = l_s[pl];
           }
         }
-    __syncthreads();  // the next group overwrites q, S, the probability parts and the statistics
+      __syncthreads();  // the next group overwrites q, S, the probability parts and the statistics
+    }
+  }
+  if (a.merge_in_cta) {
+    // every chunk of the block's queries was computed above: merge them here
+    // (the partials written by this CTA are visible to it after the barrier)
+    for (int p = warp; p < npairs; p += ATT_THREADS / 32) {
+      const int t = t0 + p / a.G, hq = hk * a.G + p % a.G;
+      const int nc = min(a.pos[t] / a.chunk + 1, c_hi);
+      merge_pair(a.part + ((size_t)(t - a.t_base) * a.Hq + hq) * a.max_chunks * (128 + 4), nc, 128, lane, a.out,
+                 (size_t)t * a.Hq * 128 + hq * 128, 0);
+    }
   }
 }
 
@@ -566,19 +634,7 @@ __global__ void attn_merge_kernel(const float* __restrict__ part, const int32_t*
     if (lane == 0) dev_flag(DEVERR_CAPACITY);
     nc = max_chunks;
   }
-  const float* base = part + ((size_t)tl * Hq + hq) * max_chunks * (d + 4);
-  float M = -INFINITY;
-  for (int c = 0; c < nc; ++c) M = fmaxf(M, base[(size_t)c * (d + 4) + d]);
-  float L = 0.f;
-  float o[4] = {0.f, 0.f, 0.f, 0.f};
-  const int ne = d / 32;
-  for (int c = 0; c < nc; ++c) {
-    const float* rec = base + (size_t)c * (d + 4);
-    const float w = expf(rec[d] - M);
-    L = fmaf(rec[d + 1], w, L);
-    for (int k = 0; k < ne; ++k) o[k] = fmaf(rec[lane + 32 * k], w, o[k]);
-  }
-  for (int k = 0; k < ne; ++k) store_act(out, (size_t)t * Hq * d + hq * d + lane + 32 * k, o[k] / L, f32);
+  merge_pair(part + ((size_t)tl * Hq + hq) * max_chunks * (d + 4), nc, d, lane, out, (size_t)t * Hq * d + hq * d, f32);
 }
 
 }  // namespace bi

@@ -43,21 +43,29 @@ constexpr int GEMM_BK = 64;  // k per k-block (128 bytes of bf16: one swizzled s
 // the box, so in shared memory every k-block is a [rows][128 B] slab with the
 // 128-byte swizzle -- the layout ldmatrix reads without bank conflicts.  Few,
 // large TMA operations per stage keep each SM streaming near its peak rate.
-template <int BN>
+//
+// Consumer warps: RW = BN/32 row groups x KS k-phases.  Warp (rw, kp) owns the
+// weight rows [32 rw, 32 rw + 32) and all 32 token columns, and takes the k16
+// steps whose index within their 64-k block is congruent to kp modulo KS: its
+// accumulators are the KS-interleaved accumulator set kp of those outputs.
+// Every weight and token fragment is therefore read from shared memory once
+// per row group, and the sets meet in a fixed tree after the K loop.
+// MT: 32-row token tiles sharing each weight stage (M-blocking; a property of
+// the launch, not of the arithmetic: every element still sees the same
+// instruction sequence).  MT > 1 only with 128-row weight tiles.
+template <int BN, int MT = 1>
 struct GemmCfg {
   static constexpr int KBS = BN == 128 ? 2 : 4;
   static constexpr int W_BYTES = KBS * BN * 128;
-  static constexpr int X_BYTES = KBS * GEMM_BM * 128;
+  static constexpr int X_BYTES = KBS * GEMM_BM * MT * 128;
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
-  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;
-  static constexpr int RW = BN / 32;      // warps along the weight rows (32 rows each)
-  static constexpr int TW = 4 / RW;       // warps along the token columns
-  static constexpr int NT = GEMM_BM / TW / 8;  // n8 token tiles per warp
+  static constexpr int RW = BN / 32;      // row groups (32 weight rows each)
   // Interleaved accumulator sets per output element (a property of the matrix
-  // shape through BN, never of M): enough independent mma chains per warp
-  // (2 row tiles x NT x KS = 8) to cover the tensor-pipe latency.
-  static constexpr int KS = NT >= 4 ? 1 : 4 / NT;
+  // shape through BN, never of M), one per k-phase warp of a row group.
+  static constexpr int KS = 4 / RW;
+  static constexpr int RED_BYTES = KS > 1 ? 4 * 32 * 32 * 4 : 0;  // cross-warp partial sums
+  static constexpr int STAGES = (212 * 1024 - RED_BYTES) / STAGE_BYTES;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + RED_BYTES + 1024;
 };
 
 // Fused RoPE + KV-append epilogue of the QKV projection (bf16 mode).  The
@@ -82,13 +90,14 @@ struct RopeEpi {
 
 // Work item -> (split, row group, token tile).  Splits > 1 only in the
 // non-invariant FAST variant, which then writes fp32 partials per split.
-template <int BN, int EPI>
+template <int BN, int EPI, int MT>
 __global__ void __launch_bounds__(160, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                      void* __restrict__ y, int ldy, int y_f32, int M, int N, int K, int m_tiles, int n_groups,
                      int splits, float* __restrict__ partial, const int* __restrict__ mcount, int mmult,
                      const RopeEpi re) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, MT>;
+  static_assert(MT == 1 || C::KS == 1, "M-blocking needs one k-phase per warp");
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::STAGES];
   __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
@@ -99,7 +108,24 @@ __global__ void __launch_bounds__(160, 1)
   // which add exact zeros to the accumulators
   const int kstages_total = (K / GEMM_BK + C::KBS - 1) / C::KBS;
   const int ks_per_split = (kstages_total + splits - 1) / splits;
-  const int n_items = splits * n_groups * m_tiles;
+  const int m_groups = (m_tiles + MT - 1) / MT;  // MT token tiles per work item
+  const int n_items = splits * n_groups * m_groups;
+  // Work item -> (split, weight row group, token group).  Token group fastest by
+  // default (CTAs working at the same time share weight tiles in L2); with a
+  // device-side row count, token group slowest, so the live first token tiles
+  // are spread over all CTAs.
+  const bool mg_major = mcount != nullptr;
+  auto decode_item = [&](int item, int& sp, int& g, int& mg) {
+    if (mg_major) {
+      g = item % n_groups;
+      sp = (item / n_groups) % splits;
+      mg = item / (n_groups * splits);
+    } else {
+      mg = item % m_groups;
+      g = (item / m_groups) % n_groups;
+      sp = item / (m_groups * n_groups);
+    }
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -116,30 +142,39 @@ __global__ void __launch_bounds__(160, 1)
       prefetch_tmap(&tmX);
       // Prologue: the first ring stages of weight tiles depend on no earlier
       // kernel, so they are requested before waiting for the previous launch.
+      // (With a device-side row count only token group 0 is sure to be live:
+      // it is live unless the count is zero, and then the prefetched stages
+      // are drained before the CTA exits.)
       int pre = 0;
-      if (mcount == nullptr && (int)blockIdx.x < n_items) {
-        const int item = blockIdx.x;
-        const int g = (item / m_tiles) % n_groups;
-        const int ks0 = (item / (m_tiles * n_groups)) * ks_per_split;
-        const int ks1 = min(kstages_total, ks0 + ks_per_split);
-        pre = max(0, min(C::STAGES, ks1 - ks0));
-        for (int s = 0; s < pre; ++s) {
-          mbar_arrive_expect_tx(&full_bar[s], C::STAGE_BYTES);
-          tma_load_3d(smem + s * C::STAGE_BYTES, &tmW, 0, g * BN, (ks0 + s) * C::KBS, &full_bar[s]);
+      if ((int)blockIdx.x < n_items) {
+        int sp, g, mg;
+        decode_item(blockIdx.x, sp, g, mg);
+        if (mcount == nullptr || mg == 0) {
+          const int ks0 = sp * ks_per_split;
+          const int ks1 = min(kstages_total, ks0 + ks_per_split);
+          pre = max(0, min(C::STAGES, ks1 - ks0));
+          for (int s = 0; s < pre; ++s) {
+            mbar_arrive_expect_tx(&full_bar[s], C::STAGE_BYTES);
+            tma_load_3d(smem + s * C::STAGE_BYTES, &tmW, 0, g * BN, (ks0 + s) * C::KBS, &full_bar[s]);
+          }
         }
       }
       pdl_wait();
       pdl_trigger();
       // rows beyond a device-side count (selective recompute) are not computed
       const int Me = mcount ? min(M, *mcount * mmult) : M;
+      if (pre > 0 && Me <= 0) {  // nothing to compute: wait for the prefetched stages, then leave
+        for (int s = 0; s < pre; ++s) (void)mbar_wait(&full_bar[s], 0u);
+        return;
+      }
       int stage = 0;
       uint32_t phase = 0;
       bool first = true;
       for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int mt = item % m_tiles;
+        int sp, g, mg;
+        decode_item(item, sp, g, mg);
+        const int mt = mg * MT;  // first token tile of the item
         if (mt * GEMM_BM >= Me) continue;
-        const int g = (item / m_tiles) % n_groups;
-        const int sp = item / (m_tiles * n_groups);
         const int ks0 = sp * ks_per_split;
         const int ks1 = min(kstages_total, ks0 + ks_per_split);
         for (int ks = ks0; ks < ks1; ++ks) {
@@ -164,99 +199,199 @@ __global__ void __launch_bounds__(160, 1)
   pdl_trigger();
 
   // ---------------- consumers
-  const int rw = warp % C::RW, tw = warp / C::RW;
+  const int rw = warp % C::RW, kp = warp / C::RW;
   const int row0 = rw * 32;                      // weight rows [row0, row0+32) of the tile
-  const int tok0 = tw * (GEMM_BM / C::TW);       // token columns [tok0, tok0 + 8*NT)
   const int g8 = lane >> 2, t4 = lane & 3;
+  float* red = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);  // [warp][32 values][32 lanes]
   int stage = 0;
   uint32_t phase = 0;
+  // A ring wait that runs out (error flag set) stops this warp's waits and
+  // math, but it keeps meeting the named barriers so no warp waits forever.
+  bool dead = false;
   const int Me = mcount ? min(M, *mcount * mmult) : M;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    const int mt = item % m_tiles;
-    if (mt * GEMM_BM >= Me) continue;
-    const int g = (item / m_tiles) % n_groups;
-    const int sp = item / (m_tiles * n_groups);
+    int sp, g, mg;
+    decode_item(item, sp, g, mg);
+    const int mt0 = mg * MT;
+    if (mt0 * GEMM_BM >= Me) continue;
     const int ks0 = sp * ks_per_split;
     const int ks1 = min(kstages_total, ks0 + ks_per_split);
-    const bool active = mt * GEMM_BM + tok0 < Me;
-    // KS interleaved accumulator sets: k16 step s (counted from k = 0) adds into
-    // set s % KS; the sets are combined in a fixed tree after the K loop.
-    float accs[C::KS][2][C::NT][4];
+    int ntvs[MT];  // n8 token tiles holding live rows, per token tile
 #pragma unroll
-    for (int q = 0; q < C::KS; ++q)
+    for (int j = 0; j < MT; ++j) ntvs[j] = max(0, min(4, (Me - (mt0 + j) * GEMM_BM + 7) / 8));
+    // accumulator set kp of this warp's outputs: k16 steps kk = kp, kp + KS, ... of every 64-k block
+    float accm[MT][2][4][4];
+#pragma unroll
+    for (int j = 0; j < MT; ++j)
 #pragma unroll
       for (int a = 0; a < 2; ++a)
 #pragma unroll
-        for (int b = 0; b < C::NT; ++b)
+        for (int b = 0; b < 4; ++b)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) accs[q][a][b][c] = 0.f;
+          for (int c = 0; c < 4; ++c) accm[j][a][b][c] = 0.f;
 
     for (int ks = ks0; ks < ks1; ++ks) {
-      if (!mbar_wait(&full_bar[stage], phase)) return;
-      if (active) {
-        const uint32_t sbase = smem_u32(smem + stage * C::STAGE_BYTES);
+      if (!dead && !mbar_wait(&full_bar[stage], phase)) dead = true;
+      const uint32_t sbase = smem_u32(smem + stage * C::STAGE_BYTES);
 #pragma unroll
-        for (int kb = 0; kb < C::KBS; ++kb) {
-          const uint32_t wb = sbase + kb * (BN * 128);
-          const uint32_t xb = sbase + C::W_BYTES + kb * (GEMM_BM * 128);
+      for (int kb = 0; kb < C::KBS && !dead; ++kb) {
+        const uint32_t wb = sbase + kb * (BN * 128);
+        const uint32_t xb = sbase + C::W_BYTES + kb * (GEMM_BM * MT * 128);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            uint32_t a[2][4];
+        for (int j = 0; j < 4 / C::KS; ++j) {
+          const int kk = kp + j * C::KS;
+          uint32_t a[2][4];
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              const int row = row0 + r * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-              ldsm_x4(swz128(wb, row, 2 * kk + (lane >> 4)), a[r][0], a[r][1], a[r][2], a[r][3]);
-            }
-            uint32_t b[C::NT][2];
-            if constexpr (C::NT >= 2) {
+          for (int r = 0; r < 2; ++r) {
+            const int row = row0 + r * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            ldsm_x4(swz128(wb, row, 2 * kk + (lane >> 4)), a[r][0], a[r][1], a[r][2], a[r][3]);
+          }
 #pragma unroll
-              for (int p = 0; p < C::NT / 2; ++p) {
-                const int tok = tok0 + p * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+          for (int j = 0; j < MT; ++j) {
+            const int ntv = ntvs[j];
+            uint32_t b[4][2];
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+              if (2 * p < ntv) {
+                const int tok = j * GEMM_BM + p * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
                 ldsm_x4(swz128(xb, tok, 2 * kk + ((lane >> 3) & 1)), b[2 * p][0], b[2 * p][1], b[2 * p + 1][0],
                         b[2 * p + 1][1]);
               }
-            } else {
-              const int tok = tok0 + (lane & 7);
-              ldsm_x2(swz128(xb, tok, 2 * kk + ((lane >> 3) & 1)), b[0][0], b[0][1]);
             }
 #pragma unroll
             for (int r = 0; r < 2; ++r)
 #pragma unroll
-              for (int nt = 0; nt < C::NT; ++nt)
-                mma_bf16_16816(accs[kk % C::KS][r][nt], a[r], b[nt][0], b[nt][1]);
+              for (int nt = 0; nt < 4; ++nt)
+                if (nt < ntv) mma_bf16_16816(accm[j][r][nt], a[r], b[nt][0], b[nt][1]);
           }
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[stage]);
+      if (lane == 0 && !dead) mbar_arrive(&empty_bar[stage]);
       if (++stage == C::STAGES) {
         stage = 0;
         phase ^= 1;
       }
     }
-    if (!active) continue;
-    float acc[2][C::NT][4];
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
+    for (int jt = 0; jt < MT; ++jt) {
+    const int mt = mt0 + jt;
+    const int ntv = ntvs[jt];
+    float (&acc)[2][4][4] = accm[jt];
+    if (ntv == 0) continue;  // uniform across the consumer warps
+    if constexpr (C::KS > 1) {
+      // The KS sets of the row group meet through shared memory: warp (rw, kp)
+      // finishes the n8 token tiles nt = kp, kp + KS, ... combining
+      // ((s0 + s1) + (s2 + s3)) (KS = 4) or s0 + s1 (KS = 2), set j coming from
+      // warp (rw, j); the epilogue work is shared by all four warps.
 #pragma unroll
-      for (int b = 0; b < C::NT; ++b)
+      for (int a = 0; a < 2; ++a)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if constexpr (C::KS == 4)
-            acc[a][b][c] = (accs[0][a][b][c] + accs[1][a][b][c]) + (accs[2][a][b][c] + accs[3][a][b][c]);
-          else if constexpr (C::KS == 2)
-            acc[a][b][c] = accs[0][a][b][c] + accs[1][a][b][c];
-          else
-            acc[a][b][c] = accs[0][a][b][c];
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) red[(warp * 32 + (a * 16 + b * 4 + c)) * 32 + lane] = acc[a][b][c];
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          if (b % C::KS != kp) continue;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int v = a * 16 + b * 4 + c;
+            const float s0 = red[(rw * 32 + v) * 32 + lane];
+            const float s1 = red[((rw + C::RW) * 32 + v) * 32 + lane];
+            if constexpr (C::KS == 4) {
+              const float s2 = red[((rw + 2) * 32 + v) * 32 + lane];
+              const float s3 = red[((rw + 3) * 32 + v) * 32 + lane];
+              acc[a][b][c] = (s0 + s1) + (s2 + s3);
+            } else {
+              acc[a][b][c] = s0 + s1;
+            }
+          }
         }
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // the next item reuses the exchange buffer
+    }
+    if (dead) continue;
 
     // ---------------- epilogue: fragment (row g8 (+8), cols 2*t4 (+1)) of each m16n8 tile
     const int nbase = g * BN + row0;
+    if constexpr (EPI == EPI_ROPE) {
+      if (splits == 1) {
+        // positions, slots and cos/sin of this thread's tokens are all fetched
+        // before any store, so the dependent loads overlap
+        const int QD = re.Hq * re.d, KD = re.Hkv * re.d, half = re.d >> 1;
+        const bool isv = nbase >= QD + KD, isq = nbase < QD;
+        const int rel = isq ? nbase : nbase - QD;
+        const int head = rel / re.d, e0 = (rel % re.d) >> 1;  // first-half element 16b
+        int pp[4][2], ss[4][2];
+        bool ok[4][2];
 #pragma unroll
-    for (int nt = 0; nt < C::NT; ++nt) {
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int m = mt * GEMM_BM + nt * 8 + 2 * t4 + j;
+            ok[nt][j] = nt % C::KS == kp && nt < ntv && m < Me;
+            pp[nt][j] = ok[nt][j] ? __ldg(re.pos + m) : 0;
+            ss[nt][j] = ok[nt][j] ? __ldg(re.slot + m) : 0;
+          }
+        float cs[4][2][2], sn[4][2][2];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int p = pp[nt][j], sl = ss[nt][j];
+            if (ok[nt][j] && (p < 0 || p >= re.cap || p >= re.table_max_pos || sl < 0 || sl >= re.n_slots)) {
+              dev_flag(DEVERR_CAPACITY);
+              ok[nt][j] = false;
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const size_t ti = (size_t)(ok[nt][j] && !isv ? p : 0) * re.d + 2 * (e0 + g8 + h * 8);
+              cs[nt][j][h] = __ldg(re.table + ti);
+              sn[nt][j][h] = __ldg(re.table + ti + 1);
+            }
+          }
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int j = i & 1, h = i >> 1;
+            if (!ok[nt][j]) continue;
+            const int m = mt * GEMM_BM + nt * 8 + 2 * t4 + j;
+            const int p = pp[nt][j], sl = ss[nt][j];
+            const int rin = g8 + h * 8;
+            if (!isv) {
+              const int ei = e0 + rin;
+              const float xa = acc[0][nt][i], xb = acc[1][nt][i];
+              const float ra = xa * cs[nt][j][h] - xb * sn[nt][j][h];
+              const float rb = xb * cs[nt][j][h] + xa * sn[nt][j][h];
+              if (isq) {
+                store_act(re.q_out, (size_t)m * QD + head * re.d + ei, ra, false);
+                store_act(re.q_out, (size_t)m * QD + head * re.d + ei + half, rb, false);
+              } else {
+                const size_t crow = (((size_t)sl * re.n_layers + re.layer) * re.Hkv + head) * re.cap + p;
+                store_act(re.kc, crow * re.d + ei, ra, false);
+                store_act(re.kc, crow * re.d + ei + half, rb, false);
+              }
+            } else {
+#pragma unroll
+              for (int r = 0; r < 2; ++r) {
+                const int ev = nbase - QD - KD + r * 16 + rin;
+                const size_t crow = (((size_t)sl * re.n_layers + re.layer) * re.Hkv + ev / re.d) * re.cap + p;
+                store_act(re.vc, crow * re.d + ev % re.d, acc[r][nt][i], false);
+              }
+            }
+          }
+        continue;
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      if (nt >= ntv || nt % C::KS != kp) continue;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int m = mt * GEMM_BM + tok0 + nt * 8 + 2 * t4 + (i & 1);
+        const int m = mt * GEMM_BM + nt * 8 + 2 * t4 + (i & 1);
         if (m >= Me) continue;
         const int rin = g8 + (i >> 1) * 8;
         if (splits > 1) {  // FAST variant: raw fp32 partial of this split
@@ -266,43 +401,13 @@ __global__ void __launch_bounds__(160, 1)
         } else if constexpr (EPI == BI_EPI_SWIGLU) {
           const int col = (nbase >> 1) + rin;  // 32-row block -> 16 output columns
           store_act(y, (size_t)m * ldy + col, silu(acc[0][nt][i]) * acc[1][nt][i], y_f32);
-        } else if constexpr (EPI == EPI_ROPE) {
-          const int p = re.pos[m], sl = re.slot[m];
-          if (p < 0 || p >= re.cap || p >= re.table_max_pos || sl < 0 || sl >= re.n_slots) {
-            dev_flag(DEVERR_CAPACITY);
-            continue;
-          }
-          const int QD = re.Hq * re.d, KD = re.Hkv * re.d, half = re.d >> 1;
-          if (nbase < QD + KD) {
-            const bool isq = nbase < QD;
-            const int rel = isq ? nbase : nbase - QD;
-            const int head = rel / re.d, ei = ((rel % re.d) >> 1) + rin;  // first-half element 16b + rin
-            const float xa = acc[0][nt][i], xb = acc[1][nt][i];
-            const float cs = re.table[(size_t)p * re.d + 2 * ei], sn = re.table[(size_t)p * re.d + 2 * ei + 1];
-            const float ra = xa * cs - xb * sn;
-            const float rb = xb * cs + xa * sn;
-            if (isq) {
-              store_act(re.q_out, (size_t)m * QD + head * re.d + ei, ra, false);
-              store_act(re.q_out, (size_t)m * QD + head * re.d + ei + half, rb, false);
-            } else {
-              const size_t crow = (((size_t)sl * re.n_layers + re.layer) * re.Hkv + head) * re.cap + p;
-              store_act(re.kc, crow * re.d + ei, ra, false);
-              store_act(re.kc, crow * re.d + ei + half, rb, false);
-            }
-          } else {
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              const int ev = nbase - QD - KD + r * 16 + rin;
-              const size_t crow = (((size_t)sl * re.n_layers + re.layer) * re.Hkv + ev / re.d) * re.cap + p;
-              store_act(re.vc, crow * re.d + ev % re.d, acc[r][nt][i], false);
-            }
-          }
         } else {
 #pragma unroll
           for (int r = 0; r < 2; ++r) store_act(y, (size_t)m * ldy + nbase + r * 16 + rin, acc[r][nt][i], y_f32);
         }
       }
     }
+    }  // token tiles of the item
   }
 }
 
@@ -475,24 +580,29 @@ size_t gemm_ws_bytes(int M, int N, int K, int mode, int variant) {
   return s > 1 ? (size_t)s * M * N * sizeof(float) : 0;
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, int MT = 1>
 static int launch_gemm_bf16_t(const CUtensorMap& tw, const CUtensorMap& tx, void* y, int ldy, int y_f32, int M, int N,
                               int K, int splits, float* partial, const int* mcount, int mmult, const RopeEpi& re,
                               cudaStream_t st) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, MT>;
   static bool attr_done = false;  // per instantiation; set once per process
   if (!attr_done) {
-    BI_CHECK_CUDA(cudaFuncSetAttribute(gemm_bf16_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    BI_CHECK_CUDA(cudaFuncSetAttribute(gemm_bf16_kernel<BN, EPI, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM));
     attr_done = true;
   }
   const int m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
   const int n_groups = N / BN;
-  const int items = splits * n_groups * m_tiles;
+  const int items = splits * n_groups * ((m_tiles + MT - 1) / MT);
   const int grid = items < num_sms() ? items : num_sms();
-  BI_TRY(launch(gemm_bf16_kernel<BN, EPI>, dim3(grid), dim3(160), C::SMEM, st, tw, tx, y, ldy, y_f32, M, N, K, m_tiles, n_groups, splits,
-                                                         partial, mcount, mmult, re));
+  BI_TRY(launch(gemm_bf16_kernel<BN, EPI, MT>, dim3(grid), dim3(160), C::SMEM, st, tw, tx, y, ldy, y_f32, M, N, K,
+                m_tiles, n_groups, splits, partial, mcount, mmult, re));
   return BI_OK;
 }
+
+// Token tiles per weight stage: 4 for 128-row weight tiles once M spans four
+// token tiles (prefill: the weight is then read once per 128 token rows), else 1.
+static int gemm_pick_mt(int bn, int M) { return bn == 128 && M >= 4 * GEMM_BM ? 4 : 1; }
 
 // mcount (optional, device int): only rows < *mcount * mmult of x are computed.
 int gemm_bf16(const void* x, int ldx, const void* w, void* y, int ldy, int y_f32, int M, int N, int K, int epi,
@@ -510,7 +620,8 @@ int gemm_bf16(const void* x, int ldx, const void* w, void* y, int ldy, int y_f32
   BI_TRY(encode_tmap_3d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, dw, sw, bw, CU_TENSOR_MAP_SWIZZLE_128B));
   const uint64_t dx[3] = {(uint64_t)GEMM_BK, (uint64_t)M, (uint64_t)(K / GEMM_BK)};
   const uint64_t sx[2] = {(uint64_t)ldx * 2, (uint64_t)GEMM_BK * 2};
-  const uint32_t bx[3] = {(uint32_t)GEMM_BK, (uint32_t)GEMM_BM, (uint32_t)kbs};
+  const int mt = gemm_pick_mt(bn, M);
+  const uint32_t bx[3] = {(uint32_t)GEMM_BK, (uint32_t)(GEMM_BM * mt), (uint32_t)kbs};
   BI_TRY(encode_tmap_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_128B));
   int splits = 1;
   if (variant == BI_VARIANT_FAST) {
@@ -529,18 +640,19 @@ int gemm_bf16(const void* x, int ldx, const void* w, void* y, int ldy, int y_f32
     BI_TRY((launch_gemm_bf16_t<32, EPI_ROPE>(tw, tx, y, ldy, y_f32, M, N, K, 1, nullptr, mcount, mmult, re, st)));
     return BI_OK;
   }
-#define BI_GEMM_CASE(BNV)                                                                                      \
-  if (bn == BNV) {                                                                                             \
-    if (epi == BI_EPI_SWIGLU)                                                                                  \
-      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_SWIGLU>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, mcount,  \
-                                                     mmult, re, st)));                                         \
-    else                                                                                                       \
-      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_NONE>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, mcount,    \
-                                                   mmult, re, st)));                                           \
+#define BI_GEMM_CASE(BNV, MTV)                                                                                  \
+  if (bn == BNV && mt == MTV) {                                                                                 \
+    if (epi == BI_EPI_SWIGLU)                                                                                   \
+      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_SWIGLU, MTV>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, mcount, \
+                                                          mmult, re, st)));                                     \
+    else                                                                                                        \
+      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_NONE, MTV>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, mcount,   \
+                                                        mmult, re, st)));                                       \
   }
-  BI_GEMM_CASE(32)
-  BI_GEMM_CASE(64)
-  BI_GEMM_CASE(128)
+  BI_GEMM_CASE(32, 1)
+  BI_GEMM_CASE(64, 1)
+  BI_GEMM_CASE(128, 1)
+  BI_GEMM_CASE(128, 4)
 #undef BI_GEMM_CASE
   if (splits > 1) {
     const int n_out = epi == BI_EPI_SWIGLU ? N / 2 : N;

@@ -82,27 +82,46 @@ static int attn_set_smem_attrs() {
                                      (int)atc_smem_bytes(1, 4)));
   BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)atc_smem_bytes(2, 4)));
-  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)atc_smem_bytes(2, 2)));
+  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)atc_smem_bytes(4, 2)));
   done = true;
   return BI_OK;
 }
 
 // np: pairs per group of the CUDA-core kernel (LayerCast, or head_dim 64); the
 // bf16 head_dim-128 path runs on tensor cores with 16-row pair tiles.
-static int attn_launch(int np, const CUtensorMap& tk, const CUtensorMap& tv, const AttnPlan& plan, const AttnArgs& a,
-                       cudaStream_t st) {
-  const dim3 grid(plan.n, a.max_chunks, a.Hkv);
+//
+// Tensor-core kernel: a CTA walks a segment of consecutive chunks of one
+// (block, kv head).  With enough (block, kv head) units to fill the GPU, one
+// segment spans all chunks and the CTA also merges (no merge launch);
+// otherwise the chunks are cut into segments so that about two CTAs per SM
+// run, and the merge kernel combines the partials.  Either way the chunk
+// partials and the merge are the same computations (work assignment only).
+// *merged reports whether this launch wrote the final outputs itself.
+static int attn_launch(int np, const CUtensorMap& tk, const CUtensorMap& tv, const AttnPlan& plan, AttnArgs a,
+                       cudaStream_t st, bool* merged) {
+  *merged = false;
   if (!a.f32 && a.d == 128) {
+    const int units = plan.n * a.Hkv;
+    const int target = 2 * num_sms();
+    int n_seg = units >= target / 2 ? 1 : std::min(a.max_chunks, (target + units - 1) / units);
+    a.seg_len = (a.max_chunks + n_seg - 1) / n_seg;
+    n_seg = (a.max_chunks + a.seg_len - 1) / a.seg_len;
+    a.merge_in_cta = n_seg == 1;
+    *merged = a.merge_in_cta != 0;
+    const dim3 grid(plan.n, n_seg, a.Hkv);
     const bool single = np <= 16;  // decode blocks: one token, G pairs
-    if (single && a.G <= 16)
+    if (single && a.G <= 8)
       BI_TRY(launch(attn_tc_kernel<1, 4>, grid, dim3(ATT_THREADS), atc_smem_bytes(1, 4), st, tk, tv, plan, a));
-    else if (single)
+    else if (single && a.G <= 16)
       BI_TRY(launch(attn_tc_kernel<2, 4>, grid, dim3(ATT_THREADS), atc_smem_bytes(2, 4), st, tk, tv, plan, a));
     else
-      BI_TRY(launch(attn_tc_kernel<2, 2>, grid, dim3(ATT_THREADS), atc_smem_bytes(2, 2), st, tk, tv, plan, a));
+      BI_TRY(launch(attn_tc_kernel<4, 2>, grid, dim3(ATT_THREADS), atc_smem_bytes(4, 2), st, tk, tv, plan, a));
     return BI_OK;
   }
+  a.seg_len = 1;
+  a.merge_in_cta = 0;
+  const dim3 grid(plan.n, a.max_chunks, a.Hkv);
   const size_t smem = att_smem_bytes(np, a.d, a.f32);
   switch (np) {
     case 4: BI_TRY(launch(attn_partial_kernel<4>, dim3(grid), dim3(ATT_THREADS), smem, st, tk, tv, plan, a)); break;
@@ -197,42 +216,58 @@ static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const
     a.q = q; a.slot = slot; a.pos = pos; a.part = part; a.t_base = t_base;
     a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.d = d; a.chunk = chunk; a.max_chunks = max_chunks;
     a.layer = layer; a.n_layers = kv->n_layers; a.cap = kv->capacity; a.f32 = f32; a.scale = scale;
-    if (p1.n) BI_TRY(attn_launch(np1, tk, tv, p1, a, st));
-    if (pm.n) BI_TRY(attn_launch(ATT_MAX_PAIRS, tk, tv, pm, a, st));
-    const int nw = (t_end - t_base) * Hq;
-    BI_TRY(launch(attn_merge_kernel, dim3((nw * 32 + 255) / 256), dim3(256), 0, st, part, pos, out, t_base, t_end - t_base, Hq, d, chunk,
-                                                              max_chunks, f32));
+    a.out = out;
+    bool m1 = true, mm = true;
+    if (p1.n) BI_TRY(attn_launch(np1, tk, tv, p1, a, st, &m1));
+    if (pm.n) BI_TRY(attn_launch(ATT_MAX_PAIRS, tk, tv, pm, a, st, &mm));
+    if (!(m1 && mm)) {  // merges every token of the group (rewriting merged ones with the same bits)
+      const int nw = (t_end - t_base) * Hq;
+      BI_TRY(launch(attn_merge_kernel, dim3((nw * 32 + 255) / 256), dim3(256), 0, st, part, pos, out, t_base,
+                    t_end - t_base, Hq, d, chunk, max_chunks, f32));
+    }
     bi0 = bi1;
   }
   return BI_OK;
 }
 
 // ------------------------------------------------------------------ LM head
+// LM-head recompute layouts.  One pass (B <= LM_ONE_PASS_ROWS): the GEMM runs
+// over 3B rows -- bf16(h) then the two exact residual parts of every row --
+// which fit one 32-row token tile, so W is read once and the flagged rows'
+// FP32 logits come for free.  Two passes (larger B): the main GEMM over B
+// rows, then one more pass over W for the two residual parts of the flagged
+// rows only (none when no row is flagged); the part bf16(h) is the main
+// pass's.  Both compute every logit with the same per-row arithmetic.
+constexpr int LM_ONE_PASS_ROWS = 10;
 struct LmWs {
-  uint16_t* h16;
-  float* logits;
+  uint16_t* hs;     // bf16 GEMM input: [B][H], or [3B][H] in the one-pass layout
+  float* logits;    // [B or 3B][V] (LayerCast: [B][V] unless the caller's buffer is used)
   LmPart* part;
   uint8_t* flag;
   int32_t* list;
   int* count;
-  uint16_t* hc3;   // [3B][H] exact bf16 parts of the flagged rows
-  float* logits_c;  // [3B][V] partial logits of the parts
+  uint16_t* hc2;    // two-pass: [2B][H] residual parts p1, p2 of the flagged rows
+  float* logits_c;  // two-pass: [2B][V] their logits
 };
-static LmWs lm_carve(Carver& cv, int B, int H, int V, int mode, bool own_logits) {
+// parts: 3 in bf16 mode with the recompute enabled, else 1
+static LmWs lm_carve(Carver& cv, int B, int H, int V, int mode, bool own_logits, int parts) {
   const int nch = (V + LM_CHUNK - 1) / LM_CHUNK;
   LmWs w{};
-  w.h16 = mode == BI_MODE_BF16 ? cv.take<uint16_t>((size_t)B * H) : nullptr;
-  w.logits = own_logits ? cv.take<float>((size_t)B * V) : nullptr;
+  const bool bf = mode == BI_MODE_BF16;
+  const int rows = (bf && parts == 3 && B <= LM_ONE_PASS_ROWS) ? 3 * B : B;
+  w.hs = bf ? cv.take<uint16_t>((size_t)rows * H) : nullptr;
+  w.logits = (bf || own_logits) ? cv.take<float>((size_t)(bf ? rows : B) * V) : nullptr;
   w.part = cv.take<LmPart>((size_t)B * nch);
   w.flag = cv.take<uint8_t>(B);
   w.list = cv.take<int32_t>(B);
   w.count = cv.take<int>(1);
-  if (mode == BI_MODE_BF16) {
-    w.hc3 = cv.take<uint16_t>((size_t)3 * B * H);
-    w.logits_c = cv.take<float>((size_t)3 * B * V);
+  if (bf && parts == 3 && B > LM_ONE_PASS_ROWS) {
+    w.hc2 = cv.take<uint16_t>((size_t)2 * B * H);
+    w.logits_c = cv.take<float>((size_t)2 * B * V);
   }
   return w;
 }
+static int lm_parts(int mode, float thresh) { return mode == BI_MODE_BF16 && thresh > 0.f ? 3 : 1; }
 
 static int lmhead_run(const float* h, const void* W, const int32_t* target, int B, int H, int V, float thresh, int mode,
                       float* logprob, float* lse, int32_t* argmax, float* margin, uint8_t* recomputed, float* logits,
@@ -244,36 +279,52 @@ static int lmhead_run(const float* h, const void* W, const int32_t* target, int 
   BI_REQUIRE(mode == BI_MODE_BF16 || mode == BI_MODE_LAYERCAST, BI_ERR_INVALID_ARG, "bi_lmhead_logprob: bad mode");
   BI_REQUIRE(aligned16(h) && aligned16(W), BI_ERR_UNSUPPORTED, "bi_lmhead_logprob: h and W must be 16-byte aligned");
   if (B == 0) return BI_OK;
+  const int parts = lm_parts(mode, thresh);
   Carver probe(nullptr);
-  lm_carve(probe, B, H, V, mode, logits == nullptr);
+  lm_carve(probe, B, H, V, mode, logits == nullptr, parts);
   BI_REQUIRE(ws && ws_bytes >= probe.used + 256, BI_ERR_WORKSPACE, "bi_lmhead_logprob: workspace %zu < %zu", ws_bytes,
              probe.used + 256);
   Carver cv(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255)));
-  LmWs w = lm_carve(cv, B, H, V, mode, logits == nullptr);
-  float* z = logits ? logits : w.logits;
+  LmWs w = lm_carve(cv, B, H, V, mode, logits == nullptr, parts);
   const int nch = (V + LM_CHUNK - 1) / LM_CHUNK;
-
+  const bool one_pass = parts == 3 && B <= LM_ONE_PASS_ROWS;
+  float* z;
   if (mode == BI_MODE_BF16) {
+    // One pass over W: rows 0..B-1 of the GEMM input are bf16(h) (the main
+    // pass); with the recompute enabled, rows B..3B-1 hold the exact split
+    // parts, whose logits are combined ((z0 + z1) + z2) only for flagged rows.
     const size_t n = (size_t)B * H;
-    BI_TRY(launch(f32_to_bf16_kernel, dim3((int)std::min<size_t>((n + 255) / 256, 4096)), dim3(256), 0, st, h, w.h16, n));
-    BI_TRY(gemm_bf16(w.h16, H, W, z, V, 1, B, V, H, BI_EPI_NONE, BI_VARIANT_INVARIANT, nullptr, 0, st));
+    const int sp = one_pass ? 3 : 1;
+    z = w.logits;
+    BI_TRY(launch(lm_split_kernel, dim3((int)std::min<size_t>((n + 255) / 256, 4096)), dim3(256), 0, st, h, w.hs, n,
+                  sp));
+    BI_TRY(gemm_bf16(w.hs, H, W, z, V, 1, sp * B, V, H, BI_EPI_NONE, BI_VARIANT_INVARIANT, nullptr, 0, st));
+    if (logits)
+      BI_CHECK_CUDA(cudaMemcpyAsync(logits, z, (size_t)B * V * sizeof(float), cudaMemcpyDeviceToDevice, st));
   } else {
+    z = logits ? logits : w.logits;
     BI_TRY(gemm_f32(h, H, W, z, V, 1, B, V, H, BI_EPI_NONE, nullptr, st));
   }
   BI_TRY(launch(lm_partial_kernel, dim3(dim3(nch, B)), dim3(LM_CHUNK), 0, st, z, V, V, target, nullptr, nullptr, w.part, nch,
-                1));
+                1, 0, nullptr));
   const float th = mode == BI_MODE_BF16 ? thresh : 0.f;
   BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, nullptr, nullptr, target, th, 0, logprob, lse,
                                                         argmax, margin, recomputed, w.flag));
-  if (mode == BI_MODE_BF16 && th > 0.f) {
-    // FP32 recompute of the flagged rows: h = p0 + p1 + p2 exactly (bf16 parts), so
-    // h.W^T = ((p0.W^T + p1.W^T) + p2.W^T) with exact products and fp32 accumulation
-    // on the tensor cores; one pass over W serves every flagged row.
-    BI_TRY(launch(lm_compact_kernel, dim3(B), dim3(256), 0, st, w.flag, B, h, H, w.list, w.count, w.hc3));
-    BI_TRY(gemm_bf16(w.hc3, H, W, w.logits_c, V, 1, 3 * B, V, H, BI_EPI_NONE, BI_VARIANT_INVARIANT, nullptr, 0, st,
-                     w.count, 3));
-    BI_TRY(launch(lm_partial_kernel, dim3(dim3(nch, B)), dim3(LM_CHUNK), 0, st, w.logits_c, V, V, target, w.list,
-                  w.count, w.part, nch, 3));
+  if (parts == 3) {
+    // FP32 logits of the flagged rows: h = p0 + p1 + p2 exactly (bf16 parts), so
+    // h.W^T = ((p0.W^T + p1.W^T) + p2.W^T) with exact products and fp32
+    // accumulation on the tensor cores.
+    if (one_pass) {  // already computed by the pass above
+      BI_TRY(launch(lm_compact_kernel, dim3(B), dim3(32), 0, st, w.flag, B, h, H, w.list, w.count, nullptr));
+      BI_TRY(launch(lm_partial_kernel, dim3(dim3(nch, B)), dim3(LM_CHUNK), 0, st, z, V, V, target, w.list, w.count,
+                    w.part, nch, 3, B, nullptr));
+    } else {  // one more pass over W for the flagged rows only (row count read on the device)
+      BI_TRY(launch(lm_compact_kernel, dim3(B), dim3(256), 0, st, w.flag, B, h, H, w.list, w.count, w.hc2));
+      BI_TRY(gemm_bf16(w.hc2, H, W, w.logits_c, V, 1, 2 * B, V, H, BI_EPI_NONE, BI_VARIANT_INVARIANT, nullptr, 0, st,
+                       w.count, 2));
+      BI_TRY(launch(lm_partial_kernel, dim3(dim3(nch, B)), dim3(LM_CHUNK), 0, st, z, V, V, target, w.list, w.count,
+                    w.part, nch, 3, 0, w.logits_c));
+    }
     BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, w.count, w.list, target, th, 1, logprob,
                                                           lse, argmax, margin, recomputed, nullptr));
   }
@@ -392,7 +443,7 @@ int bi_attention(const void* q, const bi_kv_layout* kv, int layer, const int32_t
 size_t bi_lmhead_workspace_size(int B, int H, int V, int mode) {
   if (B <= 0 || H <= 0 || V <= 0) return 0;
   Carver cv(nullptr);
-  lm_carve(cv, B, H, V, mode, true);
+  lm_carve(cv, B, H, V, mode, true, lm_parts(mode, 1.f));
   return cv.used + 256;
 }
 
@@ -612,7 +663,7 @@ int bi_lmhead_logprob_noalloc(const float* h, const void* W, const int32_t* targ
   BI_REQUIRE(B >= 0 && H > 0 && V > 0, BI_ERR_INVALID_ARG, "bi_lmhead_logprob_noalloc: bad sizes");
   if (B == 0) return BI_OK;
   Carver probe(nullptr);
-  lm_carve(probe, B, H, V, mode, logits == nullptr);
+  lm_carve(probe, B, H, V, mode, logits == nullptr, lm_parts(mode, margin_threshold));
   const size_t need = probe.used + 256;
   BI_REQUIRE(need <= (size_t)BI_NOALLOC_SCRATCH_BYTES, BI_ERR_WORKSPACE,
              "bi_lmhead_logprob_noalloc: B=%d H=%d V=%d needs %zu bytes of scratch, more than the fixed %d; "

@@ -53,7 +53,7 @@ __device__ __forceinline__ void lm_top2_warp(float& v1, int& i1, float& v2, int&
 __global__ void __launch_bounds__(LM_CHUNK)
     lm_partial_kernel(const float* __restrict__ logits, size_t ldz, int V, const int32_t* __restrict__ target,
                       const int32_t* __restrict__ rows_map, const int* __restrict__ count, LmPart* __restrict__ part,
-                      int n_chunks, int parts) {
+                      int n_chunks, int parts, int pstride, const float* __restrict__ parts_z) {
   pdl_wait();
   pdl_trigger();
   const int c = blockIdx.x, r = blockIdx.y;
@@ -63,10 +63,17 @@ __global__ void __launch_bounds__(LM_CHUNK)
   const bool ok = v < V;
   float z = -INFINITY;
   if (ok) {
-    if (parts == 3)
-      z = (logits[(size_t)(3 * r) * ldz + v] + logits[(size_t)(3 * r + 1) * ldz + v]) +
-          logits[(size_t)(3 * r + 2) * ldz + v];
-    else
+    if (parts == 3) {  // row r of the compacted list: (z0 + z1) + z2 of its row src
+      // z0 = logits row src (the main pass on p0 = bf16(h)); z1, z2 at rows
+      // src + pstride, src + 2 pstride of logits (one-pass layout, pstride > 0)
+      // or at rows 2r, 2r + 1 of parts (second pass, pstride == 0)
+      const size_t src = rows_map[r];
+      const float z0 = logits[src * ldz + v];
+      if (pstride > 0)
+        z = (z0 + logits[(src + pstride) * ldz + v]) + logits[(src + 2 * pstride) * ldz + v];
+      else
+        z = (z0 + parts_z[(size_t)(2 * r) * ldz + v]) + parts_z[(size_t)(2 * r + 1) * ldz + v];
+    } else
       z = logits[(size_t)r * ldz + v];
   }
   __shared__ float wm[LM_CHUNK / 32], ws[LM_CHUNK / 32], wv1[LM_CHUNK / 32], wv2[LM_CHUNK / 32];
@@ -170,18 +177,18 @@ __global__ void lm_merge_kernel(const LmPart* __restrict__ part, int n_chunks, i
   }
 }
 
-// Ascending compaction of the flagged rows: list[k] = k-th flagged row, and
-// that row's f32 hidden vector split exactly into three bf16 parts
-// h = p0 + p1 + p2 (p0 = bf16(h), p1 = bf16(h - p0), p2 = h - p0 - p1; 8 + 8 + 8
-// significant bits cover the 24 of an f32), stored as rows 3k, 3k+1, 3k+2 of
-// hc3.  CTA b handles row b: its rank is the number of flagged rows before it;
-// CTA 0 also writes the count.
+// Ascending compaction of the flagged rows: list[k] = k-th flagged row.  CTA
+// b handles row b: its rank is the number of flagged rows before it; CTA 0
+// also writes the count.  With hc2 != nullptr (second-pass recompute) the
+// row's f32 h is also split exactly into three bf16 parts (see
+// lm_split_kernel); p1 and p2 are stored as rows 2k, 2k+1 of hc2 (the logits
+// of p0 = bf16(h) are the main pass's).
 __global__ void lm_compact_kernel(const uint8_t* __restrict__ flag, int B, const float* __restrict__ h, int H,
-                                  int32_t* __restrict__ list, int* __restrict__ count, uint16_t* __restrict__ hc3) {
+                                  int32_t* __restrict__ list, int* __restrict__ count, uint16_t* __restrict__ hc2) {
   pdl_wait();
   pdl_trigger();
   const int b = blockIdx.x;
-  __shared__ int rank_s, total_s;
+  __shared__ int rank_s;
   if (threadIdx.x < 32) {
     int before = 0, total = 0;
     for (int i = threadIdx.x; i < B; i += 32) {
@@ -196,32 +203,45 @@ __global__ void lm_compact_kernel(const uint8_t* __restrict__ flag, int B, const
     }
     if (threadIdx.x == 0) {
       rank_s = before;
-      total_s = total;
+      if (b == 0) *count = total;
+      if (flag[b]) list[before] = b;
     }
   }
   __syncthreads();
-  if (b == 0 && threadIdx.x == 0) *count = total_s;
-  if (!flag[b]) return;
+  if (!hc2 || !flag[b]) return;
   const int k = rank_s;
-  if (threadIdx.x == 0) list[k] = b;
   for (int i = threadIdx.x; i < H; i += blockDim.x) {
     const float v = h[(size_t)b * H + i];
     const uint16_t p0 = f32_to_bf16_bits(v);
     const float r0 = v - bf16_bits_to_f32(p0);  // exact
     const uint16_t p1 = f32_to_bf16_bits(r0);
     const float r1 = r0 - bf16_bits_to_f32(p1);  // exact, at most 8 significant bits
-    hc3[(size_t)(3 * k) * H + i] = p0;
-    hc3[(size_t)(3 * k + 1) * H + i] = p1;
-    hc3[(size_t)(3 * k + 2) * H + i] = f32_to_bf16_bits(r1);
+    hc2[(size_t)(2 * k) * H + i] = p1;
+    hc2[(size_t)(2 * k + 1) * H + i] = f32_to_bf16_bits(r1);
   }
 }
 
-// h (f32) -> bf16 (round to nearest even), the main-pass LM-head input.
-__global__ void f32_to_bf16_kernel(const float* __restrict__ in, uint16_t* __restrict__ out, size_t n) {
+// LM-head GEMM input.  parts == 1: row r of out is bf16(h_r) (round to nearest
+// even).  parts == 3: h is also split exactly into three bf16 parts
+// h = p0 + p1 + p2 (p0 = bf16(h), p1 = bf16(h - p0), p2 = h - p0 - p1; 8 + 8 + 8
+// significant bits cover the 24 of an f32), stored as rows r, B + r and
+// 2B + r, so one GEMM pass over W yields both the bf16-path logits (rows
+// 0..B-1) and the parts of the FP32 logits of every row.
+__global__ void lm_split_kernel(const float* __restrict__ h, uint16_t* __restrict__ out, size_t n, int parts) {
   pdl_wait();
   pdl_trigger();
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
-    out[i] = f32_to_bf16_bits(in[i]);
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const float v = h[i];
+    const uint16_t p0 = f32_to_bf16_bits(v);
+    out[i] = p0;
+    if (parts == 3) {
+      const float r0 = v - bf16_bits_to_f32(p0);  // exact
+      const uint16_t p1 = f32_to_bf16_bits(r0);
+      const float r1 = r0 - bf16_bits_to_f32(p1);  // exact, at most 8 significant bits
+      out[n + i] = p1;
+      out[2 * n + i] = f32_to_bf16_bits(r1);
+    }
+  }
 }
 
 }  // namespace bi

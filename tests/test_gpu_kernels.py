@@ -143,6 +143,21 @@ def test_gemm_batch_invariance(bi, mode):
     _after(bi)
 
 
+@pytest.mark.parametrize("epilogue", [0, 1])
+def test_gemm_m_blocking_invariance(bi, epilogue):
+    """128-row weight tiles stream each weight stage to four token tiles once M > 32 (M-blocking): a row's
+    bits must not depend on which launch shape (one tile or a 128-row group, which slot in it) computed it."""
+    rng = np.random.default_rng(15 + epilogue)
+    N, K = 8448, 320
+    xs = synth.bf16_to_f32(synth.f32_to_bf16_bits(rng.standard_normal((300, K)).astype(np.float32)))
+    w = _bf16_dev(0.02 * rng.standard_normal((N, K)))
+    full = bi.gemm(_bf16_dev(xs), w, epilogue=epilogue, out_dtype=torch.float32).cpu()
+    for M, off in [(1, 0), (1, 299), (31, 5), (32, 100), (33, 17), (96, 3), (128, 150), (129, 40)]:
+        part = bi.gemm(_bf16_dev(xs[off:off + M]), w, epilogue=epilogue, out_dtype=torch.float32).cpu()
+        assert torch.equal(part, full[off:off + M]), (M, off)
+    _after(bi)
+
+
 def test_gemm_fast_variant_is_not_invariant_but_close(bi):
     rng = np.random.default_rng(6)
     N, K = 4096, 4096
@@ -261,6 +276,37 @@ def test_attention_invariance_decode_vs_prefill(bi, mode):
     _after(bi)
 
 
+def test_attention_invariance_across_work_splits(bi):
+    """The tensor-core kernel cuts each (query block, kv head)'s chunks into segments by how many units a launch
+    has: one segment merged inside the CTA (large decode batches), one chunk per CTA (a token alone) and
+    multi-chunk segments (a few tokens at long context).  All must give the same bits, also against the oracle."""
+    Hq, Hkv, d, cap, n = 32, 8, 128, 3072, 24
+    kv, k, v = _make_cache(bi, 0, n, Hkv, cap, d, cap, seed=21)
+    rng = np.random.default_rng(22)
+    q = torch.from_numpy(rng.standard_normal((n, Hq * d)).astype(np.float32)).cuda().to(torch.bfloat16)
+    slots = np.arange(n, dtype=np.int32)
+    pos = np.concatenate([[cap - 1, 0, 255, 256, 2047], rng.integers(0, cap, n - 5)]).astype(np.int32)
+    scale = np.float32(1.0 / math.sqrt(d))
+    run = lambda idx: bi.attention(q[idx].contiguous(), kv, 0, torch.from_numpy(slots[idx]).cuda(),
+                                   torch.from_numpy(pos[idx]).cuda(), slots[idx], pos[idx], Hq, scale).cpu()
+    full = run(np.arange(n))                  # 192 units: one segment per CTA, merged in the CTA
+    four = run(np.arange(4))                  # 32 units: segments of several chunks
+    for i in range(n):
+        alone = run(np.array([i]))            # 8 units: one chunk per CTA
+        assert torch.equal(alone[0], full[i]), i
+        if i < 4:
+            assert torch.equal(four[i], full[i]), i
+    qf = _f(q)
+    out = _f(full)
+    for t in (0, 3, 4):
+        for h in (0, 17):
+            ref = oracle.attention_query(qf[t, h * d:(h + 1) * d], k[slots[t], 0, h // 4, :pos[t] + 1],
+                                         v[slots[t], 0, h // 4, :pos[t] + 1], float(scale))
+            tol = 2e-5 * np.abs(v[slots[t], 0, h // 4]).max() + 2 ** -8 * np.abs(ref)
+            assert (np.abs(out[t, h * d:(h + 1) * d] - ref) <= tol).all(), (t, h)
+    _after(bi)
+
+
 # ------------------------------------------------------------------ LM head
 def _h_rows(B, H, seed=7):
     return synth.hidden_states(seed, B, H)
@@ -309,7 +355,7 @@ def test_lmhead_full_size_invariance_and_samples(bi):
     h = _h_rows(256, H)
     hd = torch.from_numpy(h).cuda()
     ref = {k: v.cpu() for k, v in bi.lmhead_logprob(hd, W, None, 0.1).items()}
-    for B in (1, 2, 4, 8, 16, 32, 64, 128):
+    for B in (1, 2, 4, 8, 10, 11, 16, 32, 64, 128):  # one-pass recompute up to 10 rows, two passes above
         for off in (0, 256 - B):
             o = bi.lmhead_logprob(hd[off:off + B].contiguous(), W, None, 0.1)
             for k in ("logprob", "lse", "argmax", "margin", "recomputed"):
