@@ -74,6 +74,9 @@ int bi_version(void);
 /* Device error word: kernels never trap; a bounded wait that runs out, a
  * position beyond capacity or an out-of-range id sets a bit here instead
  * (1 = wait timeout, 2 = capacity, 4 = index) and the kernel skips the access.
+ * Bits 8 and up name the first wait that ran out (a site code of the kernel:
+ * 0x11/0x12/0x13 GEMM ring empty/full/drain, 0x21/0x22 attention; higher bits
+ * carry the kernel's configuration), 0 when none did.
  * Synchronous read of the current device's word; reset != 0 clears it. */
 int bi_device_error(unsigned* flags, int reset);
 int bi_num_sms(int device); /* SM count of a device, -1 on error */

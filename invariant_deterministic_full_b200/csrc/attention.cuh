@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(ATT_THREADS)
   if (tid == 0)
     for (int L = 0; L < ATT_RING && L < total_loads; ++L) issue(L);
   int L = 0;  // next load to consume
-  auto consume_wait = [&]() -> bool { return mbar_wait(&bar[L % ATT_RING], (uint32_t)((L / ATT_RING) & 1)); };
+  auto consume_wait = [&]() -> bool { return mbar_wait(&bar[L % ATT_RING], (uint32_t)((L / ATT_RING) & 1), SITE_ATTN_CORE); };
   auto release = [&]() {  // every thread is done with load L: refill its buffer
     __syncthreads();
     if (tid == 0 && L + ATT_RING < total_loads) issue(L + ATT_RING);
@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(ATT_THREADS)
   if (tid == 0)
     for (int r = 0; r < RING; ++r) issue_next();
   int L = 0;
-  auto consume_wait = [&]() -> bool { return mbar_wait(&bar[L % RING], (uint32_t)((L / RING) & 1)); };
+  auto consume_wait = [&]() -> bool { return mbar_wait(&bar[L % RING], (uint32_t)((L / RING) & 1), SITE_ATTN_TC | (NPT << 8)); };
   auto release = [&]() {
     __syncthreads();
     if (tid == 0) issue_next();

@@ -68,6 +68,7 @@ int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStrea
 // bounded wait runs out or an index fails its check.
 enum : unsigned { DEVERR_TIMEOUT = 1u, DEVERR_CAPACITY = 2u, DEVERR_INDEX = 4u };
 __device__ unsigned g_dev_error = 0;  // one translation unit: defined here
+__device__ unsigned g_dev_site = 0;   // site code of the first wait that ran out (0: none)
 __device__ __forceinline__ void dev_flag(unsigned bit) { atomicOr(&g_dev_error, bit); }
 
 // Tensor maps (TMA descriptors), encoded through the driver entry point.
@@ -115,12 +116,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // does not complete within the iteration limit (each try_wait suspends for a
 // hardware-chosen interval, so the limit is seconds, never forever).
 constexpr uint32_t kWaitLimit = 1u << 22;
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// site: which wait ran out, reported in bits 8..15 of bi_device_error's flags.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned site = 0) {
   for (uint32_t i = 0; i < kWaitLimit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   dev_flag(DEVERR_TIMEOUT);
+  atomicCAS(&g_dev_site, 0u, site);
   return false;
 }
+enum : unsigned {
+  SITE_GEMM_EMPTY = 0x11, SITE_GEMM_FULL = 0x12, SITE_GEMM_DRAIN = 0x13,
+  SITE_ATTN_CORE = 0x21, SITE_ATTN_TC = 0x22
+};
 
 // 2D tiled TMA load into shared memory, completion counted on an mbarrier.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int c_inner, int c_outer,

@@ -163,8 +163,16 @@ __global__ void __launch_bounds__(160, 1)
       pdl_trigger();
       // rows beyond a device-side count (selective recompute) are not computed
       const int Me = mcount ? min(M, *mcount * mmult) : M;
-      if (pre > 0 && Me <= 0) {  // nothing to compute: wait for the prefetched stages, then leave
-        for (int s = 0; s < pre; ++s) (void)mbar_wait(&full_bar[s], 0u);
+      if (pre > 0 && Me <= 0) {
+        // Nothing to compute.  Each prefetched stage's barrier also expects its
+        // token tile: load those (row 0 on, in bounds or zero-filled) so the
+        // barriers complete, wait for them, then leave.
+        int sp, g, mg;
+        decode_item(blockIdx.x, sp, g, mg);
+        for (int s = 0; s < pre; ++s)
+          tma_load_3d(smem + s * C::STAGE_BYTES + C::W_BYTES, &tmX, 0, 0, (sp * ks_per_split + s) * C::KBS,
+                      &full_bar[s]);
+        for (int s = 0; s < pre; ++s) (void)mbar_wait(&full_bar[s], 0u, SITE_GEMM_DRAIN);
         return;
       }
       int stage = 0;
@@ -180,7 +188,7 @@ __global__ void __launch_bounds__(160, 1)
         for (int ks = ks0; ks < ks1; ++ks) {
           uint8_t* sb = smem + stage * C::STAGE_BYTES;
           if (!(first && ks - ks0 < pre)) {
-            if (!mbar_wait(&empty_bar[stage], phase ^ 1)) return;
+            if (!mbar_wait(&empty_bar[stage], phase ^ 1, SITE_GEMM_EMPTY | (EPI << 12))) return;
             mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
             tma_load_3d(sb, &tmW, 0, g * BN, ks * C::KBS, &full_bar[stage]);
           }
@@ -231,7 +239,7 @@ __global__ void __launch_bounds__(160, 1)
           for (int c = 0; c < 4; ++c) accm[j][a][b][c] = 0.f;
 
     for (int ks = ks0; ks < ks1; ++ks) {
-      if (!dead && !mbar_wait(&full_bar[stage], phase)) dead = true;
+      if (!dead && !mbar_wait(&full_bar[stage], phase, SITE_GEMM_FULL | (EPI << 12))) dead = true;
       const uint32_t sbase = smem_u32(smem + stage * C::STAGE_BYTES);
 #pragma unroll
       for (int kb = 0; kb < C::KBS && !dead; ++kb) {

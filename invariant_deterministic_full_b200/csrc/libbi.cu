@@ -305,7 +305,7 @@ static int lmhead_run(const float* h, const void* W, const int32_t* target, int 
     z = logits ? logits : w.logits;
     BI_TRY(gemm_f32(h, H, W, z, V, 1, B, V, H, BI_EPI_NONE, nullptr, st));
   }
-  BI_TRY(launch(lm_partial_kernel, dim3(dim3(nch, B)), dim3(LM_CHUNK), 0, st, z, V, V, target, nullptr, nullptr, w.part, nch,
+  BI_TRY(launch(lm_partial_kernel, dim3(dim3((nch + LM_CPB - 1) / LM_CPB, B)), dim3(32 * LM_CPB), 0, st, z, V, V, target, nullptr, nullptr, w.part, nch,
                 1, 0, nullptr));
   const float th = mode == BI_MODE_BF16 ? thresh : 0.f;
   BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, nullptr, nullptr, target, th, 0, logprob, lse,
@@ -316,13 +316,13 @@ static int lmhead_run(const float* h, const void* W, const int32_t* target, int 
     // accumulation on the tensor cores.
     if (one_pass) {  // already computed by the pass above
       BI_TRY(launch(lm_compact_kernel, dim3(B), dim3(32), 0, st, w.flag, B, h, H, w.list, w.count, nullptr));
-      BI_TRY(launch(lm_partial_kernel, dim3(dim3(nch, B)), dim3(LM_CHUNK), 0, st, z, V, V, target, w.list, w.count,
+      BI_TRY(launch(lm_partial_kernel, dim3(dim3((nch + LM_CPB - 1) / LM_CPB, B)), dim3(32 * LM_CPB), 0, st, z, V, V, target, w.list, w.count,
                     w.part, nch, 3, B, nullptr));
     } else {  // one more pass over W for the flagged rows only (row count read on the device)
       BI_TRY(launch(lm_compact_kernel, dim3(B), dim3(256), 0, st, w.flag, B, h, H, w.list, w.count, w.hc2));
       BI_TRY(gemm_bf16(w.hc2, H, W, w.logits_c, V, 1, 2 * B, V, H, BI_EPI_NONE, BI_VARIANT_INVARIANT, nullptr, 0, st,
                        w.count, 2));
-      BI_TRY(launch(lm_partial_kernel, dim3(dim3(nch, B)), dim3(LM_CHUNK), 0, st, z, V, V, target, w.list, w.count,
+      BI_TRY(launch(lm_partial_kernel, dim3(dim3((nch + LM_CPB - 1) / LM_CPB, B)), dim3(32 * LM_CPB), 0, st, z, V, V, target, w.list, w.count,
                     w.part, nch, 3, 0, w.logits_c));
     }
     BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, w.count, w.list, target, th, 1, logprob,
@@ -354,12 +354,14 @@ int bi_num_sms(int device) {
 }
 
 int bi_device_error(unsigned* flags, int reset) {
-  unsigned v = 0;
+  unsigned v = 0, site = 0;
   BI_CHECK_CUDA(cudaMemcpyFromSymbol(&v, g_dev_error, sizeof(v)));
-  if (flags) *flags = v;
+  BI_CHECK_CUDA(cudaMemcpyFromSymbol(&site, g_dev_site, sizeof(site)));
+  if (flags) *flags = (v & 0xffu) | (site << 8);
   if (reset) {
     unsigned z = 0;
     BI_CHECK_CUDA(cudaMemcpyToSymbol(g_dev_error, &z, sizeof(z)));
+    BI_CHECK_CUDA(cudaMemcpyToSymbol(g_dev_site, &z, sizeof(z)));
   }
   return BI_OK;
 }

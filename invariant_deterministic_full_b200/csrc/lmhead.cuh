@@ -6,11 +6,12 @@
 // Precision-Invariant", method section: top-two logit margin, FP32 LM-head
 // recompute only when it falls below a threshold.)
 //
-// Per row and per chunk of BI_VOCAB_CHUNK = 256 logits (thread j <-> logit j):
-//   max (exact), sum exp(z - max) with a fixed tree (xor-butterfly per warp,
-//   then the 8 warp sums in ascending order), top-1 and top-2 as (value, id)
-//   under the total order "larger value, then lower id" (exact, order-free),
-//   and the target logit if the target falls in the chunk.
+// Per row and per chunk of BI_VOCAB_CHUNK = 256 logits, one warp (lane l holds
+// logits l, l + 32, ..., l + 224 of the chunk): max (exact), sum exp(z - max)
+// with a fixed tree (each lane's 8 terms in ascending order, then an xor
+// butterfly), top-1 and top-2 as (value, id) under the total order "larger
+// value, then lower id" (exact, order-free), and the target logit if the
+// target falls in the chunk.
 // Merge per row: M = max over chunks (exact); S = sum_c s_c exp(m_c - M):
 //   lane i of one warp sums chunks i, i+32, ... in ascending order, then a
 //   fixed xor-butterfly; lse = M + ln S; top-2 merged exactly.
@@ -44,79 +45,78 @@ __device__ __forceinline__ void lm_top2_warp(float& v1, int& i1, float& v2, int&
   }
 }
 
-// Grid (n_chunks, B).  logits: [rows][ldz] f32.  Row r of the grid is
-// logits row r; rows >= *count (when count != nullptr) are skipped.
-// target: per-row target id (nullptr: none); rows_map maps grid row -> target
-// row (nullptr: identity).
-// parts == 3: the logit of row r is (z[3r] + z[3r+1]) + z[3r+2], the three
-// partial products of the exact bf16 split of an f32 hidden row.
-__global__ void __launch_bounds__(LM_CHUNK)
+// Grid (ceil(n_chunks / LM_CPB), B), LM_CPB warps per CTA, warp w taking
+// chunk blockIdx.x * LM_CPB + w of grid row blockIdx.y.  logits: [rows][ldz]
+// f32.  Row r of the grid is logits row r; rows >= *count (when count !=
+// nullptr) are skipped.  target: per-row target id (nullptr: none); rows_map
+// maps grid row -> target row (nullptr: identity).
+// parts == 3: the logit is (z0 + z1) + z2, the three partial products of the
+// exact bf16 split of an f32 hidden row (layouts below).
+constexpr int LM_CPB = 8;  // vocabulary chunks (warps) per CTA
+
+__global__ void __launch_bounds__(32 * LM_CPB)
     lm_partial_kernel(const float* __restrict__ logits, size_t ldz, int V, const int32_t* __restrict__ target,
                       const int32_t* __restrict__ rows_map, const int* __restrict__ count, LmPart* __restrict__ part,
                       int n_chunks, int parts, int pstride, const float* __restrict__ parts_z) {
   pdl_wait();
   pdl_trigger();
-  const int c = blockIdx.x, r = blockIdx.y;
+  const int r = blockIdx.y;
   if (count && r >= *count) return;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int v = c * LM_CHUNK + tid;
-  const bool ok = v < V;
-  float z = -INFINITY;
-  if (ok) {
-    if (parts == 3) {  // row r of the compacted list: (z0 + z1) + z2 of its row src
-      // z0 = logits row src (the main pass on p0 = bf16(h)); z1, z2 at rows
-      // src + pstride, src + 2 pstride of logits (one-pass layout, pstride > 0)
-      // or at rows 2r, 2r + 1 of parts (second pass, pstride == 0)
-      const size_t src = rows_map[r];
-      const float z0 = logits[src * ldz + v];
-      if (pstride > 0)
-        z = (z0 + logits[(src + pstride) * ldz + v]) + logits[(src + 2 * pstride) * ldz + v];
-      else
-        z = (z0 + parts_z[(size_t)(2 * r) * ldz + v]) + parts_z[(size_t)(2 * r + 1) * ldz + v];
-    } else
-      z = logits[(size_t)r * ldz + v];
-  }
-  __shared__ float wm[LM_CHUNK / 32], ws[LM_CHUNK / 32], wv1[LM_CHUNK / 32], wv2[LM_CHUNK / 32];
-  __shared__ int wi1[LM_CHUNK / 32], wi2[LM_CHUNK / 32];
-  __shared__ float zt_s;
-  __shared__ int has_s;
-  if (tid == 0) has_s = 0;
-  float mx = warp_max(z);
-  if (lane == 0) wm[warp] = mx;
-  float v1 = z, v2 = -INFINITY;
-  int i1 = ok ? v : 0x7fffffff, i2 = 0x7fffffff;
-  lm_top2_warp(v1, i1, v2, i2);
-  if (lane == 0) {
-    wv1[warp] = v1; wi1[warp] = i1; wv2[warp] = v2; wi2[warp] = i2;
-  }
-  __syncthreads();
-  float M = wm[0];
+  const int lane = threadIdx.x & 31;
+  const int c = blockIdx.x * LM_CPB + (threadIdx.x >> 5);
+  if (c >= n_chunks) return;
+  constexpr int PER = LM_CHUNK / 32;
+  float z[PER];
 #pragma unroll
-  for (int w = 1; w < LM_CHUNK / 32; ++w) M = fmaxf(M, wm[w]);
-  float e = ok ? expf(z - M) : 0.f;
-  e = warp_sum_fixed(e);
-  if (lane == 0) ws[warp] = e;
-  if (target) {
-    const int tr = rows_map ? rows_map[r] : r;
-    const int tg = target[tr];
-    if (ok && v == tg) {
-      zt_s = z;
-      has_s = 1;
+  for (int j = 0; j < PER; ++j) {
+    const int v = c * LM_CHUNK + lane + 32 * j;
+    float zv = -INFINITY;
+    if (v < V) {
+      if (parts == 3) {  // row r of the compacted list: (z0 + z1) + z2 of its row src
+        // z0 = logits row src (the main pass on p0 = bf16(h)); z1, z2 at rows
+        // src + pstride, src + 2 pstride of logits (one-pass layout, pstride > 0)
+        // or at rows 2r, 2r + 1 of parts (second pass, pstride == 0)
+        const size_t src = rows_map[r];
+        const float z0 = logits[src * ldz + v];
+        if (pstride > 0)
+          zv = (z0 + logits[(src + pstride) * ldz + v]) + logits[(src + 2 * pstride) * ldz + v];
+        else
+          zv = (z0 + parts_z[(size_t)(2 * r) * ldz + v]) + parts_z[(size_t)(2 * r + 1) * ldz + v];
+      } else {
+        zv = logits[(size_t)r * ldz + v];
+      }
+    }
+    z[j] = zv;
+  }
+  float mx = z[0];
+#pragma unroll
+  for (int j = 1; j < PER; ++j) mx = fmaxf(mx, z[j]);
+  const float M = warp_max(mx);
+  float v1 = -INFINITY, v2 = -INFINITY;
+  int i1 = 0x7fffffff, i2 = 0x7fffffff;
+  float e = 0.f, zt = 0.f;
+  int has = 0;
+  const int tg = target ? target[rows_map ? rows_map[r] : r] : -1;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const int v = c * LM_CHUNK + lane + 32 * j;
+    if (v < V) {
+      lm_top2_insert(v1, i1, v2, i2, z[j], v);
+      e += expf(z[j] - M);
+      if (v == tg) {
+        zt = z[j];
+        has = 1;
+      }
     }
   }
-  __syncthreads();
-  if (tid == 0) {
-    float S = 0.f;
-    for (int w = 0; w < LM_CHUNK / 32; ++w) S += ws[w];
-    float a1 = wv1[0], a2 = wv2[0];
-    int j1 = wi1[0], j2 = wi2[0];
-    for (int w = 1; w < LM_CHUNK / 32; ++w) {
-      lm_top2_insert(a1, j1, a2, j2, wv1[w], wi1[w]);
-      lm_top2_insert(a1, j1, a2, j2, wv2[w], wi2[w]);
-    }
+  const float S = warp_sum_fixed(e);
+  lm_top2_warp(v1, i1, v2, i2);
+  const unsigned hb = __ballot_sync(0xffffffffu, has);
+  zt = __shfl_sync(0xffffffffu, zt, hb ? __ffs(hb) - 1 : 0);
+  if (lane == 0) {
     LmPart pr;
-    pr.mx = M; pr.sum = S; pr.v1 = a1; pr.i1 = j1; pr.v2 = a2; pr.i2 = j2;
-    pr.has_t = has_s; pr.zt = has_s ? zt_s : 0.f;
+    pr.mx = M; pr.sum = S; pr.v1 = v1; pr.i1 = i1; pr.v2 = v2; pr.i2 = i2;
+    pr.has_t = hb != 0; pr.zt = hb ? zt : 0.f;
     part[(size_t)r * n_chunks + c] = pr;
   }
 }

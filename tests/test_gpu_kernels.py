@@ -346,6 +346,23 @@ def test_lmhead_vs_oracle_small_vocab(bi, mode):
     _after(bi)
 
 
+@pytest.mark.parametrize("B", [4, 24])  # one-pass and second-pass recompute layouts
+def test_lmhead_recompute_enabled_but_no_row_flagged(bi, B):
+    """With the recompute on but no row under the threshold, the second pass has a device-side row count of 0: it
+    must finish cleanly (no wait running out) and leave the main-pass results."""
+    H, V = 512, 4096
+    rng = np.random.default_rng(31)
+    W = _bf16_dev(0.02 * rng.standard_normal((V, H)))
+    hd = torch.from_numpy(_h_rows(B, H) * 4).cuda()
+    off = bi.lmhead_logprob(hd, W, None, threshold=0.0)
+    tiny = bi.lmhead_logprob(hd, W, None, threshold=1e-30)
+    torch.cuda.synchronize()
+    if int(tiny["recomputed"].sum()) == 0:
+        for k in ("logprob", "lse", "argmax", "margin"):
+            assert torch.equal(tiny[k], off[k]), k
+    _after(bi)
+
+
 def test_lmhead_full_size_invariance_and_samples(bi):
     """LM head alone at hidden 4096, vocab 128256: each row bitwise equal across batch 1..256."""
     H, V = 4096, 128256
