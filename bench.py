@@ -153,6 +153,30 @@ def step_bytes(cfg, B, ctx_lens, f32_kv=False):
     return w + B * H * 2 + kv
 
 
+# DRAM bytes (read + write) of the weight-streaming GEMM launches of one decode step at batch 32, from one ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum) of the same shapes on the 2-layer 8B-width case; the
+# per-layer figures scale to 32 layers (the weights per launch do not depend on the layer count).  Valid only for
+# the GEMM source that was captured, recognised by its SHA-256.
+GEMM_TRAFFIC = {"gemm_source_sha256": "de83f7b649dffd5be7d645cecaf8447a529282393c0be1c1ac6f1d4787707863",
+                "batch": 32, "per_layer_bytes": 438855680, "lm_head_bytes": 1066563328}
+
+
+def gemm_traffic_per_launch(cfg, B):
+    """Measured DRAM bytes per launch of the timed GEMM set, or None when they no longer apply."""
+    import hashlib
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "invariant_deterministic_full_b200", "csrc",
+                       "gemm.cuh")
+    try:
+        with open(src, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    if h != GEMM_TRAFFIC["gemm_source_sha256"] or B != GEMM_TRAFFIC["batch"] or cfg["hidden"] != 4096:
+        return None
+    L = cfg["n_layers"]
+    return (L * GEMM_TRAFFIC["per_layer_bytes"] + GEMM_TRAFFIC["lm_head_bytes"]) / (4 * L + 1)
+
+
 def gemm_bytes(cfg, B):
     """Algorithmic bytes of the weight-streaming GEMM launches of one bf16 decode step (weights + inputs + outputs)."""
     L, H, Hq, Hkv, d, F, V = (cfg["n_layers"], cfg["hidden"], cfg["n_heads"], cfg["n_kv_heads"], cfg["head_dim"],
@@ -250,7 +274,7 @@ def time_gemms(m, B, reps=3):
     L, H, F = cfg["n_layers"], cfg["hidden"], cfg["ffn"]
     QD = cfg["n_heads"] * cfg["head_dim"]
     x_h, x_q, x_f = (torch.randn(B, n, device=dev).to(torch.bfloat16) for n in (H, QD, F))
-    o_qkv = torch.empty(B, w["w_qkv"].shape[1], dtype=torch.float32, device=dev)
+    o_qkv = torch.empty(B, w["w_qkv"].shape[1], dtype=torch.bfloat16, device=dev)
     o_h = torch.empty(B, H, dtype=torch.bfloat16, device=dev)
     o_f = torch.empty(B, F, dtype=torch.bfloat16, device=dev)
     o_lm = torch.empty(B, cfg["vocab"], dtype=torch.float32, device=dev)
@@ -413,8 +437,11 @@ def main_ours(args):
         gms = time_gemms(m, B)
         gb, gl = gemm_bytes(cfg, B)
         ach = gb / (gms / 1e3) / 1e9
+        tr = gemm_traffic_per_launch(cfg, B)
         line["roofline"] = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
-                            "frac": round(ach / hbm, 4), "traffic": None,
+                            "frac": round(ach / hbm, 4), "traffic": round(tr) if tr else None,
+                            "traffic_note": "DRAM read+write bytes per launch (ncu, same GEMM shapes, 2-layer case "
+                                            "scaled to 32 layers)" if tr else "no capture for this GEMM source/batch",
                             "kernel": "gemm_bf16_kernel (weight-streaming mma.sync GEMM)",
                             "per_launch": f"{gb / gl / 1e6:.1f} MB algorithmic over {gl} launches, "
                                           f"{gms / gl * 1e3:.1f} us average",
@@ -427,15 +454,19 @@ def main_ours(args):
         line["e2e"] = {"value": round(B * min(K, 32) / (e["ms"] / 1e3) * ws, 2), "unit": "tok/s",
                        "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"]}
     # batch sweep and the non-invariant comparison (same weights)
-    extra = {}
+    extra, extra_frac = {}, {}
     for b in sweep:
         if b == B:
             extra[str(b)] = round(value / ws, 2)
+            extra_frac[str(b)] = round(step_frac, 4)
             continue
         rb = run_decode(m, b, P, min(K, 32), W, 1, rank)
         extra[str(b)] = round(b * min(K, 32) / (rb["ms"] / 1e3), 2)
+        bb = sum(step_bytes(cfg, b, [c] * b, f32_kv=(mode == 1)) for c in rb["ctx_lens"])
+        extra_frac[str(b)] = round(bb / (rb["ms"] / 1e3) / 1e9 / hbm, 4)
     if extra:
         line["sweep_tok_s_per_gpu"] = extra
+        line["sweep_hbm_roofline_frac"] = extra_frac
     if not args.no_fast:
         mf = mdl.Model(cfg, mode=mode, variant=1, n_slots=n_slots, capacity=cap, init="device")
         rf = run_decode(mf, B, P, K, W, 1, rank)
