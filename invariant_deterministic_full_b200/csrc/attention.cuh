@@ -29,6 +29,7 @@ constexpr int ATT_CHUNK = BI_ATTN_CHUNK;  // 256
 constexpr int ATT_MAX_PAIRS = 32;         // (query, q-head) pairs per CTA
 constexpr int ATT_MAX_BLOCKS = 1024;      // query blocks per launch
 constexpr int ATT_TOKEN_GROUP = 1024;     // tokens per partials workspace pass
+constexpr int ATT_MAX_QB = 64;            // tokens per query block
 
 struct AttnPlan {
   int n;
@@ -54,6 +55,39 @@ struct AttnArgs {
 // two routes give the same bits.
 __device__ __forceinline__ void merge_pair(const float* __restrict__ base, int nc, int d, int lane,
                                            void* __restrict__ out, size_t off, int f32) {
+  constexpr int NCR = 4;  // up to NCR chunks: every operand is loaded first, then the same arithmetic runs
+  if (nc <= NCR) {
+    float mc[NCR], lc[NCR], ac[NCR][4];
+#pragma unroll
+    for (int c = 0; c < NCR; ++c) {
+      if (c < nc) {
+        const float* rec = base + (size_t)c * (d + 4);
+        mc[c] = rec[d];
+        lc[c] = rec[d + 1];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) ac[c][k] = k < d / 32 ? rec[lane + 32 * k] : 0.f;
+      }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < NCR; ++c)
+      if (c < nc) M = fmaxf(M, mc[c]);
+    float L = 0.f;
+    float o[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < NCR; ++c) {
+      if (c < nc) {
+        const float w = expf(mc[c] - M);
+        L = fmaf(lc[c], w, L);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) o[k] = fmaf(ac[c][k], w, o[k]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k < d / 32) store_act(out, off + lane + 32 * k, o[k] / L, f32);
+    return;
+  }
   float M = -INFINITY;
   for (int c = 0; c < nc; ++c) M = fmaxf(M, base[(size_t)c * (d + 4) + d]);
   float L = 0.f;
@@ -363,15 +397,18 @@ __device__ __forceinline__ uint32_t atc_poff(int r, int j) {
   return (uint32_t)(r * 512 + (((c & ~7) | ((c ^ r) & 7)) << 4) + (j & 7) * 2);
 }
 
+constexpr int ATC_THREADS = ATT_THREADS + 32;  // 8 consumer warps + 1 producer warp
+
 template <int NPT, int RING>
-__global__ void __launch_bounds__(ATT_THREADS)
+__global__ void __launch_bounds__(ATC_THREADS)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ AttnPlan plan, const AttnArgs a) {
   pdl_wait();
   pdl_trigger();
   constexpr int NP = 8 * NPT;  // pairs per group
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar[RING];
+  __shared__ __align__(8) uint64_t full_bar[RING];
+  __shared__ __align__(8) uint64_t empty_bar[RING];
   __shared__ float m_s[NP], l_s[NP];
   __shared__ int live_s[NP];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -401,40 +438,51 @@ __global__ void __launch_bounds__(ATT_THREADS)
   auto nsub_of = [&](int c) { return (min(a.chunk, pmax - c * a.chunk + 1) + ATT_SUB - 1) / ATT_SUB; };
 
   if (tid == 0) {
-    for (int r = 0; r < RING; ++r) mbar_init(&bar[r], 1);
+    for (int r = 0; r < RING; ++r) {
+      mbar_init(&full_bar[r], 1);
+      mbar_init(&empty_bar[r], ATT_THREADS / 32);
+    }
     fence_mbar_init();
   }
   __syncthreads();
-  // Load stream (thread 0): for each chunk of the segment, for each pair
-  // group, the chunk's K sub-tiles then its V sub-tiles.  The ring runs
-  // across chunk boundaries, so the next chunk's keys arrive while this
-  // chunk's values are consumed.
-  int lp = 0, pc = c_lo, pg = 0, pli = 0, pns = nsub_of(c_lo);
-  auto issue_next = [&]() {
-    if (pc >= c_hi) return;
-    const bool isv = pli >= pns;
-    const int st = isv ? pli - pns : pli;
-    mbar_arrive_expect_tx(&bar[lp % RING], SUB);
-    tma_load_3d(smem + (lp % RING) * SUB, isv ? &tmV : &tmK, 0, cache_base + pc * a.chunk + st * ATT_SUB, 0,
-                &bar[lp % RING]);
-    ++lp;
-    if (++pli == 2 * pns) {
-      pli = 0;
-      if (++pg == ngroups) {
-        pg = 0;
-        if (++pc < c_hi) pns = nsub_of(pc);
+
+  if (warp == ATT_THREADS / 32) {
+    // ---- producer warp, one lane: for each chunk of the segment, for each pair
+    // group, the chunk's K sub-tiles then its V sub-tiles.  A slot is refilled
+    // once all eight consumer warps have released it, so the stream runs ahead
+    // of the slowest warp by up to RING sub-tiles, across chunk boundaries.
+    if (lane == 0) {
+      int lp = 0;
+      for (int pc = c_lo; pc < c_hi; ++pc) {
+        const int pns = nsub_of(pc);
+        for (int pg = 0; pg < ngroups; ++pg)
+          for (int pli = 0; pli < 2 * pns; ++pli, ++lp) {
+            const int slot = lp % RING;
+            if (lp >= RING && !mbar_wait(&empty_bar[slot], (uint32_t)(((lp / RING) - 1) & 1), SITE_ATTN_TC | 0x80))
+              return;
+            const bool isv = pli >= pns;
+            const int st = isv ? pli - pns : pli;
+            mbar_arrive_expect_tx(&full_bar[slot], SUB);
+            tma_load_3d(smem + slot * SUB, isv ? &tmV : &tmK, 0, cache_base + pc * a.chunk + st * ATT_SUB, 0,
+                        &full_bar[slot]);
+          }
       }
     }
-  };
-  if (tid == 0)
-    for (int r = 0; r < RING; ++r) issue_next();
+    return;
+  }
+
+  // ---- consumer warps.  A ring wait that runs out sets the error flag; the warp
+  // then goes on (on stale data) so every named barrier is still met.
   int L = 0;
-  auto consume_wait = [&]() -> bool { return mbar_wait(&bar[L % RING], (uint32_t)((L / RING) & 1), SITE_ATTN_TC | (NPT << 8)); };
-  auto release = [&]() {
-    __syncthreads();
-    if (tid == 0) issue_next();
+  auto consume_wait = [&]() {
+    (void)mbar_wait(&full_bar[L % RING], (uint32_t)((L / RING) & 1), SITE_ATTN_TC | (NPT << 8));
+  };
+  auto release = [&]() {  // this warp is done with slot L
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[L % RING]);
     ++L;
   };
+  auto cbar = []() { asm volatile("bar.sync 1, %0;" ::"n"(ATT_THREADS) : "memory"); };
 
   // score work of a warp: key tile kt of each 64-key sub-tile, pair tiles pt = spt, spt + 2, ...
   constexpr int SPT = NPT == 1 ? 1 : NPT / 2;  // pair tiles per warp in the score phase
@@ -442,42 +490,51 @@ __global__ void __launch_bounds__(ATT_THREADS)
   const int spt0 = NPT == 1 ? 0 : (warp >> 2);
   const bool score_warp = NPT > 1 || warp < 4;
 
+  // positions of the block's queries (consecutive tokens of one slot), read once
+  __shared__ int pos_s[ATT_MAX_QB];
+  for (int i = tid; i < nq; i += ATT_THREADS) pos_s[i] = a.pos[t0 + i];
+  // q tile (bf16, 128-byte swizzle per half; padded rows are zero) and the q^T
+  // fragments (B operand) of this warp's pair tiles; with one pair group they
+  // are loaded once for the whole segment
+  uint32_t qb[SPT][8][2];
+  auto load_q = [&](int pg0, int gp) {
+    for (int idx = tid; idx < NP * 16; idx += ATT_THREADS) {  // 16 chunks of 8 elements per row
+      const int row = idx >> 4, ch = idx & 15;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (row < gp) {
+        const int p = pg0 + row;
+        const int i = p / a.G, g = p % a.G;
+        v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.q) +
+                                            (size_t)(t0 + i) * a.Hq * 128 + (hk * a.G + g) * 128 + ch * 8);
+      }
+      const int half = ch >> 3, cc = ch & 7;
+      *reinterpret_cast<uint4*>(qt + half * (NP * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
+    }
+    cbar();
+    if (score_warp) {
+#pragma unroll
+      for (int u = 0; u < SPT; ++u)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int row = (spt0 + 2 * u) * 8 + (lane & 7);
+          const int half = kk >> 2, ch = 2 * (kk & 3) + ((lane >> 3) & 1);
+          ldsm_x2(qt_s + half * (NP * 128) + row * 128 + ((ch ^ (row & 7)) << 4), qb[u][kk][0], qb[u][kk][1]);
+        }
+    }
+  };
+  if (ngroups == 1) load_q(0, npairs);
+
   for (int c = c_lo; c < c_hi; ++c) {
     const int key0 = c * a.chunk;
     const int nvalid = min(a.chunk, pmax - key0 + 1);
     const int nsub = (nvalid + ATT_SUB - 1) / ATT_SUB;
     for (int pg0 = 0; pg0 < npairs; pg0 += NP) {
       const int gp = min(NP, npairs - pg0);
-      // q tile (bf16, 128-byte swizzle per half); padded rows are zero
-      for (int idx = tid; idx < NP * 16; idx += ATT_THREADS) {  // 16 chunks of 8 elements per row
-        const int row = idx >> 4, ch = idx & 15;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (row < gp) {
-          const int p = pg0 + row;
-          const int i = p / a.G, g = p % a.G;
-          v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.q) +
-                                              (size_t)(t0 + i) * a.Hq * 128 + (hk * a.G + g) * 128 + ch * 8);
-        }
-        const int half = ch >> 3, cc = ch & 7;
-        *reinterpret_cast<uint4*>(qt + half * (NP * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
-      }
-      __syncthreads();
-      // q^T fragments (B operand) of this warp's pair tiles, kept for the whole chunk
-      uint32_t qb[SPT][8][2];
-      if (score_warp) {
-#pragma unroll
-        for (int u = 0; u < SPT; ++u)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const int row = (spt0 + 2 * u) * 8 + (lane & 7);
-            const int half = kk >> 2, ch = 2 * (kk & 3) + ((lane >> 3) & 1);
-            ldsm_x2(qt_s + half * (NP * 128) + row * 128 + ((ch ^ (row & 7)) << 4), qb[u][kk][0], qb[u][kk][1]);
-          }
-      }
+      if (ngroups > 1) load_q(pg0, gp);
 
       // ---- scores: S[pair][key] = scale * (K[key] . q[pair])
       for (int st = 0; st < nsub; ++st) {
-        if (!consume_wait()) return;
+        consume_wait();
         if (score_warp) {
           const uint32_t kb = smem_u32(smem + (L % RING) * SUB);
           float acc[SPT][4];
@@ -504,13 +561,14 @@ __global__ void __launch_bounds__(ATT_THREADS)
         }
         release();
       }
+      cbar();  // every score of the chunk is in S
 
       // ---- softmax of the live pair rows: max (exact), exp, l = lane-strided ascending sums then
       // butterfly; the probabilities go out as three exact bf16 parts (zeros past the valid keys).
       // Rows past the group's pairs are not computed: they only reach output columns never stored.
       for (int pl = warp; pl < gp; pl += ATT_THREADS / 32) {
         const int i = (pg0 + pl) / a.G;
-        const int lim = a.pos[t0 + i] - key0;
+        const int lim = pos_s[i] - key0;
         float mx = -INFINITY;
 #pragma unroll
         for (int k = 0; k < ATT_CHUNK / 32; ++k) {
@@ -541,7 +599,7 @@ __global__ void __launch_bounds__(ATT_THREADS)
           live_s[pl] = lim >= 0;
         }
       }
-      __syncthreads();
+      cbar();
 
       // ---- P.V: warp w owns head elements 16w..16w+15 (one m16 tile of V^T)
       float pacc[3][NPT][4];
@@ -550,7 +608,7 @@ __global__ void __launch_bounds__(ATT_THREADS)
 #pragma unroll
         for (int u = 0; u < NPT; ++u) pacc[q][u][0] = pacc[q][u][1] = pacc[q][u][2] = pacc[q][u][3] = 0.f;
       for (int st = 0; st < nsub; ++st) {
-        if (!consume_wait()) return;
+        consume_wait();
         uint8_t* vbuf = smem + (L % RING) * SUB;
         const int vrows = nvalid - st * ATT_SUB;  // valid rows of this sub-tile
         if (vrows < ATT_SUB) {  // zero the rows past the last valid key
@@ -558,7 +616,7 @@ __global__ void __launch_bounds__(ATT_THREADS)
             const int r = vrows + (idx >> 4), ch = idx & 15;
             *reinterpret_cast<uint4*>(vbuf + (ch >> 3) * 8192 + r * 128 + ((ch & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
           }
-          __syncthreads();
+          cbar();
         }
         const uint32_t vb = smem_u32(vbuf);
         const int nk16 = min(4, (vrows + 15) / 16);
@@ -604,7 +662,7 @@ __global__ void __launch_bounds__(ATT_THREADS)
             rec[129] = l_s[pl];
           }
         }
-      __syncthreads();  // the next group overwrites q, S, the probability parts and the statistics
+      cbar();  // the next group overwrites q, S, the probability parts and the statistics
     }
   }
   if (a.merge_in_cta) {
@@ -612,7 +670,7 @@ __global__ void __launch_bounds__(ATT_THREADS)
     // (the partials written by this CTA are visible to it after the barrier)
     for (int p = warp; p < npairs; p += ATT_THREADS / 32) {
       const int t = t0 + p / a.G, hq = hk * a.G + p % a.G;
-      const int nc = min(a.pos[t] / a.chunk + 1, c_hi);
+      const int nc = min(pos_s[t - t0] / a.chunk + 1, c_hi);
       merge_pair(a.part + ((size_t)(t - a.t_base) * a.Hq + hq) * a.max_chunks * (128 + 4), nc, 128, lane, a.out,
                  (size_t)t * a.Hq * 128 + hq * 128, 0);
     }

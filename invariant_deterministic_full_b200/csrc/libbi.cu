@@ -78,8 +78,8 @@ static int attn_set_smem_attrs() {
                                      (int)att_smem_bytes(16, 128, 1)));
   BI_CHECK_CUDA(cudaFuncSetAttribute(attn_partial_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)att_smem_bytes(32, 128, 1)));
-  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<1, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)atc_smem_bytes(1, 4)));
+  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<1, 5>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)atc_smem_bytes(1, 5)));
   BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)atc_smem_bytes(2, 4)));
   BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -112,11 +112,11 @@ static int attn_launch(int np, const CUtensorMap& tk, const CUtensorMap& tv, con
     const dim3 grid(plan.n, n_seg, a.Hkv);
     const bool single = np <= 16;  // decode blocks: one token, G pairs
     if (single && a.G <= 8)
-      BI_TRY(launch(attn_tc_kernel<1, 4>, grid, dim3(ATT_THREADS), atc_smem_bytes(1, 4), st, tk, tv, plan, a));
+      BI_TRY(launch(attn_tc_kernel<1, 5>, grid, dim3(ATC_THREADS), atc_smem_bytes(1, 5), st, tk, tv, plan, a));
     else if (single && a.G <= 16)
-      BI_TRY(launch(attn_tc_kernel<2, 4>, grid, dim3(ATT_THREADS), atc_smem_bytes(2, 4), st, tk, tv, plan, a));
+      BI_TRY(launch(attn_tc_kernel<2, 4>, grid, dim3(ATC_THREADS), atc_smem_bytes(2, 4), st, tk, tv, plan, a));
     else
-      BI_TRY(launch(attn_tc_kernel<4, 2>, grid, dim3(ATT_THREADS), atc_smem_bytes(4, 2), st, tk, tv, plan, a));
+      BI_TRY(launch(attn_tc_kernel<4, 2>, grid, dim3(ATC_THREADS), atc_smem_bytes(4, 2), st, tk, tv, plan, a));
     return BI_OK;
   }
   a.seg_len = 1;
@@ -150,7 +150,7 @@ static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const
   const int chunk = attn_chunk_for(T, variant);
   // query-block size (work assignment only): a CTA streams one KV chunk and loops over
   // the block's (query, head) pairs 32 at a time; blocks hold up to 256 pairs.
-  const int QB = std::max(1, std::min(64, 256 / G));
+  const int QB = std::max(1, std::min(ATT_MAX_QB, 256 / G));
 
   // validation + plan: blocks of <= QB adjacent tokens of one slot at consecutive positions
   int max_pos = 0;
