@@ -53,9 +53,13 @@ constexpr int GEMM_BK = 64;  // k per k-block (128 bytes of bf16: one swizzled s
 // MT: 32-row token tiles sharing each weight stage (M-blocking; a property of
 // the launch, not of the arithmetic: every element still sees the same
 // instruction sequence).  MT > 1 only with 128-row weight tiles.
-template <int BN, int MT = 1>
+// CPS: CTAs per SM.  1: one persistent CTA per SM with a ~212 KB ring.  2:
+// two CTAs of ~112 KB each, for launches with between 1x and 2x as many work
+// items as SMs -- an SM that holds two row groups then streams both at once
+// instead of one after the other, so the extra groups do not double its time.
+template <int BN, int MT = 1, int CPS = 1>
 struct GemmCfg {
-  static constexpr int KBS = BN == 128 ? 2 : 4;
+  static constexpr int KBS = BN == 128 ? (CPS == 2 ? 1 : 2) : 4;
   static constexpr int W_BYTES = KBS * BN * 128;
   static constexpr int X_BYTES = KBS * GEMM_BM * MT * 128;
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
@@ -63,8 +67,11 @@ struct GemmCfg {
   // Interleaved accumulator sets per output element (a property of the matrix
   // shape through BN, never of M), one per k-phase warp of a row group.
   static constexpr int KS = 4 / RW;
-  static constexpr int RED_BYTES = KS > 1 ? 4 * 32 * 32 * 4 : 0;  // cross-warp partial sums
-  static constexpr int STAGES = (212 * 1024 - RED_BYTES) / STAGE_BYTES;
+  // cross-warp partial sums: each warp parks the 8 values x 32 lanes of every
+  // n8 token tile that another warp of its row group finishes
+  static constexpr int RED_TILES = KS > 1 ? 4 - 4 / KS : 0;
+  static constexpr int RED_BYTES = 4 * RED_TILES * 8 * 32 * 4;
+  static constexpr int STAGES = ((CPS == 2 ? 112 : 212) * 1024 - RED_BYTES) / STAGE_BYTES;
   static constexpr int SMEM = STAGES * STAGE_BYTES + RED_BYTES + 1024;
 };
 
@@ -90,13 +97,13 @@ struct RopeEpi {
 
 // Work item -> (split, row group, token tile).  Splits > 1 only in the
 // non-invariant FAST variant, which then writes fp32 partials per split.
-template <int BN, int EPI, int MT>
-__global__ void __launch_bounds__(160, 1)
+template <int BN, int EPI, int MT, int CPS>
+__global__ void __launch_bounds__(160, CPS)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                      void* __restrict__ y, int ldy, int y_f32, int M, int N, int K, int m_tiles, int n_groups,
                      int splits, float* __restrict__ partial, const int* __restrict__ mcount, int mmult,
                      const RopeEpi re) {
-  using C = GemmCfg<BN, MT>;
+  using C = GemmCfg<BN, MT, CPS>;
   static_assert(MT == 1 || C::KS == 1, "M-blocking needs one k-phase per warp");
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::STAGES];
@@ -292,32 +299,36 @@ __global__ void __launch_bounds__(160, 1)
       // finishes the n8 token tiles nt = kp, kp + KS, ... combining
       // ((s0 + s1) + (s2 + s3)) (KS = 4) or s0 + s1 (KS = 2), set j coming from
       // warp (rw, j); the epilogue work is shared by all four warps.
+      // slot of tile b among the RED_TILES tiles that warp (rw, j) parks: the tiles it
+      // does not finish, in ascending order
+      auto slot = [&](int b, int j) { return b / C::KS * (C::KS - 1) + (b % C::KS) - (b % C::KS > j ? 1 : 0); };
+      auto cell = [&](int w, int sl, int a, int c) { return ((w * C::RED_TILES + sl) * 8 + a * 4 + c) * 32 + lane; };
 #pragma unroll
-      for (int a = 0; a < 2; ++a)
+      for (int b = 0; b < 4; ++b) {
+        if (b % C::KS == kp) continue;
 #pragma unroll
-        for (int b = 0; b < 4; ++b)
+        for (int a = 0; a < 2; ++a)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) red[(warp * 32 + (a * 16 + b * 4 + c)) * 32 + lane] = acc[a][b][c];
+          for (int c = 0; c < 4; ++c) red[cell(warp, slot(b, kp), a, c)] = acc[a][b][c];
+      }
       asm volatile("bar.sync 1, 128;" ::: "memory");
 #pragma unroll
-      for (int a = 0; a < 2; ++a)
+      for (int b = 0; b < 4; ++b) {
+        if (b % C::KS != kp) continue;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          if (b % C::KS != kp) continue;
+        for (int a = 0; a < 2; ++a)
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const int v = a * 16 + b * 4 + c;
-            const float s0 = red[(rw * 32 + v) * 32 + lane];
-            const float s1 = red[((rw + C::RW) * 32 + v) * 32 + lane];
-            if constexpr (C::KS == 4) {
-              const float s2 = red[((rw + 2) * 32 + v) * 32 + lane];
-              const float s3 = red[((rw + 3) * 32 + v) * 32 + lane];
-              acc[a][b][c] = (s0 + s1) + (s2 + s3);
-            } else {
-              acc[a][b][c] = s0 + s1;
-            }
+            float sv[4];
+#pragma unroll
+            for (int j = 0; j < C::KS; ++j)
+              sv[j] = j == kp ? acc[a][b][c] : red[cell(rw + C::RW * j, slot(b, j), a, c)];
+            if constexpr (C::KS == 4)
+              acc[a][b][c] = (sv[0] + sv[1]) + (sv[2] + sv[3]);
+            else
+              acc[a][b][c] = sv[0] + sv[1];
           }
-        }
+      }
       asm volatile("bar.sync 1, 128;" ::: "memory");  // the next item reuses the exchange buffer
     }
     if (dead) continue;
@@ -567,7 +578,10 @@ static int gemm_pick_bn(int N) {
 // Split factor of the FAST variant: more K splits for small M so that the
 // grid fills the SMs (the usual library heuristic) -- which is exactly what
 // makes the result depend on the batch size.
-static int gemm_kbs(int bn) { return bn == 128 ? GemmCfg<128>::KBS : (bn == 64 ? GemmCfg<64>::KBS : GemmCfg<32>::KBS); }
+static int gemm_kbs(int bn, int cps = 1) {
+  if (bn == 128) return cps == 2 ? GemmCfg<128, 1, 2>::KBS : GemmCfg<128>::KBS;
+  return bn == 64 ? GemmCfg<64>::KBS : GemmCfg<32>::KBS;
+}
 
 static int gemm_fast_splits(int M, int n_items, int kstages) {
   const int sms = num_sms();
@@ -588,24 +602,32 @@ size_t gemm_ws_bytes(int M, int N, int K, int mode, int variant) {
   return s > 1 ? (size_t)s * M * N * sizeof(float) : 0;
 }
 
-template <int BN, int EPI, int MT = 1>
+template <int BN, int EPI, int MT = 1, int CPS = 1>
 static int launch_gemm_bf16_t(const CUtensorMap& tw, const CUtensorMap& tx, void* y, int ldy, int y_f32, int M, int N,
                               int K, int splits, float* partial, const int* mcount, int mmult, const RopeEpi& re,
                               cudaStream_t st) {
-  using C = GemmCfg<BN, MT>;
+  using C = GemmCfg<BN, MT, CPS>;
   static bool attr_done = false;  // per instantiation; set once per process
   if (!attr_done) {
-    BI_CHECK_CUDA(cudaFuncSetAttribute(gemm_bf16_kernel<BN, EPI, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::SMEM));
+    BI_CHECK_CUDA(cudaFuncSetAttribute(gemm_bf16_kernel<BN, EPI, MT, CPS>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
     attr_done = true;
   }
   const int m_tiles = (M + GEMM_BM - 1) / GEMM_BM;
   const int n_groups = N / BN;
   const int items = splits * n_groups * ((m_tiles + MT - 1) / MT);
-  const int grid = items < num_sms() ? items : num_sms();
-  BI_TRY(launch(gemm_bf16_kernel<BN, EPI, MT>, dim3(grid), dim3(160), C::SMEM, st, tw, tx, y, ldy, y_f32, M, N, K,
-                m_tiles, n_groups, splits, partial, mcount, mmult, re));
+  const int grid = items < CPS * num_sms() ? items : CPS * num_sms();
+  BI_TRY(launch(gemm_bf16_kernel<BN, EPI, MT, CPS>, dim3(grid), dim3(160), C::SMEM, st, tw, tx, y, ldy, y_f32, M, N,
+                K, m_tiles, n_groups, splits, partial, mcount, mmult, re));
   return BI_OK;
+}
+
+// Two CTAs per SM when the launch has between 1x and 2x as many work items as
+// SMs (one token tile per item, no split).
+static int gemm_pick_cps(int bn, int M, int N, int mt, int splits) {
+  if (mt != 1 || splits != 1) return 1;
+  const int items = (N / bn) * ((M + GEMM_BM - 1) / GEMM_BM);
+  return items > num_sms() && items <= 2 * num_sms() ? 2 : 1;
 }
 
 // Token tiles per weight stage: 4 for 128-row weight tiles once M spans four
@@ -618,7 +640,15 @@ int gemm_bf16(const void* x, int ldx, const void* w, void* y, int ldy, int y_f32
               const RopeEpi* rope = nullptr) {
   const RopeEpi re = rope ? *rope : RopeEpi{};
   const int bn = gemm_pick_bn(N);
-  const int kbs = gemm_kbs(bn);
+  const int mt = gemm_pick_mt(bn, M);
+  int splits = 1;
+  if (variant == BI_VARIANT_FAST) {
+    const int items = (N / bn) * ((M + GEMM_BM - 1) / GEMM_BM);
+    const int kbs1 = gemm_kbs(bn);
+    splits = gemm_fast_splits(M, items, (K / GEMM_BK + kbs1 - 1) / kbs1);
+  }
+  const int cps = gemm_pick_cps(bn, M, N, mt, splits);
+  const int kbs = gemm_kbs(bn, cps);
   // 3-D views {64 k, rows, k-block}: the k-block dimension (stride 128 B) is the
   // outermost of the box, so a box lands as kbs swizzled [rows][128 B] slabs.
   CUtensorMap tw, tx;
@@ -628,14 +658,8 @@ int gemm_bf16(const void* x, int ldx, const void* w, void* y, int ldy, int y_f32
   BI_TRY(encode_tmap_3d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, dw, sw, bw, CU_TENSOR_MAP_SWIZZLE_128B));
   const uint64_t dx[3] = {(uint64_t)GEMM_BK, (uint64_t)M, (uint64_t)(K / GEMM_BK)};
   const uint64_t sx[2] = {(uint64_t)ldx * 2, (uint64_t)GEMM_BK * 2};
-  const int mt = gemm_pick_mt(bn, M);
   const uint32_t bx[3] = {(uint32_t)GEMM_BK, (uint32_t)(GEMM_BM * mt), (uint32_t)kbs};
   BI_TRY(encode_tmap_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_128B));
-  int splits = 1;
-  if (variant == BI_VARIANT_FAST) {
-    const int items = (N / bn) * ((M + GEMM_BM - 1) / GEMM_BM);
-    splits = gemm_fast_splits(M, items, (K / GEMM_BK + kbs - 1) / kbs);
-  }
   float* partial = nullptr;
   if (splits > 1) {
     const size_t need = (size_t)splits * M * N * sizeof(float);
@@ -645,22 +669,28 @@ int gemm_bf16(const void* x, int ldx, const void* w, void* y, int ldy, int y_f32
   if (epi == EPI_ROPE) {
     if (bn != 32 || splits > 1 || !rope)
       return set_error(BI_ERR_UNSUPPORTED, "fused RoPE epilogue needs the 32-row tile and no split");
-    BI_TRY((launch_gemm_bf16_t<32, EPI_ROPE>(tw, tx, y, ldy, y_f32, M, N, K, 1, nullptr, mcount, mmult, re, st)));
+    if (cps == 2)
+      BI_TRY((launch_gemm_bf16_t<32, EPI_ROPE, 1, 2>(tw, tx, y, ldy, y_f32, M, N, K, 1, nullptr, mcount, mmult, re, st)));
+    else
+      BI_TRY((launch_gemm_bf16_t<32, EPI_ROPE, 1, 1>(tw, tx, y, ldy, y_f32, M, N, K, 1, nullptr, mcount, mmult, re, st)));
     return BI_OK;
   }
-#define BI_GEMM_CASE(BNV, MTV)                                                                                  \
-  if (bn == BNV && mt == MTV) {                                                                                 \
+#define BI_GEMM_CASE(BNV, MTV, CPSV)                                                                            \
+  if (bn == BNV && mt == MTV && cps == CPSV) {                                                                  \
     if (epi == BI_EPI_SWIGLU)                                                                                   \
-      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_SWIGLU, MTV>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, mcount, \
-                                                          mmult, re, st)));                                     \
+      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_SWIGLU, MTV, CPSV>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial,   \
+                                                                mcount, mmult, re, st)));                       \
     else                                                                                                        \
-      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_NONE, MTV>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial, mcount,   \
-                                                        mmult, re, st)));                                       \
+      BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_NONE, MTV, CPSV>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial,     \
+                                                              mcount, mmult, re, st)));                         \
   }
-  BI_GEMM_CASE(32, 1)
-  BI_GEMM_CASE(64, 1)
-  BI_GEMM_CASE(128, 1)
-  BI_GEMM_CASE(128, 4)
+  BI_GEMM_CASE(32, 1, 1)
+  BI_GEMM_CASE(64, 1, 1)
+  BI_GEMM_CASE(128, 1, 1)
+  BI_GEMM_CASE(128, 4, 1)
+  BI_GEMM_CASE(32, 1, 2)
+  BI_GEMM_CASE(64, 1, 2)
+  BI_GEMM_CASE(128, 1, 2)
 #undef BI_GEMM_CASE
   if (splits > 1) {
     const int n_out = epi == BI_EPI_SWIGLU ? N / 2 : N;
