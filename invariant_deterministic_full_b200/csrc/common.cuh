@@ -115,11 +115,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait: returns false (and flags the device error word) if the phase
 // does not complete within the iteration limit (each try_wait suspends for a
 // hardware-chosen interval, so the limit is seconds, never forever).
-constexpr uint32_t kWaitLimit = 1u << 22;
+// Bounded waits: a wait gives up after kWaitNs of wall-clock time (the
+// global nanosecond timer), whatever each try_wait costs.
+constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 // site: which wait ran out, reported in bits 8..15 of bi_device_error's flags.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned site = 0) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitNs) break;
+  }
   dev_flag(DEVERR_TIMEOUT);
   atomicCAS(&g_dev_site, 0u, site);
   return false;

@@ -4,8 +4,8 @@
 
 namespace bi {
 
-constexpr int NORM_THREADS = 256;
-constexpr int NORM_MAX_CHUNKS = 8;  // 8-element chunks per thread: H <= 256*8*8 = 16384
+constexpr int NORM_THREADS = 128;
+constexpr int NORM_MAX_CHUNKS = 16;  // 8-element chunks per thread: H <= 128*16*8 = 16384
 
 // Load/store 8 consecutive activation values (bf16: one 16-byte access; f32: two).
 __device__ __forceinline__ void load8(const void* base, size_t off, bool f32, float* v) {
@@ -37,10 +37,66 @@ __device__ __forceinline__ float as_stored(float v, bool f32) {
   return f32 ? v : bf16_bits_to_f32(f32_to_bf16_bits(v));
 }
 
-// One CTA per row.  Thread i owns the 8-element chunks i, i + 256, ... of the
-// row; its partial sum of squares runs over them in ascending order, then a
-// fixed xor-butterfly inside each warp, then the 8 warp sums are added in
-// ascending warp order (every thread repeats that same sequential sum).
+// One row, NORM_THREADS threads (tid = 0 .. NORM_THREADS-1).  Thread i owns
+// the 8-element chunks i, i + NORM_THREADS, ... of the row; its partial sum of
+// squares runs over them in ascending order, then a fixed xor-butterfly inside
+// each warp, then the warp sums are added in ascending warp order (every
+// thread repeats that same sequential sum).  r = x (+ res_in, rounded as
+// stored), written to res_out; y = (r * inv) * gamma.  The row is read twice
+// (sum of squares, then the outputs) so that no chunk is held in registers;
+// both passes compute r the same way.  `bar` synchronises the NORM_THREADS
+// threads (a CTA barrier, or a named barrier inside a larger CTA).
+template <typename Bar>
+__device__ __forceinline__ void rmsnorm_row(const void* __restrict__ x, const void* __restrict__ res_in,
+                                            void* __restrict__ res_out, const uint16_t* __restrict__ gamma,
+                                            void* __restrict__ y, float* __restrict__ y32, int row, int H, float eps,
+                                            int f32, int tid, float* wsum, Bar bar) {
+  const int nch = H / 8;
+  const size_t rbase = (size_t)row * H;
+  auto load_r = [&](int ch, float* v) {
+    load8(x, rbase + ch * 8, f32, v);
+    if (res_in) {
+      float r[8];
+      load8(res_in, rbase + ch * 8, f32, r);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = as_stored(v[j] + r[j], f32);
+    }
+  };
+  float ss = 0.f;
+  for (int ch = tid; ch < nch; ch += NORM_THREADS) {
+    float v[8];
+    load_r(ch, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ss = fmaf(v[j], v[j], ss);
+  }
+  ss = warp_sum_fixed(ss);
+  if ((tid & 31) == 0) wsum[tid >> 5] = ss;
+  bar();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < NORM_THREADS / 32; ++w) tot += wsum[w];
+  const float inv = 1.0f / sqrtf(tot / (float)H + eps);
+  bar();  // wsum may be reused by the next row
+  for (int ch = tid; ch < nch; ch += NORM_THREADS) {
+    float v[8];
+    load_r(ch, v);
+    if (res_out) store8(res_out, rbase + ch * 8, f32, v);
+    const uint4 gu = *reinterpret_cast<const uint4*>(gamma + ch * 8);
+    const float gm[8] = {bf16lo(gu.x), bf16hi(gu.x), bf16lo(gu.y), bf16hi(gu.y),
+                         bf16lo(gu.z), bf16hi(gu.z), bf16lo(gu.w), bf16hi(gu.w)};
+    float o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j] = v[j] * inv * gm[j];
+    store8(y, rbase + ch * 8, f32, o);
+    if (y32) {
+      float4* p = reinterpret_cast<float4*>(y32 + rbase + ch * 8);
+      p[0] = make_float4(o[0], o[1], o[2], o[3]);
+      p[1] = make_float4(o[4], o[5], o[6], o[7]);
+    }
+  }
+}
+
+// One CTA per row (see rmsnorm_row).
 __global__ void __launch_bounds__(NORM_THREADS)
     rmsnorm_kernel(const void* __restrict__ x, const void* __restrict__ res_in, void* __restrict__ res_out,
                    const uint16_t* __restrict__ gamma, void* __restrict__ y, float* __restrict__ y32, int H, float eps,
@@ -48,52 +104,7 @@ __global__ void __launch_bounds__(NORM_THREADS)
   pdl_wait();
   pdl_trigger();
   __shared__ float wsum[NORM_THREADS / 32];
-  const int row = blockIdx.x;
-  const int nch = H / 8;
-  const size_t rbase = (size_t)row * H;
-  float v[NORM_MAX_CHUNKS][8];
-  float ss = 0.f;
-#pragma unroll
-  for (int c = 0; c < NORM_MAX_CHUNKS; ++c) {
-    const int ch = threadIdx.x + c * NORM_THREADS;
-    if (ch < nch) {
-      load8(x, rbase + ch * 8, f32, v[c]);
-      if (res_in) {
-        float r[8];
-        load8(res_in, rbase + ch * 8, f32, r);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[c][j] = as_stored(v[c][j] + r[j], f32);
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) ss = fmaf(v[c][j], v[c][j], ss);
-    }
-  }
-  ss = warp_sum_fixed(ss);
-  if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  float tot = 0.f;
-#pragma unroll
-  for (int w = 0; w < NORM_THREADS / 32; ++w) tot += wsum[w];
-  const float inv = 1.0f / sqrtf(tot / (float)H + eps);
-#pragma unroll
-  for (int c = 0; c < NORM_MAX_CHUNKS; ++c) {
-    const int ch = threadIdx.x + c * NORM_THREADS;
-    if (ch < nch) {
-      if (res_out) store8(res_out, rbase + ch * 8, f32, v[c]);
-      const uint4 gu = *reinterpret_cast<const uint4*>(gamma + ch * 8);
-      const float gm[8] = {bf16lo(gu.x), bf16hi(gu.x), bf16lo(gu.y), bf16hi(gu.y),
-                           bf16lo(gu.z), bf16hi(gu.z), bf16lo(gu.w), bf16hi(gu.w)};
-      float o[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) o[j] = v[c][j] * inv * gm[j];
-      store8(y, rbase + ch * 8, f32, o);
-      if (y32) {
-        float4* p = reinterpret_cast<float4*>(y32 + rbase + ch * 8);
-        p[0] = make_float4(o[0], o[1], o[2], o[3]);
-        p[1] = make_float4(o[4], o[5], o[6], o[7]);
-      }
-    }
-  }
+  rmsnorm_row(x, res_in, res_out, gamma, y, y32, blockIdx.x, H, eps, f32, threadIdx.x, wsum, [] { __syncthreads(); });
 }
 
 // Row of element i of a head (size d) in the "paired" QKV layout: within every
