@@ -53,7 +53,9 @@ def parse():
 
 
 # ---------------------------------------------------------------- distributed plumbing
-def dist_init(args):
+def dist_init(args, backend="nccl"):
+    """One process per GPU (torchrun env).  Replicas only: the process group carries the barrier around the timed
+    region and the max-over-ranks of the measured time, never data."""
     import torch
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -61,9 +63,10 @@ def dist_init(args):
     if ws > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return ws, rank, local
 
@@ -79,9 +82,14 @@ def max_over_ranks(x, ws):
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if dist.get_backend() == "nccl" else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(units_per_rank, ms_max, ws):
+    """Whole-job throughput of ws replicas: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * ws / (ms_max / 1e3)
 
 
 # ---------------------------------------------------------------- clocks during the timed region
@@ -410,7 +418,7 @@ def main_ours(args):
     m = mdl.Model(cfg, mode=mode, n_slots=n_slots, capacity=cap, init="device", device="cuda")
     r = run_decode(m, B, P, K, W, ws, rank)
     ms = max_over_ranks(r["ms"], ws)
-    value = B * K * ws / (ms / 1e3)
+    value = replica_throughput(B * K, ms, ws)
     hbm, tf_burst, tf_sus, src = peaks()
     sb = step_bytes(cfg, B, [0] * B, f32_kv=(mode == 1))  # weights + rows at one position, per step
     kv_row = cfg["n_layers"] * cfg["n_kv_heads"] * cfg["head_dim"] * 2 * (4 if mode else 2)
