@@ -165,8 +165,8 @@ def step_bytes(cfg, B, ctx_lens, f32_kv=False):
 # capture (dram__bytes_read.sum + dram__bytes_write.sum) of the same shapes on the 2-layer 8B-width case; the
 # per-layer figures scale to 32 layers (the weights per launch do not depend on the layer count).  Valid only for
 # the GEMM source that was captured, recognised by its SHA-256.
-GEMM_TRAFFIC = {"gemm_source_sha256": "de83f7b649dffd5be7d645cecaf8447a529282393c0be1c1ac6f1d4787707863",
-                "batch": 32, "per_layer_bytes": 438855680, "lm_head_bytes": 1066563328}
+GEMM_TRAFFIC = {"gemm_source_sha256": "662885a36d6864faa79376ae5dbfe3f06cc721f738cf31c3d9c1fbe2e47f4d1e",
+                "batch": 32, "per_layer_bytes": 440052096, "lm_head_bytes": 1065866496}
 
 
 def gemm_traffic_per_launch(cfg, B):
