@@ -44,6 +44,7 @@ def parse():
     ap.add_argument("--sweep", default="1,4,8,16,32", help="extra batch sizes to report ('' = none)")
     ap.add_argument("--no-fast", action="store_true", help="skip the non-invariant FAST-variant comparison")
     ap.add_argument("--no-layercast", action="store_true", help="skip the LayerCast-mode line")
+    ap.add_argument("--no-lmhead", action="store_true", help="skip the LM-head-alone timing")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -273,6 +274,50 @@ def run_decode(m, B, P, K, W, ws, rank, graph=True):
     return rec
 
 
+def time_lmhead(m, batches=(1, 4, 32, 256), reps=20):
+    """The LM-head logprob alone (hidden 4096, vocab 128256): per batch, the time of one bi_lmhead_logprob call with
+    the selective recompute at threshold 0.1 and with it disabled, the recompute rate, and the weight GB/s."""
+    import ctypes
+    import torch
+    import synth
+    from invariant_deterministic_full_b200._lib import lib
+    W = m.w["lm_head"]
+    V, H = W.shape
+    dev = m.device
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    res = {}
+    for B in batches:
+        h = torch.from_numpy(synth.hidden_states(7, B, H)).to(dev)
+        out = [torch.empty(B, dtype=t, device=dev) for t in (torch.float32, torch.float32, torch.int32, torch.float32,
+                                                               torch.uint8)]
+        wsb = lib.bi_lmhead_workspace_size(B, H, V, 0)
+        ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+        p = lambda t: ctypes.c_void_p(t.data_ptr())
+
+        def call(th):
+            rc = lib.bi_lmhead_logprob(p(h), p(W), None, B, H, V, th, 0, *[p(o) for o in out], None, p(ws), wsb, st)
+            assert rc == 0, lib.bi_last_error()
+
+        row = {}
+        for name, th in (("recompute", 0.1), ("no_recompute", 0.0)):
+            for _ in range(3):
+                call(th)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                call(th)
+            e1.record()
+            e1.synchronize()
+            us = e0.elapsed_time(e1) / reps * 1e3
+            row[name + "_us"] = round(us, 1)
+            if name == "recompute":
+                row["recompute_rate"] = round(float(out[4].float().mean().item()), 4)
+        row["weight_GBps"] = round(V * H * 2 / (row["no_recompute_us"] * 1e-6) / 1e9, 1)
+        row["recompute_overhead"] = round(row["recompute_us"] / row["no_recompute_us"] - 1, 4)
+        res[str(B)] = row
+    return res
+
+
 def time_gemms(m, B, reps=3):
     """Average duration of the weight-streaming GEMM launches of one decode step, timed alone with CUDA events
     on the launching stream (all layers' four projections + the LM-head GEMM, B token rows)."""
@@ -483,6 +528,10 @@ def main_ours(args):
         mf.close()
         del mf
         torch.cuda.empty_cache()
+    if mode == 0 and not args.no_lmhead and cfg["hidden"] == 4096:
+        line["lmhead_alone"] = {"config": "hidden 4096, vocab 128256, bf16 W, fp32 rows N(0,1) RMS-normalised "
+                                          "(seed 7), threshold 0.1 vs recompute off",
+                                "per_batch": time_lmhead(m)}
     if mode == 0 and not args.no_layercast:
         ml = mdl.Model(cfg, mode=1, n_slots=max(B, 1), capacity=cap, init="device")
         rl = run_decode(ml, B, P, min(K, 16), W, 1, rank)

@@ -94,14 +94,19 @@ long long bi_launch_count(void);
  *   or 4, set by N alone) that are added in a fixed tree at the end.
  *   ("Meituan bitwise train/infer consistency": TP rewritten to full-K
  *   computation instead of segmented reduce-scatter.)
- * mode BI_MODE_BF16: x is bf16.  mode BI_MODE_LAYERCAST: x is f32 and w is
- *   upcast to f32 in registers; products and sums are fp32 FMA.
+ * mode BI_MODE_BF16: x is bf16.  mode BI_MODE_LAYERCAST: x is f32 and the
+ *   products are fp32-exact: every x is split exactly into three bf16 parts
+ *   (x = p0 + p1 + p2, 8+8+8 significant bits), each part times the bf16 w is
+ *   an exact product accumulated in fp32 on the tensor cores (full K,
+ *   ascending, as above), and the three sums are added as (y0 + y1) + y2
+ *   before the epilogue.
  * y_dtype: BI_DTYPE_BF16 (round-to-nearest-even) or BI_DTYPE_F32.
  * epilogue BI_EPI_SWIGLU: w rows are gate/up interleaved by BI_GU_INTERLEAVE
  *   and y has N/2 columns: y = silu(gate) * up, silu(g) = g / (1 + exp(-g)).
  * Requirements: K % 64 == 0, N % 64 == 0, ldx % 8 == 0 (16-byte rows),
  *   x, w 16-byte aligned; else BI_ERR_UNSUPPORTED.
- * Workspace: bi_gemm_workspace_size() bytes (0 for the invariant variant). */
+ * Workspace: bi_gemm_workspace_size() bytes (0 for the invariant bf16 mode;
+ *   LayerCast needs room for the split rows and their three partial sums). */
 size_t bi_gemm_workspace_size(int M, int N, int K, int mode, int variant);
 int bi_gemm(const void* x, int ldx, const void* w, void* y, int ldy, int y_dtype, int M, int N, int K,
             int epilogue, int mode, int variant, void* ws, size_t ws_bytes, void* stream);

@@ -593,8 +593,16 @@ static int gemm_fast_splits(int M, int n_items, int kstages) {
   return s;
 }
 
+// LayerCast on tensor cores: rows of x per pass (bounds the workspace)
+constexpr int LC_ROWS = 256;
+static size_t lc_ws_bytes(int M, int N, int K) {
+  const size_t mb = (size_t)std::min(M, LC_ROWS);
+  return 3 * mb * K * 2 + 3 * mb * N * 4 + 512;
+}
+
 size_t gemm_ws_bytes(int M, int N, int K, int mode, int variant) {
-  if (variant != BI_VARIANT_FAST || mode != BI_MODE_BF16) return 0;
+  if (mode == BI_MODE_LAYERCAST) return M > 0 ? lc_ws_bytes(M, N, K) : 0;
+  if (variant != BI_VARIANT_FAST) return 0;
   const int bn = gemm_pick_bn(N);
   const int items = (N / bn) * ((M + GEMM_BM - 1) / GEMM_BM);
   const int kbs = gemm_kbs(bn);
@@ -714,6 +722,77 @@ int gemm_f32(const float* x, int ldx, const void* w, void* y, int ldy, int y_f32
   else
     BI_TRY(launch(gemm_f32_kernel<BI_EPI_NONE>, dim3(grid), dim3(256), 0, st, x, ldx, reinterpret_cast<const uint16_t*>(w), y, ldy, y_f32, M,
                                                        N, K, count));
+  return BI_OK;
+}
+
+// ---------------------------------------------------------------- LayerCast on tensor cores
+// FP32 products with bf16 weights, on the tensor cores: every f32 activation
+// is split exactly into three bf16 parts x = p0 + p1 + p2 (p0 = bf16(x),
+// p1 = bf16(x - p0), p2 = x - p0 - p1: 8 + 8 + 8 significant bits), every
+// product of a part with a bf16 weight is exact, and each part's products are
+// accumulated in fp32 over the full K in the invariant GEMM.  The three
+// accumulations are added as (y0 + y1) + y2, then the epilogue runs in fp32.
+// ("Give Me FP32 or Give Me Death?", LayerCast section: bf16-stored weights,
+// FP32 computation.)  Per element this is independent of M, so prefill and
+// decode stay bitwise equal.
+__global__ void lc_split_kernel(const float* __restrict__ x, int ldx, int mb, int K, uint16_t* __restrict__ xs) {
+  pdl_wait();
+  pdl_trigger();
+  const size_t n = (size_t)mb * K;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t r = i / K, k = i % K;
+    const float v = x[r * ldx + k];
+    const uint16_t p0 = f32_to_bf16_bits(v);
+    const float r0 = v - bf16_bits_to_f32(p0);  // exact
+    const uint16_t p1 = f32_to_bf16_bits(r0);
+    const float r1 = r0 - bf16_bits_to_f32(p1);  // exact, at most 8 significant bits
+    xs[i] = p0;
+    xs[n + i] = p1;
+    xs[2 * n + i] = f32_to_bf16_bits(r1);
+  }
+}
+
+__global__ void lc_combine_kernel(const float* __restrict__ yt, int mb, int N, void* __restrict__ y, int ldy,
+                                  int y_f32, int swiglu) {
+  pdl_wait();
+  pdl_trigger();
+  const int n_out = swiglu ? N / 2 : N;
+  const size_t total = (size_t)mb * n_out;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total; idx += (size_t)gridDim.x * blockDim.x) {
+    const int r = (int)(idx / n_out), c = (int)(idx % n_out);
+    auto z = [&](int col) {
+      return (yt[(size_t)r * N + col] + yt[(size_t)(mb + r) * N + col]) + yt[(size_t)(2 * mb + r) * N + col];
+    };
+    float v;
+    if (swiglu) {
+      const int blk = c / BI_GU_INTERLEAVE, rr = c % BI_GU_INTERLEAVE;
+      v = silu(z(blk * 2 * BI_GU_INTERLEAVE + rr)) * z(blk * 2 * BI_GU_INTERLEAVE + BI_GU_INTERLEAVE + rr);
+    } else {
+      v = z(c);
+    }
+    store_act(y, (size_t)r * ldy + c, v, y_f32);
+  }
+}
+
+int gemm_layercast(const float* x, int ldx, const void* w, void* y, int ldy, int y_f32, int M, int N, int K, int epi,
+                   void* ws, size_t ws_bytes, cudaStream_t st) {
+  const size_t need = lc_ws_bytes(M, N, K);
+  BI_REQUIRE(ws && ws_bytes >= need, BI_ERR_WORKSPACE, "bi_gemm LayerCast: workspace %zu < %zu", ws_bytes, need);
+  const int MB = std::min(M, LC_ROWS);
+  uint16_t* xs = reinterpret_cast<uint16_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
+  float* yt = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(xs + (size_t)3 * MB * K) + 255) & ~uintptr_t(255));
+  const int n_out = epi == BI_EPI_SWIGLU ? N / 2 : N;
+  for (int m0 = 0; m0 < M; m0 += MB) {
+    const int mb = std::min(MB, M - m0);
+    const size_t n = (size_t)mb * K;
+    BI_TRY(launch(lc_split_kernel, dim3((int)std::min<size_t>((n + 255) / 256, 8 * (size_t)num_sms())), dim3(256), 0,
+                  st, x + (size_t)m0 * ldx, ldx, mb, K, xs));
+    BI_TRY(gemm_bf16(xs, K, w, yt, N, 1, 3 * mb, N, K, BI_EPI_NONE, BI_VARIANT_INVARIANT, nullptr, 0, st));
+    const size_t tot = (size_t)mb * n_out;
+    void* yb = reinterpret_cast<uint8_t*>(y) + (size_t)m0 * ldy * (y_f32 ? 4 : 2);
+    BI_TRY(launch(lc_combine_kernel, dim3((int)std::min<size_t>((tot + 255) / 256, 8 * (size_t)num_sms())), dim3(256),
+                  0, st, yt, mb, N, yb, ldy, y_f32, epi == BI_EPI_SWIGLU ? 1 : 0));
+  }
   return BI_OK;
 }
 

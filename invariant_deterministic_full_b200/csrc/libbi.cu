@@ -50,7 +50,7 @@ static int gemm_run(const void* x, int ldx, const void* w, void* y, int ldy, int
   if (M == 0) return BI_OK;
   const int y_f32 = y_dtype == BI_DTYPE_F32;
   if (mode == BI_MODE_LAYERCAST)
-    return gemm_f32(reinterpret_cast<const float*>(x), ldx, w, y, ldy, y_f32, M, N, K, epi, nullptr, st);
+    return gemm_layercast(reinterpret_cast<const float*>(x), ldx, w, y, ldy, y_f32, M, N, K, epi, ws, ws_bytes, st);
   return gemm_bf16(x, ldx, w, y, ldy, y_f32, M, N, K, epi, variant, ws, ws_bytes, st);
 }
 
