@@ -536,7 +536,8 @@ def main_ours(args):
         ml = mdl.Model(cfg, mode=1, n_slots=max(B, 1), capacity=cap, init="device")
         rl = run_decode(ml, B, P, min(K, 16), W, 1, rank)
         line["layercast"] = {"value": round(B * min(K, 16) / (rl["ms"] / 1e3), 2), "unit": "tok/s",
-                             "batch": B, "note": "bf16 weights upcast in registers, fp32 FMA, fp32 activations/KV"}
+                             "batch": B, "note": "bf16 weights, fp32 activations/KV; projections as exact fp32 "
+                                                 "products on tensor cores (3-way bf16 split of the activations)"}
         ml.close()
         del ml
     if rank == 0 and not args.no_cpu:
