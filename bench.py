@@ -165,22 +165,32 @@ def step_bytes(cfg, B, ctx_lens, f32_kv=False):
 # DRAM bytes (read + write) of the weight-streaming GEMM launches of one decode step at batch 32, from one ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum) of the same shapes on the 2-layer 8B-width case; the
 # per-layer figures scale to 32 layers (the weights per launch do not depend on the layer count).  Valid only for
-# the GEMM source that was captured, recognised by its SHA-256.
-GEMM_TRAFFIC = {"gemm_source_sha256": "662885a36d6864faa79376ae5dbfe3f06cc721f738cf31c3d9c1fbe2e47f4d1e",
+# the GEMM kernel source that was captured, recognised by gemm_bf16_source_digest.
+GEMM_TRAFFIC = {"gemm_bf16_source_sha256": "987ba4cf7027c4880d0eca32dc2805afa56d0b0fc8691a2705d5c149efa4f80a",
                 "batch": 32, "per_layer_bytes": 440052096, "lm_head_bytes": 1065866496}
+
+
+def gemm_bf16_source_digest(text):
+    """sha256 of the part of gemm.cuh that decides the bf16 GEMM's memory traffic: everything up to the FAST split
+    heuristic (tile configs, the kernel, the tile and ring pickers) plus its launch and dispatch code.  Workspace
+    sizing and the LayerCast split/combine kernels are left out, since they do not touch this kernel."""
+    import hashlib
+    a = text.index("static int gemm_fast_splits")
+    b0 = text.index("template <int BN, int EPI, int MT = 1, int CPS = 1>\nstatic int launch_gemm_bf16_t")
+    b1 = text.index("int gemm_f32(")
+    return hashlib.sha256((text[:a] + text[b0:b1]).encode()).hexdigest()
 
 
 def gemm_traffic_per_launch(cfg, B):
     """Measured DRAM bytes per launch of the timed GEMM set, or None when they no longer apply."""
-    import hashlib
     src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "invariant_deterministic_full_b200", "csrc",
                        "gemm.cuh")
     try:
-        with open(src, "rb") as f:
-            h = hashlib.sha256(f.read()).hexdigest()
-    except OSError:
+        with open(src) as f:
+            h = gemm_bf16_source_digest(f.read())
+    except (OSError, ValueError):
         return None
-    if h != GEMM_TRAFFIC["gemm_source_sha256"] or B != GEMM_TRAFFIC["batch"] or cfg["hidden"] != 4096:
+    if h != GEMM_TRAFFIC["gemm_bf16_source_sha256"] or B != GEMM_TRAFFIC["batch"] or cfg["hidden"] != 4096:
         return None
     L = cfg["n_layers"]
     return (L * GEMM_TRAFFIC["per_layer_bytes"] + GEMM_TRAFFIC["lm_head_bytes"]) / (4 * L + 1)

@@ -104,7 +104,8 @@ long long bi_launch_count(void);
  * epilogue BI_EPI_SWIGLU: w rows are gate/up interleaved by BI_GU_INTERLEAVE
  *   and y has N/2 columns: y = silu(gate) * up, silu(g) = g / (1 + exp(-g)).
  * Requirements: K % 64 == 0, N % 64 == 0, ldx % 8 == 0 (16-byte rows),
- *   x, w 16-byte aligned; else BI_ERR_UNSUPPORTED.
+ *   x, w 16-byte aligned; else BI_ERR_UNSUPPORTED.  M == 0 is a no-op
+ *   (x and y may then be NULL); w NULL is BI_ERR_INVALID_ARG.
  * Workspace: bi_gemm_workspace_size() bytes (0 for the invariant bf16 mode;
  *   LayerCast needs room for the split rows and their three partial sums). */
 size_t bi_gemm_workspace_size(int M, int N, int K, int mode, int variant);

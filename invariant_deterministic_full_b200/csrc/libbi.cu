@@ -36,7 +36,7 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // ------------------------------------------------------------------ GEMM
 static int gemm_run(const void* x, int ldx, const void* w, void* y, int ldy, int y_dtype, int M, int N, int K, int epi,
                     int mode, int variant, void* ws, size_t ws_bytes, cudaStream_t st) {
-  BI_REQUIRE(x && w && y, BI_ERR_INVALID_ARG, "bi_gemm: NULL pointer");
+  BI_REQUIRE(w && ((x && y) || M == 0), BI_ERR_INVALID_ARG, "bi_gemm: NULL pointer");
   BI_REQUIRE(M >= 0 && N > 0 && K > 0, BI_ERR_INVALID_ARG, "bi_gemm: bad sizes M=%d N=%d K=%d", M, N, K);
   BI_REQUIRE(K % 64 == 0 && N % 64 == 0, BI_ERR_UNSUPPORTED, "bi_gemm: need K %% 64 == 0 and N %% 64 == 0 (N=%d K=%d)",
              N, K);

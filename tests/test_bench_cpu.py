@@ -1,0 +1,59 @@
+"""Host-side bookkeeping of bench.py: the algorithmic byte counts behind the roofline fractions, the stored ncu
+traffic and its source guard, and the clock-record parser (no GPU)."""
+import pytest
+
+import bench
+from synth import configs
+
+L8 = configs.LLAMA8B
+# Llama 3.1 8B: 8,030,261,248 parameters (embedding and LM head untied); its model card rounds this to 8.03B.
+LLAMA31_8B_PARAMS = 8_030_261_248
+
+
+def test_step_weight_bytes_match_the_published_parameter_count():
+    # A decode step streams every weight once except the embedding table, of which it gathers only B rows.
+    embed = L8["vocab"] * L8["hidden"]
+    assert bench.step_bytes(L8, 0, []) == 2 * (LLAMA31_8B_PARAMS - embed)
+
+
+@pytest.mark.parametrize("ctx", [0, 1, 517, 4095])
+def test_step_kv_bytes_are_128_kib_per_position(ctx):
+    # GQA with 8 KV heads of 128: k and v, bf16, 32 layers -> 128 KiB per cached position of one sequence.
+    w = bench.step_bytes(L8, 0, [])
+    got = bench.step_bytes(L8, 1, [ctx]) - w - 2 * L8["hidden"]
+    assert got == (ctx + 2) * 128 * 1024  # positions 0..ctx read, one position written
+    assert bench.step_bytes(L8, 1, [ctx], f32_kv=True) - w - 2 * L8["hidden"] == 2 * got
+
+
+def test_gemm_set_is_four_projections_per_layer_plus_the_lm_head():
+    tot, n = bench.gemm_bytes(L8, 32)
+    assert n == 4 * L8["n_layers"] + 1
+    assert bench.gemm_bytes(L8, 0)[0] == bench.step_bytes(L8, 0, []) - 2 * L8["n_layers"] * 2 * L8["hidden"] - 2 * L8["hidden"]
+    assert tot / n == pytest.approx(117.4e6, rel=1e-3)
+
+
+def test_stored_gemm_traffic_applies_to_this_source_and_equals_the_algorithmic_bytes():
+    src = open(bench.os.path.join(bench.ROOT, "invariant_deterministic_full_b200", "csrc", "gemm.cuh")).read()
+    assert len(bench.gemm_bf16_source_digest(src)) == 64  # the digest's landmarks are all present
+    t = bench.gemm_traffic_per_launch(L8, 32)
+    if t is None:
+        pytest.skip("GEMM kernel source changed since the stored ncu capture: traffic is reported as null")
+    tot, n = bench.gemm_bytes(L8, 32)
+    assert t == pytest.approx(tot / n, rel=0.01)  # no re-reads beyond the algorithmic bytes
+    assert bench.gemm_traffic_per_launch(L8, 16) is None  # captured at batch 32 only
+
+
+def test_gemm_source_digest_ignores_code_outside_the_bf16_kernel():
+    src = open(bench.os.path.join(bench.ROOT, "invariant_deterministic_full_b200", "csrc", "gemm.cuh")).read()
+    h = bench.gemm_bf16_source_digest(src)
+    assert bench.gemm_bf16_source_digest(src + "\n// trailing helper\n") == h
+    i = src.index("__global__ void __launch_bounds__(160, CPS)")
+    assert bench.gemm_bf16_source_digest(src[:i] + " " + src[i:]) != h
+
+
+def test_clock_summary_median_and_reasons():
+    c = bench.ClockSampler(0)
+    row = lambda mhz, pc: ["0", str(mhz), "1965", "700", "0x4", "Not Active", "Not Active", "Not Active", pc]
+    c.rows = [row(1965, "Not Active"), row(1800, "Active"), row(1965, "Not Active"), ["garbage"]]
+    s = c.summary()
+    assert s == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}

@@ -158,6 +158,26 @@ def test_gemm_m_blocking_invariance(bi, epilogue):
     _after(bi)
 
 
+def test_gemm_layercast_row_blocks_and_empty(bi):
+    """LayerCast runs the exact 3-part split in passes of at most 256 token rows: a row's bits must not depend on
+    which pass (or which batch) computed it; M = 0 is a no-op."""
+    rng = np.random.default_rng(17)
+    N, K = 1024, 512
+    xs = rng.standard_normal((600, K)).astype(np.float32)
+    w = _bf16_dev(0.02 * rng.standard_normal((N, K)))
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    full = bi.gemm(dev(xs), w, mode=1, out_dtype=torch.float32).cpu()
+    for M, off in [(1, 599), (255, 0), (256, 100), (257, 3), (300, 290)]:
+        part = bi.gemm(dev(xs[off:off + M]), w, mode=1, out_dtype=torch.float32).cpu()
+        assert torch.equal(part, full[off:off + M]), (M, off)
+    ref = oracle.gemm(xs[:8].astype(np.float64), synth.f32_to_bf16_bits(_f(w).astype(np.float32)))
+    bound = K * 2.0 ** -24 * (np.abs(xs[:8]).astype(np.float64) @ np.abs(_f(w)).T)
+    assert (np.abs(_f(full[:8]) - ref) <= bound + 1e-30).all()
+    empty = bi.gemm(dev(xs[:0]), w, mode=1, out_dtype=torch.float32)
+    assert empty.shape == (0, N)
+    _after(bi)
+
+
 def test_gemm_fast_variant_is_not_invariant_but_close(bi):
     rng = np.random.default_rng(6)
     N, K = 4096, 4096
