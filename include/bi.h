@@ -25,6 +25,12 @@
  *    the host during the call only.  Layouts are row-major, contiguous unless
  *    a leading dimension is given.
  *  - bf16 = IEEE bfloat16 bit pattern (uint16); f32 = IEEE binary32.
+ *  - Kernels use programmatic dependent launch: a library kernel may start
+ *    while the library kernel before it on the stream is finishing.  The GEMM
+ *    reads its weight w before it waits for that kernel; every other operand
+ *    of every call is touched only after the wait.  So a GEMM weight must not
+ *    be the output of the library call enqueued just before it (kernels of the
+ *    caller's own, copies and other libraries are waited for in full).
  */
 #ifndef BI_H
 #define BI_H

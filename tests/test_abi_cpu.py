@@ -53,6 +53,9 @@ def test_gemm_validation(L):
     assert lib.bi_gemm(fake, 64, ctypes.c_void_p((1 << 20) + 2), fake, 64, 0, 4, 64, 64, 0, 0, 0, None, 0,
                        None) == L.BI_ERR_UNSUPPORTED
     assert lib.bi_gemm(fake, 64, fake, fake, 64, 0, 0, 64, 64, 0, 0, 0, None, 0, None) == L.BI_OK  # M = 0: no work
+    assert lib.bi_gemm(None, 64, fake, None, 64, 0, 0, 64, 64, 0, 0, 0, None, 0, None) == L.BI_OK  # empty x, y
+    assert lib.bi_gemm(None, 64, None, None, 64, 0, 0, 64, 64, 0, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
+    assert lib.bi_gemm(fake, 64, fake, None, 64, 0, 4, 64, 64, 0, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
     assert lib.bi_gemm_workspace_size(4, 64, 64, 0, 0) == 0
 
 
