@@ -81,10 +81,17 @@ int bi_version(void);
  * position beyond capacity or an out-of-range id sets a bit here instead
  * (1 = wait timeout, 2 = capacity, 4 = index) and the kernel skips the access.
  * Bits 8 and up name the first wait that ran out (a site code of the kernel:
- * 0x11/0x12/0x13 GEMM ring empty/full/drain, 0x21/0x22 attention; higher bits
- * carry the kernel's configuration), 0 when none did.
+ * 0x11/0x12/0x13 GEMM ring empty/full/drain, 0x21/0x22 attention, 0x31 the
+ * wait self-test; higher bits carry the kernel's configuration), 0 when none
+ * did.  Every wait gives up after about 1 s of wall-clock time.
  * Synchronous read of the current device's word; reset != 0 clears it. */
 int bi_device_error(unsigned* flags, int reset);
+/* Failure-path check of the bounded waits, without faulting the GPU: one CTA
+ * waits on a barrier that nothing completes; after about 1 s the wait gives up,
+ * sets bit 1 of the device error word with site code 0x31, and the kernel
+ * returns, leaving the context usable.  Asynchronous on the stream; read the
+ * outcome with bi_device_error after synchronising. */
+int bi_selftest_wait_timeout(void* stream);
 int bi_num_sms(int device); /* SM count of a device, -1 on error */
 /* Number of kernels the library has launched in this process (host-side
  * counter, incremented at every launch site; not thread-safe). */

@@ -69,6 +69,7 @@ SIGNATURES = {
     "bi_device_error": (I, [ctypes.POINTER(ctypes.c_uint), I]),
     "bi_num_sms": (I, [I]),
     "bi_launch_count": (ctypes.c_longlong, []),
+    "bi_selftest_wait_timeout": (I, [P]),
     "bi_gemm_workspace_size": (SZ, [I, I, I, I, I]),
     "bi_gemm": (I, [P, I, P, P, I, I, I, I, I, I, I, I, P, SZ, P]),
     "bi_rmsnorm": (I, [P, P, P, P, P, P, I, I, F, I, P]),

@@ -139,7 +139,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
 }
 enum : unsigned {
   SITE_GEMM_EMPTY = 0x11, SITE_GEMM_FULL = 0x12, SITE_GEMM_DRAIN = 0x13,
-  SITE_ATTN_CORE = 0x21, SITE_ATTN_TC = 0x22
+  SITE_ATTN_CORE = 0x21, SITE_ATTN_TC = 0x22, SITE_SELFTEST = 0x31
 };
 
 // 2D tiled TMA load into shared memory, completion counted on an mbarrier.

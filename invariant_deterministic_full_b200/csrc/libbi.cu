@@ -331,6 +331,22 @@ static int lmhead_run(const float* h, const void* W, const int32_t* target, int 
   return BI_OK;
 }
 
+// Failure-path check of the bounded waits: one thread waits on an mbarrier that
+// nothing arrives at (no copy is in flight), so the wait runs out after kWaitNs,
+// records the timeout bit and SITE_SELFTEST in the device error word and the
+// kernel returns normally.
+__global__ void wait_selftest_kernel() {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0u, SITE_SELFTEST);
+}
+
 }  // namespace bi
 
 // ====================================================================== C ABI
@@ -363,6 +379,12 @@ int bi_device_error(unsigned* flags, int reset) {
     BI_CHECK_CUDA(cudaMemcpyToSymbol(g_dev_error, &z, sizeof(z)));
     BI_CHECK_CUDA(cudaMemcpyToSymbol(g_dev_site, &z, sizeof(z)));
   }
+  return BI_OK;
+}
+
+int bi_selftest_wait_timeout(void* stream) {
+  clear_error();
+  BI_TRY(launch(wait_selftest_kernel, dim3(1), dim3(32), 0, as_stream(stream)));
   return BI_OK;
 }
 

@@ -121,6 +121,11 @@ def greedy_advance(argmax, ids, pos):
     check(lib.bi_greedy_advance(_ptr(argmax), _ptr(ids), _ptr(pos), ids.shape[0], _stream()), "bi_greedy_advance")
 
 
+def selftest_wait_timeout():
+    """Enqueue the bounded-wait failure check (bi_selftest_wait_timeout) on the current stream."""
+    check(lib.bi_selftest_wait_timeout(_stream()), "bi_selftest_wait_timeout")
+
+
 def device_error(reset=True):
     v = ctypes.c_uint(0)
     check(lib.bi_device_error(ctypes.byref(v), 1 if reset else 0), "bi_device_error")

@@ -13,8 +13,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def L():
-    from invariant_deterministic_full_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._lib_builder().build()
     from invariant_deterministic_full_b200 import _lib
     return _lib
 
