@@ -361,9 +361,11 @@ def time_gemms(m, B, reps=3):
     return e0.elapsed_time(e1) / reps
 
 
-def run_e2e(m, B, P, K, rank):
+def run_e2e(m, B, P, K, rank, graph=True):
     """Same metric through the public API with host buffers: per step an H2D copy of the step's inputs from
-    pinned host memory, bi_decode_step, and a D2H read of the step's results; the host feeds the next ids."""
+    pinned host memory, bi_decode_step, and a D2H read of the step's results; the host feeds the next ids.
+    graph=True: the step is bi_decode_step captured once in a CUDA graph (after one eager step) and replayed,
+    the way a serving loop issues it; graph=False: bi_decode_step is called eagerly every step."""
     import numpy as np
     import torch
     import synth
@@ -383,18 +385,34 @@ def run_e2e(m, B, P, K, rank):
     d_in = torch.empty(4, B, dtype=torch.int32, device=dev)
     out = m.alloc_out(B)
     slots_h = torch.arange(B, dtype=torch.int32)
+    max_pos = P + K + 1
+    pos_plan = torch.full((B,), max_pos, dtype=torch.int32)  # the last position the steps reach, for planning
+    m.workspace(B, B, max_pos)
+
+    def one_step():
+        m.step_dev(B, d_in[0], d_in[1], d_in[2], slots_h, pos_plan, d_in[3], B, None, out, max_pos=max_pos)
+
     st = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     cur = P
+    run, g = one_step, None
     for it in range(K + 1):
         if it == 1:
+            if graph:  # capture after the eager first step (one-time library set-up stays outside the capture)
+                g = torch.cuda.CUDAGraph()
+                s = torch.cuda.Stream()
+                s.wait_stream(st)
+                with torch.cuda.graph(g, stream=s):
+                    one_step()
+                st.wait_stream(s)
+                run = g.replay
             e0.record()
         h_in[0].copy_(torch.from_numpy(nxt))
         h_in[1].copy_(slots_h)
         h_in[2].fill_(cur)
         h_in[3].copy_(torch.arange(B, dtype=torch.int32))
         d_in.copy_(h_in, non_blocking=True)
-        m.step_dev(B, d_in[0], d_in[1], d_in[2], slots_h, h_in[2].clone(), d_in[3], B, None, out)
+        run()
         h_out_ids.copy_(out["argmax"], non_blocking=True)
         h_out_lp.copy_(out["logprob"], non_blocking=True)
         st.synchronize()
@@ -403,6 +421,8 @@ def run_e2e(m, B, P, K, rank):
     e1.record()
     e1.synchronize()
     ms = e0.elapsed_time(e1)
+    if g is not None:
+        del g
     return dict(ms=ms, h2d=4 * B * 4, d2h=B * 4 + B * 4)
 
 
@@ -513,9 +533,14 @@ def main_ours(args):
         line["roofline"] = {"bound": "alu", "achieved": None, "peak": None, "unit": "TFLOP/s", "frac": None,
                             "traffic": None}
     if rank == 0 and not args.no_e2e:
-        e = run_e2e(m, B, P, min(K, 32), rank)
-        line["e2e"] = {"value": round(B * min(K, 32) / (e["ms"] / 1e3) * ws, 2), "unit": "tok/s",
-                       "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"]}
+        ke = min(K, 32)
+        e = run_e2e(m, B, P, ke, rank, graph=True)
+        ee = run_e2e(m, B, P, ke, rank, graph=False)
+        line["e2e"] = {"value": round(B * ke / (e["ms"] / 1e3) * ws, 2), "unit": "tok/s",
+                       "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
+                       "call": "bi_decode_step captured once in a CUDA graph, replayed per step between the "
+                               "pinned H2D copy of the step's inputs and the D2H read of its results",
+                       "eager_value": round(B * ke / (ee["ms"] / 1e3) * ws, 2)}
     # batch sweep and the non-invariant comparison (same weights)
     extra, extra_frac = {}, {}
     for b in sweep:
