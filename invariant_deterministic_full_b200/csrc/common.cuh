@@ -142,15 +142,6 @@ enum : unsigned {
   SITE_ATTN_CORE = 0x21, SITE_ATTN_TC = 0x22, SITE_SELFTEST = 0x31
 };
 
-// 2D tiled TMA load into shared memory, completion counted on an mbarrier.
-__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int c_inner, int c_outer,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-          "r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c_inner), "r"(c_outer), "r"(smem_u32(bar))
-      : "memory");
-}
 // 3D tiled TMA load (coordinates innermost first).
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, int c0, int c1, int c2,
                                             uint64_t* bar) {
