@@ -55,9 +55,11 @@ enum { BI_MODE_BF16 = 0, BI_MODE_LAYERCAST = 1 };
 /* BI_MODE_BF16: bf16 activations and KV cache, bf16 x bf16 products with fp32
  *   accumulation on tensor cores, fp32 softmax/norm arithmetic.
  * BI_MODE_LAYERCAST: the "LayerCast" scheme of "Give Me FP32 or Give Me
- *   Death?" (LayerCast section): weights stay bf16 in memory and are cast to
- *   fp32 in registers just before use; every product and sum is fp32 FMA;
- *   activations and KV cache are fp32. */
+ *   Death?" (LayerCast section): weights stay bf16 in memory and the
+ *   arithmetic is fp32; activations and KV cache are fp32.  Projections take
+ *   exact fp32 products on the tensor cores (see bi_gemm); the LM head,
+ *   attention and norms use fp32 FMA on the CUDA cores, with the bf16
+ *   weights cast to fp32 in registers. */
 enum { BI_VARIANT_INVARIANT = 0, BI_VARIANT_FAST = 1 };
 /* BI_VARIANT_FAST is the non-invariant comparison baseline: split-K GEMMs
  * whose split factor is chosen from the row count M and the SM count, and
