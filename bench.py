@@ -46,6 +46,7 @@ def parse():
     ap.add_argument("--no-layercast", action="store_true", help="skip the LayerCast-mode line")
     ap.add_argument("--no-lmhead", action="store_true", help="skip the LM-head-alone timing")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill throughput line")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--layers", type=int, default=0,
@@ -282,6 +283,40 @@ def run_decode(m, B, P, K, W, ws, rank, graph=True):
     if graph:
         del g
     return rec
+
+
+def prefill_flops(cfg, B, P):
+    """FLOPs of one batched prefill of B prompts of P tokens with the LM head on each prompt's last token:
+    2 x projection weights x tokens, causal attention (q.k and p.v over positions 0..t of every q head), LM head."""
+    L, H, Hq, Hkv, d, F, V = (cfg["n_layers"], cfg["hidden"], cfg["n_heads"], cfg["n_kv_heads"], cfg["head_dim"],
+                              cfg["ffn"], cfg["vocab"])
+    proj = (Hq + 2 * Hkv) * d * H + H * Hq * d + 3 * F * H
+    att = 2 * 2 * d * Hq * L * B * (P * (P + 1) // 2)
+    return 2 * L * proj * B * P + att + 2 * V * H * B
+
+
+def time_prefill(m, B, P, rank, reps=2):
+    """Device time of the batched prefill of B prompts of P tokens (one bi_decode_step over B*P tokens), averaged
+    over reps identical calls after an untimed one; every call writes the same KV rows."""
+    import numpy as np
+    import torch
+    import synth
+    V = m.cfg["vocab"]
+    prompts = [synth.prompt_tokens(1000 * rank + r, P, V) for r in range(B)]
+    ids = np.concatenate(prompts).astype(np.int32)
+    slots = np.repeat(np.arange(B), P).astype(np.int32)
+    pos = np.tile(np.arange(P), B).astype(np.int32)
+    lm = np.full(B * P, -1, dtype=np.int32)
+    lm[np.arange(B) * P + P - 1] = np.arange(B)
+    m.step(ids, slots, pos, lm)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        m.step(ids, slots, pos, lm)
+    e1.record()
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps
 
 
 def time_lmhead(m, batches=(1, 4, 32, 256), reps=20):
@@ -532,6 +567,15 @@ def main_ours(args):
     else:
         line["roofline"] = {"bound": "alu", "achieved": None, "peak": None, "unit": "TFLOP/s", "frac": None,
                             "traffic": None}
+    if rank == 0 and mode == 0 and not args.no_prefill:
+        pms = time_prefill(m, B, P, rank)
+        pf = prefill_flops(cfg, B, P)
+        line["prefill"] = {"tokens": B * P, "ms": round(pms, 3), "tok_s": round(B * P / (pms / 1e3), 1),
+                           "tflops": round(pf / (pms / 1e3) / 1e12, 1), "peak_tflops": tf_burst,
+                           "frac": round(pf / (pms / 1e3) / 1e12 / tf_burst, 4),
+                           "note": f"one bi_decode_step over {B} prompts x {P} tokens, LM head on each last token; "
+                                   f"FLOPs = 2 x projection weights x tokens + causal attention + LM head; peak = "
+                                   f"{src} cuBLAS bf16 (burst); mma.sync tensor-core GEMMs"}
     if rank == 0 and not args.no_e2e:
         ke = min(K, 32)
         e = run_e2e(m, B, P, ke, rank, graph=True)

@@ -57,3 +57,13 @@ def test_clock_summary_median_and_reasons():
     c.rows = [row(1965, "Not Active"), row(1800, "Active"), row(1965, "Not Active"), ["garbage"]]
     s = c.summary()
     assert s == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+
+
+def test_prefill_flops_from_the_parameter_count():
+    c = L8
+    L, H, V, d, Hq = c["n_layers"], c["hidden"], c["vocab"], c["head_dim"], c["n_heads"]
+    matmul_params = LLAMA31_8B_PARAMS - 2 * V * H - H - 2 * L * H  # projections only: no embedding, LM head, norms
+    B, P = 3, 5
+    causal_pairs = B * P * (P + 1) // 2  # (query, key) pairs with key <= query, per head and layer
+    want = 2 * matmul_params * B * P + 4 * d * Hq * L * causal_pairs + 2 * V * H * B
+    assert bench.prefill_flops(c, B, P) == want
