@@ -496,6 +496,8 @@ int bi_ctx_create(const bi_model_desc* desc, const bi_weights* w, const bi_kv_la
              BI_ERR_UNSUPPORTED, "bi_ctx_create: hidden/ffn/vocab/projection sizes must be multiples of 64");
   BI_REQUIRE(d.head_dim == 64 || d.head_dim == 128, BI_ERR_UNSUPPORTED, "bi_ctx_create: head_dim must be 64 or 128");
   BI_REQUIRE(d.hidden <= 16384, BI_ERR_UNSUPPORTED, "bi_ctx_create: hidden > 16384");
+  BI_REQUIRE(d.n_heads / d.n_kv_heads <= ATT_MAX_PAIRS, BI_ERR_UNSUPPORTED,
+             "bi_ctx_create: %d q heads per kv head (max %d)", d.n_heads / d.n_kv_heads, ATT_MAX_PAIRS);
   BI_REQUIRE(w->embed && w->lm_head && w->final_norm && w->attn_norm && w->ffn_norm && w->w_qkv && w->w_o &&
                  w->w_gu && w->w_down && w->rope && w->rope_max_pos > 0,
              BI_ERR_INVALID_ARG, "bi_ctx_create: NULL weight pointer");
@@ -596,8 +598,10 @@ int bi_decode_step(bi_ctx* ctx, const bi_batch* batch, const bi_step_out* out, v
   BI_REQUIRE(n_lm == 0 || (out->logprob && out->lse && out->argmax && out->margin && out->recomputed),
              BI_ERR_INVALID_ARG, "bi_decode_step: NULL output array");
   int max_pos = 0;
-  for (int t = 0; t < T; ++t) {
-    const int p = batch->pos_host[t];
+  for (int t = 0; t < T; ++t) {  // every host-checkable argument is checked before the first launch
+    const int sl = batch->slot_host[t], p = batch->pos_host[t];
+    BI_REQUIRE(sl >= 0 && sl < ctx->kv.n_slots, BI_ERR_INVALID_ARG, "bi_decode_step: token %d slot %d of %d", t, sl,
+               ctx->kv.n_slots);
     BI_REQUIRE(p >= 0 && p < ctx->kv.capacity && p < w.rope_max_pos, BI_ERR_CAPACITY,
                "bi_decode_step: token %d position %d beyond KV capacity %d / RoPE table %d", t, p, ctx->kv.capacity,
                w.rope_max_pos);

@@ -100,6 +100,10 @@ def test_ctx_validation(L):
     bad = L.ModelDesc(1, 250, 4, 4, 64, 1024, 4096, 1e-5, 0, 0, 0.1)
     assert lib.bi_ctx_create(ctypes.byref(bad), ctypes.byref(w), ctypes.byref(kv), ctypes.byref(c2)) == \
         L.BI_ERR_UNSUPPORTED
+    bad = L.ModelDesc(1, 4096, 64, 1, 64, 1024, 4096, 1e-5, 0, 0, 0.1)  # 64 q heads on one kv head
+    kv1 = L.KvLayout(1 << 20, 1 << 20, 2, 1, 1, 64, 64, 0)
+    assert lib.bi_ctx_create(ctypes.byref(bad), ctypes.byref(w), ctypes.byref(kv1), ctypes.byref(c2)) == \
+        L.BI_ERR_UNSUPPORTED
     bad = L.ModelDesc(1, 256, 6, 4, 64, 1024, 4096, 1e-5, 0, 0, 0.1)
     assert lib.bi_ctx_create(ctypes.byref(bad), ctypes.byref(w), ctypes.byref(kv), ctypes.byref(c2)) == \
         L.BI_ERR_INVALID_ARG
@@ -125,6 +129,14 @@ def test_decode_step_capacity_and_workspace_rejected_on_host(L):
     b.n_lm = 4  # more output rows than tokens
     assert lib.bi_decode_step(ctx, ctypes.byref(b), ctypes.byref(o), ctypes.c_void_p(fake), need, None) == \
         L.BI_ERR_INVALID_ARG
+    # a slot outside the cache is rejected before anything is launched (here a launch would fail with BI_ERR_CUDA)
+    b.n_lm = 3
+    slot[1] = 2  # the tiny context has 2 slots
+    c0 = lib.bi_launch_count()
+    assert lib.bi_decode_step(ctx, ctypes.byref(b), ctypes.byref(o), ctypes.c_void_p(fake), need, None) == \
+        L.BI_ERR_INVALID_ARG
+    assert b"slot" in lib.bi_last_error()
+    assert lib.bi_launch_count() == c0
     lib.bi_ctx_destroy(ctx)
 
 
