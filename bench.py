@@ -649,9 +649,15 @@ def main_reference(args):
             "warmup": args.warmup, "ms_per_step": round(per_tok * 1e3, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
             "data": "synthetic: same recipe as the GPU arm",
-            "config": {"workload": "llama3.1-8b-shape greedy decode, 1 token per step (bounded CPU sample)",
-                       "model": "llama3.1-8b-shape (random init)", "global_batch": 1, "seq_len": 1,
-                       "parallelism": "host cores"},
+            "config": {"workload": f"llama3.1-8b-shape greedy decode, batch {args.batch} per GPU, prompt "
+                                   f"{args.prompt}, {args.steps} timed steps (positions {args.prompt + 1 + args.warmup}"
+                                   f"..{args.prompt + args.warmup + args.steps})",
+                       "model": "llama3.1-8b-shape (random init)", "global_batch": args.batch * args.gpus,
+                       "seq_len": args.prompt + args.warmup + args.steps + 1, "parallelism": "host cores (rank 0)",
+                       "mode": args.mode, "variant": "invariant", "margin_threshold": 0.1,
+                       "sample": "each step is a bounded sample of the workload: the oracle's time per decode token "
+                                 "(tokens are independent on the host, so tok/s does not depend on the batch); "
+                                 "see cpu_baseline.sample"},
             "cpu_baseline": cb,
             "e2e": {"value": round(v, 4), "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "wall_s": round(wall, 1)}
