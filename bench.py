@@ -167,19 +167,23 @@ def step_bytes(cfg, B, ctx_lens, f32_kv=False):
 # capture (dram__bytes_read.sum + dram__bytes_write.sum) of the same shapes on the 2-layer 8B-width case; the
 # per-layer figures scale to 32 layers (the weights per launch do not depend on the layer count).  Valid only for
 # the GEMM kernel source that was captured, recognised by gemm_bf16_source_digest.
-GEMM_TRAFFIC = {"gemm_bf16_source_sha256": "987ba4cf7027c4880d0eca32dc2805afa56d0b0fc8691a2705d5c149efa4f80a",
+GEMM_TRAFFIC = {"gemm_bf16_source_sha256": "9667a87af3277e94aaefde6dba3cb9b705671f2b4e455c485749f0d50f49eb40",
                 "batch": 32, "per_layer_bytes": 440052096, "lm_head_bytes": 1065866496}
 
 
 def gemm_bf16_source_digest(text):
-    """sha256 of the part of gemm.cuh that decides the bf16 GEMM's memory traffic: everything up to the FAST split
-    heuristic (tile configs, the kernel, the tile and ring pickers) plus its launch and dispatch code.  Workspace
-    sizing and the LayerCast split/combine kernels are left out, since they do not touch this kernel."""
+    """sha256 of the code (comments and whitespace removed) of the part of gemm.cuh that decides the bf16 GEMM's
+    memory traffic: everything up to the FAST split heuristic (tile configs, the kernel, the tile and ring pickers)
+    plus its launch and dispatch code.  Workspace sizing and the LayerCast split/combine kernels are left out, since
+    they do not touch this kernel."""
     import hashlib
+    import re
     a = text.index("static int gemm_fast_splits")
     b0 = text.index("template <int BN, int EPI, int MT = 1, int CPS = 1>\nstatic int launch_gemm_bf16_t")
     b1 = text.index("int gemm_f32(")
-    return hashlib.sha256((text[:a] + text[b0:b1]).encode()).hexdigest()
+    code = re.sub(r"/\*.*?\*/", " ", text[:a] + text[b0:b1], flags=re.S)  # comments and layout do not count
+    code = re.sub(r"//[^\n]*", " ", code)
+    return hashlib.sha256(" ".join(code.split()).encode()).hexdigest()
 
 
 def gemm_traffic_per_launch(cfg, B):

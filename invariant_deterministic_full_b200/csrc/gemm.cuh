@@ -19,16 +19,20 @@
 // Weight tiles (BN rows x 64 k) and token tiles (32 rows x 64 k) stream by TMA
 // (128-byte swizzle) into a multi-stage shared-memory ring filled by one
 // producer warp; four consumer warps read them with ldmatrix.  The grid is
-// persistent (at most one CTA per SM), each CTA walking its work items
+// persistent (one CTA per SM, or two with half the ring each when a launch
+// has between one and two work items per SM), each CTA walking its work items
 // (row group x token tile) so the ring never drains between items.
 //
-// LayerCast path (gemm_f32_kernel): the weight is upcast from bf16 to fp32 in
-// registers and every product/sum is an fp32 FMA ("Give Me FP32 or Give Me
-// Death?", LayerCast section).  Element order: lane l of a warp owns the
-// k-slices [256 i + 8 l, 256 i + 8 l + 8) for i = 0, 1, ...; it accumulates
-// them with sequential FMAs in ascending k, and the 32 lane partials are then
-// combined by a fixed xor-butterfly.  This is the same for every M and every
-// row/token tiling.
+// LayerCast ("Give Me FP32 or Give Me Death?", LayerCast section: bf16-stored
+// weights, fp32 arithmetic) has two routes.  Projections (gemm_layercast, at
+// the end of this file) split each f32 activation exactly into three bf16
+// parts and run them through gemm_bf16_kernel.  The LM head
+// (gemm_f32_kernel) upcasts the weight from bf16 to fp32 in registers and
+// takes every product and sum as an fp32 FMA.  Element order there: lane l of
+// a warp owns the k-slices [256 i + 8 l, 256 i + 8 l + 8) for i = 0, 1, ...;
+// it accumulates them with sequential FMAs in ascending k, and the 32 lane
+// partials are then combined by a fixed xor-butterfly.  This is the same for
+// every M and every row/token tiling.
 #pragma once
 #include "common.cuh"
 

@@ -48,7 +48,8 @@ def test_gemm_source_digest_ignores_code_outside_the_bf16_kernel():
     h = bench.gemm_bf16_source_digest(src)
     assert bench.gemm_bf16_source_digest(src + "\n// trailing helper\n") == h
     i = src.index("__global__ void __launch_bounds__(160, CPS)")
-    assert bench.gemm_bf16_source_digest(src[:i] + " " + src[i:]) != h
+    assert bench.gemm_bf16_source_digest(src[:i] + "// a comment\n  /* and another */ " + src[i:]) == h
+    assert bench.gemm_bf16_source_digest(src[:i] + "constexpr int kExtra = 1;\n" + src[i:]) != h
 
 
 def test_clock_summary_median_and_reasons():
