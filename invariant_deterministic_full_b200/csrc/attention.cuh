@@ -18,6 +18,17 @@
 //     later queries share the tile or not);
 //   * merge over chunks 0..pos/CH: M = max m_c, L = sum_c l_c exp(m_c - M),
 //     o = sum_c acc_c exp(m_c - M), all in ascending chunk order; out = o / L.
+// Those are the CUDA-core kernel's sums (f32 KV, or head size 64).  The
+// tensor-core kernel (bf16 KV, head size 128) keeps the chunk grid, the
+// denominator tree and the merge, and differs in two sums:
+//   * the score is eight mma.sync m16n8k16 steps over the head dimension in
+//     ascending order, each adding 16 exact products into the (key, pair)
+//     fp32 accumulator;
+//   * the numerator splits every p exactly into three bf16 parts; each part's
+//     products with V accumulate in fp32 over the chunk's keys in ascending
+//     16-key steps, and the parts are added as (a0 + a1) + a2.
+// Which kernel runs depends on the KV dtype and head size alone, so prefill
+// and decode always share one.
 // A query's result depends only on its q and the cache rows 0..pos it reads.
 #pragma once
 #include "common.cuh"
