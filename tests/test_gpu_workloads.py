@@ -137,3 +137,59 @@ def test_qwen_32k_chunked_prefill_and_decode_agree(pkg):
     torch.cuda.synchronize()
     assert ops.device_error() == 0
     m.close()
+
+
+def test_bench_decode_configuration_matches_eager_greedy(pkg):
+    """The decode configuration bench.py times on the Llama-3.1-8B shape -- one batched prefill of 32 prompts, then
+    the decode step captured in a CUDA graph with the greedy advance on the device and the attention planned for the
+    last position the replays reach -- gives the greedy tokens and logprobs of eager decoding, bit for bit (eager:
+    every prompt prefilled alone, one bi_decode_step per step)."""
+    model, ops = pkg
+    cfg = configs.LLAMA8B
+    B, P, n = 32, 64, 4
+    m = model.Model(cfg, mode=0, n_slots=B, capacity=P + n + 8, init="device")
+    V = cfg["vocab"]
+    prompts = [synth.prompt_tokens(r, P, V) for r in range(B)]
+    seqs, rec = model.greedy_generate(m, prompts, n)
+
+    ids = np.concatenate(prompts).astype(np.int32)
+    slots = np.repeat(np.arange(B), P).astype(np.int32)
+    pos = np.tile(np.arange(P), B).astype(np.int32)
+    lm = np.full(B * P, -1, dtype=np.int32)
+    lm[np.arange(B) * P + P - 1] = np.arange(B)
+    o = m.step(ids, slots, pos, lm)
+    assert o["argmax"].cpu().numpy().tolist() == [s[P] for s in seqs]
+    dev = m.device
+    ids_d = o["argmax"].clone()
+    pos_d = torch.full((B,), P, dtype=torch.int32, device=dev)
+    slot_d = torch.arange(B, dtype=torch.int32, device=dev)
+    lm_d = torch.arange(B, dtype=torch.int32, device=dev)
+    slots_h = torch.arange(B, dtype=torch.int32)
+    pos_plan = torch.full((B,), P + n, dtype=torch.int32)
+    out = m.alloc_out(B)
+    m.workspace(B, B, P + n + 1)
+
+    def one_step():
+        m.step_dev(B, ids_d, slot_d, pos_d, slots_h, pos_plan, lm_d, B, None, out, max_pos=P + n + 1)
+        ops.greedy_advance(out["argmax"], ids_d, pos_d)
+
+    got = []
+    one_step()  # eager first step, as in the bench (one-time set-up stays outside the capture)
+    torch.cuda.synchronize()
+    got.append((out["argmax"].cpu().numpy().copy(), out["logprob"].cpu().numpy().copy()))
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=s):
+        one_step()
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(n - 1):
+        g.replay()
+        torch.cuda.synchronize()
+        got.append((out["argmax"].cpu().numpy().copy(), out["logprob"].cpu().numpy().copy()))
+    del g
+    for j, (am, lp) in enumerate(got):
+        assert np.array_equal(am, rec["argmax"][:, j]), j
+        assert np.array_equal(lp, rec["logprob"][:, j]), j
+    assert ops.device_error() == 0
+    m.close()
