@@ -156,3 +156,12 @@ def test_attention_validation(L):
     kv.head_dim = 96
     pos[1] = 1
     assert lib.bi_attention(*args(slot, pos)) == L.BI_ERR_UNSUPPORTED
+
+
+def test_failing_cuda_call_maps_to_bi_err_cuda(L):
+    import torch
+    if torch.cuda.is_available():  # the call below must fail inside CUDA, never launch on a real device
+        pytest.skip("needs a machine without a usable GPU")
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.lib.bi_rmsnorm(fake, None, None, fake, fake, None, 2, 64, 1e-5, 0, None) == L.BI_ERR_CUDA
+    assert L.lib.bi_last_error()
