@@ -553,7 +553,8 @@ def main_ours(args):
             "hbm_roofline_frac_step": round(step_frac, 4),
             "recompute_rate": r["recompute_rate"],
             "gpu_launches": int(r["launches"] * K),
-            "clocks": r["clocks"]}
+            "clocks": r["clocks"],
+            "gpu": torch.cuda.get_device_name(torch.cuda.current_device())}
     # dominant kernel: the weight-streaming GEMM (all projections of one step + LM head), timed alone
     if mode == 0:
         gms = time_gemms(m, B)

@@ -7,6 +7,8 @@
 #include <cstring>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>  // header-only NVTX v3: ranges cost a pointer check unless a profiler attaches
+
 #include "host_common.cuh"
 #include "gemm.cuh"
 #include "norm_rope.cuh"
@@ -352,6 +354,13 @@ __global__ void wait_selftest_kernel() {
 // ====================================================================== C ABI
 using namespace bi;
 
+// One NVTX range per C-ABI call, named after the call (nested calls nest).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+#define BI_RANGE(name) const NvtxRange bi_nvtx_range_(name)
+
 struct bi_ctx {
   bi_model_desc desc;
   bi_weights w;
@@ -383,6 +392,7 @@ int bi_device_error(unsigned* flags, int reset) {
 }
 
 int bi_selftest_wait_timeout(void* stream) {
+  BI_RANGE("bi_selftest_wait_timeout");
   clear_error();
   BI_TRY(launch(wait_selftest_kernel, dim3(1), dim3(32), 0, as_stream(stream)));
   return BI_OK;
@@ -395,12 +405,14 @@ size_t bi_gemm_workspace_size(int M, int N, int K, int mode, int variant) {
 
 int bi_gemm(const void* x, int ldx, const void* w, void* y, int ldy, int y_dtype, int M, int N, int K, int epilogue,
             int mode, int variant, void* ws, size_t ws_bytes, void* stream) {
+  BI_RANGE("bi_gemm");
   clear_error();
   return gemm_run(x, ldx, w, y, ldy, y_dtype, M, N, K, epilogue, mode, variant, ws, ws_bytes, as_stream(stream));
 }
 
 int bi_rmsnorm(const void* x, const void* residual_in, void* residual_out, const void* gamma, void* y, float* y_f32,
                int M, int H, float eps, int mode, void* stream) {
+  BI_RANGE("bi_rmsnorm");
   clear_error();
   BI_REQUIRE(x && gamma && y, BI_ERR_INVALID_ARG, "bi_rmsnorm: NULL pointer");
   BI_REQUIRE(M >= 0 && H > 0 && H % 8 == 0 && H <= NORM_THREADS * NORM_MAX_CHUNKS * 8, BI_ERR_UNSUPPORTED,
@@ -417,6 +429,7 @@ int bi_rmsnorm(const void* x, const void* residual_in, void* residual_out, const
 }
 
 int bi_rope_table_fill(float* table, int max_pos, int head_dim, double theta, void* stream) {
+  BI_RANGE("bi_rope_table_fill");
   clear_error();
   BI_REQUIRE(table && max_pos > 0 && head_dim > 0 && head_dim % 2 == 0 && theta > 0, BI_ERR_INVALID_ARG,
              "bi_rope_table_fill: bad arguments");
@@ -437,6 +450,7 @@ int bi_rope_table_fill(float* table, int max_pos, int head_dim, double theta, vo
 int bi_rope_kv_append(const float* qkv, const float* rope, int rope_max_pos, void* q_out, const bi_kv_layout* kv,
                       int layer, const int32_t* slot, const int32_t* pos, int T, int Hq, int qk_paired, int mode,
                       void* stream) {
+  BI_RANGE("bi_rope_kv_append");
   clear_error();
   BI_REQUIRE(qkv && rope && q_out && kv && kv->k && kv->v && slot && pos, BI_ERR_INVALID_ARG,
              "bi_rope_kv_append: NULL pointer");
@@ -459,6 +473,7 @@ size_t bi_attention_workspace_size(int T, int Hq, int head_dim, int max_pos) {
 int bi_attention(const void* q, const bi_kv_layout* kv, int layer, const int32_t* slot, const int32_t* pos,
                  const int32_t* slot_host, const int32_t* pos_host, void* out, int T, int Hq, float scale, int mode,
                  int variant, void* ws, size_t ws_bytes, void* stream) {
+  BI_RANGE("bi_attention");
   clear_error();
   return attention_run(q, kv, layer, slot, pos, slot_host, pos_host, out, T, Hq, scale, mode, variant, ws, ws_bytes,
                        as_stream(stream));
@@ -474,6 +489,7 @@ size_t bi_lmhead_workspace_size(int B, int H, int V, int mode) {
 int bi_lmhead_logprob(const float* h, const void* W, const int32_t* target, int B, int H, int V,
                       float margin_threshold, int mode, float* logprob, float* lse, int32_t* argmax, float* margin,
                       uint8_t* recomputed, float* logits, void* ws, size_t ws_bytes, void* stream) {
+  BI_RANGE("bi_lmhead_logprob");
   clear_error();
   return lmhead_run(h, W, target, B, H, V, margin_threshold, mode, logprob, lse, argmax, margin, recomputed, logits,
                     ws, ws_bytes, as_stream(stream));
@@ -586,6 +602,7 @@ __global__ void gather_lm_rows_kernel(const int32_t* __restrict__ lm_row, const 
 
 int bi_decode_step(bi_ctx* ctx, const bi_batch* batch, const bi_step_out* out, void* ws, size_t ws_bytes,
                    void* stream) {
+  BI_RANGE("bi_decode_step");
   clear_error();
   BI_REQUIRE(ctx && batch && out, BI_ERR_INVALID_ARG, "bi_decode_step: NULL pointer");
   const bi_model_desc& d = ctx->desc;
@@ -687,6 +704,7 @@ static int noalloc_scratch_ptr(void** out) {
 int bi_lmhead_logprob_noalloc(const float* h, const void* W, const int32_t* target, int B, int H, int V,
                               float margin_threshold, int mode, float* logprob, float* lse, int32_t* argmax,
                               float* margin, uint8_t* recomputed, float* logits, void* stream) {
+  BI_RANGE("bi_lmhead_logprob_noalloc");
   clear_error();
   BI_REQUIRE(B >= 0 && H > 0 && V > 0, BI_ERR_INVALID_ARG, "bi_lmhead_logprob_noalloc: bad sizes");
   if (B == 0) return BI_OK;
@@ -706,6 +724,7 @@ int bi_lmhead_logprob_noalloc(const float* h, const void* W, const int32_t* targ
 }
 
 int bi_greedy_advance(const int32_t* argmax, int32_t* ids, int32_t* pos, int B, void* stream) {
+  BI_RANGE("bi_greedy_advance");
   clear_error();
   BI_REQUIRE(argmax && ids && pos && B >= 0, BI_ERR_INVALID_ARG, "bi_greedy_advance: bad arguments");
   if (B == 0) return BI_OK;
@@ -715,6 +734,7 @@ int bi_greedy_advance(const int32_t* argmax, int32_t* ids, int32_t* pos, int B, 
 
 int bi_synth_fill_bf16(uint16_t* dst, int64_t rows, int64_t cols, uint64_t key, double std, int interleave, int phase,
                        void* stream) {
+  BI_RANGE("bi_synth_fill_bf16");
   clear_error();
   BI_REQUIRE(dst && rows >= 0 && cols > 0 && (phase == 0 || phase == 1), BI_ERR_INVALID_ARG,
              "bi_synth_fill_bf16: bad arguments");
