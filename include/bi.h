@@ -232,7 +232,9 @@ int bi_lmhead_logprob(const float* h, const void* W, const int32_t* target, int 
  *    the need of the recompute-enabled case).
  *  - The first call on a device looks up the array's device address (once per
  *    device, with that device current); make that first call before any
- *    stream capture.
+ *    stream capture.  The address is kept for the life of the process: a
+ *    cudaDeviceReset destroys the array with everything else on the device,
+ *    so do not call this entry point again in that process after a reset.
  *  - All calls share the one array: calls whose GPU work overlaps (different
  *    streams, or host threads racing) corrupt each other's scratch.  Issue
  *    them in one stream order.  Nothing in the array needs to start zeroed.

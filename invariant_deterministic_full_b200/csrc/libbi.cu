@@ -684,7 +684,9 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[BI_NOALLOC_SCRATCH_BY
 
 // Device address of the array on each device.  Host code cannot use the
 // symbol itself (on the host it names a stand-in, not device memory), so the
-// address is looked up once per device, with that device current.
+// address is looked up once per device, with that device current, and kept
+// for the life of the process (a device reset invalidates it; the header
+// tells callers not to use this entry point after one).
 static int noalloc_scratch_ptr(void** out) {
   static std::mutex mu;
   static std::vector<void*> addr;

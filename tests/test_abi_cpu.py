@@ -1,6 +1,11 @@
 """The C-ABI library loads, exports every symbol include/bi.h declares, and
 rejects invalid arguments on the host with status codes (no GPU needed: every
-case here fails validation before any CUDA call)."""
+case here fails validation before any CUDA call).
+
+The validation cases pass placeholder device addresses that are never meant to
+be dereferenced.  They run only where the library's own CUDA runtime sees no
+device (the `host_only` fixture asks the library, not torch), so a broken check
+can never turn into a launch on a real GPU."""
 import ctypes
 import os
 import re
@@ -17,6 +22,13 @@ def L():
     __graft_entry__._lib_builder().build()
     from invariant_deterministic_full_b200 import _lib
     return _lib
+
+
+@pytest.fixture
+def host_only(L):
+    if L.lib.bi_num_sms(0) > 0:
+        pytest.skip("placeholder device addresses are only passed where the library sees no CUDA device")
+    return L
 
 
 def _declared():
@@ -40,7 +52,8 @@ def test_version_and_status_codes(L):
         (1, 2, 3, 4, 5)
 
 
-def test_gemm_validation(L):
+def test_gemm_validation(host_only):
+    L = host_only
     lib = L.lib
     fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
     assert lib.bi_gemm(None, 64, fake, fake, 64, 0, 4, 64, 64, 0, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
@@ -59,7 +72,8 @@ def test_gemm_validation(L):
     assert lib.bi_gemm_workspace_size(4, 64, 64, 0, 0) == 0
 
 
-def test_rmsnorm_lmhead_validation(L):
+def test_rmsnorm_lmhead_validation(host_only):
+    L = host_only
     lib = L.lib
     fake = ctypes.c_void_p(1 << 20)
     assert lib.bi_rmsnorm(None, None, None, fake, fake, None, 2, 64, 1e-5, 0, None) == L.BI_ERR_INVALID_ARG
@@ -86,7 +100,8 @@ def _tiny_ctx(L, capacity=64, mode=0):
     return rc, ctx, kv
 
 
-def test_ctx_validation(L):
+def test_ctx_validation(host_only):
+    L = host_only
     lib = L.lib
     rc, ctx, kv = _tiny_ctx(L)
     assert rc == L.BI_OK and ctx.value
@@ -110,7 +125,8 @@ def test_ctx_validation(L):
     lib.bi_ctx_destroy(ctx)
 
 
-def test_decode_step_capacity_and_workspace_rejected_on_host(L):
+def test_decode_step_capacity_and_workspace_rejected_on_host(host_only):
+    L = host_only
     lib = L.lib
     rc, ctx, _ = _tiny_ctx(L, capacity=64)
     assert rc == L.BI_OK
@@ -140,7 +156,8 @@ def test_decode_step_capacity_and_workspace_rejected_on_host(L):
     lib.bi_ctx_destroy(ctx)
 
 
-def test_attention_validation(L):
+def test_attention_validation(host_only):
+    L = host_only
     lib = L.lib
     fake = 1 << 20
     kv = L.KvLayout(fake, fake, 2, 1, 4, 64, 64, 0)
@@ -158,10 +175,10 @@ def test_attention_validation(L):
     assert lib.bi_attention(*args(slot, pos)) == L.BI_ERR_UNSUPPORTED
 
 
-def test_failing_cuda_call_maps_to_bi_err_cuda(L):
-    import torch
-    if torch.cuda.is_available():  # the call below must fail inside CUDA, never launch on a real device
-        pytest.skip("needs a machine without a usable GPU")
+def test_failing_cuda_call_maps_to_bi_err_cuda(host_only):
+    # With no device visible to the library's runtime, the launch fails on the host (no CUDA device), which must
+    # come back as BI_ERR_CUDA with a message; nothing reaches a GPU.
+    L = host_only
     fake = ctypes.c_void_p(1 << 20)
     assert L.lib.bi_rmsnorm(fake, None, None, fake, fake, None, 2, 64, 1e-5, 0, None) == L.BI_ERR_CUDA
     assert L.lib.bi_last_error()
