@@ -64,6 +64,8 @@ def _load():
         lib.or_lmhead.argtypes = [P, P, P, I, I, I, P, P]
         lib.or_forward.restype = I
         lib.or_forward.argtypes = [ctypes.POINTER(_Cfg), ctypes.POINTER(_W), I, P, I, P, P, P]
+        lib.or_forward_ctx.restype = I
+        lib.or_forward_ctx.argtypes = [ctypes.POINTER(_Cfg), ctypes.POINTER(_W), I, P, I, I, P, P, P, P, P, P, P]
         _lib = lib
     return _lib
 
@@ -156,3 +158,33 @@ def forward(cfg, weights, tokens, targets=None, mode=OR_BF16, want_h=False):
     if rc != 0:
         raise MemoryError("oracle forward: allocation failed")
     return res, h
+
+
+def forward_ctx(cfg, weights, tokens, k_ctx=None, v_ctx=None, targets=None, mode=OR_BF16, want_h=False,
+                want_kv=False):
+    """Forward of new tokens that follow earlier positions of the same sequence, given those positions' stored
+    keys and values per layer (k_ctx, v_ctx: [L, n_ctx, Hkv*d]; None for none).  Returns res [n,5], h [n,H] or
+    None, and (k, v) [L, n, Hkv*d] of the new tokens or None."""
+    lib = _load()
+    c = _Cfg(cfg["n_layers"], cfg["hidden"], cfg["n_heads"], cfg["n_kv_heads"], cfg["head_dim"], cfg["ffn"],
+             cfg["vocab"], float(cfg["eps"]), float(cfg["rope_theta"]))
+    keep = {n: _u16(weights[n]) for n in _WNAMES}
+    w = _W(*[keep[n].ctypes.data for n in _WNAMES])
+    tok = np.ascontiguousarray(tokens, dtype=np.int32)
+    n = tok.shape[0]
+    L, KD = cfg["n_layers"], cfg["n_kv_heads"] * cfg["head_dim"]
+    n_ctx = 0 if k_ctx is None else int(np.shape(k_ctx)[1])
+    kc = None if k_ctx is None else _f64(k_ctx)
+    vc = None if v_ctx is None else _f64(v_ctx)
+    assert kc is None or (kc.shape == (L, n_ctx, KD) and vc is not None and vc.shape == kc.shape)
+    tg = None if targets is None else np.ascontiguousarray(targets, dtype=np.int32)
+    res = np.empty((n, 5), dtype=np.float64)
+    h = np.empty((n, cfg["hidden"]), dtype=np.float64) if want_h else None
+    ko = np.empty((L, n, KD), dtype=np.float64) if want_kv else None
+    vo = np.empty((L, n, KD), dtype=np.float64) if want_kv else None
+    ptr = lambda a: None if a is None else a.ctypes.data
+    rc = lib.or_forward_ctx(ctypes.byref(c), ctypes.byref(w), int(mode), tok.ctypes.data, n, n_ctx, ptr(kc),
+                            ptr(vc), ptr(tg), res.ctypes.data, ptr(h), ptr(ko), ptr(vo))
+    if rc != 0:
+        raise MemoryError("oracle forward: allocation failed")
+    return res, h, ((ko, vo) if want_kv else None)

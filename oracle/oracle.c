@@ -182,21 +182,29 @@ void or_lmhead(const double* h, const uint16_t* W, const int* target, int B, int
 
 static double silu(double x) { return x / (1.0 + exp(-x)); }
 
-/* Full forward of ONE sequence of n tokens (positions 0..n-1, causal).
- * For each position t: res[t][0..4] as in or_logit_stats for target[t]
- * (target NULL or < 0: the argmax).  h_out (optional, [n][H]): the final
- * norm output before any bf16 rounding (the FP32-recompute input).
+/* Forward of ONE sequence: n new tokens at positions n_ctx .. n_ctx+n-1 that
+ * follow n_ctx earlier positions whose per-layer keys and values (after RoPE,
+ * as stored: rounded to bf16 in OR_BF16) are given in k_ctx, v_ctx
+ * ([L][n_ctx][Hkv*d], NULL when n_ctx == 0).  Causal: new token t attends to
+ * the n_ctx earlier positions and to new tokens 0..t, in ascending position
+ * order.  For each new token t: res[t][0..4] as in or_logit_stats for
+ * target[t] (target NULL or < 0: the argmax).  h_out (optional, [n][H]): the
+ * final norm output before any bf16 rounding (the FP32-recompute input).
+ * k_out, v_out (optional, [L][n][Hkv*d]): the new tokens' stored keys and
+ * values, which a later call can take as its context.
  * Returns 0 on success, -1 on allocation failure. */
-int or_forward(const or_cfg* c, const or_weights* w, int mode, const int* tokens, int n, const int* target,
-               double* res, double* h_out) {
+int or_forward_ctx(const or_cfg* c, const or_weights* w, int mode, const int* tokens, int n, int n_ctx,
+                   const double* k_ctx, const double* v_ctx, const int* target, double* res, double* h_out,
+                   double* k_out, double* v_out) {
   const int H = c->hidden, Hq = c->n_heads, Hkv = c->n_kv_heads, d = c->head_dim, F = c->ffn, V = c->vocab;
   const int QD = Hq * d, KD = Hkv * d, group = Hq / Hkv;
+  const int nt = n_ctx + n; /* positions visible to the last new token */
   const double scale = 1.0 / sqrt((double)d);
   size_t big = (size_t)n * (size_t)(F > H ? F : H);
   double *r = calloc((size_t)n * H, 8), *u = calloc((size_t)n * H, 8), *q = calloc((size_t)n * QD, 8),
          *k = calloc((size_t)n * KD, 8), *vv = calloc((size_t)n * KD, 8), *o = calloc((size_t)n * QD, 8),
          *y = calloc(big, 8), *g = calloc((size_t)n * F, 8), *up = calloc((size_t)n * F, 8),
-         *kh = calloc((size_t)n * d, 8), *vh = calloc((size_t)n * d, 8);
+         *kh = calloc((size_t)nt * d, 8), *vh = calloc((size_t)nt * d, 8);
   if (!r || !u || !q || !k || !vv || !o || !y || !g || !up || !kh || !vh) return -1;
 
   for (int t = 0; t < n; ++t)
@@ -220,23 +228,29 @@ int or_forward(const or_cfg* c, const or_weights* w, int mode, const int* tokens
     or_gemm(u, wk, k, n, KD, H);
     or_gemm(u, wv, vv, n, KD, H);
     for (int t = 0; t < n; ++t) {
-      or_rope(q + (size_t)t * QD, Hq, d, t, c->rope_theta);
-      or_rope(k + (size_t)t * KD, Hkv, d, t, c->rope_theta);
+      or_rope(q + (size_t)t * QD, Hq, d, n_ctx + t, c->rope_theta);
+      or_rope(k + (size_t)t * KD, Hkv, d, n_ctx + t, c->rope_theta);
     }
     for (size_t i = 0; i < (size_t)n * QD; ++i) q[i] = rb(mode, q[i]);
     for (size_t i = 0; i < (size_t)n * KD; ++i) {
       k[i] = rb(mode, k[i]);
       vv[i] = rb(mode, vv[i]);
     }
+    if (k_out) memcpy(k_out + (size_t)l * n * KD, k, sizeof(double) * (size_t)n * KD);
+    if (v_out) memcpy(v_out + (size_t)l * n * KD, vv, sizeof(double) * (size_t)n * KD);
+    const double* kc = k_ctx ? k_ctx + (size_t)l * n_ctx * KD : NULL;
+    const double* vc = v_ctx ? v_ctx + (size_t)l * n_ctx * KD : NULL;
     for (int hk = 0; hk < Hkv; ++hk) {
-      for (int j = 0; j < n; ++j)
+      for (int j = 0; j < nt; ++j) /* keys in position order: the context, then the new tokens */
         for (int e = 0; e < d; ++e) {
-          kh[(size_t)j * d + e] = k[(size_t)j * KD + hk * d + e];
-          vh[(size_t)j * d + e] = vv[(size_t)j * KD + hk * d + e];
+          const int jn = j - n_ctx;
+          kh[(size_t)j * d + e] = jn < 0 ? kc[(size_t)j * KD + hk * d + e] : k[(size_t)jn * KD + hk * d + e];
+          vh[(size_t)j * d + e] = jn < 0 ? vc[(size_t)j * KD + hk * d + e] : vv[(size_t)jn * KD + hk * d + e];
         }
       for (int hq = hk * group; hq < (hk + 1) * group; ++hq)
-        for (int t = 0; t < n; ++t) /* query t sees keys 0..t */
-          or_attention_query(q + (size_t)t * QD + hq * d, kh, vh, t + 1, d, scale, o + (size_t)t * QD + hq * d);
+        for (int t = 0; t < n; ++t) /* query at position n_ctx + t sees keys 0..n_ctx + t */
+          or_attention_query(q + (size_t)t * QD + hq * d, kh, vh, n_ctx + t + 1, d, scale,
+                             o + (size_t)t * QD + hq * d);
     }
     for (size_t i = 0; i < (size_t)n * QD; ++i) o[i] = rb(mode, o[i]);
     or_gemm(o, wo, y, n, H, QD);
@@ -261,4 +275,11 @@ int or_forward(const or_cfg* c, const or_weights* w, int mode, const int* tokens
   free(tg);
   free(r); free(u); free(q); free(k); free(vv); free(o); free(y); free(g); free(up); free(kh); free(vh);
   return 0;
+}
+
+/* Full forward of ONE sequence of n tokens (positions 0..n-1, causal): the
+ * call above with no earlier positions. */
+int or_forward(const or_cfg* c, const or_weights* w, int mode, const int* tokens, int n, const int* target,
+               double* res, double* h_out) {
+  return or_forward_ctx(c, w, mode, tokens, n, 0, NULL, NULL, target, res, h_out, NULL, NULL);
 }

@@ -220,3 +220,24 @@ def test_bf16_forward_each_storage_point_matters(brute_case, point):
     ref, href = _brute_bf16(cfg, w, tok, skip=point)
     dev = max(np.abs(got - ref).max(), np.abs(h - href).max())
     assert dev > 1e-7, f"leaving out {point} is invisible on this case"
+
+
+@pytest.mark.parametrize("mode", [oracle.OR_EXACT, oracle.OR_BF16])
+def test_forward_with_context_equals_whole_sequence(mode):
+    """Decoding new tokens after a context given as stored keys/values gives, bit for bit, what the whole-sequence
+    forward gives at those positions (the forward with a context is the pinned forward, resumed)."""
+    cfg = configs.shrink(configs.TINY, n_layers=2, hidden=64, n_heads=4, n_kv_heads=2, head_dim=16, ffn=96,
+                         vocab=128)
+    w = synth.model_weights(cfg, seed=23, std=0.1)
+    tok = synth.tokens(synth.key(23, 1), 11, cfg["vocab"])
+    full, hf = oracle.forward(cfg, w, tok, mode=mode, want_h=True)
+    _, _, (k7, v7) = oracle.forward_ctx(cfg, w, tok[:7], mode=mode, want_kv=True)
+    res, h, (k4, v4) = oracle.forward_ctx(cfg, w, tok[7:], k7, v7, mode=mode, want_h=True, want_kv=True)
+    assert np.array_equal(res, full[7:]) and np.array_equal(h, hf[7:])
+    # the keys/values handed on are the stored ones (bf16 values in OR_BF16)
+    if mode == oracle.OR_BF16:
+        assert np.array_equal(k4, oracle.round_bf16(k4)) and np.array_equal(v7, oracle.round_bf16(v7))
+    # a different context changes the result (the context is really read); reordering the context keys does
+    # not change the attention sums beyond fp64 rounding, scaling the values does
+    res2, _, _ = oracle.forward_ctx(cfg, w, tok[7:], k7, 2 * v7, mode=mode)
+    assert not np.array_equal(res2[:, 0], res[:, 0])
