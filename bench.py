@@ -166,36 +166,41 @@ def step_bytes(cfg, B, ctx_lens, f32_kv=False):
 # DRAM bytes (read + write) of the weight-streaming GEMM launches of one decode step at batch 32, from one ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum) of the same shapes on the 2-layer 8B-width case; the
 # per-layer figures scale to 32 layers (the weights per launch do not depend on the layer count).  Valid only for
-# the GEMM kernel source that was captured, recognised by gemm_bf16_source_digest.
-GEMM_TRAFFIC = {"gemm_bf16_source_sha256": "9667a87af3277e94aaefde6dba3cb9b705671f2b4e455c485749f0d50f49eb40",
-                "batch": 32, "per_layer_bytes": 440052096, "lm_head_bytes": 1065866496}
+# the GEMM kernel source that was captured, recognised by gemm_source_digest; None until a capture of this source.
+GEMM_TRAFFIC = {"gemm_source_sha256": None, "batch": 32, "per_layer_bytes": None, "lm_head_bytes": None}
+
+CSRC = os.path.join(ROOT, "invariant_deterministic_full_b200", "csrc")
 
 
-def gemm_bf16_source_digest(text):
-    """sha256 of the code (comments and whitespace removed) of the part of gemm.cuh that decides the bf16 GEMM's
-    memory traffic: everything up to the FAST split heuristic (tile configs, the kernel, the tile and ring pickers)
-    plus its launch and dispatch code.  Workspace sizing and the LayerCast split/combine kernels are left out, since
-    they do not touch this kernel."""
+def gemm_source_digest(tc_text, mma_text, plan_text):
+    """sha256 of the code (comments and whitespace removed) that decides the GEMM's memory traffic: the whole
+    tcgen05 and mma.sync kernel files, and the launch planning and dispatch of gemm.cuh (from the tile plan to the
+    end of the bf16 dispatcher).  The FAST split heuristic, workspace sizing and the LayerCast kernels are left
+    out."""
     import hashlib
     import re
-    a = text.index("static int gemm_fast_splits")
-    b0 = text.index("template <int BN, int EPI, int MT = 1, int CPS = 1>\nstatic int launch_gemm_bf16_t")
-    b1 = text.index("int gemm_f32(")
-    code = re.sub(r"/\*.*?\*/", " ", text[:a] + text[b0:b1], flags=re.S)  # comments and layout do not count
+    a = plan_text.index("struct TcPlan {")
+    b = plan_text.index("// LayerCast on tensor cores: rows of x per pass")
+    c0 = plan_text.index("template <int BN, int MT, int KS, int EPI>\nstatic int launch_tc_t")
+    c1 = plan_text.index("int gemm_f32(")
+    code = re.sub(r"/\*.*?\*/", " ", tc_text + mma_text + plan_text[a:b] + plan_text[c0:c1], flags=re.S)
     code = re.sub(r"//[^\n]*", " ", code)
     return hashlib.sha256(" ".join(code.split()).encode()).hexdigest()
 
 
+def current_gemm_digest():
+    txt = lambda n: open(os.path.join(CSRC, n)).read()
+    return gemm_source_digest(txt("gemm_tc.cuh"), txt("gemm_mma.cuh"), txt("gemm.cuh"))
+
+
 def gemm_traffic_per_launch(cfg, B):
     """Measured DRAM bytes per launch of the timed GEMM set, or None when they no longer apply."""
-    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "invariant_deterministic_full_b200", "csrc",
-                       "gemm.cuh")
     try:
-        with open(src) as f:
-            h = gemm_bf16_source_digest(f.read())
+        h = current_gemm_digest()
     except (OSError, ValueError):
         return None
-    if h != GEMM_TRAFFIC["gemm_bf16_source_sha256"] or B != GEMM_TRAFFIC["batch"] or cfg["hidden"] != 4096:
+    if (GEMM_TRAFFIC["gemm_source_sha256"] is None or h != GEMM_TRAFFIC["gemm_source_sha256"]
+            or B != GEMM_TRAFFIC["batch"] or cfg["hidden"] != 4096):
         return None
     L = cfg["n_layers"]
     return (L * GEMM_TRAFFIC["per_layer_bytes"] + GEMM_TRAFFIC["lm_head_bytes"]) / (4 * L + 1)
@@ -466,12 +471,17 @@ def run_e2e(m, B, P, K, rank, graph=True):
 
 
 class CpuSample:
-    """The fp64 oracle as it stands, on the host cores: one decode token through 8B-width models of 0 and 4
-    layers (both with the 128256-row LM head); the per-layer time is scaled to 32 layers -> tok/s."""
+    """The fp64 oracle as it stands, on the host cores: NEW teacher-forced decode tokens at the positions of the
+    timed steps (after a PROMPT-token prompt and the warm-up steps), through 8B-width models of 0 and 4 layers
+    (both with the 128256-row LM head); every token attends to a context of that many cached positions per layer
+    (seeded synthetic keys/values: the arithmetic per token is the workload's).  The per-layer time is scaled to
+    32 layers -> tok/s."""
 
     LAYERS = 4
+    NEW = 4
 
-    def __init__(self):
+    def __init__(self, prompt=512, warmup=4):
+        import numpy as np
         import oracle
         import synth
         from synth import configs
@@ -481,30 +491,37 @@ class CpuSample:
         self.cfg0 = configs.shrink(self.cfg32, n_layers=0)
         self.wL = synth.model_weights(self.cfgL)
         self.w0 = {k: (v[:0] if (v.ndim == 3 or k in ("attn_norm", "ffn_norm")) else v) for k, v in self.wL.items()}
-        self.tok = synth.prompt_tokens(0, 1, self.cfgL["vocab"])
+        self.pos0 = prompt + 1 + warmup  # position of the first timed decode step
+        self.tok = synth.prompt_tokens(0, self.NEW, self.cfgL["vocab"])
+        KD = self.cfgL["n_kv_heads"] * self.cfgL["head_dim"]
+        kv = synth.normal_f64(synth.key(77, 1), 2 * self.LAYERS * self.pos0 * KD)
+        kv = oracle.round_bf16(kv.reshape(2, self.LAYERS, self.pos0, KD))  # stored as bf16, as the path stores them
+        self.k_ctx, self.v_ctx = kv[0], kv[1]
+        self.k0 = np.zeros((0, self.pos0, KD))
 
     def once(self):
         t = time.perf_counter()
-        self.oracle.forward(self.cfg0, self.w0, self.tok)
+        self.oracle.forward_ctx(self.cfg0, self.w0, self.tok, self.k0, self.k0)
         t0 = time.perf_counter() - t
         t = time.perf_counter()
-        self.oracle.forward(self.cfgL, self.wL, self.tok)
+        self.oracle.forward_ctx(self.cfgL, self.wL, self.tok, self.k_ctx, self.v_ctx)
         tL = time.perf_counter() - t
         per_layer = max(tL - t0, 1e-9) / self.LAYERS
-        return t0 + per_layer * self.cfg32["n_layers"], t0, tL
+        return (t0 + per_layer * self.cfg32["n_layers"]) / self.NEW, t0, tL
 
     def describe(self, n, t0, tL):
-        return (f"fp64 oracle forward of 1 decode token through 0- and {self.LAYERS}-layer 8B-width models (both with "
-                f"the 128256-row LM head); per-layer time scaled to 32 layers; median of {n} repeats "
-                f"({t0:.3f} s, {tL:.3f} s per forward)")
+        return (f"fp64 oracle, {self.NEW} teacher-forced decode tokens at positions {self.pos0}..{self.pos0 + self.NEW - 1}"
+                f" (each attending to {self.pos0}+ cached positions per layer) through 0- and {self.LAYERS}-layer "
+                f"8B-width models with the 128256-row LM head; per-layer time scaled to 32 layers; median of {n} "
+                f"repeats ({t0:.3f} s, {tL:.3f} s per call)")
 
 
 def cores():
     return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
 
 
-def cpu_baseline(seconds):
-    cs = CpuSample()
+def cpu_baseline(seconds, prompt=512, warmup=4):
+    cs = CpuSample(prompt, warmup)
     t_end = time.time() + seconds
     runs = []
     while not runs or time.time() < t_end:
@@ -565,7 +582,7 @@ def main_ours(args):
                             "frac": round(ach / hbm, 4), "traffic": round(tr) if tr else None,
                             "traffic_note": "DRAM read+write bytes per launch (ncu, same GEMM shapes, 2-layer case "
                                             "scaled to 32 layers)" if tr else "no capture for this GEMM source/batch",
-                            "kernel": "gemm_bf16_kernel (weight-streaming mma.sync GEMM)",
+                            "kernel": "gemm_tc_kernel (weight-streaming tcgen05/TMEM GEMM)",
                             "per_launch": f"{gb / gl / 1e6:.1f} MB algorithmic over {gl} launches, "
                                           f"{gms / gl * 1e3:.1f} us average",
                             "peak_source": f"{src} hbm_gbs (copy), kernel timed alone"}
@@ -580,7 +597,7 @@ def main_ours(args):
                            "frac": round(pf / (pms / 1e3) / 1e12 / tf_burst, 4),
                            "note": f"one bi_decode_step over {B} prompts x {P} tokens, LM head on each last token; "
                                    f"FLOPs = 2 x projection weights x tokens + causal attention + LM head; peak = "
-                                   f"{src} cuBLAS bf16 (burst); mma.sync tensor-core GEMMs"}
+                                   f"{src} cuBLAS bf16 (burst); tcgen05 tensor-core GEMMs"}
     if rank == 0 and not args.no_e2e:
         ke = min(K, 32)
         e = run_e2e(m, B, P, ke, rank, graph=True)
@@ -605,10 +622,20 @@ def main_ours(args):
         line["sweep_tok_s_per_gpu"] = extra
         line["sweep_hbm_roofline_frac"] = extra_frac
     if not args.no_fast:
+        # the non-invariant variant at the headline batch and at the small batches where its split-K is active
         mf = mdl.Model(cfg, mode=mode, variant=1, n_slots=n_slots, capacity=cap, init="device")
         rf = run_decode(mf, B, P, K, W, 1, rank)
-        line["fast_variant"] = {"value": round(B * K / (rf["ms"] / 1e3), 2), "unit": "tok/s",
-                                "note": "non-invariant split-K / batch-dependent KV split, same weights and batch"}
+        per = {}
+        for b in sorted({1, 4, 8} - {B}):
+            rb = run_decode(mf, b, P, min(K, 32), W, 1, rank)
+            per[str(b)] = round(b * min(K, 32) / (rb["ms"] / 1e3), 2)
+        per[str(B)] = round(B * K / (rf["ms"] / 1e3), 2)
+        inv = {k: v for k, v in extra.items() if k in per}
+        line["fast_variant"] = {"value": per[str(B)], "unit": "tok/s", "per_batch": per,
+                                "invariant_per_batch": inv,
+                                "invariant_over_fast": {k: round(inv[k] / per[k], 4) for k in inv},
+                                "note": "non-invariant variant on the same weights: split-K chosen from the batch "
+                                        "(active at batch <= 16) and a KV split chosen from the batch"}
         mf.close()
         del mf
         torch.cuda.empty_cache()
@@ -625,7 +652,7 @@ def main_ours(args):
         ml.close()
         del ml
     if rank == 0 and not args.no_cpu:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds) if ws == 1 else None
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds, P, W) if ws == 1 else None
     m.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -639,7 +666,7 @@ def main_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    cs = CpuSample()
+    cs = CpuSample(args.prompt, args.warmup)
     for _ in range(args.warmup):
         cs.once()
     t0 = time.perf_counter()

@@ -51,7 +51,7 @@ typedef enum {
   BI_ERR_CUDA = 5         /* a CUDA runtime/driver call failed at launch */
 } bi_status;
 
-enum { BI_MODE_BF16 = 0, BI_MODE_LAYERCAST = 1 };
+enum { BI_MODE_BF16 = 0, BI_MODE_LAYERCAST = 1, BI_MODE_FP32 = 2 };
 /* BI_MODE_BF16: bf16 activations and KV cache, bf16 x bf16 products with fp32
  *   accumulation on tensor cores, fp32 softmax/norm arithmetic.
  * BI_MODE_LAYERCAST: the "LayerCast" scheme of "Give Me FP32 or Give Me
@@ -59,7 +59,13 @@ enum { BI_MODE_BF16 = 0, BI_MODE_LAYERCAST = 1 };
  *   arithmetic is fp32; activations and KV cache are fp32.  Projections take
  *   exact fp32 products on the tensor cores (see bi_gemm); the LM head,
  *   attention and norms use fp32 FMA on the CUDA cores, with the bf16
- *   weights cast to fp32 in registers. */
+ *   weights cast to fp32 in registers.
+ * BI_MODE_FP32: full FP32 storage, the arm LayerCast is compared with in
+ *   "Give Me FP32 or Give Me Death?" (LayerCast section; jiaxiangli.netlify.app
+ *   write-up, section 4): the projection, embedding and LM-head weights are f32
+ *   in memory (the norm gains stay bf16), activations and KV cache are f32,
+ *   and every product and sum is an fp32 FMA on the CUDA cores.  A reference
+ *   arm for the precision study, not a fast path. */
 enum { BI_VARIANT_INVARIANT = 0, BI_VARIANT_FAST = 1 };
 /* BI_VARIANT_FAST is the non-invariant comparison baseline: split-K GEMMs
  * whose split factor is chosen from the row count M and the SM count, and
@@ -67,7 +73,7 @@ enum { BI_VARIANT_INVARIANT = 0, BI_VARIANT_FAST = 1 };
  * deterministic for a fixed shape but change with batch size.  Not a product
  * path; it exists so the cost of invariance can be measured. */
 enum { BI_DTYPE_BF16 = 0, BI_DTYPE_F32 = 1 };
-enum { BI_EPI_NONE = 0, BI_EPI_SWIGLU = 1 };
+enum { BI_EPI_NONE = 0, BI_EPI_SWIGLU = 1, BI_EPI_ROPE_KV_APPEND = 2 };
 
 /* Granule of the gate/up interleave used by BI_EPI_SWIGLU: the fused weight
  * holds 16 gate rows, then the 16 up rows of the same output columns, etc. */
@@ -99,47 +105,6 @@ int bi_num_sms(int device); /* SM count of a device, -1 on error */
  * counter, incremented at every launch site; not thread-safe). */
 long long bi_launch_count(void);
 
-/* ------------------------------------------------------------------ GEMM
- * y[m][n] = sum_k x[m][k] * w[n][k]   (x: [M][K] with leading dim ldx,
- *   w: bf16 [N][K] contiguous, y: [M][N] with leading dim ldy).
- * Invariant variant: each output element is accumulated in fp32 over the
- *   FULL K range in ascending K order, by the same instruction sequence for
- *   any M (no split-K; the row tile and K loop do not depend on M).  The
- *   16-wide K steps go round-robin into a fixed number of accumulators (1, 2
- *   or 4, set by N alone) that are added in a fixed tree at the end.
- *   ("Meituan bitwise train/infer consistency": TP rewritten to full-K
- *   computation instead of segmented reduce-scatter.)
- * mode BI_MODE_BF16: x is bf16.  mode BI_MODE_LAYERCAST: x is f32 and the
- *   products are fp32-exact: every x is split exactly into three bf16 parts
- *   (x = p0 + p1 + p2, 8+8+8 significant bits), each part times the bf16 w is
- *   an exact product accumulated in fp32 on the tensor cores (full K,
- *   ascending, as above), and the three sums are added as (y0 + y1) + y2
- *   before the epilogue.
- * y_dtype: BI_DTYPE_BF16 (round-to-nearest-even) or BI_DTYPE_F32.
- * epilogue BI_EPI_SWIGLU: w rows are gate/up interleaved by BI_GU_INTERLEAVE
- *   and y has N/2 columns: y = silu(gate) * up, silu(g) = g / (1 + exp(-g)).
- * Requirements: K % 64 == 0, N % 64 == 0, ldx % 8 == 0 (16-byte rows),
- *   x, w 16-byte aligned; else BI_ERR_UNSUPPORTED.  M == 0 is a no-op
- *   (x and y may then be NULL); w NULL is BI_ERR_INVALID_ARG.
- * Workspace: bi_gemm_workspace_size() bytes (0 for the invariant bf16 mode;
- *   LayerCast needs room for the split rows and their three partial sums). */
-size_t bi_gemm_workspace_size(int M, int N, int K, int mode, int variant);
-int bi_gemm(const void* x, int ldx, const void* w, void* y, int ldy, int y_dtype, int M, int N, int K,
-            int epilogue, int mode, int variant, void* ws, size_t ws_bytes, void* stream);
-
-/* --------------------------------------------------------------- RMSNorm
- * Per row m (fused residual add, as in a pre-norm decoder):
- *   r'  = x + residual_in          (residual_in NULL: r' = x)
- *   residual_out = r' (rounded to the activation dtype; may alias residual_in)
- *   y   = r' / sqrt(mean(r'^2) + eps) * gamma        (activation dtype)
- *   y_f32 (optional, f32) = the same value before rounding.
- * The mean of squares is a fixed reduction tree over H (per-thread strided
- * partials, fixed shuffle tree, ascending cross-warp sum) that does not
- * depend on M.  Activation dtype: bf16 (BI_MODE_BF16) or f32 (LAYERCAST).
- * gamma: bf16 [H].  H % 8 == 0 and H <= 16384. */
-int bi_rmsnorm(const void* x, const void* residual_in, void* residual_out, const void* gamma, void* y,
-               float* y_f32, int M, int H, float eps, int mode, void* stream);
-
 /* --------------------------------------------------------------- KV cache
  * k and v: [n_slots][n_layers][n_kv_heads][capacity][head_dim], dtype bf16
  * (BI_MODE_BF16) or f32 (BI_MODE_LAYERCAST).  Position p of slot s is row p. */
@@ -155,7 +120,85 @@ typedef struct {
  * (i, i + d/2).  table: device, caller-allocated max_pos*head_dim floats. */
 int bi_rope_table_fill(float* table, int max_pos, int head_dim, double theta, void* stream);
 
-/* Rotary embedding + KV append for T tokens after the QKV projection.
+/* ------------------------------------------------------------------ GEMM
+ * y[m][n] = sum_k x[m][k] * w[n][k]   (x: [M][K] with leading dim ldx,
+ *   w: bf16 [N][K] contiguous, y: [M][N] with leading dim ldy).
+ * Invariant variant ("Meituan bitwise train/infer consistency": TP rewritten
+ *   to full-K computation instead of segmented reduce-scatter, one reduction
+ *   path shared by Prefill and Decode): each output element is accumulated in
+ *   fp32 over the FULL K range by tensor-core MMA instructions of K = 16 in
+ *   ascending K, the k16 steps going round-robin into KS interleaved
+ *   accumulators that are added in a fixed tree at the end: KS = 4 for
+ *   matrices of N <= 8192 rows, 1 for larger N divisible by 128, else 2.
+ *   ((s0 + s1) + (s2 + s3), s0 + s1 or s0.)  KS is a property of the matrix,
+ *   never of M: no split-K, and a row's result does not depend on the other
+ *   rows of the call, nor on which tensor-core path (mma.sync for at most 32
+ *   rows, tcgen05 above: the same arithmetic) runs it.
+ * n_full: 0 when w is a whole weight matrix; else the output rows of the
+ *   matrix that w is a contiguous row shard of (tensor parallelism), which
+ *   then fixes KS, so a shard's rows are bitwise the unsharded call's.  A
+ *   shard must hold whole 128/KS-row tiles (else BI_ERR_UNSUPPORTED).
+ * mode BI_MODE_BF16: x is bf16.  mode BI_MODE_LAYERCAST: x is f32 and the
+ *   products are fp32-exact: every x is split exactly into three bf16 parts
+ *   (x = p0 + p1 + p2, 8+8+8 significant bits), each part times the bf16 w is
+ *   an exact product accumulated in fp32 on the tensor cores (full K,
+ *   ascending, as above), and the three sums are added as (y0 + y1) + y2
+ *   before the epilogue.
+ * y_dtype: BI_DTYPE_BF16 (round-to-nearest-even) or BI_DTYPE_F32.
+ * epilogue BI_EPI_SWIGLU: w rows are gate/up interleaved by BI_GU_INTERLEAVE
+ *   and y has N/2 columns: y = silu(gate) * up, silu(g) = g / (1 + exp(-g)).
+ * epilogue BI_EPI_ROPE_KV_APPEND (BI_MODE_BF16, invariant variant only): the
+ *   QKV projection of one decoder layer with rotate-half RoPE and the KV-cache
+ *   append in its epilogue (the pages name the steps, not the fusion, which
+ *   is this library's).  w is one layer of bi_weights.w_qkv (q and k heads in
+ *   the paired row order described there), N = (Hq + 2 Hkv) * head_dim.  The
+ *   f32 projection of each q and k head is rotated at pos[m] with the f32
+ *   table of bi_rope_table_fill (for the pair (a, b) = (x[i], x[i + d/2]):
+ *   a' = a c - b s, b' = b c + a s), then q is stored (bf16, natural element
+ *   order) to epi->q_out [M][Hq * head_dim] and k, v (bf16) to the cache
+ *   epi->kv at (slot[m], epi->layer, head, pos[m]).  y and ldy are unused (y
+ *   may be NULL).  A row whose slot or position is out of range sets the
+ *   capacity bit of the device error word and is skipped.  epi must be NULL
+ *   for the other epilogues.
+ * Requirements: K % 64 == 0, N % 64 == 0, ldx % 8 == 0 (16-byte rows),
+ *   x, w 16-byte aligned; else BI_ERR_UNSUPPORTED.  M == 0 is a no-op
+ *   (x and y may then be NULL); w NULL is BI_ERR_INVALID_ARG.
+ * Workspace: bi_gemm_workspace_size() bytes (0 for the invariant bf16 mode;
+ *   LayerCast needs room for the split rows and their three partial sums). */
+typedef struct {
+  const float* rope;      /* device RoPE table from bi_rope_table_fill */
+  int rope_max_pos;       /* positions the table holds */
+  void* q_out;            /* device [M][n_heads * head_dim] bf16 */
+  const bi_kv_layout* kv; /* host struct; kv->k and kv->v are the device cache (bf16) */
+  int layer;              /* layer of the cache the rows are appended to */
+  const int32_t* slot;    /* device [M]: KV slot of each row */
+  const int32_t* pos;     /* device [M]: position of each row in its slot */
+  int n_heads;            /* Hq (Hkv and head_dim come from kv) */
+} bi_epi_args;
+size_t bi_gemm_workspace_size(int M, int N, int K, int mode, int variant);
+int bi_gemm(const void* x, int ldx, const void* w, void* y, int ldy, int y_dtype, int M, int N, int K, int n_full,
+            int epilogue, const bi_epi_args* epi, int mode, int variant, void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------- RMSNorm
+ * Per row m (fused residual add, as in a pre-norm decoder):
+ *   r'  = x + residual_in          (residual_in NULL: r' = x)
+ *   residual_out = r' (rounded to the activation dtype; may alias residual_in)
+ *   y   = r' / sqrt(mean(r'^2) + eps) * gamma        (activation dtype)
+ *   y_f32 (optional, f32) = the same value before rounding.
+ * The mean of squares is a fixed reduction tree over H (per-thread strided
+ * partials, fixed shuffle tree, ascending cross-warp sum) that does not
+ * depend on M ("Meituan bitwise train/infer consistency", key-practices list:
+ * batch-invariant operators with one reduction order for training, Prefill
+ * and Decode; the pages do not name RMSNorm, the architecture comes from the
+ * model shapes of the workloads).  Activation dtype: bf16 (BI_MODE_BF16) or
+ * f32 (LAYERCAST).  gamma: bf16 [H].  H % 8 == 0 and H <= 16384. */
+int bi_rmsnorm(const void* x, const void* residual_in, void* residual_out, const void* gamma, void* y,
+               float* y_f32, int M, int H, float eps, int mode, void* stream);
+
+/* Rotary embedding + KV append for T tokens after the QKV projection (the
+ * pages are silent on positional encoding: rotate-half RoPE of the Llama- and
+ * Qwen-shaped workloads, no frequency scaling; the LayerCast and FAST paths
+ * use this kernel, the bf16 invariant path the fused GEMM epilogue).
  * qkv: f32 [T][(Hq + 2*Hkv) * d] (q heads, then k heads, then v heads).
  * q_out: [T][Hq*d] activation dtype; k and v rows are written to the cache at
  * (slot[t], layer, head, pos[t]).  slot/pos: device int32 [T].
@@ -200,9 +243,9 @@ int bi_attention(const void* q, const bi_kv_layout* kv, int layer, const int32_t
  *   h is split exactly into three bf16 parts (h = p0 + p1 + p2; 8+8+8
  *   significant bits), each product with W is exact, the three products are
  *   accumulated in fp32 on the tensor cores and added as (z0 + z1) + z2.
- *   p0 = bf16(h) is the main-pass input.  For B <= 10 one GEMM pass over W
+ *   p0 = bf16(h) is the main-pass input.  For B <= 42 one GEMM pass over W
  *   computes the main logits and the parts of every row (3B token rows in
- *   one 32-row token tile, W read once); for larger B a second pass over W
+ *   one 128-row token tile, W read once); for larger B a second pass over W
  *   computes p1.W^T and p2.W^T of the flagged rows only, when there are any.
  *   Their lse, logprob and argmax are replaced; margin keeps the bf16-path
  *   value that triggered the recompute;
@@ -216,6 +259,28 @@ size_t bi_lmhead_workspace_size(int B, int H, int V, int mode);
 int bi_lmhead_logprob(const float* h, const void* W, const int32_t* target, int B, int H, int V,
                       float margin_threshold, int mode, float* logprob, float* lse, int32_t* argmax, float* margin,
                       uint8_t* recomputed, float* logits, void* ws, size_t ws_bytes, void* stream);
+
+/* The LM head in stages, for callers that shard the vocabulary across ranks
+ * (tensor parallelism: "Meituan bitwise train/infer consistency", TP item --
+ * each rank computes its vocabulary rows over the full K, the logits are
+ * gathered, and the fixed-order reduction runs on the whole row).
+ * bi_lmhead_split: out (bf16 [parts*B][H], device) = the GEMM rows of
+ *   bi_lmhead_logprob: rows 0..B-1 = bf16(h) (round to nearest even); with
+ *   parts == 3 also the exact residual parts p1 (rows B..2B-1) and p2 (rows
+ *   2B..3B-1), h = p0 + p1 + p2.
+ * bi_lmhead_from_logits: z (f32 [parts*B][V], device) = those rows times W^T
+ *   (any row-sharded GEMM whose shards are concatenated by vocabulary id);
+ *   runs the vocabulary-chunk partials, the ascending merge, the margin test
+ *   and -- parts == 3 and margin_threshold > 0 -- the FP32 recompute of the
+ *   flagged rows from (z0 + z1) + z2, with the outputs of bi_lmhead_logprob.
+ *   Given the same logits, every output is bitwise that of bi_lmhead_logprob
+ *   (the same kernels, arguments and order).  Workspace:
+ *   bi_lmhead_logits_workspace_size(B, V) bytes. */
+int bi_lmhead_split(const float* h, int B, int H, int parts, void* out, void* stream);
+size_t bi_lmhead_logits_workspace_size(int B, int V);
+int bi_lmhead_from_logits(const float* z, int B, int V, int parts, const int32_t* target, float margin_threshold,
+                          float* logprob, float* lse, int32_t* argmax, float* margin, uint8_t* recomputed, void* ws,
+                          size_t ws_bytes, void* stream);
 
 /* LM-head logprob for callers that cannot allocate device memory.  (No
  * counterpart on the pages: this is an interface convenience, not part of
@@ -247,10 +312,16 @@ int bi_lmhead_logprob_noalloc(const float* h, const void* W, const int32_t* targ
 /* ------------------------------------------------------------ Decode step
  * A whole decoder forward for a batch of tokens (any mix of prefill chunks and
  * decode tokens of many slots: continuous batching), followed by the LM-head
- * logprob above for the tokens that ask for it.  Weights: bf16, caller-owned,
- * device pointers; layouts below.  Architecture: pre-norm Llama-style decoder
- * (RMSNorm, GQA attention with rotate-half RoPE, SwiGLU MLP, untied LM head,
- * no biases). */
+ * logprob above for the tokens that ask for it.  This is the pages' unit of
+ * consistency: "Meituan bitwise train/infer consistency" (opening summary and
+ * key-practices list) asks that a token's probability be bit-identical
+ * whichever way it is computed -- Prefill or Decode, any batch -- and every
+ * step here is one of the fixed-order calls above, so a token's logprob
+ * depends only on its own sequence.  Weights: bf16, caller-owned, device
+ * pointers; layouts below.  Architecture (the pages are silent; the
+ * workloads' Llama-3.1-8B and Qwen2.5-7B shapes): pre-norm decoder with
+ * RMSNorm, GQA attention with rotate-half RoPE, SwiGLU MLP, untied LM head,
+ * no biases. */
 typedef struct {
   int n_layers, hidden, n_heads, n_kv_heads, head_dim, ffn, vocab;
   float eps;
@@ -277,6 +348,9 @@ typedef struct {
   int rope_max_pos;
 } bi_weights;
 
+/* A context only records the model description and the caller's weight and
+ * KV-cache pointers (no device memory, no launch); it checks that the shapes
+ * are ones the kernels implement (the pages are silent on interfaces). */
 typedef struct bi_ctx bi_ctx;
 int bi_ctx_create(const bi_model_desc* desc, const bi_weights* w, const bi_kv_layout* kv, bi_ctx** out);
 int bi_ctx_destroy(bi_ctx* ctx);
@@ -306,6 +380,13 @@ typedef struct {
 size_t bi_decode_workspace_size(const bi_ctx* ctx, int max_tokens, int max_lm_rows, int max_pos);
 int bi_decode_step(bi_ctx* ctx, const bi_batch* batch, const bi_step_out* out, void* ws, size_t ws_bytes,
                    void* stream);
+
+/* Embedding gather (the first step of bi_decode_step, for callers that run
+ * the layers themselves, e.g. a tensor-parallel orchestration): x[t] =
+ * embed[ids[t]] in the activation dtype of mode (bf16 values, exact in f32).
+ * ids: device int32 [T]; embed: bf16 [V][H]; x: [T][H].  An id outside
+ * [0, V) sets the index bit of the device error word and gives a zero row. */
+int bi_embed(const int32_t* ids, const void* embed, int T, int H, int V, int mode, void* x, void* stream);
 
 /* Greedy feedback for a device-resident decode loop: for b < B,
  * ids[b] = argmax[b] and pos[b] += 1 (device int32 arrays). */

@@ -4,8 +4,9 @@ The compute path is libbi.so (hand-written CUDA, C ABI in include/bi.h); this
 package only marshals arguments to it.  There is no CPU fallback: importing
 the binding raises if the library is missing.
 """
-from ._lib import (BiError, lib, MODE_BF16, MODE_LAYERCAST, VARIANT_INVARIANT, VARIANT_FAST, DTYPE_BF16, DTYPE_F32,
-                   EPI_NONE, EPI_SWIGLU, GU_INTERLEAVE, ATTN_CHUNK, VOCAB_CHUNK)
+from ._lib import (BiError, lib, MODE_BF16, MODE_LAYERCAST, MODE_FP32, VARIANT_INVARIANT, VARIANT_FAST, DTYPE_BF16,
+                   DTYPE_F32, EPI_NONE, EPI_SWIGLU, EPI_ROPE_KV_APPEND, GU_INTERLEAVE, ATTN_CHUNK, VOCAB_CHUNK)
 
-__all__ = ["BiError", "lib", "MODE_BF16", "MODE_LAYERCAST", "VARIANT_INVARIANT", "VARIANT_FAST", "DTYPE_BF16",
-           "DTYPE_F32", "EPI_NONE", "EPI_SWIGLU", "GU_INTERLEAVE", "ATTN_CHUNK", "VOCAB_CHUNK"]
+__all__ = ["BiError", "lib", "MODE_BF16", "MODE_LAYERCAST", "MODE_FP32", "VARIANT_INVARIANT", "VARIANT_FAST",
+           "DTYPE_BF16", "DTYPE_F32", "EPI_NONE", "EPI_SWIGLU", "EPI_ROPE_KV_APPEND", "GU_INTERLEAVE", "ATTN_CHUNK",
+           "VOCAB_CHUNK"]

@@ -13,10 +13,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "lib", "libbi.so")
 
 BI_OK, BI_ERR_INVALID_ARG, BI_ERR_UNSUPPORTED, BI_ERR_WORKSPACE, BI_ERR_CAPACITY, BI_ERR_CUDA = range(6)
-MODE_BF16, MODE_LAYERCAST = 0, 1
+MODE_BF16, MODE_LAYERCAST, MODE_FP32 = 0, 1, 2
 VARIANT_INVARIANT, VARIANT_FAST = 0, 1
 DTYPE_BF16, DTYPE_F32 = 0, 1
-EPI_NONE, EPI_SWIGLU = 0, 1
+EPI_NONE, EPI_SWIGLU, EPI_ROPE_KV_APPEND = 0, 1, 2
 GU_INTERLEAVE = 16
 ATTN_CHUNK = 256
 VOCAB_CHUNK = 256
@@ -40,6 +40,11 @@ SZ = ctypes.c_size_t
 class KvLayout(ctypes.Structure):
     _fields_ = [("k", P), ("v", P), ("n_slots", I), ("n_layers", I), ("n_kv_heads", I), ("capacity", I),
                 ("head_dim", I), ("dtype", I)]
+
+
+class EpiArgs(ctypes.Structure):
+    _fields_ = [("rope", P), ("rope_max_pos", I), ("q_out", P), ("kv", ctypes.POINTER(KvLayout)), ("layer", I),
+                ("slot", P), ("pos", P), ("n_heads", I)]
 
 
 class ModelDesc(ctypes.Structure):
@@ -71,7 +76,7 @@ SIGNATURES = {
     "bi_launch_count": (ctypes.c_longlong, []),
     "bi_selftest_wait_timeout": (I, [P]),
     "bi_gemm_workspace_size": (SZ, [I, I, I, I, I]),
-    "bi_gemm": (I, [P, I, P, P, I, I, I, I, I, I, I, I, P, SZ, P]),
+    "bi_gemm": (I, [P, I, P, P, I, I, I, I, I, I, I, ctypes.POINTER(EpiArgs), I, I, P, SZ, P]),
     "bi_rmsnorm": (I, [P, P, P, P, P, P, I, I, F, I, P]),
     "bi_rope_table_fill": (I, [P, I, I, D, P]),
     "bi_rope_kv_append": (I, [P, P, I, P, ctypes.POINTER(KvLayout), I, P, P, I, I, I, I, P]),
@@ -80,12 +85,16 @@ SIGNATURES = {
     "bi_lmhead_workspace_size": (SZ, [I, I, I, I]),
     "bi_lmhead_logprob": (I, [P, P, P, I, I, I, F, I, P, P, P, P, P, P, P, SZ, P]),
     "bi_lmhead_logprob_noalloc": (I, [P, P, P, I, I, I, F, I, P, P, P, P, P, P, P]),
+    "bi_lmhead_split": (I, [P, I, I, I, P, P]),
+    "bi_lmhead_logits_workspace_size": (SZ, [I, I]),
+    "bi_lmhead_from_logits": (I, [P, I, I, I, P, F, P, P, P, P, P, P, SZ, P]),
     "bi_ctx_create": (I, [ctypes.POINTER(ModelDesc), ctypes.POINTER(Weights), ctypes.POINTER(KvLayout),
                           ctypes.POINTER(P)]),
     "bi_ctx_destroy": (I, [P]),
     "bi_decode_workspace_size": (SZ, [P, I, I, I]),
     "bi_decode_step": (I, [P, ctypes.POINTER(Batch), ctypes.POINTER(StepOut), P, SZ, P]),
     "bi_greedy_advance": (I, [P, P, P, I, P]),
+    "bi_embed": (I, [P, P, I, I, I, I, P, P]),
     "bi_synth_fill_bf16": (I, [P, ctypes.c_int64, ctypes.c_int64, ctypes.c_uint64, D, I, I, P]),
 }
 

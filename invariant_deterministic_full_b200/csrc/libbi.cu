@@ -34,26 +34,60 @@ struct Carver {
 };
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+static bool mode_ok(int mode) { return mode == BI_MODE_BF16 || mode == BI_MODE_LAYERCAST || mode == BI_MODE_FP32; }
+// Activations and the KV cache are f32 in LayerCast and FP32 modes.
+static int act_f32(int mode) { return mode != BI_MODE_BF16 ? 1 : 0; }
 
 // ------------------------------------------------------------------ GEMM
 static int gemm_run(const void* x, int ldx, const void* w, void* y, int ldy, int y_dtype, int M, int N, int K, int epi,
-                    int mode, int variant, void* ws, size_t ws_bytes, cudaStream_t st) {
-  BI_REQUIRE(w && ((x && y) || M == 0), BI_ERR_INVALID_ARG, "bi_gemm: NULL pointer");
+                    const bi_epi_args* ea, int mode, int variant, void* ws, size_t ws_bytes, cudaStream_t st,
+                    int n_full = 0) {
+  const bool rope = epi == BI_EPI_ROPE_KV_APPEND;
+  BI_REQUIRE(w && ((x && (y || rope)) || M == 0), BI_ERR_INVALID_ARG, "bi_gemm: NULL pointer");
   BI_REQUIRE(M >= 0 && N > 0 && K > 0, BI_ERR_INVALID_ARG, "bi_gemm: bad sizes M=%d N=%d K=%d", M, N, K);
+  BI_REQUIRE(n_full == 0 || (n_full >= N && n_full % 64 == 0), BI_ERR_INVALID_ARG,
+             "bi_gemm: n_full=%d must be 0 or the full matrix's rows (>= N=%d, a multiple of 64)", n_full, N);
   BI_REQUIRE(K % 64 == 0 && N % 64 == 0, BI_ERR_UNSUPPORTED, "bi_gemm: need K %% 64 == 0 and N %% 64 == 0 (N=%d K=%d)",
              N, K);
   BI_REQUIRE(ldx >= K && ldx % 8 == 0, BI_ERR_UNSUPPORTED, "bi_gemm: ldx=%d must be >= K and a multiple of 8", ldx);
+  BI_REQUIRE(epi == BI_EPI_NONE || epi == BI_EPI_SWIGLU || rope, BI_ERR_INVALID_ARG, "bi_gemm: bad epilogue %d", epi);
   const int n_out = epi == BI_EPI_SWIGLU ? N / 2 : N;
-  BI_REQUIRE(ldy >= n_out, BI_ERR_INVALID_ARG, "bi_gemm: ldy=%d < output columns %d", ldy, n_out);
+  BI_REQUIRE(rope || ldy >= n_out, BI_ERR_INVALID_ARG, "bi_gemm: ldy=%d < output columns %d", ldy, n_out);
   BI_REQUIRE(aligned16(x) && aligned16(w), BI_ERR_UNSUPPORTED, "bi_gemm: x and w must be 16-byte aligned");
-  BI_REQUIRE(epi == BI_EPI_NONE || epi == BI_EPI_SWIGLU, BI_ERR_INVALID_ARG, "bi_gemm: bad epilogue %d", epi);
-  BI_REQUIRE(mode == BI_MODE_BF16 || mode == BI_MODE_LAYERCAST, BI_ERR_INVALID_ARG, "bi_gemm: bad mode %d", mode);
+  BI_REQUIRE(mode_ok(mode), BI_ERR_INVALID_ARG, "bi_gemm: bad mode %d", mode);
   BI_REQUIRE(y_dtype == BI_DTYPE_BF16 || y_dtype == BI_DTYPE_F32, BI_ERR_INVALID_ARG, "bi_gemm: bad y dtype");
+  BI_REQUIRE(rope == (ea != nullptr), BI_ERR_INVALID_ARG, "bi_gemm: epilogue arguments %s",
+             rope ? "missing for BI_EPI_ROPE_KV_APPEND" : "given for an epilogue that takes none");
+  RopeEpi re{};
+  if (rope) {
+    BI_REQUIRE(mode == BI_MODE_BF16 && variant == BI_VARIANT_INVARIANT, BI_ERR_UNSUPPORTED,
+               "bi_gemm: BI_EPI_ROPE_KV_APPEND needs BI_MODE_BF16 and the invariant variant");
+    const bi_kv_layout* kv = ea->kv;
+    BI_REQUIRE(kv && kv->k && kv->v && ea->rope && ea->q_out && ea->slot && ea->pos, BI_ERR_INVALID_ARG,
+               "bi_gemm: NULL RoPE/KV epilogue argument");
+    BI_REQUIRE(kv->dtype == BI_DTYPE_BF16, BI_ERR_INVALID_ARG, "bi_gemm: the RoPE/KV epilogue needs a bf16 cache");
+    BI_REQUIRE(kv->head_dim == 64 || kv->head_dim == 128, BI_ERR_UNSUPPORTED, "bi_gemm: head_dim %d", kv->head_dim);
+    BI_REQUIRE(ea->n_heads > 0 && kv->n_kv_heads > 0 && ea->n_heads % kv->n_kv_heads == 0, BI_ERR_INVALID_ARG,
+               "bi_gemm: Hq=%d Hkv=%d", ea->n_heads, kv->n_kv_heads);
+    BI_REQUIRE(N == (ea->n_heads + 2 * kv->n_kv_heads) * kv->head_dim, BI_ERR_INVALID_ARG,
+               "bi_gemm: N=%d is not (Hq + 2 Hkv) * head_dim", N);
+    BI_REQUIRE(ea->layer >= 0 && ea->layer < kv->n_layers && kv->n_slots > 0 && kv->capacity > 0 &&
+                   ea->rope_max_pos > 0,
+               BI_ERR_INVALID_ARG, "bi_gemm: bad cache layer/shape");
+    BI_REQUIRE(aligned16(ea->q_out) && aligned16(kv->k) && aligned16(kv->v), BI_ERR_UNSUPPORTED,
+               "bi_gemm: q_out and the cache must be 16-byte aligned");
+    re = RopeEpi{ea->rope, ea->rope_max_pos, ea->q_out, kv->k, kv->v, ea->slot, ea->pos,
+                 ea->n_heads, kv->n_kv_heads, kv->head_dim, ea->layer, kv->n_layers, kv->n_slots, kv->capacity};
+  }
   if (M == 0) return BI_OK;
   const int y_f32 = y_dtype == BI_DTYPE_F32;
+  if (mode == BI_MODE_FP32)
+    return gemm_f32(reinterpret_cast<const float*>(x), ldx, w, y, ldy, y_f32, M, N, K, epi, nullptr, st, true);
   if (mode == BI_MODE_LAYERCAST)
-    return gemm_layercast(reinterpret_cast<const float*>(x), ldx, w, y, ldy, y_f32, M, N, K, epi, ws, ws_bytes, st);
-  return gemm_bf16(x, ldx, w, y, ldy, y_f32, M, N, K, epi, variant, ws, ws_bytes, st);
+    return gemm_layercast(reinterpret_cast<const float*>(x), ldx, w, y, ldy, y_f32, M, N, K, epi, ws, ws_bytes, st,
+                          n_full);
+  return gemm_bf16(x, ldx, w, y, ldy, y_f32, M, N, K, epi, variant, ws, ws_bytes, st, nullptr, 1,
+                   rope ? &re : nullptr, n_full);
 }
 
 // ------------------------------------------------------------------ attention
@@ -143,7 +177,8 @@ static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const
   BI_REQUIRE(d == 64 || d == 128, BI_ERR_UNSUPPORTED, "bi_attention: head_dim %d (need 64 or 128)", d);
   BI_REQUIRE(Hkv > 0 && Hq > 0 && Hq % Hkv == 0, BI_ERR_INVALID_ARG, "bi_attention: Hq=%d Hkv=%d", Hq, Hkv);
   BI_REQUIRE(layer >= 0 && layer < kv->n_layers, BI_ERR_INVALID_ARG, "bi_attention: layer %d", layer);
-  const int f32 = mode == BI_MODE_LAYERCAST;
+  BI_REQUIRE(mode_ok(mode), BI_ERR_INVALID_ARG, "bi_attention: bad mode %d", mode);
+  const int f32 = act_f32(mode);
   BI_REQUIRE(kv->dtype == (f32 ? BI_DTYPE_F32 : BI_DTYPE_BF16), BI_ERR_INVALID_ARG,
              "bi_attention: KV dtype does not match the mode");
   if (T == 0) return BI_OK;
@@ -235,12 +270,13 @@ static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const
 // ------------------------------------------------------------------ LM head
 // LM-head recompute layouts.  One pass (B <= LM_ONE_PASS_ROWS): the GEMM runs
 // over 3B rows -- bf16(h) then the two exact residual parts of every row --
-// which fit one 32-row token tile, so W is read once and the flagged rows'
-// FP32 logits come for free.  Two passes (larger B): the main GEMM over B
+// which fit one 128-row token tile of the tensor-core MMA, so W is read once
+// and the flagged rows' FP32 logits come for free (the MMA costs the same for
+// 3 or 126 live rows).  Two passes (larger B): the main GEMM over B
 // rows, then one more pass over W for the two residual parts of the flagged
 // rows only (none when no row is flagged); the part bf16(h) is the main
 // pass's.  Both compute every logit with the same per-row arithmetic.
-constexpr int LM_ONE_PASS_ROWS = 10;
+constexpr int LM_ONE_PASS_ROWS = 42;
 struct LmWs {
   uint16_t* hs;     // bf16 GEMM input: [B][H], or [3B][H] in the one-pass layout
   float* logits;    // [B or 3B][V] (LayerCast: [B][V] unless the caller's buffer is used)
@@ -278,7 +314,7 @@ static int lmhead_run(const float* h, const void* W, const int32_t* target, int 
              "bi_lmhead_logprob: NULL pointer");
   BI_REQUIRE(B >= 0 && H > 0 && V > 0, BI_ERR_INVALID_ARG, "bi_lmhead_logprob: bad sizes");
   BI_REQUIRE(H % 64 == 0 && V % 64 == 0, BI_ERR_UNSUPPORTED, "bi_lmhead_logprob: need H, V multiples of 64");
-  BI_REQUIRE(mode == BI_MODE_BF16 || mode == BI_MODE_LAYERCAST, BI_ERR_INVALID_ARG, "bi_lmhead_logprob: bad mode");
+  BI_REQUIRE(mode_ok(mode), BI_ERR_INVALID_ARG, "bi_lmhead_logprob: bad mode");
   BI_REQUIRE(aligned16(h) && aligned16(W), BI_ERR_UNSUPPORTED, "bi_lmhead_logprob: h and W must be 16-byte aligned");
   if (B == 0) return BI_OK;
   const int parts = lm_parts(mode, thresh);
@@ -305,7 +341,7 @@ static int lmhead_run(const float* h, const void* W, const int32_t* target, int 
       BI_CHECK_CUDA(cudaMemcpyAsync(logits, z, (size_t)B * V * sizeof(float), cudaMemcpyDeviceToDevice, st));
   } else {
     z = logits ? logits : w.logits;
-    BI_TRY(gemm_f32(h, H, W, z, V, 1, B, V, H, BI_EPI_NONE, nullptr, st));
+    BI_TRY(gemm_f32(h, H, W, z, V, 1, B, V, H, BI_EPI_NONE, nullptr, st, mode == BI_MODE_FP32));
   }
   BI_TRY(launch(lm_partial_kernel, dim3(dim3((nch + LM_CPB - 1) / LM_CPB, B)), dim3(32 * LM_CPB), 0, st, z, V, V, target, nullptr, nullptr, w.part, nch,
                 1, 0, nullptr));
@@ -329,6 +365,55 @@ static int lmhead_run(const float* h, const void* W, const int32_t* target, int 
     }
     BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, w.count, w.list, target, th, 1, logprob,
                                                           lse, argmax, margin, recomputed, nullptr));
+  }
+  return BI_OK;
+}
+
+// The LM head's stages for callers that shard the vocabulary across ranks
+// (tensor parallelism): the split of h into the GEMM rows, then everything
+// after the GEMM on given logits.  The same kernels with the same arguments as
+// the one-pass route of lmhead_run, so a row's results are the same bits.
+struct LmStageWs {
+  LmPart* part;
+  uint8_t* flag;
+  int32_t* list;
+  int* count;
+};
+static LmStageWs lm_stage_carve(Carver& cv, int B, int V) {
+  const int nch = (V + LM_CHUNK - 1) / LM_CHUNK;
+  LmStageWs w{};
+  w.part = cv.take<LmPart>((size_t)B * nch);
+  w.flag = cv.take<uint8_t>(B);
+  w.list = cv.take<int32_t>(B);
+  w.count = cv.take<int>(1);
+  return w;
+}
+
+static int lm_from_logits_run(const float* z, int B, int V, int parts, const int32_t* target, float thresh,
+                              float* logprob, float* lse, int32_t* argmax, float* margin, uint8_t* recomputed,
+                              void* ws, size_t ws_bytes, cudaStream_t st) {
+  BI_REQUIRE(z && logprob && lse && argmax && margin && recomputed, BI_ERR_INVALID_ARG,
+             "bi_lmhead_from_logits: NULL pointer");
+  BI_REQUIRE(B >= 0 && V > 0 && (parts == 1 || parts == 3), BI_ERR_INVALID_ARG, "bi_lmhead_from_logits: bad sizes");
+  if (B == 0) return BI_OK;
+  Carver probe(nullptr);
+  lm_stage_carve(probe, B, V);
+  BI_REQUIRE(ws && ws_bytes >= probe.used + 256, BI_ERR_WORKSPACE, "bi_lmhead_from_logits: workspace %zu < %zu",
+             ws_bytes, probe.used + 256);
+  Carver cv(reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255)));
+  LmStageWs w = lm_stage_carve(cv, B, V);
+  const int nch = (V + LM_CHUNK - 1) / LM_CHUNK;
+  const float th = parts == 3 ? thresh : 0.f;
+  BI_TRY(launch(lm_partial_kernel, dim3((nch + LM_CPB - 1) / LM_CPB, B), dim3(32 * LM_CPB), 0, st, z, (size_t)V, V,
+                target, nullptr, nullptr, w.part, nch, 1, 0, nullptr));
+  BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, nullptr, nullptr,
+                target, th, 0, logprob, lse, argmax, margin, recomputed, w.flag));
+  if (parts == 3 && thresh > 0.f) {
+    BI_TRY(launch(lm_compact_kernel, dim3(B), dim3(32), 0, st, w.flag, B, nullptr, 0, w.list, w.count, nullptr));
+    BI_TRY(launch(lm_partial_kernel, dim3((nch + LM_CPB - 1) / LM_CPB, B), dim3(32 * LM_CPB), 0, st, z, (size_t)V, V,
+                  target, w.list, w.count, w.part, nch, 3, B, nullptr));
+    BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, w.count, w.list,
+                  target, th, 1, logprob, lse, argmax, margin, recomputed, nullptr));
   }
   return BI_OK;
 }
@@ -403,11 +488,12 @@ size_t bi_gemm_workspace_size(int M, int N, int K, int mode, int variant) {
   return gemm_ws_bytes(M, N, K, mode, variant);
 }
 
-int bi_gemm(const void* x, int ldx, const void* w, void* y, int ldy, int y_dtype, int M, int N, int K, int epilogue,
-            int mode, int variant, void* ws, size_t ws_bytes, void* stream) {
+int bi_gemm(const void* x, int ldx, const void* w, void* y, int ldy, int y_dtype, int M, int N, int K, int n_full,
+            int epilogue, const bi_epi_args* epi, int mode, int variant, void* ws, size_t ws_bytes, void* stream) {
   BI_RANGE("bi_gemm");
   clear_error();
-  return gemm_run(x, ldx, w, y, ldy, y_dtype, M, N, K, epilogue, mode, variant, ws, ws_bytes, as_stream(stream));
+  return gemm_run(x, ldx, w, y, ldy, y_dtype, M, N, K, epilogue, epi, mode, variant, ws, ws_bytes, as_stream(stream),
+                  n_full);
 }
 
 int bi_rmsnorm(const void* x, const void* residual_in, void* residual_out, const void* gamma, void* y, float* y_f32,
@@ -417,14 +503,14 @@ int bi_rmsnorm(const void* x, const void* residual_in, void* residual_out, const
   BI_REQUIRE(x && gamma && y, BI_ERR_INVALID_ARG, "bi_rmsnorm: NULL pointer");
   BI_REQUIRE(M >= 0 && H > 0 && H % 8 == 0 && H <= NORM_THREADS * NORM_MAX_CHUNKS * 8, BI_ERR_UNSUPPORTED,
              "bi_rmsnorm: H=%d (need H %% 8 == 0, H <= 16384)", H);
-  BI_REQUIRE(mode == BI_MODE_BF16 || mode == BI_MODE_LAYERCAST, BI_ERR_INVALID_ARG, "bi_rmsnorm: bad mode");
+  BI_REQUIRE(mode_ok(mode), BI_ERR_INVALID_ARG, "bi_rmsnorm: bad mode");
   BI_REQUIRE(aligned16(x) && aligned16(gamma) && aligned16(y) && (!residual_in || aligned16(residual_in)) &&
                  (!residual_out || aligned16(residual_out)) && (!y_f32 || aligned16(y_f32)),
              BI_ERR_UNSUPPORTED, "bi_rmsnorm: buffers must be 16-byte aligned");
   if (M == 0) return BI_OK;
   BI_TRY(launch(rmsnorm_kernel, dim3(M), dim3(NORM_THREADS), 0, as_stream(stream), x, residual_in, residual_out,
                                                             reinterpret_cast<const uint16_t*>(gamma), y, y_f32, H, eps,
-                                                            mode == BI_MODE_LAYERCAST));
+                                                            act_f32(mode)));
   return BI_OK;
 }
 
@@ -455,12 +541,12 @@ int bi_rope_kv_append(const float* qkv, const float* rope, int rope_max_pos, voi
   BI_REQUIRE(qkv && rope && q_out && kv && kv->k && kv->v && slot && pos, BI_ERR_INVALID_ARG,
              "bi_rope_kv_append: NULL pointer");
   BI_REQUIRE(layer >= 0 && layer < kv->n_layers && T >= 0 && Hq > 0, BI_ERR_INVALID_ARG, "bi_rope_kv_append: bad args");
-  BI_REQUIRE(kv->dtype == (mode == BI_MODE_LAYERCAST ? BI_DTYPE_F32 : BI_DTYPE_BF16), BI_ERR_INVALID_ARG,
+  BI_REQUIRE(mode_ok(mode) && kv->dtype == (act_f32(mode) ? BI_DTYPE_F32 : BI_DTYPE_BF16), BI_ERR_INVALID_ARG,
              "bi_rope_kv_append: KV dtype does not match the mode");
   if (T == 0) return BI_OK;
   BI_TRY(launch(rope_append_kernel, dim3(T), dim3(256), 0, as_stream(stream), qkv, rope, rope_max_pos, q_out, kv->k, kv->v, slot, pos, Hq,
                                                        kv->n_kv_heads, kv->head_dim, layer, kv->n_layers, kv->n_slots,
-                                                       kv->capacity, mode == BI_MODE_LAYERCAST, qk_paired ? 1 : 0));
+                                                       kv->capacity, act_f32(mode), qk_paired ? 1 : 0));
   return BI_OK;
 }
 
@@ -495,6 +581,34 @@ int bi_lmhead_logprob(const float* h, const void* W, const int32_t* target, int 
                     ws, ws_bytes, as_stream(stream));
 }
 
+int bi_lmhead_split(const float* h, int B, int H, int parts, void* out, void* stream) {
+  BI_RANGE("bi_lmhead_split");
+  clear_error();
+  BI_REQUIRE(h && out && B >= 0 && H > 0 && (parts == 1 || parts == 3), BI_ERR_INVALID_ARG,
+             "bi_lmhead_split: bad arguments");
+  if (B == 0) return BI_OK;
+  const size_t n = (size_t)B * H;
+  BI_TRY(launch(lm_split_kernel, dim3((int)std::min<size_t>((n + 255) / 256, 4096)), dim3(256), 0, as_stream(stream),
+                h, reinterpret_cast<uint16_t*>(out), n, parts));
+  return BI_OK;
+}
+
+size_t bi_lmhead_logits_workspace_size(int B, int V) {
+  if (B <= 0 || V <= 0) return 0;
+  Carver cv(nullptr);
+  lm_stage_carve(cv, B, V);
+  return cv.used + 256;
+}
+
+int bi_lmhead_from_logits(const float* z, int B, int V, int parts, const int32_t* target, float margin_threshold,
+                          float* logprob, float* lse, int32_t* argmax, float* margin, uint8_t* recomputed, void* ws,
+                          size_t ws_bytes, void* stream) {
+  BI_RANGE("bi_lmhead_from_logits");
+  clear_error();
+  return lm_from_logits_run(z, B, V, parts, target, margin_threshold, logprob, lse, argmax, margin, recomputed, ws,
+                            ws_bytes, as_stream(stream));
+}
+
 int bi_ctx_create(const bi_model_desc* desc, const bi_weights* w, const bi_kv_layout* kv, bi_ctx** out) {
   clear_error();
   BI_REQUIRE(desc && w && kv && out, BI_ERR_INVALID_ARG, "bi_ctx_create: NULL pointer");
@@ -503,7 +617,7 @@ int bi_ctx_create(const bi_model_desc* desc, const bi_weights* w, const bi_kv_la
                  d.vocab > 0,
              BI_ERR_INVALID_ARG, "bi_ctx_create: bad model sizes");
   BI_REQUIRE(d.n_heads % d.n_kv_heads == 0, BI_ERR_INVALID_ARG, "bi_ctx_create: n_heads %% n_kv_heads != 0");
-  BI_REQUIRE(d.mode == BI_MODE_BF16 || d.mode == BI_MODE_LAYERCAST, BI_ERR_INVALID_ARG, "bi_ctx_create: bad mode");
+  BI_REQUIRE(mode_ok(d.mode), BI_ERR_INVALID_ARG, "bi_ctx_create: bad mode");
   BI_REQUIRE(d.variant == BI_VARIANT_INVARIANT || d.variant == BI_VARIANT_FAST, BI_ERR_INVALID_ARG,
              "bi_ctx_create: bad variant");
   const int QKV = (d.n_heads + 2 * d.n_kv_heads) * d.head_dim;
@@ -520,7 +634,7 @@ int bi_ctx_create(const bi_model_desc* desc, const bi_weights* w, const bi_kv_la
   BI_REQUIRE(kv->k && kv->v && kv->n_layers == d.n_layers && kv->n_kv_heads == d.n_kv_heads &&
                  kv->head_dim == d.head_dim && kv->n_slots > 0 && kv->capacity > 0,
              BI_ERR_INVALID_ARG, "bi_ctx_create: KV layout does not match the model");
-  BI_REQUIRE(kv->dtype == (d.mode == BI_MODE_LAYERCAST ? BI_DTYPE_F32 : BI_DTYPE_BF16), BI_ERR_INVALID_ARG,
+  BI_REQUIRE(kv->dtype == (act_f32(d.mode) ? BI_DTYPE_F32 : BI_DTYPE_BF16), BI_ERR_INVALID_ARG,
              "bi_ctx_create: KV dtype does not match the mode");
   bi_ctx* c = new (std::nothrow) bi_ctx;
   BI_REQUIRE(c, BI_ERR_INVALID_ARG, "bi_ctx_create: out of host memory");
@@ -550,7 +664,7 @@ struct StepWs {
 };
 
 static StepWs step_carve(Carver& cv, const bi_model_desc& d, int T, int n_lm, int max_pos) {
-  const size_t es = d.mode == BI_MODE_LAYERCAST ? 4 : 2;
+  const size_t es = act_f32(d.mode) ? 4 : 2;
   const int QD = d.n_heads * d.head_dim, KD = d.n_kv_heads * d.head_dim;
   StepWs s{};
   s.res = cv.take<uint8_t>((size_t)T * d.hidden * es);
@@ -631,38 +745,45 @@ int bi_decode_step(bi_ctx* ctx, const bi_batch* batch, const bi_step_out* out, v
   cudaStream_t st = as_stream(stream);
   const int H = d.hidden, Hq = d.n_heads, Hkv = d.n_kv_heads, hd = d.head_dim, F = d.ffn;
   const int QD = Hq * hd, KD = Hkv * hd, QKV = QD + 2 * KD;
-  const int f32 = d.mode == BI_MODE_LAYERCAST;
+  const int f32 = act_f32(d.mode);
   const int act_dtype = f32 ? BI_DTYPE_F32 : BI_DTYPE_BF16;
-  const size_t wbytes = 2;
+  const size_t wbytes = d.mode == BI_MODE_FP32 ? 4 : 2;  // projection weights; the norm gains are bf16 in every mode
   const float scale = 1.0f / std::sqrt((float)hd);
   auto lw = [&](const void* base, size_t per_layer, int l) {
     return reinterpret_cast<const void*>(reinterpret_cast<const uint8_t*>(base) + per_layer * l * wbytes);
   };
+  auto lg = [&](const void* base, int l) {  // per-layer norm gain (bf16)
+    return reinterpret_cast<const void*>(reinterpret_cast<const uint8_t*>(base) + (size_t)H * l * 2);
+  };
 
-  BI_TRY(launch(embed_kernel, dim3(T), dim3(256), 0, st, batch->ids, reinterpret_cast<const uint16_t*>(w.embed), s.y, H, d.vocab, f32));
+  if (d.mode == BI_MODE_FP32)
+    BI_TRY(launch(embed_kernel<float>, dim3(T), dim3(256), 0, st, batch->ids, reinterpret_cast<const float*>(w.embed),
+                  s.y, H, d.vocab, f32));
+  else
+    BI_TRY(launch(embed_kernel<uint16_t>, dim3(T), dim3(256), 0, st, batch->ids,
+                  reinterpret_cast<const uint16_t*>(w.embed), s.y, H, d.vocab, f32));
   for (int l = 0; l < d.n_layers; ++l) {
-    const void* g_attn = lw(w.attn_norm, H, l);
-    const void* g_ffn = lw(w.ffn_norm, H, l);
+    const void* g_attn = lg(w.attn_norm, l);
+    const void* g_ffn = lg(w.ffn_norm, l);
     BI_TRY(bi_rmsnorm(s.y, l == 0 ? nullptr : s.res, s.res, g_attn, s.u, nullptr, T, H, d.eps, d.mode, stream));
     if (f32 || d.variant == BI_VARIANT_FAST) {  // projection, then RoPE + KV append as a kernel
       BI_TRY(gemm_run(s.u, H, lw(w.w_qkv, (size_t)QKV * H, l), s.qkv, QKV, BI_DTYPE_F32, T, QKV, H, BI_EPI_NONE,
-                      d.mode, d.variant, s.gemm, s.gemm_bytes, st));
+                      nullptr, d.mode, d.variant, s.gemm, s.gemm_bytes, st));
       BI_TRY(bi_rope_kv_append(s.qkv, w.rope, w.rope_max_pos, s.q, &ctx->kv, l, batch->slot, batch->pos, T, Hq, 1,
                                d.mode, stream));
     } else {  // RoPE + KV append in the projection's epilogue
-      RopeEpi re{w.rope, w.rope_max_pos, s.q, ctx->kv.k, ctx->kv.v, batch->slot, batch->pos,
-                 Hq, Hkv, hd, l, ctx->kv.n_layers, ctx->kv.n_slots, ctx->kv.capacity};
-      BI_TRY(gemm_bf16(s.u, H, lw(w.w_qkv, (size_t)QKV * H, l), s.qkv, QKV, 1, T, QKV, H, EPI_ROPE,
-                       BI_VARIANT_INVARIANT, nullptr, 0, st, nullptr, 1, &re));
+      const bi_epi_args ea{w.rope, w.rope_max_pos, s.q, &ctx->kv, l, batch->slot, batch->pos, Hq};
+      BI_TRY(gemm_run(s.u, H, lw(w.w_qkv, (size_t)QKV * H, l), nullptr, QKV, BI_DTYPE_BF16, T, QKV, H,
+                      BI_EPI_ROPE_KV_APPEND, &ea, d.mode, d.variant, nullptr, 0, st));
     }
     BI_TRY(attention_run(s.q, &ctx->kv, l, batch->slot, batch->pos, batch->slot_host, batch->pos_host, s.o, T, Hq,
                          scale, d.mode, d.variant, s.attn, s.attn_bytes, st));
-    BI_TRY(gemm_run(s.o, QD, lw(w.w_o, (size_t)H * QD, l), s.y, H, act_dtype, T, H, QD, BI_EPI_NONE, d.mode,
+    BI_TRY(gemm_run(s.o, QD, lw(w.w_o, (size_t)H * QD, l), s.y, H, act_dtype, T, H, QD, BI_EPI_NONE, nullptr, d.mode,
                     d.variant, s.gemm, s.gemm_bytes, st));
     BI_TRY(bi_rmsnorm(s.y, s.res, s.res, g_ffn, s.u, nullptr, T, H, d.eps, d.mode, stream));
-    BI_TRY(gemm_run(s.u, H, lw(w.w_gu, (size_t)2 * F * H, l), s.a, F, act_dtype, T, 2 * F, H, BI_EPI_SWIGLU, d.mode,
+    BI_TRY(gemm_run(s.u, H, lw(w.w_gu, (size_t)2 * F * H, l), s.a, F, act_dtype, T, 2 * F, H, BI_EPI_SWIGLU, nullptr, d.mode,
                     d.variant, s.gemm, s.gemm_bytes, st));
-    BI_TRY(gemm_run(s.a, F, lw(w.w_down, (size_t)H * F, l), s.y, H, act_dtype, T, H, F, BI_EPI_NONE, d.mode,
+    BI_TRY(gemm_run(s.a, F, lw(w.w_down, (size_t)H * F, l), s.y, H, act_dtype, T, H, F, BI_EPI_NONE, nullptr, d.mode,
                     d.variant, s.gemm, s.gemm_bytes, st));
   }
   BI_TRY(bi_rmsnorm(s.y, s.res, s.res, w.final_norm, s.u, s.h32, T, H, d.eps, d.mode, stream));
@@ -723,6 +844,21 @@ int bi_lmhead_logprob_noalloc(const float* h, const void* W, const int32_t* targ
   // so nothing needs clearing between calls.
   return lmhead_run(h, W, target, B, H, V, margin_threshold, mode, logprob, lse, argmax, margin, recomputed, logits,
                     scratch, BI_NOALLOC_SCRATCH_BYTES, as_stream(stream));
+}
+
+int bi_embed(const int32_t* ids, const void* embed, int T, int H, int V, int mode, void* x, void* stream) {
+  BI_RANGE("bi_embed");
+  clear_error();
+  BI_REQUIRE(ids && embed && x && T >= 0 && H > 0 && V > 0, BI_ERR_INVALID_ARG, "bi_embed: bad arguments");
+  BI_REQUIRE(mode_ok(mode), BI_ERR_INVALID_ARG, "bi_embed: bad mode");
+  if (T == 0) return BI_OK;
+  if (mode == BI_MODE_FP32)
+    BI_TRY(launch(embed_kernel<float>, dim3(T), dim3(256), 0, as_stream(stream), ids,
+                  reinterpret_cast<const float*>(embed), x, H, V, 1));
+  else
+    BI_TRY(launch(embed_kernel<uint16_t>, dim3(T), dim3(256), 0, as_stream(stream), ids,
+                  reinterpret_cast<const uint16_t*>(embed), x, H, V, act_f32(mode)));
+  return BI_OK;
 }
 
 int bi_greedy_advance(const int32_t* argmax, int32_t* ids, int32_t* pos, int B, void* stream) {

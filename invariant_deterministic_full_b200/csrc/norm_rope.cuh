@@ -162,7 +162,9 @@ __global__ void rope_append_kernel(const float* __restrict__ qkv, const float* _
 }
 
 // x[t][:] = E[ids[t]][:] in the activation dtype.
-__global__ void embed_kernel(const int32_t* __restrict__ ids, const uint16_t* __restrict__ E, void* __restrict__ x,
+// E: bf16 (ET = uint16_t) or f32 (ET = float, FP32-storage mode) [V][H].
+template <typename ET>
+__global__ void embed_kernel(const int32_t* __restrict__ ids, const ET* __restrict__ E, void* __restrict__ x,
                              int H, int V, int f32) {
   pdl_wait();
   pdl_trigger();
@@ -173,8 +175,14 @@ __global__ void embed_kernel(const int32_t* __restrict__ ids, const uint16_t* __
     for (int i = threadIdx.x; i < H; i += blockDim.x) store_act(x, (size_t)t * H + i, 0.f, f32);
     return;
   }
-  for (int i = threadIdx.x; i < H; i += blockDim.x)
-    store_act(x, (size_t)t * H + i, bf16_bits_to_f32(E[(size_t)id * H + i]), f32);
+  for (int i = threadIdx.x; i < H; i += blockDim.x) {
+    float v;
+    if constexpr (sizeof(ET) == 2)
+      v = bf16_bits_to_f32(E[(size_t)id * H + i]);
+    else
+      v = E[(size_t)id * H + i];
+    store_act(x, (size_t)t * H + i, v, f32);
+  }
 }
 
 __global__ void greedy_advance_kernel(const int32_t* __restrict__ argmax, int32_t* __restrict__ ids,

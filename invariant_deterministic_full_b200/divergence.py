@@ -14,9 +14,12 @@ random-init weights instead of the pages' benchmarks:
   and without the selective FP32 LM-head recompute.
 
 The reference run is LayerCast: the same bf16 weights with fp32 arithmetic,
-activations and KV cache.  Batch invariance is measured the same way: one
-configuration run on every prompt alone and on all prompts in one batch, for
-the invariant path and for the non-invariant FAST variant.
+activations and KV cache.  The FP32-storage arm (BI_MODE_FP32: the same weight
+values held as f32, fp32 FMA everywhere) is run too, so LayerCast is compared
+with what it replaces -- in agreement and in measured memory.  Batch invariance
+is measured the same way: one configuration run on every prompt alone and on
+all prompts in one batch, for the invariant path and for the non-invariant FAST
+variant.
 """
 import argparse
 import json
@@ -27,7 +30,7 @@ import numpy as np
 import synth
 from synth import configs
 
-from ._lib import MODE_BF16, MODE_LAYERCAST, VARIANT_FAST, VARIANT_INVARIANT
+from ._lib import MODE_BF16, MODE_FP32, MODE_LAYERCAST, VARIANT_FAST, VARIANT_INVARIANT
 
 
 def divergence_index(a, b):
@@ -110,6 +113,7 @@ def study(cfg, n_prompts=16, prompt_len=64, n_steps=64, threshold=0.1, seed0=200
     cap = prompt_len + n_steps + 1
     run = lambda **k: _run(model_mod, cfg, prompts, n_steps, capacity=cap, **k)
     ref, _, w_lc, kv_lc = run(mode=MODE_LAYERCAST, variant=VARIANT_INVARIANT, threshold=0.0, alone=False)
+    fp, _, w_fp, kv_fp = run(mode=MODE_FP32, variant=VARIANT_INVARIANT, threshold=0.0, alone=False)
     b0, _, w_bf, kv_bf = run(mode=MODE_BF16, variant=VARIANT_INVARIANT, threshold=0.0, alone=False)
     b1, rate, _, _ = run(mode=MODE_BF16, variant=VARIANT_INVARIANT, threshold=threshold, alone=False)
     inv1, _, _, _ = run(mode=MODE_BF16, variant=VARIANT_INVARIANT, threshold=threshold, alone=True)
@@ -118,17 +122,21 @@ def study(cfg, n_prompts=16, prompt_len=64, n_steps=64, threshold=0.1, seed0=200
     strip = lambda c: {k: v for k, v in c.items() if k != "indices"}
     no_rc, rc = compare(ref, b0), compare(ref, b1)
     kv_tokens = n_prompts * cap
-    lc, fp = memory_bytes(cfg, kv_tokens, "layercast"), memory_bytes(cfg, kv_tokens, "fp32")
+    lc, fpb = memory_bytes(cfg, kv_tokens, "layercast"), memory_bytes(cfg, kv_tokens, "fp32")
     return {
         "config": cfg["name"], "n_layers": cfg["n_layers"], "prompts": n_prompts, "prompt_len": prompt_len,
         "steps": n_steps, "threshold": threshold,
         "vs_layercast": {"bf16_no_recompute": strip(no_rc), "bf16_selective_recompute": strip(rc),
                          "recompute_gain_pp": 100.0 * (rc["exact_agreement"] - no_rc["exact_agreement"]),
                          "recompute_rate": rate},
+        "vs_fp32": {"layercast": strip(compare(fp, ref)), "bf16_no_recompute": strip(compare(fp, b0)),
+                    "bf16_selective_recompute": strip(compare(fp, b1))},
         "batch_alone_vs_batched": {"invariant": strip(compare(inv1, b1)), "fast": strip(compare(f_1, f_n))},
         "memory": {"allocated_weights_bf16": w_bf, "allocated_weights_layercast": w_lc,
-                   "allocated_kv_bf16": kv_bf, "allocated_kv_layercast": kv_lc,
-                   "layercast_bytes": lc, "fp32_storage_bytes": fp, "layercast_saving_vs_fp32": 1.0 - lc / fp,
+                   "allocated_weights_fp32": w_fp, "allocated_kv_bf16": kv_bf, "allocated_kv_layercast": kv_lc,
+                   "allocated_kv_fp32": kv_fp,
+                   "measured_layercast_saving_vs_fp32": 1.0 - (w_lc + kv_lc) / (w_fp + kv_fp),
+                   "layercast_bytes": lc, "fp32_storage_bytes": fpb, "layercast_saving_vs_fp32": 1.0 - lc / fpb,
                    "kv_positions": kv_tokens},
     }
 

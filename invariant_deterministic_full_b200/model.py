@@ -13,8 +13,8 @@ import torch
 
 import synth
 from . import ops
-from ._lib import (lib, check, ModelDesc, Weights, Batch, StepOut, MODE_BF16, MODE_LAYERCAST, VARIANT_INVARIANT,
-                   GU_INTERLEAVE)
+from ._lib import (lib, check, ModelDesc, Weights, Batch, StepOut, MODE_BF16, MODE_LAYERCAST, MODE_FP32,
+                   VARIANT_INVARIANT, GU_INTERLEAVE)
 
 
 def _to_dev_bf16(bits, device):
@@ -74,6 +74,10 @@ class Model:
         else:
             self.host_weights = None
             self.w = self._device_init(seed)
+        if mode == MODE_FP32:
+            # FP32 storage: the same weight values held as f32 (an exact upcast; the norm gains stay bf16)
+            for k in ("embed", "lm_head", "w_qkv", "w_o", "w_gu", "w_down"):
+                self.w[k] = self.w[k].float()
         self.rope_max_pos = capacity
         self.rope = ops.rope_table(capacity, d, cfg["rope_theta"], device)
         self.kv = ops.KVCache(n_slots, L, Hkv, capacity, d, mode, device)

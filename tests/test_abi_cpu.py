@@ -56,19 +56,41 @@ def test_gemm_validation(host_only):
     L = host_only
     lib = L.lib
     fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
-    assert lib.bi_gemm(None, 64, fake, fake, 64, 0, 4, 64, 64, 0, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
-    assert lib.bi_gemm(fake, 96, fake, fake, 64, 0, 4, 64, 96, 0, 0, 0, None, 0, None) == L.BI_ERR_UNSUPPORTED
+    assert lib.bi_gemm(None, 64, fake, fake, 64, 0, 4, 64, 64, 0, 0, None, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
+    assert lib.bi_gemm(fake, 96, fake, fake, 64, 0, 4, 64, 96, 0, 0, None, 0, 0, None, 0, None) == L.BI_ERR_UNSUPPORTED
     assert b"K % 64" in lib.bi_last_error()
-    assert lib.bi_gemm(fake, 64, fake, fake, 64, 0, 4, 96, 64, 0, 0, 0, None, 0, None) == L.BI_ERR_UNSUPPORTED
-    assert lib.bi_gemm(fake, 60, fake, fake, 64, 0, 4, 64, 64, 0, 0, 0, None, 0, None) == L.BI_ERR_UNSUPPORTED
-    assert lib.bi_gemm(fake, 64, fake, fake, 16, 0, 4, 64, 64, 0, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
-    assert lib.bi_gemm(fake, 64, fake, fake, 64, 0, 4, 64, 64, 7, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
-    assert lib.bi_gemm(fake, 64, ctypes.c_void_p((1 << 20) + 2), fake, 64, 0, 4, 64, 64, 0, 0, 0, None, 0,
+    assert lib.bi_gemm(fake, 64, fake, fake, 64, 0, 4, 96, 64, 0, 0, None, 0, 0, None, 0, None) == L.BI_ERR_UNSUPPORTED
+    assert lib.bi_gemm(fake, 60, fake, fake, 64, 0, 4, 64, 64, 0, 0, None, 0, 0, None, 0, None) == L.BI_ERR_UNSUPPORTED
+    assert lib.bi_gemm(fake, 64, fake, fake, 16, 0, 4, 64, 64, 0, 0, None, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
+    assert lib.bi_gemm(fake, 64, fake, fake, 64, 0, 4, 64, 64, 0, 7, None, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
+    assert lib.bi_gemm(fake, 64, ctypes.c_void_p((1 << 20) + 2), fake, 64, 0, 4, 64, 64, 0, 0, None, 0, 0, None, 0,
                        None) == L.BI_ERR_UNSUPPORTED
-    assert lib.bi_gemm(fake, 64, fake, fake, 64, 0, 0, 64, 64, 0, 0, 0, None, 0, None) == L.BI_OK  # M = 0: no work
-    assert lib.bi_gemm(None, 64, fake, None, 64, 0, 0, 64, 64, 0, 0, 0, None, 0, None) == L.BI_OK  # empty x, y
-    assert lib.bi_gemm(None, 64, None, None, 64, 0, 0, 64, 64, 0, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
-    assert lib.bi_gemm(fake, 64, fake, None, 64, 0, 4, 64, 64, 0, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
+    assert lib.bi_gemm(fake, 64, fake, fake, 64, 0, 0, 64, 64, 0, 0, None, 0, 0, None, 0, None) == L.BI_OK  # M = 0: no work
+    assert lib.bi_gemm(None, 64, fake, None, 64, 0, 0, 64, 64, 0, 0, None, 0, 0, None, 0, None) == L.BI_OK  # empty x, y
+    assert lib.bi_gemm(None, 64, None, None, 64, 0, 0, 64, 64, 0, 0, None, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
+    assert lib.bi_gemm(fake, 64, fake, None, 64, 0, 4, 64, 64, 0, 0, None, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
+    # RoPE + KV-append epilogue: its arguments are required, checked against the cache, and bf16 invariant only
+    kv = L.KvLayout(1 << 20, 1 << 20, 2, 1, 2, 64, 64, 0)
+    ea = L.EpiArgs(1 << 20, 64, 1 << 20, ctypes.pointer(kv), 0, 1 << 20, 1 << 20, 4)  # N = (4 + 2*2) * 64 = 512
+    R = L.EPI_ROPE_KV_APPEND
+    assert lib.bi_gemm(fake, 64, fake, None, 0, 0, 4, 512, 64, 0, R, None, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
+    assert lib.bi_gemm(fake, 64, fake, fake, 512, 0, 4, 512, 64, 0, 0, ctypes.byref(ea), 0, 0, None, 0, None) == \
+        L.BI_ERR_INVALID_ARG  # arguments given for an epilogue that takes none
+    assert lib.bi_gemm(fake, 64, fake, None, 0, 0, 4, 512, 64, 0, R, ctypes.byref(ea), 1, 0, None, 0, None) == \
+        L.BI_ERR_UNSUPPORTED  # LayerCast
+    assert lib.bi_gemm(fake, 64, fake, None, 0, 0, 4, 512, 64, 0, R, ctypes.byref(ea), 0, 1, None, 0, None) == \
+        L.BI_ERR_UNSUPPORTED  # FAST variant
+    assert lib.bi_gemm(fake, 64, fake, None, 0, 0, 4, 576, 64, 0, R, ctypes.byref(ea), 0, 0, None, 0, None) == \
+        L.BI_ERR_INVALID_ARG  # N is not (Hq + 2 Hkv) * head_dim
+    ea.layer = 1
+    assert lib.bi_gemm(fake, 64, fake, None, 0, 0, 4, 512, 64, 0, R, ctypes.byref(ea), 0, 0, None, 0, None) == \
+        L.BI_ERR_INVALID_ARG  # layer beyond the cache
+    ea.layer = 0
+    assert lib.bi_gemm(fake, 64, fake, None, 0, 0, 0, 512, 64, 0, R, ctypes.byref(ea), 0, 0, None, 0, None) == L.BI_OK
+    # n_full names the whole matrix a row shard belongs to: at least N rows, a multiple of 64
+    assert lib.bi_gemm(fake, 64, fake, fake, 64, 0, 4, 128, 64, 64, 0, None, 0, 0, None, 0, None) == L.BI_ERR_INVALID_ARG
+    assert lib.bi_gemm(fake, 64, fake, fake, 64, 0, 4, 128, 64, 200, 0, None, 0, 0, None, 0, None) == \
+        L.BI_ERR_INVALID_ARG
     assert lib.bi_gemm_workspace_size(4, 64, 64, 0, 0) == 0
 
 

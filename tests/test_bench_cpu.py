@@ -33,8 +33,7 @@ def test_gemm_set_is_four_projections_per_layer_plus_the_lm_head():
 
 
 def test_stored_gemm_traffic_applies_to_this_source_and_equals_the_algorithmic_bytes():
-    src = open(bench.os.path.join(bench.ROOT, "invariant_deterministic_full_b200", "csrc", "gemm.cuh")).read()
-    assert len(bench.gemm_bf16_source_digest(src)) == 64  # the digest's landmarks are all present
+    assert len(bench.current_gemm_digest()) == 64  # the digest's landmarks are all present
     t = bench.gemm_traffic_per_launch(L8, 32)
     if t is None:
         pytest.skip("GEMM kernel source changed since the stored ncu capture: traffic is reported as null")
@@ -43,13 +42,19 @@ def test_stored_gemm_traffic_applies_to_this_source_and_equals_the_algorithmic_b
     assert bench.gemm_traffic_per_launch(L8, 16) is None  # captured at batch 32 only
 
 
-def test_gemm_source_digest_ignores_code_outside_the_bf16_kernel():
-    src = open(bench.os.path.join(bench.ROOT, "invariant_deterministic_full_b200", "csrc", "gemm.cuh")).read()
-    h = bench.gemm_bf16_source_digest(src)
-    assert bench.gemm_bf16_source_digest(src + "\n// trailing helper\n") == h
-    i = src.index("__global__ void __launch_bounds__(160, CPS)")
-    assert bench.gemm_bf16_source_digest(src[:i] + "// a comment\n  /* and another */ " + src[i:]) == h
-    assert bench.gemm_bf16_source_digest(src[:i] + "constexpr int kExtra = 1;\n" + src[i:]) != h
+def test_gemm_source_digest_ignores_comments_and_code_outside_the_kernel():
+    rd = lambda n: open(bench.os.path.join(bench.CSRC, n)).read()
+    tc, mma, plan = rd("gemm_tc.cuh"), rd("gemm_mma.cuh"), rd("gemm.cuh")
+    h = bench.gemm_source_digest(tc, mma, plan)
+    assert bench.gemm_source_digest(tc, mma, plan + "\n// trailing helper\n") == h
+    i = tc.index("template <int BN, int MT, int XR, int KS, int EPI, int CPS>")
+    assert bench.gemm_source_digest(tc[:i] + "// a comment\n  /* and another */ " + tc[i:], mma, plan) == h
+    assert bench.gemm_source_digest(tc[:i] + "constexpr int kExtra = 1;\n" + tc[i:], mma, plan) != h
+    assert bench.gemm_source_digest(tc, mma + "static int kMore = 4;\n", plan) != h
+    j = plan.index("static TcPlan tc_plan(")
+    assert bench.gemm_source_digest(tc, mma, plan[:j] + "static int kOther = 2;\n" + plan[j:]) != h
+    k = plan.index("size_t gemm_ws_bytes(")  # workspace sizing does not decide the traffic
+    assert bench.gemm_source_digest(tc, mma, plan[:k] + "static int kWs = 3;\n" + plan[k:]) == h
 
 
 def test_clock_summary_median_and_reasons():

@@ -25,3 +25,56 @@ def test_divergence_study_tiny():
         assert 0.0 <= c["exact_agreement"] <= 1.0 and c["exact_agreement"] + c["diverged"] == pytest.approx(1.0)
     assert 0.0 <= v["recompute_rate"] <= 1.0
     assert ops.device_error() == 0
+
+
+def _oracle_greedy(cfg, w, prompt, n_steps, mode):
+    """The oracle's own greedy run: the prompt, then one token at a time after the stored keys/values.
+    Returns the generated tokens and the oracle's top-2 margin at each choice."""
+    import numpy as np
+    import oracle
+    res, _, (k, v) = oracle.forward_ctx(cfg, w, prompt, mode=mode, want_kv=True)
+    toks, margins = [int(res[-1, 2])], [float(res[-1, 3])]
+    for _ in range(n_steps):
+        res, _, (k1, v1) = oracle.forward_ctx(cfg, w, np.array(toks[-1:], np.int32), k, v, mode=mode, want_kv=True)
+        k, v = np.concatenate([k, k1], axis=1), np.concatenate([v, v1], axis=1)
+        toks.append(int(res[-1, 2]))
+        margins.append(float(res[-1, 3]))
+    return toks, margins
+
+
+def test_divergence_index_matches_the_oracles_greedy_runs():
+    """The study's bf16-vs-LayerCast divergence index on the tiny config is the oracle's own: its greedy runs in
+    bf16-storage emulation and in exact fp64 give the same first differing position, wherever the oracle's top-2
+    margin is clear (> 0.05) at every choice up to it (else either token is a correct greedy choice)."""
+    import numpy as np
+    import torch
+    import synth
+    from invariant_deterministic_full_b200 import divergence as dv, model as mdl, ops
+    from invariant_deterministic_full_b200._lib import MODE_BF16, MODE_LAYERCAST
+    import oracle
+    assert torch.cuda.is_available()
+    cfg = configs.TINY
+    w = synth.model_weights(cfg)
+    prompts = [synth.prompt_tokens(2000 + r, 16, cfg["vocab"]) for r in range(6)]
+    n_steps = 24
+
+    def gpu_run(mode):
+        m = mdl.Model(cfg, mode=mode, n_slots=len(prompts), capacity=64, margin_threshold=0.0, host_weights=w)
+        seqs, _ = mdl.greedy_generate(m, prompts, n_steps)
+        m.close()
+        return [s[16:] for s in seqs]
+
+    g_bf, g_lc = gpu_run(MODE_BF16), gpu_run(MODE_LAYERCAST)
+    checked = 0
+    for p, gb, gl in zip(prompts, g_bf, g_lc):
+        ob, mb = _oracle_greedy(cfg, w, p, n_steps, oracle.OR_BF16)
+        oe, me = _oracle_greedy(cfg, w, p, n_steps, oracle.OR_EXACT)
+        i_or = dv.divergence_index(ob, oe)
+        last = len(ob) - 1 if i_or is None else i_or
+        if min(mb[: last + 1]) <= 0.05 or min(me[: last + 1]) <= 0.05:
+            continue  # a near-tie before the divergence: either greedy token is correct
+        assert gb[: last + 1] == ob[: last + 1] and gl[: last + 1] == oe[: last + 1]
+        assert dv.divergence_index(gb, gl) == i_or
+        checked += 1
+    assert checked >= 3, f"only {checked} prompts had clear margins"
+    assert ops.device_error() == 0

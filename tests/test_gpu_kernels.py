@@ -131,13 +131,13 @@ def test_gemm_batch_invariance(bi, mode):
     """Row r of x.W^T is bitwise the same whatever the number of rows and the row's position."""
     rng = np.random.default_rng(5)
     N, K = 4096, 1024
-    xs = rng.standard_normal((100, K)).astype(np.float32)
+    xs = rng.standard_normal((300, K)).astype(np.float32)
     if mode == 0:
         xs = synth.bf16_to_f32(synth.f32_to_bf16_bits(xs))
     w = _bf16_dev(0.02 * rng.standard_normal((N, K)))
     dev = lambda a: (_bf16_dev(a) if mode == 0 else torch.from_numpy(np.ascontiguousarray(a)).cuda())
     full = bi.gemm(dev(xs), w, mode=mode, out_dtype=torch.float32).cpu()
-    for M, off in [(1, 0), (1, 57), (4, 30), (31, 2), (32, 40), (33, 17), (64, 36)]:
+    for M, off in [(1, 0), (1, 57), (4, 30), (31, 2), (32, 40), (33, 17), (64, 36), (129, 40), (257, 43)]:
         part = bi.gemm(dev(xs[off:off + M]), w, mode=mode, out_dtype=torch.float32).cpu()
         assert torch.equal(part, full[off:off + M]), (M, off)
     _after(bi)
@@ -188,6 +188,63 @@ def test_gemm_fast_variant_is_not_invariant_but_close(bi):
     f32 = bi.gemm(_bf16_dev(xs), w, variant=1, out_dtype=torch.float32).cpu()
     assert torch.allclose(f1[0], inv[0], rtol=1e-4, atol=1e-4)
     assert not torch.equal(f1[0], f32[0])  # split-K chosen from M changes the bits
+    _after(bi)
+
+
+@pytest.mark.parametrize("d,Hq,Hkv", [(128, 4, 2), (64, 4, 4)])
+def test_gemm_rope_kv_epilogue_vs_oracle(bi, d, Hq, Hkv):
+    """bi_gemm with BI_EPI_ROPE_KV_APPEND through the C ABI: q (natural order) and the appended k, v rows against
+    the oracle's fp64 projection and rotate-half RoPE (or_rope), at positions on both sides of a 256-key chunk;
+    every cache row not written stays untouched; v equals the unfused projection bit for bit."""
+    from invariant_deterministic_full_b200.model import pair_heads
+    from invariant_deterministic_full_b200.ops import KVCache, rope_table
+    rng = np.random.default_rng(d + Hq)
+    K, theta, cap, L = 256, 10000.0, 600, 2
+    QD, KD = Hq * d, Hkv * d
+    slot = np.array([0, 2, 1, 2, 0], dtype=np.int32)
+    pos = np.array([0, 255, 256, 511, 7], dtype=np.int32)
+    M = len(slot)
+    x = synth.bf16_to_f32(synth.f32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32)))
+    wq, wk, wv = (synth.f32_to_bf16_bits((0.05 * rng.standard_normal((n, K))).astype(np.float32))
+                  for n in (QD, KD, KD))
+    wf = np.concatenate([pair_heads(wq, d), pair_heads(wk, d), wv])
+    kv = KVCache(3, L, Hkv, cap, d)
+    table = rope_table(cap, d, theta)
+    sd, pd = torch.from_numpy(slot).cuda(), torch.from_numpy(pos).cuda()
+    wd = torch.from_numpy(wf.view(np.int16)).cuda().view(torch.bfloat16)
+    q = bi.gemm_rope_kv(_bf16_dev(x), wd, table, cap, kv, 1, sd, pd, Hq)
+    torch.cuda.synchronize()
+    # oracle: fp64 projection then rotate-half RoPE at each row's position
+    x64 = x.astype(np.float64)
+    qr = oracle.gemm(x64, wq)
+    kr = oracle.gemm(x64, wk)
+    vr = oracle.gemm(x64, wv)
+    qr = np.stack([oracle.rope(qr[m], Hq, d, int(pos[m]), theta) for m in range(M)])
+    kr = np.stack([oracle.rope(kr[m], Hkv, d, int(pos[m]), theta) for m in range(M)])
+    ax = np.abs(x64)
+    bq = K * 2.0 ** -24 * (ax @ np.abs(synth.bf16_to_f32(wq)).T)
+    bk = K * 2.0 ** -24 * (ax @ np.abs(synth.bf16_to_f32(wk)).T)
+    bv = K * 2.0 ** -24 * (ax @ np.abs(synth.bf16_to_f32(wv)).T)
+    # a rotated element mixes two products: twice the projection bound of its pair, the f32 table (2^-24
+    # relative) and the final bf16 rounding (half an ulp, 2^-8 relative)
+    pair = lambda b, H: np.maximum(b, b.reshape(M, H, 2, d // 2)[:, :, ::-1].reshape(M, H * d))
+    gq = _f(q)
+    assert (np.abs(gq - qr) <= 2.0 ** -8 * np.abs(qr) + 2 * pair(bq, Hq) + 2.0 ** -22 * np.abs(qr) + 1e-7).all()
+    kc, vc = _f(kv.k), _f(kv.v)
+    for m in range(M):
+        gk = kc[slot[m], 1, :, pos[m]].reshape(KD)
+        gv = vc[slot[m], 1, :, pos[m]].reshape(KD)
+        assert (np.abs(gk - kr[m]) <= 2.0 ** -8 * np.abs(kr[m]) + 2 * pair(bk, Hkv)[m] + 1e-7).all(), m
+        assert (np.abs(gv - vr[m]) <= 2.0 ** -8 * np.abs(vr[m]) + bv[m] + 1e-7).all(), m
+    written = np.zeros((3, L, cap), dtype=bool)
+    written[slot, 1, pos] = True
+    assert not np.any(kc.transpose(0, 1, 3, 2, 4)[~written]) and not np.any(vc.transpose(0, 1, 3, 2, 4)[~written])
+    # the unfused route (f32 projection, then the RoPE/append kernel) stores the same v bits
+    qkv32 = bi.gemm(_bf16_dev(x), wd, out_dtype=torch.float32)
+    kv2 = KVCache(3, L, Hkv, cap, d)
+    bi.rope_kv_append(qkv32, table, cap, kv2, 1, sd, pd, Hq, qk_paired=True)
+    torch.cuda.synchronize()
+    assert torch.equal(kv2.v, kv.v)
     _after(bi)
 
 
@@ -366,20 +423,28 @@ def test_lmhead_vs_oracle_small_vocab(bi, mode):
     _after(bi)
 
 
-@pytest.mark.parametrize("B", [4, 24])  # one-pass and second-pass recompute layouts
+@pytest.mark.parametrize("B", [4, 24, 64])  # one-pass and second-pass recompute layouts
 def test_lmhead_recompute_enabled_but_no_row_flagged(bi, B):
-    """With the recompute on but no row under the threshold, the second pass has a device-side row count of 0: it
-    must finish cleanly (no wait running out) and leave the main-pass results."""
+    """With the recompute on but no row under the threshold, the recompute stage has a device-side row count of 0:
+    it must finish cleanly (no wait running out) and leave the main-pass results.  Every row's top logit is made
+    to stand out: W row 7b + 1 is bf16(h_b / |h_b|), so z = |h_b| (about 90) there against about 2 elsewhere,
+    and no margin can fall under the threshold 1.0."""
     H, V = 512, 4096
     rng = np.random.default_rng(31)
-    W = _bf16_dev(0.02 * rng.standard_normal((V, H)))
-    hd = torch.from_numpy(_h_rows(B, H) * 4).cuda()
+    h = _h_rows(B, H) * 4
+    Wf = 0.02 * rng.standard_normal((V, H))
+    for b in range(B):
+        Wf[7 * b + 1] = h[b] / np.linalg.norm(h[b])
+    W = _bf16_dev(Wf)
+    hd = torch.from_numpy(h).cuda()
     off = bi.lmhead_logprob(hd, W, None, threshold=0.0)
-    tiny = bi.lmhead_logprob(hd, W, None, threshold=1e-30)
+    on = bi.lmhead_logprob(hd, W, None, threshold=1.0)
     torch.cuda.synchronize()
-    if int(tiny["recomputed"].sum()) == 0:
-        for k in ("logprob", "lse", "argmax", "margin"):
-            assert torch.equal(tiny[k], off[k]), k
+    assert int(on["recomputed"].sum()) == 0
+    assert float(on["margin"].min()) > 50.0
+    assert torch.equal(on["argmax"].cpu(), torch.arange(B, dtype=torch.int32) * 7 + 1)
+    for k in ("logprob", "lse", "argmax", "margin"):
+        assert torch.equal(on[k], off[k]), k
     _after(bi)
 
 
@@ -392,7 +457,7 @@ def test_lmhead_full_size_invariance_and_samples(bi):
     h = _h_rows(256, H)
     hd = torch.from_numpy(h).cuda()
     ref = {k: v.cpu() for k, v in bi.lmhead_logprob(hd, W, None, 0.1).items()}
-    for B in (1, 2, 4, 8, 10, 11, 16, 32, 64, 128):  # one-pass recompute up to 10 rows, two passes above
+    for B in (1, 2, 4, 8, 10, 11, 16, 32, 42, 43, 64, 128):  # one-pass recompute up to 42 rows, two passes above
         for off in (0, 256 - B):
             o = bi.lmhead_logprob(hd[off:off + B].contiguous(), W, None, 0.1)
             for k in ("logprob", "lse", "argmax", "margin", "recomputed"):

@@ -41,7 +41,7 @@ def test_gemm_writes_only_its_rows_columns_and_workspace(api, mode):
     y = ybuf[1:M + 1]
     wsb = lib.bi_gemm_workspace_size(M, N, K, mode, 0)
     ws = torch.full((wsb + 4096,), 0xFF, dtype=torch.uint8, device="cuda")
-    check(lib.bi_gemm(x.data_ptr(), K, w.data_ptr(), y.data_ptr(), N + pad, 1, M, N, K, 0, mode, 0, ws.data_ptr(),
+    check(lib.bi_gemm(x.data_ptr(), K, w.data_ptr(), y.data_ptr(), N + pad, 1, M, N, K, 0, 0, None, mode, 0, ws.data_ptr(),
                       wsb, ops._stream()), "bi_gemm")
     torch.cuda.synchronize()
     assert torch.isnan(ybuf[0]).all() and torch.isnan(ybuf[M + 1]).all()
