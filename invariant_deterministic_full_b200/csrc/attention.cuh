@@ -688,6 +688,261 @@ __global__ void __launch_bounds__(ATC_THREADS)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Decode schedule of the same computation (one query per block, G <= 8 q
+// heads: one 8-pair tile).  attn_tc_kernel<1, RING> walks each chunk as
+// scores -> softmax -> P.V, so at every chunk boundary the next chunk's keys
+// are only requested while P.V of the current one drains the ring.  Here a
+// CTA first streams the K rows of its whole segment (at most ATD_SEG chunks)
+// and keeps every score in shared memory, then streams the V rows, running
+// each chunk's softmax just before its P.V.  The K stream and the V stream
+// each run back to back through the ring, and all eight warps score: warps
+// 0-3 the even 64-key sub-tiles, warps 4-7 the odd ones.  Every score, every
+// softmax and every P.V chain is the instruction sequence of attn_tc_kernel
+// (each score one warp's chain of 8 ascending k16 mma over the head; the same
+// lane-strided max and denominator; the same 3-part P split and per-part
+// chains over ascending 16-key steps; the same record and merge), so the two
+// kernels, and prefill and decode, give the same bits.
+constexpr int ATD_SEG = 3;                   // chunks per CTA (scores of all of them are kept)
+constexpr int ATD_SST = ATD_SEG * 256 + 4;  // row stride of the score rows (floats)
+constexpr int ATD_RING = 4;                // K/V sub-tiles in flight per CTA (two CTAs fit an SM)
+
+__host__ __device__ inline size_t atd_smem_bytes(int ring) {
+  return (size_t)ring * 16384  // K/V sub-tiles: [2 halves][64 keys][128 B]
+         + 8 * 256             // q tile: [2 halves][8 pairs][128 B]
+         + 8 * ATD_SST * 4     // scores [8][ATD_SST]
+         + 3 * 8 * 512         // probability parts of one chunk [3][8][256 keys] bf16, swizzled
+         + 1024;
+}
+
+template <int RING>
+__global__ void __launch_bounds__(ATC_THREADS)
+    attn_dec_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ AttnPlan plan, const AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int NP = 8;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[RING];
+  __shared__ __align__(8) uint64_t empty_bar[RING];
+  __shared__ float m_s[NP], l_s[NP];
+  __shared__ int live_s[NP];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int b = blockIdx.x, sg = blockIdx.y, hk = blockIdx.z;
+  if (b >= plan.n) return;
+  const int t0 = plan.blk[b].x;  // one query per block
+  const int s = a.slot[t0];
+  const int pmax = a.pos[t0];
+  const int c_lo = sg * a.seg_len;
+  int c_hi = min(pmax / a.chunk + 1, c_lo + a.seg_len);
+  if (c_hi > a.max_chunks) {  // device position beyond what the launch was planned for
+    if (threadIdx.x == 0) dev_flag(DEVERR_CAPACITY);
+    c_hi = a.max_chunks;
+  }
+  if (c_lo >= c_hi) return;
+  const int npairs = a.G;  // <= 8
+  const int cache_base = ((s * a.n_layers + a.layer) * a.Hkv + hk) * a.cap;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g8 = lane >> 2, t4 = lane & 3;
+  constexpr uint32_t SUB = 16384;
+  uint8_t* qt = smem + RING * SUB;                             // [2][NP][128 B]
+  float* S = reinterpret_cast<float*>(qt + NP * 256);          // [NP][ATD_SST]
+  uint8_t* Pp = reinterpret_cast<uint8_t*>(S + NP * ATD_SST);  // [3][NP][512 B]
+  const uint32_t qt_s = smem_u32(qt), pp_s = smem_u32(Pp);
+  auto nsub_of = [&](int c) { return (min(a.chunk, pmax - c * a.chunk + 1) + ATT_SUB - 1) / ATT_SUB; };
+
+  if (tid == 0) {
+    for (int r = 0; r < RING; ++r) {
+      mbar_init(&full_bar[r], 1);
+      mbar_init(&empty_bar[r], ATT_THREADS / 32);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == ATT_THREADS / 32) {
+    // ---- producer warp, one lane: every K sub-tile of the segment, then every V sub-tile
+    if (lane == 0) {
+      int lp = 0;
+      for (int isv = 0; isv < 2; ++isv)
+        for (int pc = c_lo; pc < c_hi; ++pc) {
+          const int pns = nsub_of(pc);
+          for (int st = 0; st < pns; ++st, ++lp) {
+            const int slot = lp % RING;
+            if (lp >= RING && !mbar_wait(&empty_bar[slot], (uint32_t)(((lp / RING) - 1) & 1), SITE_ATTN_TC | 0x90))
+              return;
+            mbar_arrive_expect_tx(&full_bar[slot], SUB);
+            tma_load_3d(smem + slot * SUB, isv ? &tmV : &tmK, 0, cache_base + pc * a.chunk + st * ATT_SUB, 0,
+                        &full_bar[slot]);
+          }
+        }
+    }
+    return;
+  }
+
+  int L = 0;
+  auto consume_wait = [&]() {
+    (void)mbar_wait(&full_bar[L % RING], (uint32_t)((L / RING) & 1), SITE_ATTN_TC | 0x100);
+  };
+  auto release = [&]() {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[L % RING]);
+    ++L;
+  };
+  auto cbar = []() { asm volatile("bar.sync 1, %0;" ::"n"(ATT_THREADS) : "memory"); };
+
+  // q tile (bf16, 128-byte swizzle per half; rows past the group are zero) and the q^T fragments
+  for (int idx = tid; idx < NP * 16; idx += ATT_THREADS) {
+    const int row = idx >> 4, ch = idx & 15;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (row < npairs)
+      v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.q) + (size_t)t0 * a.Hq * 128 +
+                                          (hk * a.G + row) * 128 + ch * 8);
+    const int half = ch >> 3, cc = ch & 7;
+    *reinterpret_cast<uint4*>(qt + half * (NP * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
+  }
+  cbar();
+  const int kt = warp & 3, par = warp >> 2;  // 16-key slice of a sub-tile; sub-tile parity this warp scores
+  uint32_t qb[8][2];
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const int row = lane & 7;
+    const int half = kk >> 2, ch = 2 * (kk & 3) + ((lane >> 3) & 1);
+    ldsm_x2(qt_s + half * (NP * 128) + row * 128 + ((ch ^ (row & 7)) << 4), qb[kk][0], qb[kk][1]);
+  }
+
+  // ---- phase 1: scores of every chunk of the segment, S[pair][(c - c_lo) * 256 + key]
+  for (int c = c_lo; c < c_hi; ++c) {
+    const int nsub = nsub_of(c);
+    float* Sc = S + (c - c_lo) * 256;
+    for (int st = 0; st < nsub; ++st) {
+      consume_wait();
+      if ((st & 1) == par) {
+        const uint32_t kb = smem_u32(smem + (L % RING) * SUB);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int krow = kt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int half = kk >> 2, ch = 2 * (kk & 3) + (lane >> 4);
+          uint32_t ka[4];
+          ldsm_x4(kb + half * 8192 + krow * 128 + ((ch ^ (krow & 7)) << 4), ka[0], ka[1], ka[2], ka[3]);
+          mma_bf16_16816(acc, ka, qb[kk][0], qb[kk][1]);
+        }
+        const int pr = 2 * t4;
+        const int j = st * ATT_SUB + kt * 16 + g8;
+        Sc[pr * ATD_SST + j] = acc[0] * a.scale;
+        Sc[(pr + 1) * ATD_SST + j] = acc[1] * a.scale;
+        Sc[pr * ATD_SST + j + 8] = acc[2] * a.scale;
+        Sc[(pr + 1) * ATD_SST + j + 8] = acc[3] * a.scale;
+      }
+      release();
+    }
+  }
+  cbar();  // every score is in S
+
+  // ---- phase 2: per chunk, softmax then P.V (the V stream)
+  const int lim0 = pmax;
+  for (int c = c_lo; c < c_hi; ++c) {
+    const int key0 = c * a.chunk;
+    const int nvalid = min(a.chunk, pmax - key0 + 1);
+    const int nsub = (nvalid + ATT_SUB - 1) / ATT_SUB;
+    const float* Sc = S + (c - c_lo) * 256;
+    for (int pl = warp; pl < npairs; pl += ATT_THREADS / 32) {
+      const int lim = lim0 - key0;  // keys j <= lim are visible to the query
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < ATT_CHUNK / 32; ++k) {
+        const int j = lane + 32 * k;
+        if (j <= lim && j < nvalid) mx = fmaxf(mx, Sc[pl * ATD_SST + j]);
+      }
+      mx = warp_max(mx);
+      float sum = 0.f;
+#pragma unroll
+      for (int k = 0; k < ATT_CHUNK / 32; ++k) {
+        const int j = lane + 32 * k;
+        float pj = 0.f;
+        if (j <= lim && j < nvalid) pj = expf(Sc[pl * ATD_SST + j] - mx);
+        sum += pj;
+        const uint16_t p0 = f32_to_bf16_bits(pj);
+        const float r0 = pj - bf16_bits_to_f32(p0);
+        const uint16_t p1 = f32_to_bf16_bits(r0);
+        const uint16_t p2 = f32_to_bf16_bits(r0 - bf16_bits_to_f32(p1));
+        const uint32_t off = atc_poff(pl, j);
+        *reinterpret_cast<uint16_t*>(Pp + 0 * (NP * 512) + off) = p0;
+        *reinterpret_cast<uint16_t*>(Pp + 1 * (NP * 512) + off) = p1;
+        *reinterpret_cast<uint16_t*>(Pp + 2 * (NP * 512) + off) = p2;
+      }
+      sum = warp_sum_fixed(sum);
+      if (lane == 0) {
+        m_s[pl] = mx;
+        l_s[pl] = sum;
+        live_s[pl] = lim >= 0;
+      }
+    }
+    cbar();
+
+    // P.V: warp w owns head elements 16w..16w+15 (one m16 tile of V^T)
+    float pacc[3][4];
+#pragma unroll
+    for (int q = 0; q < 3; ++q) pacc[q][0] = pacc[q][1] = pacc[q][2] = pacc[q][3] = 0.f;
+    for (int st = 0; st < nsub; ++st) {
+      consume_wait();
+      uint8_t* vbuf = smem + (L % RING) * SUB;
+      const int vrows = nvalid - st * ATT_SUB;
+      if (vrows < ATT_SUB) {  // zero the rows past the last valid key
+        for (int idx = tid; idx < (ATT_SUB - vrows) * 16; idx += ATT_THREADS) {
+          const int r = vrows + (idx >> 4), ch = idx & 15;
+          *reinterpret_cast<uint4*>(vbuf + (ch >> 3) * 8192 + r * 128 + ((ch & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        cbar();
+      }
+      const uint32_t vb = smem_u32(vbuf);
+      const int nk16 = min(4, (vrows + 15) / 16);
+      for (int kk = 0; kk < nk16; ++kk) {
+        uint32_t va[4];
+        {
+          const int krow = kk * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+          const int e0 = warp * 16 + ((lane >> 3) & 1) * 8;
+          const int half = e0 >> 6, ch = (e0 & 63) >> 3;
+          ldsm_x4_trans(vb + half * 8192 + krow * 128 + ((ch ^ (krow & 7)) << 4), va[0], va[1], va[2], va[3]);
+        }
+        const int j0 = st * ATT_SUB + kk * 16;
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
+          uint32_t pb0, pb1;
+          const int row = lane & 7;
+          ldsm_x2(pp_s + q * (NP * 512) + atc_poff(row, j0 + ((lane >> 3) & 1) * 8), pb0, pb1);
+          mma_bf16_16816(pacc[q], va, pb0, pb1);
+        }
+      }
+      release();
+    }
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int pl = 2 * t4 + cc;
+      if (pl >= npairs || !live_s[pl]) continue;
+      const int hq = hk * a.G + pl;
+      float* rec = a.part + (((size_t)(t0 - a.t_base) * a.Hq + hq) * a.max_chunks + c) * (128 + 4);
+      const int e = warp * 16 + g8;
+      rec[e] = (pacc[0][cc] + pacc[1][cc]) + pacc[2][cc];
+      rec[e + 8] = (pacc[0][2 + cc] + pacc[1][2 + cc]) + pacc[2][2 + cc];
+      if (warp == 0 && g8 == 0) {
+        rec[128] = m_s[pl];
+        rec[129] = l_s[pl];
+      }
+    }
+    cbar();  // the next chunk overwrites the probability parts and the statistics
+  }
+  if (a.merge_in_cta) {
+    for (int p = warp; p < npairs; p += ATT_THREADS / 32) {
+      const int hq = hk * a.G + p;
+      const int nc = min(pmax / a.chunk + 1, c_hi);
+      merge_pair(a.part + ((size_t)(t0 - a.t_base) * a.Hq + hq) * a.max_chunks * (128 + 4), nc, 128, lane, a.out,
+                 (size_t)t0 * a.Hq * 128 + hq * 128, 0);
+    }
+  }
+}
+
 // One warp per (token, q head): fixed ascending merge of the chunk partials.
 __global__ void attn_merge_kernel(const float* __restrict__ part, const int32_t* __restrict__ pos, void* __restrict__ out,
                                   int t_base, int T, int Hq, int d, int chunk, int max_chunks, int f32) {

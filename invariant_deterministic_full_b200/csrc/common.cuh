@@ -151,6 +151,11 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
 }
+// Bring [p, p + bytes) into L2 without waiting (bytes a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -204,6 +209,16 @@ __device__ __forceinline__ float load_act(const void* base, size_t idx, bool f32
 }
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+
+// Rotate-half RoPE of the pair (a, b) = (x[i], x[i + d/2]) by (c, s):
+// a' = a c - b s, b' = b c + a s, with the rounding spelled out (the second
+// product rounded, the first fused) so that every kernel that rotates -- the
+// two GEMM epilogues and the standalone kernel -- gives the same bits; left to
+// the compiler, a*c - b*s may be contracted differently in each.
+__device__ __forceinline__ void rope_rotate(float a, float b, float c, float s, float& ra, float& rb) {
+  ra = __fmaf_rn(a, c, -__fmul_rn(b, s));
+  rb = __fmaf_rn(b, c, __fmul_rn(a, s));
+}
 
 // Fixed butterfly sum over the 32 lanes: every lane ends with the same value
 // (each level adds the same two operands, only their order differs, and fp

@@ -467,8 +467,7 @@ __global__ void __launch_bounds__(TC_THREADS, CPS)
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float2 cs = __ldg(tb + i);
-              ra[i] = v[i] * cs.x - v[16 + i] * cs.y;
-              rb[i] = v[16 + i] * cs.x + v[i] * cs.y;
+              rope_rotate(v[i], v[16 + i], cs.x, cs.y, ra[i], rb[i]);
             }
             size_t base;
             void* dst;

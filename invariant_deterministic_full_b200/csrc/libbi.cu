@@ -114,12 +114,12 @@ static int attn_set_smem_attrs() {
                                      (int)att_smem_bytes(16, 128, 1)));
   BI_CHECK_CUDA(cudaFuncSetAttribute(attn_partial_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)att_smem_bytes(32, 128, 1)));
-  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<1, 5>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)atc_smem_bytes(1, 5)));
   BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)atc_smem_bytes(2, 4)));
   BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)atc_smem_bytes(4, 2)));
+  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_dec_kernel<ATD_RING>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)atd_smem_bytes(ATD_RING)));
   done = true;
   return BI_OK;
 }
@@ -138,17 +138,20 @@ static int attn_launch(int np, const CUtensorMap& tk, const CUtensorMap& tv, con
                        cudaStream_t st, bool* merged) {
   *merged = false;
   if (!a.f32 && a.d == 128) {
+    const bool single = np <= 16;  // decode blocks: one token, G pairs
+    const bool dec = single && a.G <= 8;  // the decode schedule: one 8-pair tile, at most ATD_SEG chunks per CTA
     const int units = plan.n * a.Hkv;
     const int target = 2 * num_sms();
     int n_seg = units >= target / 2 ? 1 : std::min(a.max_chunks, (target + units - 1) / units);
     a.seg_len = (a.max_chunks + n_seg - 1) / n_seg;
+    if (dec) a.seg_len = std::min(a.seg_len, ATD_SEG);
     n_seg = (a.max_chunks + a.seg_len - 1) / a.seg_len;
     a.merge_in_cta = n_seg == 1;
     *merged = a.merge_in_cta != 0;
     const dim3 grid(plan.n, n_seg, a.Hkv);
-    const bool single = np <= 16;  // decode blocks: one token, G pairs
-    if (single && a.G <= 8)
-      BI_TRY(launch(attn_tc_kernel<1, 5>, grid, dim3(ATC_THREADS), atc_smem_bytes(1, 5), st, tk, tv, plan, a));
+    if (dec)
+      BI_TRY(launch(attn_dec_kernel<ATD_RING>, grid, dim3(ATC_THREADS), atd_smem_bytes(ATD_RING), st, tk, tv, plan,
+                    a));
     else if (single && a.G <= 16)
       BI_TRY(launch(attn_tc_kernel<2, 4>, grid, dim3(ATC_THREADS), atc_smem_bytes(2, 4), st, tk, tv, plan, a));
     else

@@ -142,8 +142,8 @@ __global__ void rope_append_kernel(const float* __restrict__ qkv, const float* _
     const float c = cs[2 * i], sn = cs[2 * i + 1];
     const int ia = paired ? paired_row(i, d) : i, ib = paired ? paired_row(i + half, d) : i + half;
     const float a = row[h * d + ia], b = row[h * d + ib];
-    const float ra = a * c - b * sn;
-    const float rb = b * c + a * sn;
+    float ra, rb;
+    rope_rotate(a, b, c, sn, ra, rb);
     if (h < Hq) {
       store_act(q_out, (size_t)t * QD + h * d + i, ra, f32);
       store_act(q_out, (size_t)t * QD + h * d + i + half, rb, f32);

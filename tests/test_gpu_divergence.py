@@ -43,10 +43,13 @@ def _oracle_greedy(cfg, w, prompt, n_steps, mode):
 
 
 def test_divergence_index_matches_the_oracles_greedy_runs():
-    """The study's bf16-vs-LayerCast divergence index on the tiny config is the oracle's own: its greedy runs in
-    bf16-storage emulation and in exact fp64 give the same first differing position, wherever the oracle's top-2
-    margin is clear (> 0.05) at every choice up to it (else either token is a correct greedy choice)."""
-    import numpy as np
+    """The study's bf16-vs-LayerCast divergence on the tiny config against the oracle's own greedy runs in
+    bf16-storage emulation and in exact fp64.  A greedy choice is decided where the oracle's top-2 margin is clear
+    of the path's logit error: > 0.05 for bf16 (the parity bound), > 1e-3 for LayerCast (1e-5 relative).  On each
+    prompt's decided stretch the GPU's bf16 tokens are the oracle's bf16 tokens and its LayerCast tokens the exact
+    oracle's; a bf16/exact divergence sits at a near-tie by nature, so the GPU's divergence index is never before
+    the end of the stretch, and prompts whose whole run is decided and agrees give no divergence on the GPU either.
+    The LM head is drawn with std 0.25 so that most margins are clear."""
     import torch
     import synth
     from invariant_deterministic_full_b200 import divergence as dv, model as mdl, ops
@@ -54,8 +57,10 @@ def test_divergence_index_matches_the_oracles_greedy_runs():
     import oracle
     assert torch.cuda.is_available()
     cfg = configs.TINY
+    V, H = cfg["vocab"], cfg["hidden"]
     w = synth.model_weights(cfg)
-    prompts = [synth.prompt_tokens(2000 + r, 16, cfg["vocab"]) for r in range(6)]
+    w["lm_head"] = synth.normal_bf16(synth.key(synth.WEIGHT_SEED, synth.S_LMHEAD), V * H, 0.25).reshape(V, H)
+    prompts = [synth.prompt_tokens(2000 + r, 16, V) for r in range(24)]
     n_steps = 24
 
     def gpu_run(mode):
@@ -65,16 +70,19 @@ def test_divergence_index_matches_the_oracles_greedy_runs():
         return [s[16:] for s in seqs]
 
     g_bf, g_lc = gpu_run(MODE_BF16), gpu_run(MODE_LAYERCAST)
-    checked = 0
+    decided, whole = 0, 0
     for p, gb, gl in zip(prompts, g_bf, g_lc):
         ob, mb = _oracle_greedy(cfg, w, p, n_steps, oracle.OR_BF16)
         oe, me = _oracle_greedy(cfg, w, p, n_steps, oracle.OR_EXACT)
-        i_or = dv.divergence_index(ob, oe)
-        last = len(ob) - 1 if i_or is None else i_or
-        if min(mb[: last + 1]) <= 0.05 or min(me[: last + 1]) <= 0.05:
-            continue  # a near-tie before the divergence: either greedy token is correct
-        assert gb[: last + 1] == ob[: last + 1] and gl[: last + 1] == oe[: last + 1]
-        assert dv.divergence_index(gb, gl) == i_or
-        checked += 1
-    assert checked >= 3, f"only {checked} prompts had clear margins"
+        nb = next((i for i, m in enumerate(mb) if m <= 0.05), len(mb))  # bf16 choices decided before nb
+        ne = next((i for i, m in enumerate(me) if m <= 1e-3), len(me))  # exact choices decided before ne
+        assert gb[:nb] == ob[:nb] and gl[:ne] == oe[:ne]
+        n = min(nb, ne)
+        i_or, i_gpu = dv.divergence_index(ob, oe), dv.divergence_index(gb, gl)
+        assert (i_or is None or i_or >= n) and (i_gpu is None or i_gpu >= n)
+        if n == len(ob) and i_or is None:
+            assert i_gpu is None
+            whole += 1
+        decided += n
+    assert decided >= 150 and whole >= 3, (decided, whole)
     assert ops.device_error() == 0

@@ -239,12 +239,23 @@ def test_gemm_rope_kv_epilogue_vs_oracle(bi, d, Hq, Hkv):
     written = np.zeros((3, L, cap), dtype=bool)
     written[slot, 1, pos] = True
     assert not np.any(kc.transpose(0, 1, 3, 2, 4)[~written]) and not np.any(vc.transpose(0, 1, 3, 2, 4)[~written])
-    # the unfused route (f32 projection, then the RoPE/append kernel) stores the same v bits
+    # the unfused route (f32 projection, then the RoPE/append kernel) rotates with the same rounding: same bits
     qkv32 = bi.gemm(_bf16_dev(x), wd, out_dtype=torch.float32)
     kv2 = KVCache(3, L, Hkv, cap, d)
-    bi.rope_kv_append(qkv32, table, cap, kv2, 1, sd, pd, Hq, qk_paired=True)
+    q2 = bi.rope_kv_append(qkv32, table, cap, kv2, 1, sd, pd, Hq, qk_paired=True)
     torch.cuda.synchronize()
-    assert torch.equal(kv2.v, kv.v)
+    assert torch.equal(kv2.v, kv.v) and torch.equal(kv2.k, kv.k) and torch.equal(q2, q)
+    # the same rows inside a launch of more than 32 rows (the tcgen05 kernel) give the same bits
+    reps = 9  # 45 rows: the five tokens repeated, each copy at its own slot and position
+    slot_r = np.concatenate([slot + 0 * i for i in range(reps)]).astype(np.int32)
+    pos_r = np.concatenate([pos + 0 * i for i in range(reps)]).astype(np.int32)
+    kv3 = KVCache(3, L, Hkv, cap, d)
+    xr = np.concatenate([x] * reps)
+    q3 = bi.gemm_rope_kv(_bf16_dev(xr), wd, table, cap, kv3, 1, torch.from_numpy(slot_r).cuda(),
+                         torch.from_numpy(pos_r).cuda(), Hq)
+    torch.cuda.synchronize()
+    assert torch.equal(q3[:M], q) and torch.equal(q3[-M:], q)
+    assert torch.equal(kv3.k, kv.k) and torch.equal(kv3.v, kv.v)
     _after(bi)
 
 
