@@ -374,7 +374,8 @@ def time_lmhead(m, batches=(1, 4, 32, 256), reps=20):
 
 def time_gemms(m, B, reps=3):
     """Average duration of the weight-streaming GEMM launches of one decode step, timed alone with CUDA events
-    on the launching stream (all layers' four projections + the LM-head GEMM, B token rows)."""
+    on the launching stream (all layers' four projections + the LM-head GEMM, B token rows).  The launches are
+    captured once in a CUDA graph and replayed, so the host never paces the GPU between them."""
     import torch
     from invariant_deterministic_full_b200 import ops
     cfg, w, dev = m.cfg, m.w, m.device
@@ -394,14 +395,23 @@ def time_gemms(m, B, reps=3):
             ops.gemm(x_f, w["w_down"][l], out=o_h)
         ops.gemm(x_h, w["lm_head"], out=o_lm)
 
-    once()
+    once()  # one-time library set-up outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=st):
+        once()
+    torch.cuda.current_stream().wait_stream(st)
+    g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(reps):
-        once()
+        g.replay()
     e1.record()
     e1.synchronize()
+    del g
     return e0.elapsed_time(e1) / reps
 
 

@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(160, CPS)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                      void* __restrict__ y, int ldy, int y_f32, int M, int N, int K, int m_tiles, int n_groups,
                      int splits, float* __restrict__ partial, const int* __restrict__ mcount, int mmult,
-                     const RopeEpi re, const uint8_t* __restrict__ wl2) {
+                     const RopeEpi re) {
   using C = GemmCfg<BN, MT, CPS>;
   static_assert(MT == 1 || C::KS == 1, "M-blocking needs one k-phase per warp");
   extern __shared__ uint8_t smem_raw[];
@@ -138,16 +138,6 @@ __global__ void __launch_bounds__(160, CPS)
             mbar_arrive_expect_tx(&full_bar[s], C::STAGE_BYTES);
             tma_load_3d(smem + s * C::STAGE_BYTES, &tmW, 0, g * BN, (ks0 + s) * C::KBS, &full_bar[s]);
           }
-        }
-      }
-      if (wl2 != nullptr) {
-        // A matrix that fits in L2 (wl2 set by the host): every weight row group
-        // this CTA will stream (BN contiguous rows of K) is requested into L2 now,
-        // so the whole matrix streams from HBM while the previous kernel finishes.
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-          int sp, g, mg;
-          decode_item(item, sp, g, mg);
-          if (mg == 0) prefetch_l2(wl2 + (size_t)g * BN * K * 2, (uint32_t)BN * K * 2);
         }
       }
       pdl_wait();
@@ -445,14 +435,10 @@ static int gemm_kbs(int bn, int cps = 1) {
 }
 
 
-// Weight matrices up to this size are prefetched whole into L2 at kernel start
-// (see the kernel's producer); 0 disables it.
-constexpr size_t MMA_L2_PREFETCH_MAX = size_t(64) << 20;
-
 template <int BN, int EPI, int MT = 1, int CPS = 1>
 static int launch_gemm_bf16_t(const CUtensorMap& tw, const CUtensorMap& tx, void* y, int ldy, int y_f32, int M, int N,
                               int K, int splits, float* partial, const int* mcount, int mmult, const RopeEpi& re,
-                              cudaStream_t st, const void* w) {
+                              cudaStream_t st) {
   using C = GemmCfg<BN, MT, CPS>;
   static bool attr_done = false;  // per instantiation; set once per process
   if (!attr_done) {
@@ -464,10 +450,8 @@ static int launch_gemm_bf16_t(const CUtensorMap& tw, const CUtensorMap& tx, void
   const int n_groups = N / BN;
   const int items = splits * n_groups * ((m_tiles + MT - 1) / MT);
   const int grid = items < CPS * num_sms() ? items : CPS * num_sms();
-  const bool l2 = splits == 1 && (size_t)N * K * 2 <= MMA_L2_PREFETCH_MAX;
   BI_TRY(launch(gemm_bf16_kernel<BN, EPI, MT, CPS>, dim3(grid), dim3(160), C::SMEM, st, tw, tx, y, ldy, y_f32, M, N,
-                K, m_tiles, n_groups, splits, partial, mcount, mmult, re,
-                l2 ? reinterpret_cast<const uint8_t*>(w) : nullptr));
+                K, m_tiles, n_groups, splits, partial, mcount, mmult, re));
   return BI_OK;
 }
 
@@ -513,19 +497,19 @@ static int gemm_mma(const void* x, int ldx, const void* w, void* y, int ldy, int
     if (bn != 32 || splits > 1 || !rope)
       return set_error(BI_ERR_UNSUPPORTED, "fused RoPE epilogue needs the 32-row tile and no split");
     if (cps == 2)
-      BI_TRY((launch_gemm_bf16_t<32, EPI_ROPE, 1, 2>(tw, tx, y, ldy, y_f32, M, N, K, 1, nullptr, mcount, mmult, re, st, w)));
+      BI_TRY((launch_gemm_bf16_t<32, EPI_ROPE, 1, 2>(tw, tx, y, ldy, y_f32, M, N, K, 1, nullptr, mcount, mmult, re, st)));
     else
-      BI_TRY((launch_gemm_bf16_t<32, EPI_ROPE, 1, 1>(tw, tx, y, ldy, y_f32, M, N, K, 1, nullptr, mcount, mmult, re, st, w)));
+      BI_TRY((launch_gemm_bf16_t<32, EPI_ROPE, 1, 1>(tw, tx, y, ldy, y_f32, M, N, K, 1, nullptr, mcount, mmult, re, st)));
     return BI_OK;
   }
 #define BI_GEMM_CASE(BNV, MTV, CPSV)                                                                            \
   if (bn == BNV && mt == MTV && cps == CPSV) {                                                                  \
     if (epi == BI_EPI_SWIGLU)                                                                                   \
       BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_SWIGLU, MTV, CPSV>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial,   \
-                                                                mcount, mmult, re, st, w)));                       \
+                                                                mcount, mmult, re, st)));                       \
     else                                                                                                        \
       BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_NONE, MTV, CPSV>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial,     \
-                                                              mcount, mmult, re, st, w)));                         \
+                                                              mcount, mmult, re, st)));                         \
   }
   BI_GEMM_CASE(32, 1, 1)
   BI_GEMM_CASE(64, 1, 1)
