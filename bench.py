@@ -163,11 +163,11 @@ def step_bytes(cfg, B, ctx_lens, f32_kv=False):
     return w + B * H * 2 + kv
 
 
-# DRAM bytes (read + write) of the weight-streaming GEMM launches of one decode step at batch 32, from one ncu
-# capture (dram__bytes_read.sum + dram__bytes_write.sum) of the same shapes on the 2-layer 8B-width case; the
-# per-layer figures scale to 32 layers (the weights per launch do not depend on the layer count).  Valid only for
-# the GEMM kernel source that was captured, recognised by gemm_source_digest; None until a capture of this source.
-GEMM_TRAFFIC = {"gemm_source_sha256": None, "batch": 32, "per_layer_bytes": None, "lm_head_bytes": None}
+# DRAM bytes (read + write) of the four projection GEMM launches of one decoder layer at batch 32, from one ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum) of the same shapes on the 2-layer 8B-width case (the
+# weights per launch do not depend on the layer count).  Valid only for the GEMM kernel source that was captured,
+# recognised by gemm_source_digest; None until a capture of this source.
+GEMM_TRAFFIC = {"gemm_source_sha256": None, "batch": 32, "per_layer_bytes": None}
 
 CSRC = os.path.join(ROOT, "invariant_deterministic_full_b200", "csrc")
 
@@ -202,12 +202,12 @@ def gemm_traffic_per_launch(cfg, B):
     if (GEMM_TRAFFIC["gemm_source_sha256"] is None or h != GEMM_TRAFFIC["gemm_source_sha256"]
             or B != GEMM_TRAFFIC["batch"] or cfg["hidden"] != 4096):
         return None
-    L = cfg["n_layers"]
-    return (L * GEMM_TRAFFIC["per_layer_bytes"] + GEMM_TRAFFIC["lm_head_bytes"]) / (4 * L + 1)
+    return GEMM_TRAFFIC["per_layer_bytes"] / 4
 
 
 def gemm_bytes(cfg, B):
-    """Algorithmic bytes of the weight-streaming GEMM launches of one bf16 decode step (weights + inputs + outputs)."""
+    """Algorithmic bytes of the projection GEMM launches of one bf16 decode step (weights + inputs + outputs):
+    QKV, O, gate/up (SwiGLU output) and down of every layer."""
     L, H, Hq, Hkv, d, F, V = (cfg["n_layers"], cfg["hidden"], cfg["n_heads"], cfg["n_kv_heads"], cfg["head_dim"],
                               cfg["ffn"], cfg["vocab"])
     QKV = (Hq + 2 * Hkv) * d
@@ -216,8 +216,6 @@ def gemm_bytes(cfg, B):
     for N, K, ob in per_layer:
         tot += L * (N * K * 2 + B * K * 2 + B * (N // 2 if N == 2 * F else N) * ob)
         n += L
-    tot += V * H * 2 + B * H * 2 + B * V * 4
-    n += 1
     return tot, n
 
 
@@ -373,9 +371,9 @@ def time_lmhead(m, batches=(1, 4, 32, 256), reps=20):
 
 
 def time_gemms(m, B, reps=3):
-    """Average duration of the weight-streaming GEMM launches of one decode step, timed alone with CUDA events
-    on the launching stream (all layers' four projections + the LM-head GEMM, B token rows).  The launches are
-    captured once in a CUDA graph and replayed, so the host never paces the GPU between them."""
+    """Duration of the projection GEMM launches of one decode step, timed alone with CUDA events on the
+    launching stream (all layers' QKV, O, gate/up and down, B token rows).  The launches are captured once in a
+    CUDA graph and replayed, so the host never paces the GPU between them."""
     import torch
     from invariant_deterministic_full_b200 import ops
     cfg, w, dev = m.cfg, m.w, m.device
@@ -385,7 +383,6 @@ def time_gemms(m, B, reps=3):
     o_qkv = torch.empty(B, w["w_qkv"].shape[1], dtype=torch.bfloat16, device=dev)
     o_h = torch.empty(B, H, dtype=torch.bfloat16, device=dev)
     o_f = torch.empty(B, F, dtype=torch.bfloat16, device=dev)
-    o_lm = torch.empty(B, cfg["vocab"], dtype=torch.float32, device=dev)
 
     def once():
         for l in range(L):
@@ -393,7 +390,6 @@ def time_gemms(m, B, reps=3):
             ops.gemm(x_q, w["w_o"][l], out=o_h)
             ops.gemm(x_h, w["w_gu"][l], epilogue=1, out=o_f)
             ops.gemm(x_f, w["w_down"][l], out=o_h)
-        ops.gemm(x_h, w["lm_head"], out=o_lm)
 
     once()  # one-time library set-up outside the capture
     torch.cuda.synchronize()
@@ -582,7 +578,7 @@ def main_ours(args):
             "gpu_launches": int(r["launches"] * K),
             "clocks": r["clocks"],
             "gpu": torch.cuda.get_device_name(torch.cuda.current_device())}
-    # dominant kernel: the weight-streaming GEMM (all projections of one step + LM head), timed alone
+    # dominant kernel: the weight-streaming projection GEMM (all layers' projections of one step), timed alone
     if mode == 0:
         gms = time_gemms(m, B)
         gb, gl = gemm_bytes(cfg, B)
@@ -590,9 +586,10 @@ def main_ours(args):
         tr = gemm_traffic_per_launch(cfg, B)
         line["roofline"] = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
                             "frac": round(ach / hbm, 4), "traffic": round(tr) if tr else None,
-                            "traffic_note": "DRAM read+write bytes per launch (ncu, same GEMM shapes, 2-layer case "
-                                            "scaled to 32 layers)" if tr else "no capture for this GEMM source/batch",
-                            "kernel": "gemm_tc_kernel (weight-streaming tcgen05/TMEM GEMM)",
+                            "traffic_note": "DRAM read+write bytes per launch (ncu, the same four GEMM shapes on "
+                                            "the 2-layer case)" if tr else "no capture for this GEMM source/batch",
+                            "kernel": "gemm_bf16_kernel (weight-streaming mma.sync GEMM, <= 32 token rows)" if B <= 32
+                                      else "gemm_tc_kernel (weight-streaming tcgen05/TMEM GEMM)",
                             "per_launch": f"{gb / gl / 1e6:.1f} MB algorithmic over {gl} launches, "
                                           f"{gms / gl * 1e3:.1f} us average",
                             "peak_source": f"{src} hbm_gbs (copy), kernel timed alone"}

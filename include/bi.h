@@ -231,7 +231,10 @@ int bi_attention(const void* q, const bi_kv_layout* kv, int layer, const int32_t
  * For each row b of h (f32 [B][H], device):
  *   z = h . W^T (W bf16 [V][H]).  BI_MODE_BF16: h is rounded to bf16 and
  *   z is a bf16 x bf16 tensor-core product with fp32 accumulation.
- *   BI_MODE_LAYERCAST: z = fp32 FMA of h with W upcast to fp32.
+ *   BI_MODE_LAYERCAST: z = h . W^T with exact fp32 products: h split into
+ *   three bf16 parts h = p0 + p1 + p2, each part's products accumulated in
+ *   fp32 on the tensor cores, z = (z0 + z1) + z2.  BI_MODE_FP32: W is f32
+ *   and z is an fp32 FMA chain.
  *   lse = M + ln S over the vocabulary, reduced in BI_VOCAB_CHUNK chunks
  *   (per chunk: max, sum exp(z - max), top-1 and top-2) merged in ascending
  *   chunk order; logprob = z[target] - lse (target NULL or < 0: the argmax);

@@ -10,15 +10,15 @@
 // chosen here from M and N for speed; it is work assignment only.
 //
 // LayerCast ("Give Me FP32 or Give Me Death?", LayerCast section: bf16-stored
-// weights, fp32 arithmetic) has two routes.  Projections (gemm_layercast, at
-// the end of this file) split each f32 activation exactly into three bf16
-// parts and run them through the tcgen05 GEMM.  The LM head
-// (gemm_f32_kernel) upcasts the weight from bf16 to fp32 in registers and
-// takes every product and sum as an fp32 FMA.  Element order there: lane l of
-// a warp owns the k-slices [256 i + 8 l, 256 i + 8 l + 8) for i = 0, 1, ...;
-// it accumulates them with sequential FMAs in ascending k, and the 32 lane
-// partials are then combined by a fixed xor-butterfly.  This is the same for
-// every M and every row/token tiling.
+// weights, fp32 arithmetic): every projection and the LM head
+// (gemm_layercast, at the end of this file) split each f32 activation exactly
+// into three bf16 parts and run them through the invariant tensor-core GEMM.
+// The FP32-storage mode (f32 weights) takes every product and sum as an fp32
+// FMA (gemm_f32_kernel).  Element order there: lane l of a warp owns the
+// k-slices [256 i + 8 l, 256 i + 8 l + 8) for i = 0, 1, ...; it accumulates
+// them with sequential FMAs in ascending k, and the 32 lane partials are then
+// combined by a fixed xor-butterfly.  This is the same for every M and every
+// row/token tiling.
 #pragma once
 #include <algorithm>
 
@@ -197,9 +197,12 @@ constexpr int MMA_MAX_ROWS = 32;
 
 // LayerCast on tensor cores: rows of x per pass (bounds the workspace)
 constexpr int LC_ROWS = 256;
-static size_t lc_ws_bytes(int M, int N, int K) {
+// col_block > 0: the output columns are computed col_block at a time (a
+// multiple of 256), so the workspace holds one block's three partial products.
+static size_t lc_ws_bytes(int M, int N, int K, int col_block = 0) {
   const size_t mb = (size_t)std::min(M, LC_ROWS);
-  return 3 * mb * K * 2 + 3 * mb * N * 4 + 512;
+  const size_t nb = (size_t)(col_block > 0 ? std::min(N, col_block) : N);
+  return 3 * mb * K * 2 + 3 * mb * nb * 4 + 512;
 }
 
 size_t gemm_ws_bytes(int M, int N, int K, int mode, int variant) {
@@ -406,25 +409,36 @@ __global__ void lc_combine_kernel(const float* __restrict__ yt, int mb, int N, v
   }
 }
 
+// col_block > 0 (no SwiGLU epilogue): the columns in blocks of col_block
+// rows of w, each block's accumulation structure fixed by the whole matrix's
+// row count (n_full, else N) -- the same bits as one unblocked call.
 int gemm_layercast(const float* x, int ldx, const void* w, void* y, int ldy, int y_f32, int M, int N, int K, int epi,
-                   void* ws, size_t ws_bytes, cudaStream_t st, int n_full = 0) {
-  const size_t need = lc_ws_bytes(M, N, K);
+                   void* ws, size_t ws_bytes, cudaStream_t st, int n_full = 0, int col_block = 0) {
+  const size_t need = lc_ws_bytes(M, N, K, col_block);
   BI_REQUIRE(ws && ws_bytes >= need, BI_ERR_WORKSPACE, "bi_gemm LayerCast: workspace %zu < %zu", ws_bytes, need);
+  BI_REQUIRE(col_block == 0 || (col_block % 256 == 0 && epi != BI_EPI_SWIGLU), BI_ERR_INVALID_ARG,
+             "LayerCast column blocks: %d", col_block);
   const int MB = std::min(M, LC_ROWS);
+  const int NB = col_block > 0 ? std::min(N, col_block) : N;
+  const int nf = n_full > 0 ? n_full : N;
   uint16_t* xs = reinterpret_cast<uint16_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
   float* yt = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(xs + (size_t)3 * MB * K) + 255) & ~uintptr_t(255));
-  const int n_out = epi == BI_EPI_SWIGLU ? N / 2 : N;
+  const size_t esz = y_f32 ? 4 : 2;
   for (int m0 = 0; m0 < M; m0 += MB) {
     const int mb = std::min(MB, M - m0);
     const size_t n = (size_t)mb * K;
     BI_TRY(launch(lc_split_kernel, dim3((int)std::min<size_t>((n + 255) / 256, 8 * (size_t)num_sms())), dim3(256), 0,
                   st, x + (size_t)m0 * ldx, ldx, mb, K, xs));
-    BI_TRY(gemm_bf16(xs, K, w, yt, N, 1, 3 * mb, N, K, BI_EPI_NONE, BI_VARIANT_INVARIANT, nullptr, 0, st, nullptr, 1,
-                     nullptr, n_full));
-    const size_t tot = (size_t)mb * n_out;
-    void* yb = reinterpret_cast<uint8_t*>(y) + (size_t)m0 * ldy * (y_f32 ? 4 : 2);
-    BI_TRY(launch(lc_combine_kernel, dim3((int)std::min<size_t>((tot + 255) / 256, 8 * (size_t)num_sms())), dim3(256),
-                  0, st, yt, mb, N, yb, ldy, y_f32, epi == BI_EPI_SWIGLU ? 1 : 0));
+    for (int n0 = 0; n0 < N; n0 += NB) {
+      const int nb = std::min(NB, N - n0);
+      const int n_out = epi == BI_EPI_SWIGLU ? nb / 2 : nb;
+      BI_TRY(gemm_bf16(xs, K, reinterpret_cast<const uint16_t*>(w) + (size_t)n0 * K, yt, nb, 1, 3 * mb, nb, K,
+                       BI_EPI_NONE, BI_VARIANT_INVARIANT, nullptr, 0, st, nullptr, 1, nullptr, nf));
+      const size_t tot = (size_t)mb * n_out;
+      void* yb = reinterpret_cast<uint8_t*>(y) + ((size_t)m0 * ldy + n0) * esz;
+      BI_TRY(launch(lc_combine_kernel, dim3((int)std::min<size_t>((tot + 255) / 256, 8 * (size_t)num_sms())),
+                    dim3(256), 0, st, yt, mb, nb, yb, ldy, y_f32, epi == BI_EPI_SWIGLU ? 1 : 0));
+    }
   }
   return BI_OK;
 }

@@ -289,7 +289,11 @@ struct LmWs {
   int* count;
   uint16_t* hc2;    // two-pass: [2B][H] residual parts p1, p2 of the flagged rows
   float* logits_c;  // two-pass: [2B][V] their logits
+  void* lc;         // LayerCast: the tensor-core GEMM's split rows and partial products
+  size_t lc_bytes;
 };
+// LayerCast LM head: vocabulary columns per tensor-core pass (bounds its workspace)
+constexpr int LM_LC_COLS = 16384;
 // parts: 3 in bf16 mode with the recompute enabled, else 1
 static LmWs lm_carve(Carver& cv, int B, int H, int V, int mode, bool own_logits, int parts) {
   const int nch = (V + LM_CHUNK - 1) / LM_CHUNK;
@@ -305,6 +309,10 @@ static LmWs lm_carve(Carver& cv, int B, int H, int V, int mode, bool own_logits,
   if (bf && parts == 3 && B > LM_ONE_PASS_ROWS) {
     w.hc2 = cv.take<uint16_t>((size_t)2 * B * H);
     w.logits_c = cv.take<float>((size_t)2 * B * V);
+  }
+  if (mode == BI_MODE_LAYERCAST) {
+    w.lc_bytes = lc_ws_bytes(B, V, H, LM_LC_COLS);
+    w.lc = cv.take<uint8_t>(w.lc_bytes);
   }
   return w;
 }
@@ -342,9 +350,14 @@ static int lmhead_run(const float* h, const void* W, const int32_t* target, int 
     BI_TRY(gemm_bf16(w.hs, H, W, z, V, 1, sp * B, V, H, BI_EPI_NONE, BI_VARIANT_INVARIANT, nullptr, 0, st));
     if (logits)
       BI_CHECK_CUDA(cudaMemcpyAsync(logits, z, (size_t)B * V * sizeof(float), cudaMemcpyDeviceToDevice, st));
+  } else if (mode == BI_MODE_LAYERCAST) {
+    // exact products of fp32 h with the bf16 W on the tensor cores (three bf16
+    // parts of h, fp32 accumulation), as the LayerCast projections
+    z = logits ? logits : w.logits;
+    BI_TRY(gemm_layercast(h, H, W, z, V, 1, B, V, H, BI_EPI_NONE, w.lc, w.lc_bytes, st, V, LM_LC_COLS));
   } else {
     z = logits ? logits : w.logits;
-    BI_TRY(gemm_f32(h, H, W, z, V, 1, B, V, H, BI_EPI_NONE, nullptr, st, mode == BI_MODE_FP32));
+    BI_TRY(gemm_f32(h, H, W, z, V, 1, B, V, H, BI_EPI_NONE, nullptr, st, true));
   }
   BI_TRY(launch(lm_partial_kernel, dim3(dim3((nch + LM_CPB - 1) / LM_CPB, B)), dim3(32 * LM_CPB), 0, st, z, V, V, target, nullptr, nullptr, w.part, nch,
                 1, 0, nullptr));

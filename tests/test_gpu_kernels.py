@@ -459,6 +459,38 @@ def test_lmhead_recompute_enabled_but_no_row_flagged(bi, B):
     _after(bi)
 
 
+def test_lmhead_layercast_full_size_tensor_core_blocks(bi):
+    """LayerCast LM head at hidden 4096, vocab 128256 on the tensor cores, in vocabulary blocks: the logits are
+    bitwise those of one unblocked LayerCast bi_gemm over the whole vocabulary, every row is bitwise equal across
+    batch 1..64, and sampled rows match the exact oracle within the fp32 summation bound."""
+    H, V = 4096, 128256
+    W = torch.empty(V, H, dtype=torch.bfloat16, device="cuda")
+    kW = synth.key(synth.WEIGHT_SEED, synth.S_LMHEAD)
+    bi.synth_fill_bf16(W, V, H, kW, 0.02)
+    h = _h_rows(64, H)
+    hd = torch.from_numpy(h).cuda()
+    ref = bi.lmhead_logprob(hd, W, None, 0.1, mode=1, want_logits=True)
+    z = bi.gemm(hd, W, mode=1, out_dtype=torch.float32)
+    assert torch.equal(ref["logits"], z)
+    assert int(ref["recomputed"].sum()) == 0
+    ref = {k: v.cpu() for k, v in ref.items()}
+    for B in (1, 3, 11, 32, 40):
+        for off in (0, 64 - B):
+            o = bi.lmhead_logprob(hd[off:off + B].contiguous(), W, None, 0.1, mode=1)
+            for k in ("logprob", "lse", "argmax", "margin"):
+                assert torch.equal(o[k].cpu(), ref[k][off:off + B]), (B, off, k)
+    Wb = synth.normal_bf16(kW, V * H).reshape(V, H)
+    rows = [0, 33, 63]
+    res, zx = oracle.lmhead(h[rows].astype(np.float64), Wb, want_logits=True)
+    Wa = np.abs(synth.bf16_to_f32(Wb)).astype(np.float64)
+    for i, r in enumerate(rows):
+        bound = (H + 2) * 2.0 ** -24 * (Wa @ np.abs(h[r]).astype(np.float64))
+        assert (np.abs(ref["logits"][r].numpy() - zx[i]) <= bound).all(), r
+        assert abs(ref["logprob"][r].item() - res[i][1]) <= 1e-5 * abs(res[i][1]) + 1e-6, r
+        assert abs(ref["lse"][r].item() - res[i][0]) <= 1e-5 * abs(res[i][0]) + 1e-6, r
+    _after(bi)
+
+
 def test_lmhead_full_size_invariance_and_samples(bi):
     """LM head alone at hidden 4096, vocab 128256: each row bitwise equal across batch 1..256."""
     H, V = 4096, 128256
