@@ -16,7 +16,9 @@
 // from the weight-row tile BN, itself chosen from N alone (gemm_ks).  The
 // interleave keeps several independent mma chains per warp so the tensor-pipe
 // latency is covered even when M is small.
-// Weight tiles (BN rows x 64 k) and token tiles (32 rows x 64 k) stream by TMA
+// Weight tiles (BN rows x 64 k) and token tiles (32 rows x 64 k; only 8 or 16
+// rows are copied when M is that small, since every copied row -- zero fill
+// past M included -- costs the SM's copy engine the same time) stream by TMA
 // (128-byte swizzle) into a multi-stage shared-memory ring filled by one
 // producer warp; four consumer warps read them with ldmatrix.  The grid is
 // persistent (one CTA per SM, or two with half the ring each when a launch
@@ -76,9 +78,13 @@ __global__ void __launch_bounds__(160, CPS)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                      void* __restrict__ y, int ldy, int y_f32, int M, int N, int K, int m_tiles, int n_groups,
                      int splits, float* __restrict__ partial, const int* __restrict__ mcount, int mmult,
-                     const RopeEpi re) {
+                     const RopeEpi re, int xr) {
   using C = GemmCfg<BN, MT, CPS>;
   static_assert(MT == 1 || C::KS == 1, "M-blocking needs one k-phase per warp");
+  // Token rows per k-block slab of a stage: xr = 8 or 16 when M fits (MT = 1),
+  // else 32.  Rows of the slab past M are zero-filled by the copy and never
+  // read: the consumers stop at the last n8 tile holding live rows.
+  const uint32_t stage_tx = C::W_BYTES + C::KBS * xr * MT * 128;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::STAGES];
   __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
@@ -135,7 +141,7 @@ __global__ void __launch_bounds__(160, CPS)
           const int ks1 = min(kstages_total, ks0 + ks_per_split);
           pre = max(0, min(C::STAGES, ks1 - ks0));
           for (int s = 0; s < pre; ++s) {
-            mbar_arrive_expect_tx(&full_bar[s], C::STAGE_BYTES);
+            mbar_arrive_expect_tx(&full_bar[s], stage_tx);
             tma_load_3d(smem + s * C::STAGE_BYTES, &tmW, 0, g * BN, (ks0 + s) * C::KBS, &full_bar[s]);
           }
         }
@@ -174,7 +180,7 @@ __global__ void __launch_bounds__(160, CPS)
               timed_out = true;
               break;
             }
-            mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+            mbar_arrive_expect_tx(&full_bar[stage], stage_tx);
             tma_load_3d(sb, &tmW, 0, g * BN, ks * C::KBS, &full_bar[stage]);
             ++issued;
           }
@@ -236,7 +242,7 @@ __global__ void __launch_bounds__(160, CPS)
 #pragma unroll
       for (int kb = 0; kb < C::KBS && !dead; ++kb) {
         const uint32_t wb = sbase + kb * (BN * 128);
-        const uint32_t xb = sbase + C::W_BYTES + kb * (GEMM_BM * MT * 128);
+        const uint32_t xb = sbase + C::W_BYTES + kb * (xr * MT * 128);
 #pragma unroll
         for (int j = 0; j < 4 / C::KS; ++j) {
           const int kk = kp + j * C::KS;
@@ -438,7 +444,7 @@ static int gemm_kbs(int bn, int cps = 1) {
 template <int BN, int EPI, int MT = 1, int CPS = 1>
 static int launch_gemm_bf16_t(const CUtensorMap& tw, const CUtensorMap& tx, void* y, int ldy, int y_f32, int M, int N,
                               int K, int splits, float* partial, const int* mcount, int mmult, const RopeEpi& re,
-                              cudaStream_t st) {
+                              int xr, cudaStream_t st) {
   using C = GemmCfg<BN, MT, CPS>;
   static bool attr_done = false;  // per instantiation; set once per process
   if (!attr_done) {
@@ -451,7 +457,7 @@ static int launch_gemm_bf16_t(const CUtensorMap& tw, const CUtensorMap& tx, void
   const int items = splits * n_groups * ((m_tiles + MT - 1) / MT);
   const int grid = items < CPS * num_sms() ? items : CPS * num_sms();
   BI_TRY(launch(gemm_bf16_kernel<BN, EPI, MT, CPS>, dim3(grid), dim3(160), C::SMEM, st, tw, tx, y, ldy, y_f32, M, N,
-                K, m_tiles, n_groups, splits, partial, mcount, mmult, re));
+                K, m_tiles, n_groups, splits, partial, mcount, mmult, re, xr));
   return BI_OK;
 }
 
@@ -476,6 +482,8 @@ static int gemm_mma(const void* x, int ldx, const void* w, void* y, int ldy, int
   const int mt = gemm_pick_mt(bn, M);
   const int cps = gemm_pick_cps(bn, M, N, mt, splits);
   const int kbs = gemm_kbs(bn, cps);
+  // token rows per copied slab: the fewest multiple of 8 (8, 16 or 32) that holds M
+  const int xr = mt == 1 ? (M <= 8 ? 8 : (M <= 16 ? 16 : GEMM_BM)) : GEMM_BM;
   // 3-D views {64 k, rows, k-block}: the k-block dimension (stride 128 B) is the
   // outermost of the box, so a box lands as kbs swizzled [rows][128 B] slabs.
   CUtensorMap tw, tx;
@@ -485,7 +493,7 @@ static int gemm_mma(const void* x, int ldx, const void* w, void* y, int ldy, int
   BI_TRY(encode_tmap_3d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, dw, sw, bw, CU_TENSOR_MAP_SWIZZLE_128B));
   const uint64_t dx[3] = {(uint64_t)GEMM_BK, (uint64_t)M, (uint64_t)(K / GEMM_BK)};
   const uint64_t sx[2] = {(uint64_t)ldx * 2, (uint64_t)GEMM_BK * 2};
-  const uint32_t bx[3] = {(uint32_t)GEMM_BK, (uint32_t)(GEMM_BM * mt), (uint32_t)kbs};
+  const uint32_t bx[3] = {(uint32_t)GEMM_BK, (uint32_t)(xr * mt), (uint32_t)kbs};
   BI_TRY(encode_tmap_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, dx, sx, bx, CU_TENSOR_MAP_SWIZZLE_128B));
   float* partial = nullptr;
   if (splits > 1) {
@@ -497,19 +505,21 @@ static int gemm_mma(const void* x, int ldx, const void* w, void* y, int ldy, int
     if (bn != 32 || splits > 1 || !rope)
       return set_error(BI_ERR_UNSUPPORTED, "fused RoPE epilogue needs the 32-row tile and no split");
     if (cps == 2)
-      BI_TRY((launch_gemm_bf16_t<32, EPI_ROPE, 1, 2>(tw, tx, y, ldy, y_f32, M, N, K, 1, nullptr, mcount, mmult, re, st)));
+      BI_TRY((launch_gemm_bf16_t<32, EPI_ROPE, 1, 2>(tw, tx, y, ldy, y_f32, M, N, K, 1, nullptr, mcount, mmult, re, xr,
+                                                    st)));
     else
-      BI_TRY((launch_gemm_bf16_t<32, EPI_ROPE, 1, 1>(tw, tx, y, ldy, y_f32, M, N, K, 1, nullptr, mcount, mmult, re, st)));
+      BI_TRY((launch_gemm_bf16_t<32, EPI_ROPE, 1, 1>(tw, tx, y, ldy, y_f32, M, N, K, 1, nullptr, mcount, mmult, re, xr,
+                                                    st)));
     return BI_OK;
   }
 #define BI_GEMM_CASE(BNV, MTV, CPSV)                                                                            \
   if (bn == BNV && mt == MTV && cps == CPSV) {                                                                  \
     if (epi == BI_EPI_SWIGLU)                                                                                   \
       BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_SWIGLU, MTV, CPSV>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial,   \
-                                                                mcount, mmult, re, st)));                       \
+                                                                mcount, mmult, re, xr, st)));                   \
     else                                                                                                        \
       BI_TRY((launch_gemm_bf16_t<BNV, BI_EPI_NONE, MTV, CPSV>(tw, tx, y, ldy, y_f32, M, N, K, splits, partial,     \
-                                                              mcount, mmult, re, st)));                         \
+                                                              mcount, mmult, re, xr, st)));                     \
   }
   BI_GEMM_CASE(32, 1, 1)
   BI_GEMM_CASE(64, 1, 1)
