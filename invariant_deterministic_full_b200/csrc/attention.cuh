@@ -694,10 +694,11 @@ __global__ void __launch_bounds__(ATC_THREADS)
 // scores -> softmax -> P.V, so at every chunk boundary the next chunk's keys
 // are only requested while P.V of the current one drains the ring.  Here a
 // CTA first streams the K rows of its whole segment (at most ATD_SEG chunks)
-// and keeps every score in shared memory, then streams the V rows, running
-// each chunk's softmax just before its P.V.  The K stream and the V stream
-// each run back to back through the ring, and all eight warps score: warps
-// 0-3 the even 64-key sub-tiles, warps 4-7 the odd ones.  Every score, every
+// and keeps every score in shared memory; then it runs the softmax of every
+// (chunk, pair) of the segment, one warp each, while the first V rows arrive,
+// keeping the probability parts of every chunk; then it streams the V rows
+// through P.V without a pause at the chunk boundaries.  All eight warps score:
+// warps 0-3 the even 64-key sub-tiles, warps 4-7 the odd ones.  Every score, every
 // softmax and every P.V chain is the instruction sequence of attn_tc_kernel
 // (each score one warp's chain of 8 ascending k16 mma over the head; the same
 // lane-strided max and denominator; the same 3-part P split and per-part
@@ -705,28 +706,29 @@ __global__ void __launch_bounds__(ATC_THREADS)
 // kernels, and prefill and decode, give the same bits.
 constexpr int ATD_SEG = 3;                   // chunks per CTA (scores of all of them are kept)
 constexpr int ATD_SST = ATD_SEG * 256 + 4;  // row stride of the score rows (floats)
-constexpr int ATD_RING = 4;                // K/V sub-tiles in flight per CTA (two CTAs fit an SM)
 
-__host__ __device__ inline size_t atd_smem_bytes(int ring) {
-  return (size_t)ring * 16384  // K/V sub-tiles: [2 halves][64 keys][128 B]
-         + 8 * 256             // q tile: [2 halves][8 pairs][128 B]
-         + 8 * ATD_SST * 4     // scores [8][ATD_SST]
-         + 3 * 8 * 512         // probability parts of one chunk [3][8][256 keys] bf16, swizzled
+// Shared memory of attn_dec_kernel<RING, NP>: NP pair rows of scores and of the
+// probability parts of every chunk of the segment (NP = 4 when a kv head has at
+// most 4 q heads, which leaves room for a deeper ring at two CTAs per SM).
+__host__ __device__ inline size_t atd_smem_bytes(int ring, int np) {
+  return (size_t)ring * 16384            // K/V sub-tiles: [2 halves][64 keys][128 B]
+         + 8 * 256                       // q tile: [2 halves][8 pairs][128 B]
+         + (size_t)np * ATD_SST * 4      // scores [NP][ATD_SST]
+         + (size_t)ATD_SEG * 3 * np * 512  // probability parts [chunk][3][NP][256 keys] bf16, swizzled
          + 1024;
 }
 
-template <int RING>
+template <int RING, int NP>
 __global__ void __launch_bounds__(ATC_THREADS)
     attn_dec_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ AttnPlan plan, const AttnArgs a) {
   pdl_wait();
   pdl_trigger();
-  constexpr int NP = 8;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[RING];
   __shared__ __align__(8) uint64_t empty_bar[RING];
-  __shared__ float m_s[NP], l_s[NP];
-  __shared__ int live_s[NP];
+  __shared__ float m_s[ATD_SEG][NP], l_s[ATD_SEG][NP];
+  __shared__ int live_s[ATD_SEG][NP];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int b = blockIdx.x, sg = blockIdx.y, hk = blockIdx.z;
   if (b >= plan.n) return;
@@ -740,14 +742,15 @@ __global__ void __launch_bounds__(ATC_THREADS)
     c_hi = a.max_chunks;
   }
   if (c_lo >= c_hi) return;
-  const int npairs = a.G;  // <= 8
+  const int npairs = a.G;  // <= NP
   const int cache_base = ((s * a.n_layers + a.layer) * a.Hkv + hk) * a.cap;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, t4 = lane & 3;
   constexpr uint32_t SUB = 16384;
-  uint8_t* qt = smem + RING * SUB;                             // [2][NP][128 B]
-  float* S = reinterpret_cast<float*>(qt + NP * 256);          // [NP][ATD_SST]
-  uint8_t* Pp = reinterpret_cast<uint8_t*>(S + NP * ATD_SST);  // [3][NP][512 B]
+  constexpr int PPART = NP * 512;  // bytes of one probability part of one chunk
+  uint8_t* qt = smem + RING * SUB;                            // [2][8][128 B]
+  float* S = reinterpret_cast<float*>(qt + 8 * 256);          // [NP][ATD_SST]
+  uint8_t* Pp = reinterpret_cast<uint8_t*>(S + NP * ATD_SST);  // [ATD_SEG][3][NP][512 B]
   const uint32_t qt_s = smem_u32(qt), pp_s = smem_u32(Pp);
   auto nsub_of = [&](int c) { return (min(a.chunk, pmax - c * a.chunk + 1) + ATT_SUB - 1) / ATT_SUB; };
 
@@ -792,14 +795,14 @@ __global__ void __launch_bounds__(ATC_THREADS)
   auto cbar = []() { asm volatile("bar.sync 1, %0;" ::"n"(ATT_THREADS) : "memory"); };
 
   // q tile (bf16, 128-byte swizzle per half; rows past the group are zero) and the q^T fragments
-  for (int idx = tid; idx < NP * 16; idx += ATT_THREADS) {
+  for (int idx = tid; idx < 8 * 16; idx += ATT_THREADS) {
     const int row = idx >> 4, ch = idx & 15;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (row < npairs)
       v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.q) + (size_t)t0 * a.Hq * 128 +
                                           (hk * a.G + row) * 128 + ch * 8);
     const int half = ch >> 3, cc = ch & 7;
-    *reinterpret_cast<uint4*>(qt + half * (NP * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
+    *reinterpret_cast<uint4*>(qt + half * (8 * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
   }
   cbar();
   const int kt = warp & 3, par = warp >> 2;  // 16-key slice of a sub-tile; sub-tile parity this warp scores
@@ -808,7 +811,7 @@ __global__ void __launch_bounds__(ATC_THREADS)
   for (int kk = 0; kk < 8; ++kk) {
     const int row = lane & 7;
     const int half = kk >> 2, ch = 2 * (kk & 3) + ((lane >> 3) & 1);
-    ldsm_x2(qt_s + half * (NP * 128) + row * 128 + ((ch ^ (row & 7)) << 4), qb[kk][0], qb[kk][1]);
+    ldsm_x2(qt_s + half * (8 * 128) + row * 128 + ((ch ^ (row & 7)) << 4), qb[kk][0], qb[kk][1]);
   }
 
   // ---- phase 1: scores of every chunk of the segment, S[pair][(c - c_lo) * 256 + key]
@@ -830,58 +833,70 @@ __global__ void __launch_bounds__(ATC_THREADS)
         }
         const int pr = 2 * t4;
         const int j = st * ATT_SUB + kt * 16 + g8;
-        Sc[pr * ATD_SST + j] = acc[0] * a.scale;
-        Sc[(pr + 1) * ATD_SST + j] = acc[1] * a.scale;
-        Sc[pr * ATD_SST + j + 8] = acc[2] * a.scale;
-        Sc[(pr + 1) * ATD_SST + j + 8] = acc[3] * a.scale;
+        if (pr < NP) {
+          Sc[pr * ATD_SST + j] = acc[0] * a.scale;
+          Sc[pr * ATD_SST + j + 8] = acc[2] * a.scale;
+        }
+        if (pr + 1 < NP) {
+          Sc[(pr + 1) * ATD_SST + j] = acc[1] * a.scale;
+          Sc[(pr + 1) * ATD_SST + j + 8] = acc[3] * a.scale;
+        }
       }
       release();
     }
   }
   cbar();  // every score is in S
 
-  // ---- phase 2: per chunk, softmax then P.V (the V stream)
-  const int lim0 = pmax;
-  for (int c = c_lo; c < c_hi; ++c) {
-    const int key0 = c * a.chunk;
+  // ---- phase 2: the softmax of every (chunk, pair) of the segment, one warp each,
+  // while the V sub-tiles stream into the ring
+  const int nch = c_hi - c_lo;
+  for (int task = warp; task < nch * npairs; task += ATT_THREADS / 32) {
+    const int cl = task / npairs, pl = task % npairs;
+    const int key0 = (c_lo + cl) * a.chunk;
     const int nvalid = min(a.chunk, pmax - key0 + 1);
-    const int nsub = (nvalid + ATT_SUB - 1) / ATT_SUB;
-    const float* Sc = S + (c - c_lo) * 256;
-    for (int pl = warp; pl < npairs; pl += ATT_THREADS / 32) {
-      const int lim = lim0 - key0;  // keys j <= lim are visible to the query
-      float mx = -INFINITY;
+    const int lim = pmax - key0;  // keys j <= lim are visible to the query
+    const float* Sc = S + cl * 256;
+    float mx = -INFINITY;
 #pragma unroll
-      for (int k = 0; k < ATT_CHUNK / 32; ++k) {
-        const int j = lane + 32 * k;
-        if (j <= lim && j < nvalid) mx = fmaxf(mx, Sc[pl * ATD_SST + j]);
-      }
-      mx = warp_max(mx);
-      float sum = 0.f;
-#pragma unroll
-      for (int k = 0; k < ATT_CHUNK / 32; ++k) {
-        const int j = lane + 32 * k;
-        float pj = 0.f;
-        if (j <= lim && j < nvalid) pj = expf(Sc[pl * ATD_SST + j] - mx);
-        sum += pj;
-        const uint16_t p0 = f32_to_bf16_bits(pj);
-        const float r0 = pj - bf16_bits_to_f32(p0);
-        const uint16_t p1 = f32_to_bf16_bits(r0);
-        const uint16_t p2 = f32_to_bf16_bits(r0 - bf16_bits_to_f32(p1));
-        const uint32_t off = atc_poff(pl, j);
-        *reinterpret_cast<uint16_t*>(Pp + 0 * (NP * 512) + off) = p0;
-        *reinterpret_cast<uint16_t*>(Pp + 1 * (NP * 512) + off) = p1;
-        *reinterpret_cast<uint16_t*>(Pp + 2 * (NP * 512) + off) = p2;
-      }
-      sum = warp_sum_fixed(sum);
-      if (lane == 0) {
-        m_s[pl] = mx;
-        l_s[pl] = sum;
-        live_s[pl] = lim >= 0;
-      }
+    for (int k = 0; k < ATT_CHUNK / 32; ++k) {
+      const int j = lane + 32 * k;
+      if (j <= lim && j < nvalid) mx = fmaxf(mx, Sc[pl * ATD_SST + j]);
     }
-    cbar();
+    mx = warp_max(mx);
+    float sum = 0.f;
+    uint8_t* Pc = Pp + cl * (3 * PPART);
+#pragma unroll
+    for (int k = 0; k < ATT_CHUNK / 32; ++k) {
+      const int j = lane + 32 * k;
+      float pj = 0.f;
+      if (j <= lim && j < nvalid) pj = expf(Sc[pl * ATD_SST + j] - mx);
+      sum += pj;
+      const uint16_t p0 = f32_to_bf16_bits(pj);
+      const float r0 = pj - bf16_bits_to_f32(p0);
+      const uint16_t p1 = f32_to_bf16_bits(r0);
+      const uint16_t p2 = f32_to_bf16_bits(r0 - bf16_bits_to_f32(p1));
+      const uint32_t off = atc_poff(pl, j);
+      *reinterpret_cast<uint16_t*>(Pc + 0 * PPART + off) = p0;
+      *reinterpret_cast<uint16_t*>(Pc + 1 * PPART + off) = p1;
+      *reinterpret_cast<uint16_t*>(Pc + 2 * PPART + off) = p2;
+    }
+    sum = warp_sum_fixed(sum);
+    if (lane == 0) {
+      m_s[cl][pl] = mx;
+      l_s[cl][pl] = sum;
+      live_s[cl][pl] = lim >= 0;
+    }
+  }
+  cbar();
 
-    // P.V: warp w owns head elements 16w..16w+15 (one m16 tile of V^T)
+  // ---- phase 3: P.V of every chunk, the V stream without pauses.  Warp w owns
+  // head elements 16w..16w+15 (one m16 tile of V^T); pair rows past NP read a
+  // real row (their columns of the product are never stored).
+  for (int c = c_lo; c < c_hi; ++c) {
+    const int cl = c - c_lo;
+    const int nvalid = min(a.chunk, pmax - c * a.chunk + 1);
+    const int nsub = (nvalid + ATT_SUB - 1) / ATT_SUB;
+    const uint32_t pc_s = pp_s + cl * (3 * PPART);
     float pacc[3][4];
 #pragma unroll
     for (int q = 0; q < 3; ++q) pacc[q][0] = pacc[q][1] = pacc[q][2] = pacc[q][3] = 0.f;
@@ -910,8 +925,8 @@ __global__ void __launch_bounds__(ATC_THREADS)
 #pragma unroll
         for (int q = 0; q < 3; ++q) {
           uint32_t pb0, pb1;
-          const int row = lane & 7;
-          ldsm_x2(pp_s + q * (NP * 512) + atc_poff(row, j0 + ((lane >> 3) & 1) * 8), pb0, pb1);
+          const int row = (lane & 7) % NP;
+          ldsm_x2(pc_s + q * PPART + atc_poff(row, j0 + ((lane >> 3) & 1) * 8), pb0, pb1);
           mma_bf16_16816(pacc[q], va, pb0, pb1);
         }
       }
@@ -920,20 +935,20 @@ __global__ void __launch_bounds__(ATC_THREADS)
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
       const int pl = 2 * t4 + cc;
-      if (pl >= npairs || !live_s[pl]) continue;
+      if (pl >= npairs || !live_s[cl][pl]) continue;
       const int hq = hk * a.G + pl;
       float* rec = a.part + (((size_t)(t0 - a.t_base) * a.Hq + hq) * a.max_chunks + c) * (128 + 4);
       const int e = warp * 16 + g8;
       rec[e] = (pacc[0][cc] + pacc[1][cc]) + pacc[2][cc];
       rec[e + 8] = (pacc[0][2 + cc] + pacc[1][2 + cc]) + pacc[2][2 + cc];
       if (warp == 0 && g8 == 0) {
-        rec[128] = m_s[pl];
-        rec[129] = l_s[pl];
+        rec[128] = m_s[cl][pl];
+        rec[129] = l_s[cl][pl];
       }
     }
-    cbar();  // the next chunk overwrites the probability parts and the statistics
   }
   if (a.merge_in_cta) {
+    cbar();  // every chunk record of the CTA is written
     for (int p = warp; p < npairs; p += ATT_THREADS / 32) {
       const int hq = hk * a.G + p;
       const int nc = min(pmax / a.chunk + 1, c_hi);

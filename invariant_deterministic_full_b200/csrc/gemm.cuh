@@ -280,6 +280,9 @@ static int gemm_tc(const void* x, int ldx, const void* w, void* y, int ldy, int 
   a.K = K;
   a.m_groups = (M + p.mt * TC_TILE_M - 1) / (p.mt * TC_TILE_M);
   a.n_groups = N / p.bn;
+  // token rows of a band of the work order: about 48 MB, so that a band stays in L2
+  const size_t group_bytes = (size_t)p.mt * TC_TILE_M * K * 2;
+  a.m_band = (int)std::max<size_t>(1, std::min<size_t>(a.m_groups, (size_t(48) << 20) / group_bytes));
   a.splits = p.splits;
   a.mcount = mcount;
   a.mmult = mmult;

@@ -141,6 +141,7 @@ struct TcArgs {
   int ldy, y_f32, vec_ok;  // vec_ok: y and ldy allow 16-byte stores
   int M, N, K;
   int m_groups, n_groups, splits;
+  int m_band;              // token groups per band of the work order (see decode_item)
   float* partial;          // FAST split-K: [splits][M][N] fp32
   const int* mcount;       // optional device row count (rows >= *mcount * mmult are not computed)
   int mmult;
@@ -214,9 +215,12 @@ __global__ void __launch_bounds__(TC_THREADS, CPS)
   const int kstages_total = (nkb + C::KBS - 1) / C::KBS;  // the last stage may hold fewer k-blocks
   const int ks_per_split = (kstages_total + a.splits - 1) / a.splits;
   const int n_items = a.splits * a.n_groups * a.m_groups;
-  // Work item -> (split, weight group, token group): token group fastest (CTAs
-  // running together share weight tiles in L2), or slowest with a device row
-  // count so that the live first token group is spread over every CTA.
+  // Work item -> (split, weight group, token group).  The token groups are cut
+  // into bands of m_band groups; a band's items run weight group by weight
+  // group, token group fastest, so the CTAs running together share weight
+  // tiles, and a band's token rows (sized to stay in L2) are read from DRAM
+  // once instead of once per weight group.  With a device row count: token
+  // group slowest, so the live first token group is spread over every CTA.
   const bool mg_major = a.mcount != nullptr;
   auto decode_item = [&](int item, int& sp, int& g, int& mg) {
     if (mg_major) {
@@ -224,9 +228,15 @@ __global__ void __launch_bounds__(TC_THREADS, CPS)
       sp = (item / a.n_groups) % a.splits;
       mg = item / (a.n_groups * a.splits);
     } else {
-      mg = item % a.m_groups;
-      g = (item / a.m_groups) % a.n_groups;
-      sp = item / (a.m_groups * a.n_groups);
+      const int per_split = a.m_groups * a.n_groups;
+      sp = item / per_split;
+      const int r = item - sp * per_split;
+      const int band = r / (a.m_band * a.n_groups);
+      const int m0 = band * a.m_band;
+      const int span = min(a.m_band, a.m_groups - m0);
+      const int w = r - band * a.m_band * a.n_groups;
+      mg = m0 + w % span;
+      g = w / span;
     }
   };
 

@@ -118,8 +118,10 @@ static int attn_set_smem_attrs() {
                                      (int)atc_smem_bytes(2, 4)));
   BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)atc_smem_bytes(4, 2)));
-  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_dec_kernel<ATD_RING>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)atd_smem_bytes(ATD_RING)));
+  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_dec_kernel<4, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)atd_smem_bytes(4, 4)));
+  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_dec_kernel<3, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)atd_smem_bytes(3, 8)));
   done = true;
   return BI_OK;
 }
@@ -149,9 +151,12 @@ static int attn_launch(int np, const CUtensorMap& tk, const CUtensorMap& tv, con
     a.merge_in_cta = n_seg == 1;
     *merged = a.merge_in_cta != 0;
     const dim3 grid(plan.n, n_seg, a.Hkv);
-    if (dec)
-      BI_TRY(launch(attn_dec_kernel<ATD_RING>, grid, dim3(ATC_THREADS), atd_smem_bytes(ATD_RING), st, tk, tv, plan,
-                    a));
+    // decode: 4-pair rows for kv heads of at most 4 q heads (a 4-deep ring), else
+    // 8 (3-deep); either way two CTAs fit an SM
+    if (dec && a.G <= 4)
+      BI_TRY(launch(attn_dec_kernel<4, 4>, grid, dim3(ATC_THREADS), atd_smem_bytes(4, 4), st, tk, tv, plan, a));
+    else if (dec)
+      BI_TRY(launch(attn_dec_kernel<3, 8>, grid, dim3(ATC_THREADS), atd_smem_bytes(3, 8), st, tk, tv, plan, a));
     else if (single && a.G <= 16)
       BI_TRY(launch(attn_tc_kernel<2, 4>, grid, dim3(ATC_THREADS), atc_smem_bytes(2, 4), st, tk, tv, plan, a));
     else
