@@ -689,6 +689,271 @@ __global__ void __launch_bounds__(ATC_THREADS)
 }
 
 // ---------------------------------------------------------------------------
+// Prefill schedule of the same computation (query blocks of up to
+// ATT_MAX_QB consecutive tokens; their (query, q head) pairs in groups of 32).
+// attn_tc_kernel streams a chunk's K and V rows through its ring once per
+// pair group.  Here a CTA keeps the chunk's K rows and V rows resident in
+// shared memory (128 KB) and runs every pair group against them; the next
+// chunk's K rows are requested as soon as the last group has its scores, and
+// its V rows once the last P.V is done.  Every score, softmax, P split, P.V
+// chain, record and merge is attn_tc_kernel's instruction sequence for the
+// same element, so prefill and decode keep giving the same bits.
+constexpr int ATP_NP = 32;  // pairs per group
+__host__ __device__ inline size_t atp_smem_bytes() {
+  return (size_t)2 * 4 * 16384       // K and V rows of one chunk: 4 sub-tiles each
+         + 2 * ATP_NP * 128          // q tile: [2 halves][NP pairs][128 B]
+         + (size_t)ATP_NP * ATC_SST * 4  // scores [NP][ATC_SST]
+         + 3 * ATP_NP * 512          // probability parts [3][NP][256 keys] bf16
+         + 1024;
+}
+
+__global__ void __launch_bounds__(ATC_THREADS, 1)
+    attn_pre_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ AttnPlan plan, const AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int NP = ATP_NP, NPT = NP / 8;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_k, full_v, empty_k, empty_v;
+  __shared__ float m_s[NP], l_s[NP];
+  __shared__ int live_s[NP];
+  __shared__ int pos_s[ATT_MAX_QB];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int b = blockIdx.x, sg = blockIdx.y, hk = blockIdx.z;
+  if (b >= plan.n) return;
+  const int t0 = plan.blk[b].x, nq = plan.blk[b].y;
+  const int s = a.slot[t0];
+  const int pmax = a.pos[t0 + nq - 1];
+  const int c_lo = sg * a.seg_len;
+  int c_hi = min(pmax / a.chunk + 1, c_lo + a.seg_len);
+  if (c_hi > a.max_chunks) {  // device position beyond what the launch was planned for
+    if (threadIdx.x == 0) dev_flag(DEVERR_CAPACITY);
+    c_hi = a.max_chunks;
+  }
+  if (c_lo >= c_hi) return;
+  const int npairs = nq * a.G;
+  const int cache_base = ((s * a.n_layers + a.layer) * a.Hkv + hk) * a.cap;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g8 = lane >> 2, t4 = lane & 3;
+  constexpr uint32_t SUB = 16384;
+  uint8_t* kbuf = smem;                                        // [4 sub-tiles][16 KB]
+  uint8_t* vbuf = smem + 4 * SUB;
+  uint8_t* qt = smem + 8 * SUB;                                // [2][NP][128 B]
+  float* S = reinterpret_cast<float*>(qt + NP * 256);          // [NP][ATC_SST]
+  uint8_t* Pp = reinterpret_cast<uint8_t*>(S + NP * ATC_SST);  // [3][NP][512 B]
+  const uint32_t qt_s = smem_u32(qt), pp_s = smem_u32(Pp);
+  auto nsub_of = [&](int c) { return (min(a.chunk, pmax - c * a.chunk + 1) + ATT_SUB - 1) / ATT_SUB; };
+
+  if (tid == 0) {
+    mbar_init(&full_k, 1);
+    mbar_init(&full_v, 1);
+    mbar_init(&empty_k, ATT_THREADS / 32);
+    mbar_init(&empty_v, ATT_THREADS / 32);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == ATT_THREADS / 32) {
+    // ---- producer warp, one lane: per chunk, its K rows into kbuf, its V rows into vbuf
+    if (lane == 0) {
+      for (int pc = c_lo; pc < c_hi; ++pc) {
+        const int pns = nsub_of(pc);
+        const uint32_t par = (uint32_t)((pc - c_lo - 1) & 1);
+        for (int isv = 0; isv < 2; ++isv) {
+          uint64_t* fb = isv ? &full_v : &full_k;
+          if (pc > c_lo && !mbar_wait(isv ? &empty_v : &empty_k, par, SITE_ATTN_TC | 0xA0)) return;
+          mbar_arrive_expect_tx(fb, pns * SUB);
+          for (int st = 0; st < pns; ++st)
+            tma_load_3d((isv ? vbuf : kbuf) + st * SUB, isv ? &tmV : &tmK, 0, cache_base + pc * a.chunk + st * ATT_SUB,
+                        0, fb);
+        }
+      }
+    }
+    return;
+  }
+
+  auto cbar = []() { asm volatile("bar.sync 1, %0;" ::"n"(ATT_THREADS) : "memory"); };
+  constexpr int SPT = NPT / 2;  // pair tiles per warp in the score phase
+  const int kt = warp & 3, spt0 = warp >> 2;
+  for (int i = tid; i < nq; i += ATT_THREADS) pos_s[i] = a.pos[t0 + i];
+
+  for (int c = c_lo; c < c_hi; ++c) {
+    const uint32_t par = (uint32_t)((c - c_lo) & 1);
+    const int key0 = c * a.chunk;
+    const int nvalid = min(a.chunk, pmax - key0 + 1);
+    const int nsub = (nvalid + ATT_SUB - 1) / ATT_SUB;
+    (void)mbar_wait(&full_k, par, SITE_ATTN_TC | 0xB0);
+    for (int pg0 = 0, gi = 0; pg0 < npairs; pg0 += NP, ++gi) {
+      const int gp = min(NP, npairs - pg0);
+      // q tile of the group (bf16, 128-byte swizzle per half; padded rows are zero)
+      for (int idx = tid; idx < NP * 16; idx += ATT_THREADS) {
+        const int row = idx >> 4, ch = idx & 15;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (row < gp) {
+          const int p = pg0 + row;
+          const int i = p / a.G, g = p % a.G;
+          v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.q) +
+                                              (size_t)(t0 + i) * a.Hq * 128 + (hk * a.G + g) * 128 + ch * 8);
+        }
+        const int half = ch >> 3, cc = ch & 7;
+        *reinterpret_cast<uint4*>(qt + half * (NP * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
+      }
+      cbar();
+      uint32_t qb[SPT][8][2];
+#pragma unroll
+      for (int u = 0; u < SPT; ++u)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int row = (spt0 + 2 * u) * 8 + (lane & 7);
+          const int half = kk >> 2, ch = 2 * (kk & 3) + ((lane >> 3) & 1);
+          ldsm_x2(qt_s + half * (NP * 128) + row * 128 + ((ch ^ (row & 7)) << 4), qb[u][kk][0], qb[u][kk][1]);
+        }
+
+      // ---- scores: S[pair][key] = scale * (K[key] . q[pair]), K resident
+      for (int st = 0; st < nsub; ++st) {
+        const uint32_t kb = smem_u32(kbuf + st * SUB);
+        float acc[SPT][4];
+#pragma unroll
+        for (int u = 0; u < SPT; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int krow = kt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int half = kk >> 2, ch = 2 * (kk & 3) + (lane >> 4);
+          uint32_t ka[4];
+          ldsm_x4(kb + half * 8192 + krow * 128 + ((ch ^ (krow & 7)) << 4), ka[0], ka[1], ka[2], ka[3]);
+#pragma unroll
+          for (int u = 0; u < SPT; ++u) mma_bf16_16816(acc[u], ka, qb[u][kk][0], qb[u][kk][1]);
+        }
+#pragma unroll
+        for (int u = 0; u < SPT; ++u) {
+          const int pr = (spt0 + 2 * u) * 8 + 2 * t4;
+          const int j = st * ATT_SUB + kt * 16 + g8;
+          S[pr * ATC_SST + j] = acc[u][0] * a.scale;
+          S[(pr + 1) * ATC_SST + j] = acc[u][1] * a.scale;
+          S[pr * ATC_SST + j + 8] = acc[u][2] * a.scale;
+          S[(pr + 1) * ATC_SST + j + 8] = acc[u][3] * a.scale;
+        }
+      }
+      if (pg0 + NP >= npairs) {  // the last group has its scores: the K rows may be replaced
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_k);
+      }
+      cbar();  // every score of the group is in S
+
+      // ---- softmax of the live pair rows (attn_tc_kernel's sequence)
+      for (int pl = warp; pl < gp; pl += ATT_THREADS / 32) {
+        const int i = (pg0 + pl) / a.G;
+        const int lim = pos_s[i] - key0;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < ATT_CHUNK / 32; ++k) {
+          const int j = lane + 32 * k;
+          if (j <= lim && j < nvalid) mx = fmaxf(mx, S[pl * ATC_SST + j]);
+        }
+        mx = warp_max(mx);
+        float sum = 0.f;
+#pragma unroll
+        for (int k = 0; k < ATT_CHUNK / 32; ++k) {
+          const int j = lane + 32 * k;
+          float pj = 0.f;
+          if (j <= lim && j < nvalid) pj = expf(S[pl * ATC_SST + j] - mx);
+          sum += pj;
+          const uint16_t p0 = f32_to_bf16_bits(pj);
+          const float r0 = pj - bf16_bits_to_f32(p0);
+          const uint16_t p1 = f32_to_bf16_bits(r0);
+          const uint16_t p2 = f32_to_bf16_bits(r0 - bf16_bits_to_f32(p1));
+          const uint32_t off = atc_poff(pl, j);
+          *reinterpret_cast<uint16_t*>(Pp + 0 * (NP * 512) + off) = p0;
+          *reinterpret_cast<uint16_t*>(Pp + 1 * (NP * 512) + off) = p1;
+          *reinterpret_cast<uint16_t*>(Pp + 2 * (NP * 512) + off) = p2;
+        }
+        sum = warp_sum_fixed(sum);
+        if (lane == 0) {
+          m_s[pl] = mx;
+          l_s[pl] = sum;
+          live_s[pl] = lim >= 0;
+        }
+      }
+      if (gi == 0) {
+        // the chunk's V rows: once per chunk, zero the rows past the last valid key
+        (void)mbar_wait(&full_v, par, SITE_ATTN_TC | 0xC0);
+        const int vpad = nsub * ATT_SUB - nvalid;
+        for (int idx = tid; idx < vpad * 16; idx += ATT_THREADS) {
+          const int r = nvalid + (idx >> 4), ch = idx & 15;  // row within the chunk
+          *reinterpret_cast<uint4*>(vbuf + (r / ATT_SUB) * SUB + (ch >> 3) * 8192 + (r % ATT_SUB) * 128 +
+                                    ((ch & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      cbar();
+
+      // ---- P.V: warp w owns head elements 16w..16w+15 (one m16 tile of V^T), V resident
+      float pacc[3][NPT][4];
+#pragma unroll
+      for (int q = 0; q < 3; ++q)
+#pragma unroll
+        for (int u = 0; u < NPT; ++u) pacc[q][u][0] = pacc[q][u][1] = pacc[q][u][2] = pacc[q][u][3] = 0.f;
+      for (int st = 0; st < nsub; ++st) {
+        const uint32_t vb = smem_u32(vbuf + st * SUB);
+        const int vrows = nvalid - st * ATT_SUB;
+        const int nk16 = min(4, (vrows + 15) / 16);
+        for (int kk = 0; kk < nk16; ++kk) {
+          uint32_t va[4];
+          {
+            const int krow = kk * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+            const int e0 = warp * 16 + ((lane >> 3) & 1) * 8;
+            const int half = e0 >> 6, ch = (e0 & 63) >> 3;
+            ldsm_x4_trans(vb + half * 8192 + krow * 128 + ((ch ^ (krow & 7)) << 4), va[0], va[1], va[2], va[3]);
+          }
+          const int j0 = st * ATT_SUB + kk * 16;
+#pragma unroll
+          for (int q = 0; q < 3; ++q) {
+#pragma unroll
+            for (int u = 0; u < NPT; ++u) {
+              uint32_t pb0, pb1;
+              const int row = u * 8 + (lane & 7);
+              ldsm_x2(pp_s + q * (NP * 512) + atc_poff(row, j0 + ((lane >> 3) & 1) * 8), pb0, pb1);
+              mma_bf16_16816(pacc[q][u], va, pb0, pb1);
+            }
+          }
+        }
+      }
+      if (pg0 + NP >= npairs) {  // the last P.V of the chunk is done: the V rows may be replaced
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_v);
+      }
+      // partial record of each live pair: acc[e] = (o0 + o1) + o2, then m and l
+#pragma unroll
+      for (int u = 0; u < NPT; ++u)
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int pl = u * 8 + 2 * t4 + cc;
+          if (pl >= gp || !live_s[pl]) continue;
+          const int p = pg0 + pl;
+          const int i = p / a.G, g = p % a.G;
+          const int hq = hk * a.G + g;
+          float* rec = a.part + (((size_t)(t0 + i - a.t_base) * a.Hq + hq) * a.max_chunks + c) * (128 + 4);
+          const int e = warp * 16 + g8;
+          rec[e] = (pacc[0][u][cc] + pacc[1][u][cc]) + pacc[2][u][cc];
+          rec[e + 8] = (pacc[0][u][2 + cc] + pacc[1][u][2 + cc]) + pacc[2][u][2 + cc];
+          if (warp == 0 && g8 == 0) {
+            rec[128] = m_s[pl];
+            rec[129] = l_s[pl];
+          }
+        }
+      cbar();  // the next group overwrites q, S, the probability parts and the statistics
+    }
+  }
+  if (a.merge_in_cta) {
+    for (int p = warp; p < npairs; p += ATT_THREADS / 32) {
+      const int t = t0 + p / a.G, hq = hk * a.G + p % a.G;
+      const int nc = min(pos_s[t - t0] / a.chunk + 1, c_hi);
+      merge_pair(a.part + ((size_t)(t - a.t_base) * a.Hq + hq) * a.max_chunks * (128 + 4), nc, 128, lane, a.out,
+                 (size_t)t * a.Hq * 128 + hq * 128, 0);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Decode schedule of the same computation (one query per block, G <= 8 q
 // heads: one 8-pair tile).  attn_tc_kernel<1, RING> walks each chunk as
 // scores -> softmax -> P.V, so at every chunk boundary the next chunk's keys

@@ -97,9 +97,17 @@ static int attn_chunk_for(int T, int variant) {
   return T <= 4 ? 64 : (T <= 16 ? 128 : 256);
 }
 
+// Tokens per attention launch: as many as fit a 256 MB partials workspace (at
+// least ATT_TOKEN_GROUP), so a long prefill is a few large launches.
+constexpr size_t ATT_PART_BUDGET = size_t(256) << 20;
+static int attn_token_group(int T, int Hq, int d, int max_chunks) {
+  const size_t per_tok = (size_t)Hq * max_chunks * (d + 4) * sizeof(float);
+  const size_t by_budget = ATT_PART_BUDGET / per_tok;
+  return (int)std::min<size_t>((size_t)T, std::max<size_t>(ATT_TOKEN_GROUP, std::min<size_t>(by_budget, 1u << 20)));
+}
 static size_t attn_ws_bytes(int T, int Hq, int d, int max_pos, int chunk) {
-  const int tg = std::min(T, ATT_TOKEN_GROUP);
   const int max_chunks = max_pos / chunk + 1;
+  const int tg = attn_token_group(T, Hq, d, max_chunks);
   return (size_t)tg * Hq * max_chunks * (d + 4) * sizeof(float) + 256;
 }
 
@@ -118,6 +126,8 @@ static int attn_set_smem_attrs() {
                                      (int)atc_smem_bytes(2, 4)));
   BI_CHECK_CUDA(cudaFuncSetAttribute(attn_tc_kernel<4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)atc_smem_bytes(4, 2)));
+  BI_CHECK_CUDA(cudaFuncSetAttribute(attn_pre_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)atp_smem_bytes()));
   BI_CHECK_CUDA(cudaFuncSetAttribute(attn_dec_kernel<4, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)atd_smem_bytes(4, 4)));
   BI_CHECK_CUDA(cudaFuncSetAttribute(attn_dec_kernel<3, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -159,8 +169,8 @@ static int attn_launch(int np, const CUtensorMap& tk, const CUtensorMap& tv, con
       BI_TRY(launch(attn_dec_kernel<3, 8>, grid, dim3(ATC_THREADS), atd_smem_bytes(3, 8), st, tk, tv, plan, a));
     else if (single && a.G <= 16)
       BI_TRY(launch(attn_tc_kernel<2, 4>, grid, dim3(ATC_THREADS), atc_smem_bytes(2, 4), st, tk, tv, plan, a));
-    else
-      BI_TRY(launch(attn_tc_kernel<4, 2>, grid, dim3(ATC_THREADS), atc_smem_bytes(4, 2), st, tk, tv, plan, a));
+    else  // prefill blocks: the chunk's K and V rows resident for all pair groups
+      BI_TRY(launch(attn_pre_kernel, grid, dim3(ATC_THREADS), atp_smem_bytes(), st, tk, tv, plan, a));
     return BI_OK;
   }
   a.seg_len = 1;
@@ -216,6 +226,7 @@ static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const
   }
   const int max_chunks = max_pos / chunk + 1;
   const size_t need = attn_ws_bytes(T, Hq, d, max_pos, chunk);
+  const int tg = attn_token_group(T, Hq, d, max_chunks);
   BI_REQUIRE(ws && ws_bytes >= need, BI_ERR_WORKSPACE, "bi_attention: workspace %zu < %zu", ws_bytes, need);
 
   const int esz = f32 ? 4 : 2;
@@ -237,7 +248,7 @@ static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const
   int np1 = 4;
   while (np1 < G) np1 *= 2;
 
-  // Token groups of at most ATT_TOKEN_GROUP tokens bound the partials
+  // Token groups of at most tg tokens bound the partials
   // workspace; a group is made of whole blocks.  Within a group, single-token
   // blocks and multi-token blocks go to two launches with different pair-group
   // sizes (work assignment only).
@@ -249,7 +260,7 @@ static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const
     p1.n = 0;
     pm.n = 0;
     while (bi1 < blocks.size() && p1.n < ATT_MAX_BLOCKS && pm.n < ATT_MAX_BLOCKS &&
-           blocks[bi1].x + blocks[bi1].y - t_base <= ATT_TOKEN_GROUP) {
+           blocks[bi1].x + blocks[bi1].y - t_base <= tg) {
       if (blocks[bi1].y == 1)
         p1.blk[p1.n++] = blocks[bi1++];
       else
@@ -574,7 +585,8 @@ int bi_rope_kv_append(const float* qkv, const float* rope, int rope_max_pos, voi
 size_t bi_attention_workspace_size(int T, int Hq, int head_dim, int max_pos) {
   if (T <= 0 || Hq <= 0 || head_dim <= 0 || max_pos < 0) return 0;
   // the largest of the invariant and FAST chunkings
-  return attn_ws_bytes(T, Hq, head_dim, max_pos, 64);
+  return std::max(std::max(attn_ws_bytes(T, Hq, head_dim, max_pos, 64), attn_ws_bytes(T, Hq, head_dim, max_pos, 128)),
+                  attn_ws_bytes(T, Hq, head_dim, max_pos, 256));
 }
 
 int bi_attention(const void* q, const bi_kv_layout* kv, int layer, const int32_t* slot, const int32_t* pos,
