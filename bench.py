@@ -167,7 +167,8 @@ def step_bytes(cfg, B, ctx_lens, f32_kv=False):
 # capture (dram__bytes_read.sum + dram__bytes_write.sum) of the same shapes on the 2-layer 8B-width case (the
 # weights per launch do not depend on the layer count).  Valid only for the GEMM kernel source that was captured,
 # recognised by gemm_source_digest; None until a capture of this source.
-GEMM_TRAFFIC = {"gemm_source_sha256": None, "batch": 32, "per_layer_bytes": None}
+GEMM_TRAFFIC = {"gemm_source_sha256": "b9c5b367c4427dfa380176401f09704f39acb3137e5821b44194db8546979d18",
+                "batch": 32, "per_layer_bytes": 445870336}
 
 CSRC = os.path.join(ROOT, "invariant_deterministic_full_b200", "csrc")
 

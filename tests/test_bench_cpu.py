@@ -44,7 +44,9 @@ def test_stored_gemm_traffic_applies_to_this_source_and_equals_the_algorithmic_b
     if t is None:
         pytest.skip("GEMM kernel source changed since the stored ncu capture: traffic is reported as null")
     tot, n = bench.gemm_bytes(L8, 32)
-    assert t == pytest.approx(tot / n, rel=0.01)  # no re-reads beyond the algorithmic bytes
+    # no re-reads beyond the algorithmic bytes; the epilogues' 2-byte stores write whole 32-byte sectors, which
+    # puts the measured DRAM writes a few MB per layer above the algorithmic outputs
+    assert tot / n <= t <= 1.02 * tot / n
     assert bench.gemm_traffic_per_launch(L8, 16) is None  # captured at batch 32 only
 
 
