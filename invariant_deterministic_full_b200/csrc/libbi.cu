@@ -318,7 +318,7 @@ static LmWs lm_carve(Carver& cv, int B, int H, int V, int mode, bool own_logits,
   const int rows = (bf && parts == 3 && B <= LM_ONE_PASS_ROWS) ? 3 * B : B;
   w.hs = bf ? cv.take<uint16_t>((size_t)rows * H) : nullptr;
   w.logits = (bf || own_logits) ? cv.take<float>((size_t)(bf ? rows : B) * V) : nullptr;
-  w.part = cv.take<LmPart>((size_t)B * nch);
+  w.part = cv.take<LmPart>((size_t)(rows == 3 * B ? 2 : 1) * B * nch);  // one pass: main and exact partials
   w.flag = cv.take<uint8_t>(B);
   w.list = cv.take<int32_t>(B);
   w.count = cv.take<int>(1);
@@ -375,28 +375,27 @@ static int lmhead_run(const float* h, const void* W, const int32_t* target, int 
     z = logits ? logits : w.logits;
     BI_TRY(gemm_f32(h, H, W, z, V, 1, B, V, H, BI_EPI_NONE, nullptr, st, true));
   }
-  BI_TRY(launch(lm_partial_kernel, dim3(dim3((nch + LM_CPB - 1) / LM_CPB, B)), dim3(32 * LM_CPB), 0, st, z, V, V, target, nullptr, nullptr, w.part, nch,
-                1, 0, nullptr));
+  // FP32 logits of the flagged rows: h = p0 + p1 + p2 exactly (bf16 parts), so
+  // h.W^T = ((p0.W^T + p1.W^T) + p2.W^T) with exact products and fp32
+  // accumulation on the tensor cores.  One pass: the GEMM above computed them
+  // for every row, and one partials launch and one merge launch serve both
+  // paths (the merge picks the exact one for the flagged rows).  Two passes:
+  // the main path first, then one more pass over W for the flagged rows only
+  // (row count read on the device).
+  const bool fused = parts == 3 && one_pass;
   const float th = mode == BI_MODE_BF16 ? thresh : 0.f;
-  BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, nullptr, nullptr, target, th, 0, logprob, lse,
-                                                        argmax, margin, recomputed, w.flag));
-  if (parts == 3) {
-    // FP32 logits of the flagged rows: h = p0 + p1 + p2 exactly (bf16 parts), so
-    // h.W^T = ((p0.W^T + p1.W^T) + p2.W^T) with exact products and fp32
-    // accumulation on the tensor cores.
-    if (one_pass) {  // already computed by the pass above
-      BI_TRY(launch(lm_compact_kernel, dim3(B), dim3(32), 0, st, w.flag, B, h, H, w.list, w.count, nullptr));
-      BI_TRY(launch(lm_partial_kernel, dim3(dim3((nch + LM_CPB - 1) / LM_CPB, B)), dim3(32 * LM_CPB), 0, st, z, V, V, target, w.list, w.count,
-                    w.part, nch, 3, B, nullptr));
-    } else {  // one more pass over W for the flagged rows only (row count read on the device)
-      BI_TRY(launch(lm_compact_kernel, dim3(B), dim3(256), 0, st, w.flag, B, h, H, w.list, w.count, w.hc2));
-      BI_TRY(gemm_bf16(w.hc2, H, W, w.logits_c, V, 1, 2 * B, V, H, BI_EPI_NONE, BI_VARIANT_INVARIANT, nullptr, 0, st,
-                       w.count, 2));
-      BI_TRY(launch(lm_partial_kernel, dim3(dim3((nch + LM_CPB - 1) / LM_CPB, B)), dim3(32 * LM_CPB), 0, st, z, V, V, target, w.list, w.count,
-                    w.part, nch, 3, 0, w.logits_c));
-    }
-    BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, w.count, w.list, target, th, 1, logprob,
-                                                          lse, argmax, margin, recomputed, nullptr));
+  BI_TRY(launch(lm_partial_kernel, dim3((nch + LM_CPB - 1) / LM_CPB, fused ? 2 * B : B), dim3(32 * LM_CPB), 0, st, z,
+                (size_t)V, V, target, nullptr, nullptr, w.part, nch, fused ? 4 : 1, fused ? B : 0, nullptr));
+  BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, nullptr, nullptr, target,
+                th, fused ? 2 : 0, logprob, lse, argmax, margin, recomputed, w.flag));
+  if (parts == 3 && !one_pass) {
+    BI_TRY(launch(lm_compact_kernel, dim3(B), dim3(256), 0, st, w.flag, B, h, H, w.list, w.count, w.hc2));
+    BI_TRY(gemm_bf16(w.hc2, H, W, w.logits_c, V, 1, 2 * B, V, H, BI_EPI_NONE, BI_VARIANT_INVARIANT, nullptr, 0, st,
+                     w.count, 2));
+    BI_TRY(launch(lm_partial_kernel, dim3((nch + LM_CPB - 1) / LM_CPB, B), dim3(32 * LM_CPB), 0, st, z, (size_t)V, V,
+                  target, w.list, w.count, w.part, nch, 3, 0, w.logits_c));
+    BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, w.count, w.list,
+                  target, th, 1, logprob, lse, argmax, margin, recomputed, nullptr));
   }
   return BI_OK;
 }
@@ -414,7 +413,7 @@ struct LmStageWs {
 static LmStageWs lm_stage_carve(Carver& cv, int B, int V) {
   const int nch = (V + LM_CHUNK - 1) / LM_CHUNK;
   LmStageWs w{};
-  w.part = cv.take<LmPart>((size_t)B * nch);
+  w.part = cv.take<LmPart>((size_t)2 * B * nch);  // main and exact partials of every row
   w.flag = cv.take<uint8_t>(B);
   w.list = cv.take<int32_t>(B);
   w.count = cv.take<int>(1);
@@ -436,17 +435,11 @@ static int lm_from_logits_run(const float* z, int B, int V, int parts, const int
   LmStageWs w = lm_stage_carve(cv, B, V);
   const int nch = (V + LM_CHUNK - 1) / LM_CHUNK;
   const float th = parts == 3 ? thresh : 0.f;
-  BI_TRY(launch(lm_partial_kernel, dim3((nch + LM_CPB - 1) / LM_CPB, B), dim3(32 * LM_CPB), 0, st, z, (size_t)V, V,
-                target, nullptr, nullptr, w.part, nch, 1, 0, nullptr));
+  const bool fused = parts == 3 && thresh > 0.f;  // the one-pass layout's two paths in one launch each
+  BI_TRY(launch(lm_partial_kernel, dim3((nch + LM_CPB - 1) / LM_CPB, fused ? 2 * B : B), dim3(32 * LM_CPB), 0, st, z,
+                (size_t)V, V, target, nullptr, nullptr, w.part, nch, fused ? 4 : 1, fused ? B : 0, nullptr));
   BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, nullptr, nullptr,
-                target, th, 0, logprob, lse, argmax, margin, recomputed, w.flag));
-  if (parts == 3 && thresh > 0.f) {
-    BI_TRY(launch(lm_compact_kernel, dim3(B), dim3(32), 0, st, w.flag, B, nullptr, 0, w.list, w.count, nullptr));
-    BI_TRY(launch(lm_partial_kernel, dim3((nch + LM_CPB - 1) / LM_CPB, B), dim3(32 * LM_CPB), 0, st, z, (size_t)V, V,
-                  target, w.list, w.count, w.part, nch, 3, B, nullptr));
-    BI_TRY(launch(lm_merge_kernel, dim3((B * 32 + 127) / 128), dim3(128), 0, st, w.part, nch, B, w.count, w.list,
-                  target, th, 1, logprob, lse, argmax, margin, recomputed, nullptr));
-  }
+                target, th, fused ? 2 : 0, logprob, lse, argmax, margin, recomputed, w.flag));
   return BI_OK;
 }
 

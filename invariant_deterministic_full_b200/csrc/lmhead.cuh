@@ -45,13 +45,17 @@ __device__ __forceinline__ void lm_top2_warp(float& v1, int& i1, float& v2, int&
   }
 }
 
-// Grid (ceil(n_chunks / LM_CPB), B), LM_CPB warps per CTA, warp w taking
+// Grid (ceil(n_chunks / LM_CPB), rows), LM_CPB warps per CTA, warp w taking
 // chunk blockIdx.x * LM_CPB + w of grid row blockIdx.y.  logits: [rows][ldz]
-// f32.  Row r of the grid is logits row r; rows >= *count (when count !=
-// nullptr) are skipped.  target: per-row target id (nullptr: none); rows_map
-// maps grid row -> target row (nullptr: identity).
-// parts == 3: the logit is (z0 + z1) + z2, the three partial products of the
-// exact bf16 split of an f32 hidden row (layouts below).
+// f32.  Grid rows >= *count (when count != nullptr) are skipped.  target:
+// per-row target id (nullptr: none).  What grid row r computes:
+//   parts 1: the logits of row r (rows_map, if given, maps r -> target row);
+//   parts 3: the exact logits (z0 + z1) + z2 of the f32 hidden row src =
+//     rows_map[r] (compacted flagged rows): z0 at row src of logits, z1 and z2
+//     at rows src + pstride and src + 2 pstride (one-pass layout, pstride > 0)
+//     or at rows 2r, 2r + 1 of parts_z (second pass, pstride == 0);
+//   parts 4 (one-pass layout, every row both ways): rows r < pstride as parts
+//     1, rows r >= pstride the exact logits of row src = r - pstride.
 constexpr int LM_CPB = 8;  // vocabulary chunks (warps) per CTA
 
 __global__ void __launch_bounds__(32 * LM_CPB)
@@ -66,24 +70,23 @@ __global__ void __launch_bounds__(32 * LM_CPB)
   const int c = blockIdx.x * LM_CPB + (threadIdx.x >> 5);
   if (c >= n_chunks) return;
   constexpr int PER = LM_CHUNK / 32;
+  const bool exact = parts == 3 || (parts == 4 && r >= pstride);
+  // the hidden row this grid row belongs to (its target)
+  const int src = parts == 4 ? (exact ? r - pstride : r) : (rows_map ? rows_map[r] : r);
   float z[PER];
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
     const int v = c * LM_CHUNK + lane + 32 * j;
     float zv = -INFINITY;
     if (v < V) {
-      if (parts == 3) {  // row r of the compacted list: (z0 + z1) + z2 of its row src
-        // z0 = logits row src (the main pass on p0 = bf16(h)); z1, z2 at rows
-        // src + pstride, src + 2 pstride of logits (one-pass layout, pstride > 0)
-        // or at rows 2r, 2r + 1 of parts (second pass, pstride == 0)
-        const size_t src = rows_map[r];
-        const float z0 = logits[src * ldz + v];
+      if (!exact) {
+        zv = logits[(size_t)r * ldz + v];
+      } else {
+        const float z0 = logits[(size_t)src * ldz + v];
         if (pstride > 0)
-          zv = (z0 + logits[(src + pstride) * ldz + v]) + logits[(src + 2 * pstride) * ldz + v];
+          zv = (z0 + logits[((size_t)src + pstride) * ldz + v]) + logits[((size_t)src + 2 * pstride) * ldz + v];
         else
           zv = (z0 + parts_z[(size_t)(2 * r) * ldz + v]) + parts_z[(size_t)(2 * r + 1) * ldz + v];
-      } else {
-        zv = logits[(size_t)r * ldz + v];
       }
     }
     z[j] = zv;
@@ -96,7 +99,7 @@ __global__ void __launch_bounds__(32 * LM_CPB)
   int i1 = 0x7fffffff, i2 = 0x7fffffff;
   float e = 0.f, zt = 0.f;
   int has = 0;
-  const int tg = target ? target[rows_map ? rows_map[r] : r] : -1;
+  const int tg = target ? target[src] : -1;
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
     const int v = c * LM_CHUNK + lane + 32 * j;
@@ -121,21 +124,12 @@ __global__ void __launch_bounds__(32 * LM_CPB)
   }
 }
 
-// One warp per row.  mode_recompute = 0: main pass (writes every output and
-// sets the flag); 1: recompute pass (rows given by rows_map, writes lse,
-// logprob, argmax and recomputed = 1; margin keeps the main-pass value).
-__global__ void lm_merge_kernel(const LmPart* __restrict__ part, int n_chunks, int B, const int* __restrict__ count,
-                                const int32_t* __restrict__ rows_map, const int32_t* __restrict__ target,
-                                float thresh, int mode_recompute, float* __restrict__ logprob, float* __restrict__ lse,
-                                int32_t* __restrict__ argmax, float* __restrict__ margin,
-                                uint8_t* __restrict__ recomputed, uint8_t* __restrict__ flag) {
-  pdl_wait();
-  pdl_trigger();
-  const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const int nrows = count ? min(B, *count) : B;
-  if (r >= nrows) return;
-  const LmPart* pr = part + (size_t)r * n_chunks;
+// Merge of one row's chunk partials (one warp; every lane returns the results).
+struct LmRow {
+  float L, v1, v2, zt;
+  int i1, has;
+};
+__device__ __forceinline__ LmRow lm_merge_row(const LmPart* __restrict__ pr, int n_chunks, int lane) {
   float M = -INFINITY;
   for (int c = lane; c < n_chunks; c += 32) M = fmaxf(M, pr[c].mx);
   M = warp_max(M);
@@ -158,23 +152,54 @@ __global__ void lm_merge_kernel(const LmPart* __restrict__ part, int n_chunks, i
   const unsigned hb = __ballot_sync(0xffffffffu, has);
   const int src = hb ? __ffs(hb) - 1 : 0;
   zt = __shfl_sync(0xffffffffu, zt, src);
-  if (lane != 0) return;
-  const float L = M + logf(S);
+  LmRow o;
+  o.L = M + logf(S);
+  o.v1 = v1;
+  o.v2 = v2;
+  o.i1 = i1;
+  o.zt = zt;
+  o.has = hb != 0;
+  return o;
+}
+
+// One warp per row.  mode_recompute = 0: main pass (writes every output and
+// sets the flag); 1: recompute pass (rows given by rows_map, writes lse,
+// logprob, argmax and recomputed = 1; margin keeps the main-pass value);
+// 2: both in one launch (the one-pass layout): the main partials of row r are
+// rows r of part and its exact partials rows B + r; the flag decided by the
+// main margin picks which merge gives lse, logprob and argmax.
+__global__ void lm_merge_kernel(const LmPart* __restrict__ part, int n_chunks, int B, const int* __restrict__ count,
+                                const int32_t* __restrict__ rows_map, const int32_t* __restrict__ target,
+                                float thresh, int mode_recompute, float* __restrict__ logprob, float* __restrict__ lse,
+                                int32_t* __restrict__ argmax, float* __restrict__ margin,
+                                uint8_t* __restrict__ recomputed, uint8_t* __restrict__ flag) {
+  pdl_wait();
+  pdl_trigger();
+  const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nrows = count ? min(B, *count) : B;
+  if (r >= nrows) return;
+  LmRow m = lm_merge_row(part + (size_t)r * n_chunks, n_chunks, lane);
   const int orow = rows_map ? rows_map[r] : r;
   const int tg = target ? target[orow] : -1;
-  const float lp = (tg >= 0 && hb) ? zt - L : v1 - L;
-  lse[orow] = L;
-  logprob[orow] = lp;
-  argmax[orow] = i1;
-  if (!mode_recompute) {
-    const float mg = v1 - v2;
-    margin[orow] = mg;
-    const bool f = thresh > 0.f && mg < thresh;
-    if (flag) flag[orow] = f;
-    recomputed[orow] = 0;
-  } else {
+  if (mode_recompute == 1) {
+    if (lane != 0) return;
+    lse[orow] = m.L;
+    logprob[orow] = (tg >= 0 && m.has) ? m.zt - m.L : m.v1 - m.L;
+    argmax[orow] = m.i1;
     recomputed[orow] = 1;
+    return;
   }
+  const float mg = m.v1 - m.v2;
+  const bool f = thresh > 0.f && mg < thresh;  // uniform across the warp
+  if (mode_recompute == 2 && f) m = lm_merge_row(part + (size_t)(B + r) * n_chunks, n_chunks, lane);
+  if (lane != 0) return;
+  lse[orow] = m.L;
+  logprob[orow] = (tg >= 0 && m.has) ? m.zt - m.L : m.v1 - m.L;
+  argmax[orow] = m.i1;
+  margin[orow] = mg;
+  if (flag) flag[orow] = f;
+  recomputed[orow] = mode_recompute == 2 && f;
 }
 
 // Ascending compaction of the flagged rows: list[k] = k-th flagged row.  CTA
