@@ -690,33 +690,37 @@ __global__ void __launch_bounds__(ATC_THREADS)
 
 // ---------------------------------------------------------------------------
 // Prefill schedule of the same computation (query blocks of up to
-// ATT_MAX_QB consecutive tokens; their (query, q head) pairs in groups of 32).
+// ATT_MAX_QB consecutive tokens; their (query, q head) pairs in groups of 16).
 // attn_tc_kernel streams a chunk's K and V rows through its ring once per
 // pair group.  Here a CTA keeps the chunk's K rows and V rows resident in
-// shared memory (128 KB) and runs every pair group against them; the next
-// chunk's K rows are requested as soon as the last group has its scores, and
-// its V rows once the last P.V is done.  Every score, softmax, P split, P.V
-// chain, record and merge is attn_tc_kernel's instruction sequence for the
-// same element, so prefill and decode keep giving the same bits.
-constexpr int ATP_NP = 32;  // pairs per group
+// shared memory (128 KB) and two groups of eight consumer warps run the
+// block's pair groups against them, alternately, so that each SM keeps four
+// warps per sub-partition busy; the next chunk's K rows are requested once
+// both warp groups have their last scores, its V rows once both have done
+// their last P.V.  Every score, softmax, P split, P.V chain, record and merge
+// is attn_tc_kernel's instruction sequence for the same element, so prefill
+// and decode keep giving the same bits.
+constexpr int ATP_NP = 16;          // pairs per group
+constexpr int ATP_WG = 2;           // consumer warp groups of ATT_THREADS threads
+constexpr int ATP_THREADS = ATP_WG * ATT_THREADS + 32;
+constexpr size_t ATP_WG_BYTES = 2 * ATP_NP * 128 + (size_t)ATP_NP * ATC_SST * 4 + 3 * ATP_NP * 512;
 __host__ __device__ inline size_t atp_smem_bytes() {
-  return (size_t)2 * 4 * 16384       // K and V rows of one chunk: 4 sub-tiles each
-         + 2 * ATP_NP * 128          // q tile: [2 halves][NP pairs][128 B]
-         + (size_t)ATP_NP * ATC_SST * 4  // scores [NP][ATC_SST]
-         + 3 * ATP_NP * 512          // probability parts [3][NP][256 keys] bf16
+  return (size_t)2 * 4 * 16384  // K and V rows of one chunk: 4 sub-tiles each
+         + ATP_WG * ATP_WG_BYTES // per warp group: q tile [2][NP][128 B], scores [NP][ATC_SST], P parts [3][NP][512 B]
          + 1024;
 }
 
-__global__ void __launch_bounds__(ATC_THREADS, 1)
+__global__ void __launch_bounds__(ATP_THREADS, 1)
     attn_pre_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ AttnPlan plan, const AttnArgs a) {
   pdl_wait();
   pdl_trigger();
-  constexpr int NP = ATP_NP, NPT = NP / 8;
+  constexpr int NP = ATP_NP, NPT = NP / 8, SPT = NPT / 2;
+  constexpr int NCW = ATP_WG * ATT_THREADS / 32;  // consumer warps
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_k, full_v, empty_k, empty_v;
-  __shared__ float m_s[NP], l_s[NP];
-  __shared__ int live_s[NP];
+  __shared__ float m_s[ATP_WG][NP], l_s[ATP_WG][NP];
+  __shared__ int live_s[ATP_WG][NP];
   __shared__ int pos_s[ATT_MAX_QB];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int b = blockIdx.x, sg = blockIdx.y, hk = blockIdx.z;
@@ -732,28 +736,25 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
   }
   if (c_lo >= c_hi) return;
   const int npairs = nq * a.G;
+  const int ngroups = (npairs + NP - 1) / NP;
   const int cache_base = ((s * a.n_layers + a.layer) * a.Hkv + hk) * a.cap;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, t4 = lane & 3;
   constexpr uint32_t SUB = 16384;
-  uint8_t* kbuf = smem;                                        // [4 sub-tiles][16 KB]
+  uint8_t* kbuf = smem;  // [4 sub-tiles][16 KB]
   uint8_t* vbuf = smem + 4 * SUB;
-  uint8_t* qt = smem + 8 * SUB;                                // [2][NP][128 B]
-  float* S = reinterpret_cast<float*>(qt + NP * 256);          // [NP][ATC_SST]
-  uint8_t* Pp = reinterpret_cast<uint8_t*>(S + NP * ATC_SST);  // [3][NP][512 B]
-  const uint32_t qt_s = smem_u32(qt), pp_s = smem_u32(Pp);
   auto nsub_of = [&](int c) { return (min(a.chunk, pmax - c * a.chunk + 1) + ATT_SUB - 1) / ATT_SUB; };
 
   if (tid == 0) {
     mbar_init(&full_k, 1);
     mbar_init(&full_v, 1);
-    mbar_init(&empty_k, ATT_THREADS / 32);
-    mbar_init(&empty_v, ATT_THREADS / 32);
+    mbar_init(&empty_k, NCW);
+    mbar_init(&empty_v, NCW);
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == ATT_THREADS / 32) {
+  if (warp == NCW) {
     // ---- producer warp, one lane: per chunk, its K rows into kbuf, its V rows into vbuf
     if (lane == 0) {
       for (int pc = c_lo; pc < c_hi; ++pc) {
@@ -772,10 +773,20 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     return;
   }
 
-  auto cbar = []() { asm volatile("bar.sync 1, %0;" ::"n"(ATT_THREADS) : "memory"); };
-  constexpr int SPT = NPT / 2;  // pair tiles per warp in the score phase
-  const int kt = warp & 3, spt0 = warp >> 2;
-  for (int i = tid; i < nq; i += ATT_THREADS) pos_s[i] = a.pos[t0 + i];
+  // ---- consumer warp groups: group wg takes the pair groups gi = wg, wg + ATP_WG, ...
+  const int wg = warp / 8, wl = warp % 8;  // warp group, warp within it
+  uint8_t* wbase = smem + 8 * SUB + wg * ATP_WG_BYTES;
+  uint8_t* qt = wbase;                                         // [2][NP][128 B]
+  float* S = reinterpret_cast<float*>(qt + NP * 256);          // [NP][ATC_SST]
+  uint8_t* Pp = reinterpret_cast<uint8_t*>(S + NP * ATC_SST);  // [3][NP][512 B]
+  const uint32_t qt_s = smem_u32(qt), pp_s = smem_u32(Pp);
+  const int gbar = 1 + wg;  // named barrier of the warp group
+  auto gsync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(gbar), "n"(ATT_THREADS) : "memory"); };
+  auto csync = []() { asm volatile("bar.sync 3, %0;" ::"n"(NCW * 32) : "memory"); };  // every consumer warp
+  const int kt = wl & 3, spt0 = wl >> 2;
+  for (int i = tid; i < nq; i += NCW * 32) pos_s[i] = a.pos[t0 + i];
+  csync();  // the positions are read by both warp groups
+  const int my_last = ngroups > wg ? wg + ((ngroups - 1 - wg) / ATP_WG) * ATP_WG : -1;  // this group's last pair group
 
   for (int c = c_lo; c < c_hi; ++c) {
     const uint32_t par = (uint32_t)((c - c_lo) & 1);
@@ -783,10 +794,27 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     const int nvalid = min(a.chunk, pmax - key0 + 1);
     const int nsub = (nvalid + ATT_SUB - 1) / ATT_SUB;
     (void)mbar_wait(&full_k, par, SITE_ATTN_TC | 0xB0);
-    for (int pg0 = 0, gi = 0; pg0 < npairs; pg0 += NP, ++gi) {
+    if (my_last < 0) {  // no pair group for this warp group: the chunk's K rows are free at once
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_k);
+    }
+    bool v_ready = false;
+    auto v_prepare = [&]() {  // once per chunk, by every consumer warp: wait for V, zero the rows past the last key
+      (void)mbar_wait(&full_v, par, SITE_ATTN_TC | 0xC0);
+      const int vpad = nsub * ATT_SUB - nvalid;
+      for (int idx = tid; idx < vpad * 16; idx += NCW * 32) {
+        const int r = nvalid + (idx >> 4), ch = idx & 15;  // row within the chunk
+        *reinterpret_cast<uint4*>(vbuf + (r / ATT_SUB) * SUB + (ch >> 3) * 8192 + (r % ATT_SUB) * 128 +
+                                  ((ch & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      csync();
+      v_ready = true;
+    };
+    for (int gi = wg; gi < ngroups; gi += ATP_WG) {
+      const int pg0 = gi * NP;
       const int gp = min(NP, npairs - pg0);
       // q tile of the group (bf16, 128-byte swizzle per half; padded rows are zero)
-      for (int idx = tid; idx < NP * 16; idx += ATT_THREADS) {
+      for (int idx = tid - wg * ATT_THREADS; idx < NP * 16; idx += ATT_THREADS) {
         const int row = idx >> 4, ch = idx & 15;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (row < gp) {
@@ -798,7 +826,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         const int half = ch >> 3, cc = ch & 7;
         *reinterpret_cast<uint4*>(qt + half * (NP * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
       }
-      cbar();
+      gsync();
       uint32_t qb[SPT][8][2];
 #pragma unroll
       for (int u = 0; u < SPT; ++u)
@@ -834,14 +862,14 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
           S[(pr + 1) * ATC_SST + j + 8] = acc[u][3] * a.scale;
         }
       }
-      if (pg0 + NP >= npairs) {  // the last group has its scores: the K rows may be replaced
+      if (gi == my_last) {  // this warp group's last scores of the chunk: its K rows may be replaced
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_k);
       }
-      cbar();  // every score of the group is in S
+      gsync();  // every score of the group is in S
 
       // ---- softmax of the live pair rows (attn_tc_kernel's sequence)
-      for (int pl = warp; pl < gp; pl += ATT_THREADS / 32) {
+      for (int pl = wl; pl < gp; pl += 8) {
         const int i = (pg0 + pl) / a.G;
         const int lim = pos_s[i] - key0;
         float mx = -INFINITY;
@@ -869,24 +897,15 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         }
         sum = warp_sum_fixed(sum);
         if (lane == 0) {
-          m_s[pl] = mx;
-          l_s[pl] = sum;
-          live_s[pl] = lim >= 0;
+          m_s[wg][pl] = mx;
+          l_s[wg][pl] = sum;
+          live_s[wg][pl] = lim >= 0;
         }
       }
-      if (gi == 0) {
-        // the chunk's V rows: once per chunk, zero the rows past the last valid key
-        (void)mbar_wait(&full_v, par, SITE_ATTN_TC | 0xC0);
-        const int vpad = nsub * ATT_SUB - nvalid;
-        for (int idx = tid; idx < vpad * 16; idx += ATT_THREADS) {
-          const int r = nvalid + (idx >> 4), ch = idx & 15;  // row within the chunk
-          *reinterpret_cast<uint4*>(vbuf + (r / ATT_SUB) * SUB + (ch >> 3) * 8192 + (r % ATT_SUB) * 128 +
-                                    ((ch & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      cbar();
+      if (!v_ready) v_prepare();  // both warp groups meet here once per chunk
+      gsync();
 
-      // ---- P.V: warp w owns head elements 16w..16w+15 (one m16 tile of V^T), V resident
+      // ---- P.V: warp wl owns head elements 16 wl..16 wl + 15 (one m16 tile of V^T), V resident
       float pacc[3][NPT][4];
 #pragma unroll
       for (int q = 0; q < 3; ++q)
@@ -900,7 +919,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
           uint32_t va[4];
           {
             const int krow = kk * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-            const int e0 = warp * 16 + ((lane >> 3) & 1) * 8;
+            const int e0 = wl * 16 + ((lane >> 3) & 1) * 8;
             const int half = e0 >> 6, ch = (e0 & 63) >> 3;
             ldsm_x4_trans(vb + half * 8192 + krow * 128 + ((ch ^ (krow & 7)) << 4), va[0], va[1], va[2], va[3]);
           }
@@ -917,7 +936,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
           }
         }
       }
-      if (pg0 + NP >= npairs) {  // the last P.V of the chunk is done: the V rows may be replaced
+      if (gi == my_last) {  // this warp group's last P.V of the chunk: its V rows may be replaced
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_v);
       }
@@ -927,24 +946,30 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int pl = u * 8 + 2 * t4 + cc;
-          if (pl >= gp || !live_s[pl]) continue;
+          if (pl >= gp || !live_s[wg][pl]) continue;
           const int p = pg0 + pl;
           const int i = p / a.G, g = p % a.G;
           const int hq = hk * a.G + g;
           float* rec = a.part + (((size_t)(t0 + i - a.t_base) * a.Hq + hq) * a.max_chunks + c) * (128 + 4);
-          const int e = warp * 16 + g8;
+          const int e = wl * 16 + g8;
           rec[e] = (pacc[0][u][cc] + pacc[1][u][cc]) + pacc[2][u][cc];
           rec[e + 8] = (pacc[0][u][2 + cc] + pacc[1][u][2 + cc]) + pacc[2][u][2 + cc];
-          if (warp == 0 && g8 == 0) {
-            rec[128] = m_s[pl];
-            rec[129] = l_s[pl];
+          if (wl == 0 && g8 == 0) {
+            rec[128] = m_s[wg][pl];
+            rec[129] = l_s[wg][pl];
           }
         }
-      cbar();  // the next group overwrites q, S, the probability parts and the statistics
+      gsync();  // the next group overwrites q, S, the probability parts and the statistics
+    }
+    if (!v_ready) {  // a warp group with no pair group still takes part in the chunk's V set-up
+      v_prepare();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_v);
     }
   }
   if (a.merge_in_cta) {
-    for (int p = warp; p < npairs; p += ATT_THREADS / 32) {
+    csync();  // every chunk record of the CTA is written
+    for (int p = warp; p < npairs; p += NCW) {
       const int t = t0 + p / a.G, hq = hk * a.G + p % a.G;
       const int nc = min(pos_s[t - t0] / a.chunk + 1, c_hi);
       merge_pair(a.part + ((size_t)(t - a.t_base) * a.Hq + hq) * a.max_chunks * (128 + 4), nc, 128, lane, a.out,

@@ -170,7 +170,7 @@ static int attn_launch(int np, const CUtensorMap& tk, const CUtensorMap& tv, con
     else if (single && a.G <= 16)
       BI_TRY(launch(attn_tc_kernel<2, 4>, grid, dim3(ATC_THREADS), atc_smem_bytes(2, 4), st, tk, tv, plan, a));
     else  // prefill blocks: the chunk's K and V rows resident for all pair groups
-      BI_TRY(launch(attn_pre_kernel, grid, dim3(ATC_THREADS), atp_smem_bytes(), st, tk, tv, plan, a));
+      BI_TRY(launch(attn_pre_kernel, grid, dim3(ATP_THREADS), atp_smem_bytes(), st, tk, tv, plan, a));
     return BI_OK;
   }
   a.seg_len = 1;
