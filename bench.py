@@ -167,31 +167,31 @@ def step_bytes(cfg, B, ctx_lens, f32_kv=False):
 # capture (dram__bytes_read.sum + dram__bytes_write.sum) of the same shapes on the 2-layer 8B-width case (the
 # weights per launch do not depend on the layer count).  Valid only for the GEMM kernel source that was captured,
 # recognised by gemm_source_digest; None until a capture of this source.
-GEMM_TRAFFIC = {"gemm_source_sha256": "b9c5b367c4427dfa380176401f09704f39acb3137e5821b44194db8546979d18",
+GEMM_TRAFFIC = {"gemm_source_sha256": "e5a3c669c6a9e67f7187742aeb1b7757cb193c30795531a8557b3b3e9bc8516e",
                 "batch": 32, "per_layer_bytes": 445870336}
 
 CSRC = os.path.join(ROOT, "invariant_deterministic_full_b200", "csrc")
 
 
-def gemm_source_digest(tc_text, mma_text, plan_text):
-    """sha256 of the code (comments and whitespace removed) that decides the GEMM's memory traffic: the whole
-    tcgen05 and mma.sync kernel files, and the launch planning and dispatch of gemm.cuh (from the tile plan to the
-    end of the bf16 dispatcher).  The FAST split heuristic, workspace sizing and the LayerCast kernels are left
-    out."""
+def gemm_source_digest(mma_text, plan_text):
+    """sha256 of the code (comments and whitespace removed) that decides the dominant kernel's memory traffic: the
+    whole mma.sync kernel file (the projections of a decode step at <= 32 token rows run on it), and the launch
+    planning and dispatch of gemm.cuh (from the tile plan to the end of the bf16 dispatcher).  The tcgen05 kernel
+    (prefill), the FAST split heuristic, workspace sizing and the LayerCast kernels are left out."""
     import hashlib
     import re
     a = plan_text.index("struct TcPlan {")
     b = plan_text.index("// LayerCast on tensor cores: rows of x per pass")
     c0 = plan_text.index("template <int BN, int MT, int KS, int EPI>\nstatic int launch_tc_t")
     c1 = plan_text.index("int gemm_f32(")
-    code = re.sub(r"/\*.*?\*/", " ", tc_text + mma_text + plan_text[a:b] + plan_text[c0:c1], flags=re.S)
+    code = re.sub(r"/\*.*?\*/", " ", mma_text + plan_text[a:b] + plan_text[c0:c1], flags=re.S)
     code = re.sub(r"//[^\n]*", " ", code)
     return hashlib.sha256(" ".join(code.split()).encode()).hexdigest()
 
 
 def current_gemm_digest():
     txt = lambda n: open(os.path.join(CSRC, n)).read()
-    return gemm_source_digest(txt("gemm_tc.cuh"), txt("gemm_mma.cuh"), txt("gemm.cuh"))
+    return gemm_source_digest(txt("gemm_mma.cuh"), txt("gemm.cuh"))
 
 
 def gemm_traffic_per_launch(cfg, B):

@@ -472,12 +472,14 @@ __global__ void __launch_bounds__(TC_THREADS, CPS)
             const bool isq = n0 < QD;
             const int rel = isq ? n0 : n0 - QD;
             const int head = rel / re.d, e0 = (rel % re.d) >> 1;  // first-half element 16b
-            const float2* tb = reinterpret_cast<const float2*>(re.table) + (size_t)p * half + e0;
+            // cos/sin of the 16 pairs: 128 contiguous bytes of the table row (16-byte loads)
+            const float4* tb = reinterpret_cast<const float4*>(re.table + ((size_t)p * half + e0) * 2);
             float ra[16], rb[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float2 cs = __ldg(tb + i);
-              rope_rotate(v[i], v[16 + i], cs.x, cs.y, ra[i], rb[i]);
+            for (int i = 0; i < 8; ++i) {
+              const float4 cs = __ldg(tb + i);
+              rope_rotate(v[2 * i], v[16 + 2 * i], cs.x, cs.y, ra[2 * i], rb[2 * i]);
+              rope_rotate(v[2 * i + 1], v[16 + 2 * i + 1], cs.z, cs.w, ra[2 * i + 1], rb[2 * i + 1]);
             }
             size_t base;
             void* dst;

@@ -97,9 +97,9 @@ static int attn_chunk_for(int T, int variant) {
   return T <= 4 ? 64 : (T <= 16 ? 128 : 256);
 }
 
-// Tokens per attention launch: as many as fit a 256 MB partials workspace (at
-// least ATT_TOKEN_GROUP), so a long prefill is a few large launches.
-constexpr size_t ATT_PART_BUDGET = size_t(256) << 20;
+// Tokens per attention launch: as many as fit a 640 MB partials workspace (at
+// least ATT_TOKEN_GROUP), so a long prefill is one or a few large launches.
+constexpr size_t ATT_PART_BUDGET = size_t(640) << 20;
 static int attn_token_group(int T, int Hq, int d, int max_chunks) {
   const size_t per_tok = (size_t)Hq * max_chunks * (d + 4) * sizeof(float);
   const size_t by_budget = ATT_PART_BUDGET / per_tok;

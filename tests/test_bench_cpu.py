@@ -52,17 +52,18 @@ def test_stored_gemm_traffic_applies_to_this_source_and_equals_the_algorithmic_b
 
 def test_gemm_source_digest_ignores_comments_and_code_outside_the_kernel():
     rd = lambda n: open(bench.os.path.join(bench.CSRC, n)).read()
-    tc, mma, plan = rd("gemm_tc.cuh"), rd("gemm_mma.cuh"), rd("gemm.cuh")
-    h = bench.gemm_source_digest(tc, mma, plan)
-    assert bench.gemm_source_digest(tc, mma, plan + "\n// trailing helper\n") == h
-    i = tc.index("template <int BN, int MT, int XR, int KS, int EPI, int CPS>")
-    assert bench.gemm_source_digest(tc[:i] + "// a comment\n  /* and another */ " + tc[i:], mma, plan) == h
-    assert bench.gemm_source_digest(tc[:i] + "constexpr int kExtra = 1;\n" + tc[i:], mma, plan) != h
-    assert bench.gemm_source_digest(tc, mma + "static int kMore = 4;\n", plan) != h
-    j = plan.index("static TcPlan tc_plan(")
-    assert bench.gemm_source_digest(tc, mma, plan[:j] + "static int kOther = 2;\n" + plan[j:]) != h
-    k = plan.index("size_t gemm_ws_bytes(")  # workspace sizing does not decide the traffic
-    assert bench.gemm_source_digest(tc, mma, plan[:k] + "static int kWs = 3;\n" + plan[k:]) == h
+    mma, plan = rd("gemm_mma.cuh"), rd("gemm.cuh")
+    h = bench.gemm_source_digest(mma, plan)
+    assert bench.gemm_source_digest(mma, plan + "\n// trailing helper\n") == h
+    i = mma.index("template <int BN, int EPI, int MT, int CPS>")
+    assert bench.gemm_source_digest(mma[:i] + "// a comment\n  /* and another */ " + mma[i:], plan) == h
+    assert bench.gemm_source_digest(mma[:i] + "constexpr int kExtra = 1;\n" + mma[i:], plan) != h
+    j = plan.index("struct TcPlan {")
+    assert bench.gemm_source_digest(mma, plan[:j] + "static int kMore = 4;\n" + plan[j:]) == h  # before the plan
+    k = plan.index("static TcPlan tc_plan(")
+    assert bench.gemm_source_digest(mma, plan[:k] + "static int kMore = 4;\n" + plan[k:]) != h
+    w = plan.index("size_t gemm_ws_bytes(")  # workspace sizing does not decide the traffic
+    assert bench.gemm_source_digest(mma, plan[:w] + "static int kWs = 3;\n" + plan[w:]) == h
 
 
 def test_clock_summary_median_and_reasons():
