@@ -1056,6 +1056,7 @@ __global__ void __launch_bounds__(ATC_THREADS)
   if (warp == ATT_THREADS / 32) {
     // ---- producer warp, one lane: every K sub-tile of the segment, then every V sub-tile
     if (lane == 0) {
+      const uint64_t kvpol = l2_evict_first();  // each cached row is read once per step
       int lp = 0;
       for (int isv = 0; isv < 2; ++isv)
         for (int pc = c_lo; pc < c_hi; ++pc) {
@@ -1065,8 +1066,8 @@ __global__ void __launch_bounds__(ATC_THREADS)
             if (lp >= RING && !mbar_wait(&empty_bar[slot], (uint32_t)(((lp / RING) - 1) & 1), SITE_ATTN_TC | 0x90))
               return;
             mbar_arrive_expect_tx(&full_bar[slot], SUB);
-            tma_load_3d(smem + slot * SUB, isv ? &tmV : &tmK, 0, cache_base + pc * a.chunk + st * ATT_SUB, 0,
-                        &full_bar[slot]);
+            tma_load_3d_hint(smem + slot * SUB, isv ? &tmV : &tmK, 0, cache_base + pc * a.chunk + st * ATT_SUB, 0,
+                             &full_bar[slot], kvpol);
           }
         }
     }

@@ -127,6 +127,7 @@ __global__ void __launch_bounds__(160, CPS)
     if (lane == 0) {
       prefetch_tmap(&tmW);
       prefetch_tmap(&tmX);
+      const uint64_t wpol = l2_evict_first();  // every weight byte is read once per launch
       // Prologue: the first ring stages of weight tiles depend on no earlier
       // kernel, so they are requested before waiting for the previous launch.
       // (With a device-side row count only token group 0 is sure to be live:
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(160, CPS)
           pre = max(0, min(C::STAGES, ks1 - ks0));
           for (int s = 0; s < pre; ++s) {
             mbar_arrive_expect_tx(&full_bar[s], stage_tx);
-            tma_load_3d(smem + s * C::STAGE_BYTES, &tmW, 0, g * BN, (ks0 + s) * C::KBS, &full_bar[s]);
+            tma_load_3d_hint(smem + s * C::STAGE_BYTES, &tmW, 0, g * BN, (ks0 + s) * C::KBS, &full_bar[s], wpol);
           }
         }
       }
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(160, CPS)
               break;
             }
             mbar_arrive_expect_tx(&full_bar[stage], stage_tx);
-            tma_load_3d(sb, &tmW, 0, g * BN, ks * C::KBS, &full_bar[stage]);
+            tma_load_3d_hint(sb, &tmW, 0, g * BN, ks * C::KBS, &full_bar[stage], wpol);
             ++issued;
           }
           tma_load_3d(sb + C::W_BYTES, &tmX, 0, mt * GEMM_BM, ks * C::KBS, &full_bar[stage]);
