@@ -84,8 +84,9 @@ int encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
 // before it reads anything an earlier kernel wrote and before it writes
 // anything (so the chain of completions stays transitive), then pdl_trigger()
 // so the next kernel may be scheduled and run its independent prologue
-// (barrier set-up, weight prefetch) while this one finishes.  Both are no-ops
-// for a kernel launched without the attribute.
+// (barrier set-up, weight prefetch) while this one finishes: at once, except
+// in the norm, which first lets its own few loads land.  Both are no-ops for a
+// kernel launched without the attribute.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 

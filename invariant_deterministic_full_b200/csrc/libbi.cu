@@ -533,10 +533,21 @@ int bi_rmsnorm(const void* x, const void* residual_in, void* residual_out, const
                  (!residual_out || aligned16(residual_out)) && (!y_f32 || aligned16(y_f32)),
              BI_ERR_UNSUPPORTED, "bi_rmsnorm: buffers must be 16-byte aligned");
   if (M == 0) return BI_OK;
-  BI_TRY(launch(rmsnorm_kernel, dim3(M), dim3(NORM_THREADS), 0, as_stream(stream), x, residual_in, residual_out,
-                                                            reinterpret_cast<const uint16_t*>(gamma), y, y_f32, H, eps,
-                                                            act_f32(mode)));
-  return BI_OK;
+  const uint16_t* g16 = reinterpret_cast<const uint16_t*>(gamma);
+  const int f32 = act_f32(mode);
+  cudaStream_t st = as_stream(stream);
+  switch (norm_cpt(H)) {
+    case 1: return launch(rmsnorm_kernel<1>, dim3(M), dim3(NORM_THREADS), 0, st, x, residual_in, residual_out, g16, y,
+                          y_f32, H, eps, f32);
+    case 2: return launch(rmsnorm_kernel<2>, dim3(M), dim3(NORM_THREADS), 0, st, x, residual_in, residual_out, g16, y,
+                          y_f32, H, eps, f32);
+    case 4: return launch(rmsnorm_kernel<4>, dim3(M), dim3(NORM_THREADS), 0, st, x, residual_in, residual_out, g16, y,
+                          y_f32, H, eps, f32);
+    case 8: return launch(rmsnorm_kernel<8>, dim3(M), dim3(NORM_THREADS), 0, st, x, residual_in, residual_out, g16, y,
+                          y_f32, H, eps, f32);
+    default: return launch(rmsnorm_kernel<16>, dim3(M), dim3(NORM_THREADS), 0, st, x, residual_in, residual_out, g16,
+                           y, y_f32, H, eps, f32);
+  }
 }
 
 int bi_rope_table_fill(float* table, int max_pos, int head_dim, double theta, void* stream) {

@@ -38,37 +38,44 @@ __device__ __forceinline__ float as_stored(float v, bool f32) {
 }
 
 // One row, NORM_THREADS threads (tid = 0 .. NORM_THREADS-1).  Thread i owns
-// the 8-element chunks i, i + NORM_THREADS, ... of the row; its partial sum of
-// squares runs over them in ascending order, then a fixed xor-butterfly inside
-// each warp, then the warp sums are added in ascending warp order (every
-// thread repeats that same sequential sum).  r = x (+ res_in, rounded as
-// stored), written to res_out; y = (r * inv) * gamma.  The row is read twice
-// (sum of squares, then the outputs) so that no chunk is held in registers;
-// both passes compute r the same way.  `bar` synchronises the NORM_THREADS
-// threads (a CTA barrier, or a named barrier inside a larger CTA).
-template <typename Bar>
+// the 8-element chunks i, i + NORM_THREADS, ... of the row (at most CPT of
+// them, held in registers: every load of the thread is issued at once); its
+// partial sum of squares runs over them in ascending order, then a fixed
+// xor-butterfly inside each warp, then the warp sums are added in ascending
+// warp order (every thread repeats that same sequential sum).  r = x
+// (+ res_in, rounded as stored), written to res_out; y = (r * inv) * gamma.
+// `bar` synchronises the NORM_THREADS threads (a CTA barrier, or a named
+// barrier inside a larger CTA).
+template <int CPT, typename Bar>
 __device__ __forceinline__ void rmsnorm_row(const void* __restrict__ x, const void* __restrict__ res_in,
                                             void* __restrict__ res_out, const uint16_t* __restrict__ gamma,
                                             void* __restrict__ y, float* __restrict__ y32, int row, int H, float eps,
                                             int f32, int tid, float* wsum, Bar bar) {
   const int nch = H / 8;
   const size_t rbase = (size_t)row * H;
-  auto load_r = [&](int ch, float* v) {
-    load8(x, rbase + ch * 8, f32, v);
-    if (res_in) {
-      float r[8];
-      load8(res_in, rbase + ch * 8, f32, r);
+  float v[CPT][8];
+  uint4 gu[CPT];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = as_stored(v[j] + r[j], f32);
+  for (int i = 0; i < CPT; ++i) {
+    const int ch = tid + i * NORM_THREADS;
+    if (ch < nch) {
+      load8(x, rbase + ch * 8, f32, v[i]);
+      if (res_in) {
+        float r[8];
+        load8(res_in, rbase + ch * 8, f32, r);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[i][j] = as_stored(v[i][j] + r[j], f32);
+      }
+      gu[i] = *reinterpret_cast<const uint4*>(gamma + ch * 8);
     }
-  };
-  float ss = 0.f;
-  for (int ch = tid; ch < nch; ch += NORM_THREADS) {
-    float v[8];
-    load_r(ch, v);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) ss = fmaf(v[j], v[j], ss);
   }
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < CPT; ++i)
+    if (tid + i * NORM_THREADS < nch) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ss = fmaf(v[i][j], v[i][j], ss);
+    }
   ss = warp_sum_fixed(ss);
   if ((tid & 31) == 0) wsum[tid >> 5] = ss;
   bar();
@@ -77,34 +84,58 @@ __device__ __forceinline__ void rmsnorm_row(const void* __restrict__ x, const vo
   for (int w = 0; w < NORM_THREADS / 32; ++w) tot += wsum[w];
   const float inv = 1.0f / sqrtf(tot / (float)H + eps);
   bar();  // wsum may be reused by the next row
-  for (int ch = tid; ch < nch; ch += NORM_THREADS) {
-    float v[8];
-    load_r(ch, v);
-    if (res_out) store8(res_out, rbase + ch * 8, f32, v);
-    const uint4 gu = *reinterpret_cast<const uint4*>(gamma + ch * 8);
-    const float gm[8] = {bf16lo(gu.x), bf16hi(gu.x), bf16lo(gu.y), bf16hi(gu.y),
-                         bf16lo(gu.z), bf16hi(gu.z), bf16lo(gu.w), bf16hi(gu.w)};
-    float o[8];
+  // Every load of the row has landed: the next kernel may now be scheduled
+  // (its weight prefetch would otherwise queue ahead of these loads).
+  pdl_trigger();
 #pragma unroll
-    for (int j = 0; j < 8; ++j) o[j] = v[j] * inv * gm[j];
-    store8(y, rbase + ch * 8, f32, o);
-    if (y32) {
-      float4* p = reinterpret_cast<float4*>(y32 + rbase + ch * 8);
-      p[0] = make_float4(o[0], o[1], o[2], o[3]);
-      p[1] = make_float4(o[4], o[5], o[6], o[7]);
+  for (int i = 0; i < CPT; ++i) {
+    const int ch = tid + i * NORM_THREADS;
+    if (ch < nch) {
+      if (res_out) store8(res_out, rbase + ch * 8, f32, v[i]);
+      const float gm[8] = {bf16lo(gu[i].x), bf16hi(gu[i].x), bf16lo(gu[i].y), bf16hi(gu[i].y),
+                           bf16lo(gu[i].z), bf16hi(gu[i].z), bf16lo(gu[i].w), bf16hi(gu[i].w)};
+      float o[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = v[i][j] * inv * gm[j];
+      store8(y, rbase + ch * 8, f32, o);
+      if (y32) {
+        float4* p = reinterpret_cast<float4*>(y32 + rbase + ch * 8);
+        p[0] = make_float4(o[0], o[1], o[2], o[3]);
+        p[1] = make_float4(o[4], o[5], o[6], o[7]);
+      }
     }
   }
 }
 
-// One CTA per row (see rmsnorm_row).
+// One CTA per row (see rmsnorm_row, which also releases the next kernel once
+// the row's loads have landed); CPT: chunks per thread, the smallest of 1, 2,
+// 4, 8, 16 that covers the row.
+template <int CPT>
 __global__ void __launch_bounds__(NORM_THREADS)
     rmsnorm_kernel(const void* __restrict__ x, const void* __restrict__ res_in, void* __restrict__ res_out,
                    const uint16_t* __restrict__ gamma, void* __restrict__ y, float* __restrict__ y32, int H, float eps,
                    int f32) {
+  {
+    // Before the dependency wait, request the row's residual and gamma into
+    // L2 (a prefetch returns no value, so it cannot observe data that an
+    // earlier kernel is still writing): after the wait the row's loads find
+    // them there instead of queuing for DRAM.
+    const int esz = f32 ? 4 : 2;
+    const int rlines = res_in ? H * esz / 128 : 0, glines = H * 2 / 128;
+    for (int i = threadIdx.x; i < rlines + glines; i += NORM_THREADS) {
+      const char* pa = i < rlines ? reinterpret_cast<const char*>(res_in) + (size_t)blockIdx.x * H * esz + i * 128
+                                  : reinterpret_cast<const char*>(gamma) + (size_t)(i - rlines) * 128;
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(pa));
+    }
+  }
   pdl_wait();
-  pdl_trigger();
   __shared__ float wsum[NORM_THREADS / 32];
-  rmsnorm_row(x, res_in, res_out, gamma, y, y32, blockIdx.x, H, eps, f32, threadIdx.x, wsum, [] { __syncthreads(); });
+  rmsnorm_row<CPT>(x, res_in, res_out, gamma, y, y32, blockIdx.x, H, eps, f32, threadIdx.x, wsum,
+                   [] { __syncthreads(); });
+}
+__host__ __device__ constexpr int norm_cpt(int H) {
+  return H / 8 <= NORM_THREADS ? 1 : H / 8 <= 2 * NORM_THREADS ? 2 : H / 8 <= 4 * NORM_THREADS ? 4
+         : H / 8 <= 8 * NORM_THREADS ? 8 : 16;
 }
 
 // Row of element i of a head (size d) in the "paired" QKV layout: within every
