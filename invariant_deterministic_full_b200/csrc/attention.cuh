@@ -999,12 +999,16 @@ constexpr int ATD_SST = ATD_SEG * 256 + 4;  // row stride of the score rows (flo
 
 // Shared memory of attn_dec_kernel<RING, NP>: NP pair rows of scores and of the
 // probability parts of every chunk of the segment (NP = 4 when a kv head has at
-// most 4 q heads, which leaves room for a deeper ring at two CTAs per SM).
+// most 4 q heads, which leaves room for a deeper ring at two CTAs per SM).  With
+// NP = 4 the chunk records of the segment also stay in shared memory when the
+// CTA merges them itself (NP = 8 would then no longer fit two CTAs per SM).
+__host__ __device__ constexpr bool atd_smem_records(int np) { return np <= 4; }
 __host__ __device__ inline size_t atd_smem_bytes(int ring, int np) {
   return (size_t)ring * 16384            // K/V sub-tiles: [2 halves][64 keys][128 B]
          + 8 * 256                       // q tile: [2 halves][8 pairs][128 B]
          + (size_t)np * ATD_SST * 4      // scores [NP][ATD_SST]
          + (size_t)ATD_SEG * 3 * np * 512  // probability parts [chunk][3][NP][256 keys] bf16, swizzled
+         + (atd_smem_records(np) ? (size_t)np * ATD_SEG * (128 + 4) * 4 : 0)  // chunk records [NP][chunk][132]
          + 1024;
 }
 
@@ -1042,6 +1046,10 @@ __global__ void __launch_bounds__(ATC_THREADS)
   float* S = reinterpret_cast<float*>(qt + 8 * 256);          // [NP][ATD_SST]
   uint8_t* Pp = reinterpret_cast<uint8_t*>(S + NP * ATD_SST);  // [ATD_SEG][3][NP][512 B]
   const uint32_t qt_s = smem_u32(qt), pp_s = smem_u32(Pp);
+  // chunk records: in shared memory when this CTA merges them (no round trip
+  // through L2 between the last P.V and the merge), else in the workspace
+  const bool rec_smem = atd_smem_records(NP) && a.merge_in_cta;
+  float* recs = reinterpret_cast<float*>(Pp + ATD_SEG * 3 * NP * 512);  // [NP][ATD_SEG][132]
   auto nsub_of = [&](int c) { return (min(a.chunk, pmax - c * a.chunk + 1) + ATT_SUB - 1) / ATT_SUB; };
 
   if (tid == 0) {
@@ -1228,7 +1236,8 @@ __global__ void __launch_bounds__(ATC_THREADS)
       const int pl = 2 * t4 + cc;
       if (pl >= npairs || !live_s[cl][pl]) continue;
       const int hq = hk * a.G + pl;
-      float* rec = a.part + (((size_t)(t0 - a.t_base) * a.Hq + hq) * a.max_chunks + c) * (128 + 4);
+      float* rec = rec_smem ? recs + ((size_t)pl * ATD_SEG + (c - c_lo)) * (128 + 4)
+                            : a.part + (((size_t)(t0 - a.t_base) * a.Hq + hq) * a.max_chunks + c) * (128 + 4);
       const int e = warp * 16 + g8;
       rec[e] = (pacc[0][cc] + pacc[1][cc]) + pacc[2][cc];
       rec[e + 8] = (pacc[0][2 + cc] + pacc[1][2 + cc]) + pacc[2][2 + cc];
@@ -1243,8 +1252,9 @@ __global__ void __launch_bounds__(ATC_THREADS)
     for (int p = warp; p < npairs; p += ATT_THREADS / 32) {
       const int hq = hk * a.G + p;
       const int nc = min(pmax / a.chunk + 1, c_hi);
-      merge_pair(a.part + ((size_t)(t0 - a.t_base) * a.Hq + hq) * a.max_chunks * (128 + 4), nc, 128, lane, a.out,
-                 (size_t)t0 * a.Hq * 128 + hq * 128, 0);
+      merge_pair(rec_smem ? recs + (size_t)p * ATD_SEG * (128 + 4)
+                          : a.part + ((size_t)(t0 - a.t_base) * a.Hq + hq) * a.max_chunks * (128 + 4),
+                 nc, 128, lane, a.out, (size_t)t0 * a.Hq * 128 + hq * 128, 0);
     }
   }
 }
