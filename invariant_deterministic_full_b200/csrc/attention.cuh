@@ -57,6 +57,10 @@ struct AttnArgs {
   float scale;
   int seg_len;              // chunks per CTA (tensor-core kernel; the CUDA-core kernel takes one)
   int merge_in_cta;         // 1: one segment spans every chunk, the CTA merges and writes out
+  int pre_kv;               // 1: slot, pos and every cache row below each token's own position were written by
+                            // kernels that completed before the previous launch (a decode step with one token per
+                            // slot): attn_dec_kernel reads them and copies its first K sub-tiles before its
+                            // dependency wait
   void* out;                // [T][Hq*d] attention output (activation dtype)
 };
 
@@ -1016,8 +1020,10 @@ template <int RING, int NP>
 __global__ void __launch_bounds__(ATC_THREADS)
     attn_dec_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ AttnPlan plan, const AttnArgs a) {
-  pdl_wait();
-  pdl_trigger();
+  if (!a.pre_kv) {
+    pdl_wait();
+    pdl_trigger();
+  }
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[RING];
   __shared__ __align__(8) uint64_t empty_bar[RING];
@@ -1065,11 +1071,30 @@ __global__ void __launch_bounds__(ATC_THREADS)
     // ---- producer warp, one lane: every K sub-tile of the segment, then every V sub-tile
     if (lane == 0) {
       const uint64_t kvpol = l2_evict_first();  // each cached row is read once per step
+      // With pre_kv the first ring fill is requested before the dependency
+      // wait: K sub-tiles whose keys all lie below the token's own row (the one
+      // row the previous kernel writes), in stream order up to the first that
+      // does not.
+      int pre = 0;
+      if (a.pre_kv) {
+        for (int pc = c_lo; pc < c_hi && pre < RING; ++pc) {
+          const int pns = nsub_of(pc);
+          int st = 0;
+          for (; st < pns && pre < RING && pc * a.chunk + (st + 1) * ATT_SUB <= pmax; ++st, ++pre) {
+            mbar_arrive_expect_tx(&full_bar[pre], SUB);
+            tma_load_3d_hint(smem + pre * SUB, &tmK, 0, cache_base + pc * a.chunk + st * ATT_SUB, 0, &full_bar[pre],
+                             kvpol);
+          }
+          if (st < pns) break;
+        }
+        pdl_wait();
+      }
       int lp = 0;
       for (int isv = 0; isv < 2; ++isv)
         for (int pc = c_lo; pc < c_hi; ++pc) {
           const int pns = nsub_of(pc);
           for (int st = 0; st < pns; ++st, ++lp) {
+            if (lp < pre) continue;  // requested before the wait
             const int slot = lp % RING;
             if (lp >= RING && !mbar_wait(&empty_bar[slot], (uint32_t)(((lp / RING) - 1) & 1), SITE_ATTN_TC | 0x90))
               return;
@@ -1092,6 +1117,10 @@ __global__ void __launch_bounds__(ATC_THREADS)
     ++L;
   };
   auto cbar = []() { asm volatile("bar.sync 1, %0;" ::"n"(ATT_THREADS) : "memory"); };
+  if (a.pre_kv) {  // q, and every output, depend on the previous kernel
+    pdl_wait();
+    pdl_trigger();
+  }
 
   // q tile (bf16, 128-byte swizzle per half; rows past the group are zero) and the q^T fragments
   for (int idx = tid; idx < 8 * 16; idx += ATT_THREADS) {

@@ -186,9 +186,13 @@ static int attn_launch(int np, const CUtensorMap& tk, const CUtensorMap& tv, con
   return BI_OK;
 }
 
+// early_kv: the caller guarantees that slot, pos and the cache rows below the
+// step's positions were written before the kernel preceding this launch (the
+// decode step); with one token per slot the decode kernel may then read them
+// before its dependency wait.
 static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const int32_t* slot, const int32_t* pos,
                          const int32_t* slot_h, const int32_t* pos_h, void* out, int T, int Hq, float scale, int mode,
-                         int variant, void* ws, size_t ws_bytes, cudaStream_t st) {
+                         int variant, void* ws, size_t ws_bytes, cudaStream_t st, bool early_kv = false) {
   BI_REQUIRE(q && kv && slot && pos && slot_h && pos_h && out, BI_ERR_INVALID_ARG, "bi_attention: NULL pointer");
   BI_REQUIRE(kv->k && kv->v, BI_ERR_INVALID_ARG, "bi_attention: NULL KV cache");
   const int d = kv->head_dim, Hkv = kv->n_kv_heads;
@@ -223,6 +227,14 @@ static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const
       blocks.back().y++;
     else
       blocks.push_back(make_int2(t, 1));
+  }
+  bool one_per_slot = early_kv;
+  if (one_per_slot) {
+    std::vector<char> seen(kv->n_slots, 0);
+    for (int t = 0; t < T && one_per_slot; ++t) {
+      one_per_slot = !seen[slot_h[t]];
+      seen[slot_h[t]] = 1;
+    }
   }
   const int max_chunks = max_pos / chunk + 1;
   const size_t need = attn_ws_bytes(T, Hq, d, max_pos, chunk);
@@ -272,6 +284,7 @@ static int attention_run(const void* q, const bi_kv_layout* kv, int layer, const
     a.q = q; a.slot = slot; a.pos = pos; a.part = part; a.t_base = t_base;
     a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.d = d; a.chunk = chunk; a.max_chunks = max_chunks;
     a.layer = layer; a.n_layers = kv->n_layers; a.cap = kv->capacity; a.f32 = f32; a.scale = scale;
+    a.pre_kv = one_per_slot ? 1 : 0;
     a.out = out;
     bool m1 = true, mm = true;
     if (p1.n) BI_TRY(attn_launch(np1, tk, tv, p1, a, st, &m1));
@@ -814,7 +827,7 @@ int bi_decode_step(bi_ctx* ctx, const bi_batch* batch, const bi_step_out* out, v
                       BI_EPI_ROPE_KV_APPEND, &ea, d.mode, d.variant, nullptr, 0, st));
     }
     BI_TRY(attention_run(s.q, &ctx->kv, l, batch->slot, batch->pos, batch->slot_host, batch->pos_host, s.o, T, Hq,
-                         scale, d.mode, d.variant, s.attn, s.attn_bytes, st));
+                         scale, d.mode, d.variant, s.attn, s.attn_bytes, st, true));
     BI_TRY(gemm_run(s.o, QD, lw(w.w_o, (size_t)H * QD, l), s.y, H, act_dtype, T, H, QD, BI_EPI_NONE, nullptr, d.mode,
                     d.variant, s.gemm, s.gemm_bytes, st));
     BI_TRY(bi_rmsnorm(s.y, s.res, s.res, g_ffn, s.u, nullptr, T, H, d.eps, d.mode, stream));
