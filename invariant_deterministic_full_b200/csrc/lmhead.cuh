@@ -26,6 +26,11 @@ struct LmPart {
   int i1, i2, has_t;
 };
 
+__device__ __forceinline__ int warp_min_int(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
 // (v, i) beats (w, j) if v > w, or v == w and i < j.
 __device__ __forceinline__ bool lm_better(float v, int i, float w, int j) { return v > w || (v == w && i < j); }
 __device__ __forceinline__ void lm_top2_insert(float& v1, int& i1, float& v2, int& i2, float v, int i) {
@@ -95,25 +100,55 @@ __global__ void __launch_bounds__(32 * LM_CPB)
 #pragma unroll
   for (int j = 1; j < PER; ++j) mx = fmaxf(mx, z[j]);
   const float M = warp_max(mx);
-  float v1 = -INFINITY, v2 = -INFINITY;
-  int i1 = 0x7fffffff, i2 = 0x7fffffff;
+  const int v0 = c * LM_CHUNK + lane;  // id of z[0]; z[j] has id v0 + 32 j
   float e = 0.f, zt = 0.f;
   int has = 0;
   const int tg = target ? target[src] : -1;
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
-    const int v = c * LM_CHUNK + lane + 32 * j;
-    if (v < V) {
-      lm_top2_insert(v1, i1, v2, i2, z[j], v);
+    if (v0 + 32 * j < V) {
       e += expf(z[j] - M);
-      if (v == tg) {
+      if (v0 + 32 * j == tg) {
         zt = z[j];
         has = 1;
       }
     }
   }
   const float S = warp_sum_fixed(e);
-  lm_top2_warp(v1, i1, v2, i2);
+  // Top two (value, id) under "larger value, then lower id", from the exact
+  // max: the first is the lowest valid id whose logit equals M, the second the
+  // same rule over the chunk without the first.  Each stored value is the
+  // owner lane's logit itself (so a -0 stays -0).  Rows of exact logits need
+  // only the first: their margin is the main pass's.
+  auto owner_value = [&](int id) {
+    const int k = id - c * LM_CHUNK;  // 0..255, or out of range for "none"
+    float mine = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < PER; ++j)
+      if (lane + 32 * j == k) mine = z[j];
+    return __shfl_sync(0xffffffffu, mine, k & 31);
+  };
+  int c1 = 0x7fffffff;
+#pragma unroll
+  for (int j = PER - 1; j >= 0; --j)
+    if (v0 + 32 * j < V && z[j] == M) c1 = v0 + 32 * j;
+  const int i1 = warp_min_int(c1);
+  const float v1 = i1 == 0x7fffffff ? -INFINITY : owner_value(i1);
+  float v2 = -INFINITY;
+  int i2 = 0x7fffffff;
+  if (!exact) {
+    float m2 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < PER; ++j)
+      if (v0 + 32 * j < V && v0 + 32 * j != i1) m2 = fmaxf(m2, z[j]);
+    const float M2 = warp_max(m2);
+    int c2 = 0x7fffffff;
+#pragma unroll
+    for (int j = PER - 1; j >= 0; --j)
+      if (v0 + 32 * j < V && v0 + 32 * j != i1 && z[j] == M2) c2 = v0 + 32 * j;
+    i2 = warp_min_int(c2);
+    if (i2 != 0x7fffffff) v2 = owner_value(i2);
+  }
   const unsigned hb = __ballot_sync(0xffffffffu, has);
   zt = __shfl_sync(0xffffffffu, zt, hb ? __ffs(hb) - 1 : 0);
   if (lane == 0) {
@@ -129,22 +164,51 @@ struct LmRow {
   float L, v1, v2, zt;
   int i1, has;
 };
+// Up to LM_MERGE_REG chunks per lane (n_chunks <= 32 * LM_MERGE_REG, vocabularies
+// up to 163840) are read in one pass, every load issued at once: max, top-2 and
+// the target need no order, and each chunk's (max, sum) stays in registers for
+// the ordered sum.  Larger vocabularies take two passes over the partials.
+// Either way lane l sums chunks l, l + 32, ... in ascending order.
+constexpr int LM_MERGE_REG = 20;
 __device__ __forceinline__ LmRow lm_merge_row(const LmPart* __restrict__ pr, int n_chunks, int lane) {
-  float M = -INFINITY;
-  for (int c = lane; c < n_chunks; c += 32) M = fmaxf(M, pr[c].mx);
-  M = warp_max(M);
-  float S = 0.f, zt = 0.f;
+  float M = -INFINITY, S = 0.f, zt = 0.f;
   int has = 0;
   float v1 = -INFINITY, v2 = -INFINITY;
   int i1 = 0x7fffffff, i2 = 0x7fffffff;
-  for (int c = lane; c < n_chunks; c += 32) {
-    const LmPart q = pr[c];
-    S = fmaf(q.sum, expf(q.mx - M), S);
+  auto take = [&](const LmPart& q) {
     lm_top2_insert(v1, i1, v2, i2, q.v1, q.i1);
     lm_top2_insert(v1, i1, v2, i2, q.v2, q.i2);
     if (q.has_t) {
       has = 1;
       zt = q.zt;
+    }
+  };
+  if (n_chunks <= 32 * LM_MERGE_REG) {
+    float mxs[LM_MERGE_REG], sums[LM_MERGE_REG];
+#pragma unroll
+    for (int k = 0; k < LM_MERGE_REG; ++k) {
+      const int c = lane + 32 * k;
+      mxs[k] = -INFINITY;
+      sums[k] = 0.f;
+      if (c < n_chunks) {
+        const LmPart q = pr[c];
+        mxs[k] = q.mx;
+        sums[k] = q.sum;
+        M = fmaxf(M, q.mx);
+        take(q);
+      }
+    }
+    M = warp_max(M);
+#pragma unroll
+    for (int k = 0; k < LM_MERGE_REG; ++k)
+      if (lane + 32 * k < n_chunks) S = fmaf(sums[k], expf(mxs[k] - M), S);
+  } else {
+    for (int c = lane; c < n_chunks; c += 32) M = fmaxf(M, pr[c].mx);
+    M = warp_max(M);
+    for (int c = lane; c < n_chunks; c += 32) {
+      const LmPart q = pr[c];
+      S = fmaf(q.sum, expf(q.mx - M), S);
+      take(q);
     }
   }
   S = warp_sum_fixed(S);
