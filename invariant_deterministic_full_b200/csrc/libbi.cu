@@ -140,8 +140,9 @@ static int attn_set_smem_attrs() {
 // bf16 head_dim-128 path runs on tensor cores with 16-row pair tiles.
 //
 // Tensor-core kernel: a CTA walks a segment of consecutive chunks of one
-// (block, kv head).  With enough (block, kv head) units to fill the GPU, one
-// segment spans all chunks and the CTA also merges (no merge launch);
+// (block, kv head).  With enough (block, kv head) units (at least two thirds
+// of the SM count), one segment spans all chunks and the CTA also merges (no
+// merge launch);
 // otherwise the chunks are cut into segments so that about two CTAs per SM
 // run, and the merge kernel combines the partials.  Either way the chunk
 // partials and the merge are the same computations (work assignment only).
@@ -154,7 +155,7 @@ static int attn_launch(int np, const CUtensorMap& tk, const CUtensorMap& tv, con
     const bool dec = single && a.G <= 8;  // the decode schedule: one 8-pair tile, at most ATD_SEG chunks per CTA
     const int units = plan.n * a.Hkv;
     const int target = 2 * num_sms();
-    int n_seg = units >= target / 2 ? 1 : std::min(a.max_chunks, (target + units - 1) / units);
+    int n_seg = units >= target / 3 ? 1 : std::min(a.max_chunks, (target + units - 1) / units);
     a.seg_len = (a.max_chunks + n_seg - 1) / n_seg;
     if (dec) a.seg_len = std::min(a.seg_len, ATD_SEG);
     n_seg = (a.max_chunks + a.seg_len - 1) / a.seg_len;

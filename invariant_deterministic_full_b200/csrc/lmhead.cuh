@@ -21,10 +21,11 @@
 namespace bi {
 
 constexpr int LM_CHUNK = BI_VOCAB_CHUNK;  // 256
-struct LmPart {
+struct __align__(16) LmPart {  // 32 bytes: read as two 16-byte halves by the merge
   float mx, sum, v1, v2, zt;
   int i1, i2, has_t;
 };
+static_assert(sizeof(LmPart) == 32, "LmPart layout");
 
 __device__ __forceinline__ int warp_min_int(int v) {
 #pragma unroll
@@ -185,17 +186,30 @@ __device__ __forceinline__ LmRow lm_merge_row(const LmPart* __restrict__ pr, int
   };
   if (n_chunks <= 32 * LM_MERGE_REG) {
     float mxs[LM_MERGE_REG], sums[LM_MERGE_REG];
+    constexpr int BATCH = LM_MERGE_REG / 2;  // partials loaded per batch, all before any is used
 #pragma unroll
-    for (int k = 0; k < LM_MERGE_REG; ++k) {
-      const int c = lane + 32 * k;
-      mxs[k] = -INFINITY;
-      sums[k] = 0.f;
-      if (c < n_chunks) {
-        const LmPart q = pr[c];
-        mxs[k] = q.mx;
-        sums[k] = q.sum;
-        M = fmaxf(M, q.mx);
-        take(q);
+    for (int k0 = 0; k0 < LM_MERGE_REG; k0 += BATCH) {
+      uint4 lo[BATCH], hi[BATCH];
+#pragma unroll
+      for (int k = 0; k < BATCH; ++k) {
+        const int c = min(lane + 32 * (k0 + k), n_chunks - 1);  // in bounds; unused past n_chunks
+        const uint4* q = reinterpret_cast<const uint4*>(pr + c);
+        lo[k] = q[0];
+        hi[k] = q[1];
+      }
+#pragma unroll
+      for (int k = 0; k < BATCH; ++k) {
+        LmPart q;
+        q.mx = __uint_as_float(lo[k].x); q.sum = __uint_as_float(lo[k].y);
+        q.v1 = __uint_as_float(lo[k].z); q.v2 = __uint_as_float(lo[k].w);
+        q.zt = __uint_as_float(hi[k].x); q.i1 = (int)hi[k].y; q.i2 = (int)hi[k].z; q.has_t = (int)hi[k].w;
+        const bool ok = lane + 32 * (k0 + k) < n_chunks;
+        mxs[k0 + k] = ok ? q.mx : -INFINITY;
+        sums[k0 + k] = ok ? q.sum : 0.f;
+        if (ok) {
+          M = fmaxf(M, q.mx);
+          take(q);
+        }
       }
     }
     M = warp_max(M);
