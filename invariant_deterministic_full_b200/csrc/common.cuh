@@ -44,6 +44,12 @@ extern long long g_launches;  // host-side count of kernels launched by the libr
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 int num_sms();  // of the current device (cached per device)
 bool pdl_enabled();  // programmatic dependent launch (env BI_PDL=0 turns it off)
+// Every kernel runs with the largest shared-memory carveout, so all kernels
+// share one L1 / shared-memory split: an SM still holding CTAs of a kernel
+// with little shared memory (the norm) then also takes CTAs of the GEMM or
+// attention kernel launched behind it instead of waiting to drain.  Sets the
+// attribute the first time a thread launches `kern` on the current device.
+int ensure_carveout(const void* kern);
 
 // Launch a library kernel on `st`, with programmatic stream serialisation
 // allowed (see pdl_wait / pdl_trigger), counting it in g_launches.
@@ -59,6 +65,7 @@ int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStrea
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  BI_TRY(ensure_carveout(reinterpret_cast<const void*>(kern)));
   BI_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...));
   BI_CHECK_LAUNCH();
   return BI_OK;

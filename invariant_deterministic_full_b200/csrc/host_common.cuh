@@ -2,6 +2,7 @@
 // TMA descriptor encoding through the driver entry point, device error word.
 #pragma once
 #include <mutex>
+#include <unordered_set>
 #include <vector>
 
 #include "common.cuh"
@@ -46,6 +47,17 @@ bool pdl_enabled() {
   return on;
 }
 
+int ensure_carveout(const void* kern) {
+  int dev = 0;
+  BI_CHECK_CUDA(cudaGetDevice(&dev));
+  thread_local std::unordered_set<uint64_t> done;
+  const uint64_t key = (uint64_t)reinterpret_cast<uintptr_t>(kern) ^ ((uint64_t)dev << 56);
+  if (done.count(key)) return BI_OK;
+  BI_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared));
+  done.insert(key);
+  return BI_OK;
+}
 typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                     const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                     CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
