@@ -19,8 +19,10 @@
 //   * merge over chunks 0..pos/CH: M = max m_c, L = sum_c l_c exp(m_c - M),
 //     o = sum_c acc_c exp(m_c - M), all in ascending chunk order; out = o / L.
 // Those are the CUDA-core kernel's sums (f32 KV, or head size 64).  The
-// tensor-core kernel (bf16 KV, head size 128) keeps the chunk grid, the
-// denominator tree and the merge, and differs in two sums:
+// tensor-core kernels (bf16 KV, head size 128) keep the chunk grid and the
+// merge, and differ in three sums:
+//   * the denominator: lane i sums keys 8i, ..., 8i+7 in ascending order, then
+//     the same xor-butterfly (so each lane's probabilities are contiguous);
 //   * the score is eight mma.sync m16n8k16 steps over the head dimension in
 //     ascending order, each adding 16 exact products into the (key, pair)
 //     fp32 accumulator;
@@ -378,7 +380,8 @@ __global__ void __launch_bounds__(ATT_THREADS)
 
 // ---------------------------------------------------------------------------
 // bf16 mode on tensor cores (mma.sync m16n8k16, fp32 accumulate).  The same
-// chunk grid, masks, max and lane-strided denominator as above.  The
+// chunk grid, masks and max as above; the denominator and the probabilities
+// come from atc_softmax_row (eight contiguous keys per lane).  The
 // (query, q head) pairs are the 8-column side of every mma, so a decode group
 // of G <= 8 pairs fills at least half a tile:
 //   * scores  S^T[key][pair] = scale * sum_d K[key][d] q[pair][d]
@@ -410,6 +413,52 @@ __host__ __device__ inline size_t atc_smem_bytes(int npt, int ring) {
 __device__ __forceinline__ uint32_t atc_poff(int r, int j) {
   const int c = j >> 3;
   return (uint32_t)(r * 512 + (((c & ~7) | ((c ^ r) & 7)) << 4) + (j & 7) * 2);
+}
+
+// Softmax of one (pair, chunk) row of scores, the one sequence every
+// tensor-core schedule runs: lane l owns keys 8l .. 8l+7 of the chunk (two
+// 16-byte score loads); max over the visible keys (exact); each lane sums its
+// eight exp(s - max) in ascending key order, then the fixed xor-butterfly;
+// every probability is split exactly into three bf16 parts, stored as one
+// 16-byte vector per part at row pl of each part (zeros past the visible
+// keys).  srow: the row's 256 scores (16-byte aligned); part q of the
+// probabilities at pbase + q * part_bytes.
+__device__ __forceinline__ void atc_softmax_row(const float* __restrict__ srow, uint8_t* __restrict__ pbase,
+                                                int part_bytes, int pl, int lim, int nvalid, int lane, float& mx_out,
+                                                float& sum_out) {
+  const int j0 = lane * 8;
+  const float4 sa = *reinterpret_cast<const float4*>(srow + j0), sb = *reinterpret_cast<const float4*>(srow + j0 + 4);
+  const float sv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+  float mx = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    if (j0 + e <= lim && j0 + e < nvalid) mx = fmaxf(mx, sv[e]);
+  mx = warp_max(mx);
+  float sum = 0.f;
+  uint32_t w[3][4];
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    uint16_t q[3][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = j0 + e + h;
+      float pj = 0.f;
+      if (j <= lim && j < nvalid) pj = expf(sv[e + h] - mx);
+      sum += pj;
+      q[0][h] = f32_to_bf16_bits(pj);
+      const float r0 = pj - bf16_bits_to_f32(q[0][h]);
+      q[1][h] = f32_to_bf16_bits(r0);
+      q[2][h] = f32_to_bf16_bits(r0 - bf16_bits_to_f32(q[1][h]));
+    }
+#pragma unroll
+    for (int t = 0; t < 3; ++t) w[t][e >> 1] = (uint32_t)q[t][0] | ((uint32_t)q[t][1] << 16);
+  }
+  const uint32_t off = atc_poff(pl, j0);
+#pragma unroll
+  for (int t = 0; t < 3; ++t)
+    *reinterpret_cast<uint4*>(pbase + t * part_bytes + off) = make_uint4(w[t][0], w[t][1], w[t][2], w[t][3]);
+  mx_out = mx;
+  sum_out = warp_sum_fixed(sum);
 }
 
 constexpr int ATC_THREADS = ATT_THREADS + 32;  // 8 consumer warps + 1 producer warp
@@ -578,36 +627,13 @@ __global__ void __launch_bounds__(ATC_THREADS)
       }
       cbar();  // every score of the chunk is in S
 
-      // ---- softmax of the live pair rows: max (exact), exp, l = lane-strided ascending sums then
-      // butterfly; the probabilities go out as three exact bf16 parts (zeros past the valid keys).
-      // Rows past the group's pairs are not computed: they only reach output columns never stored.
+      // ---- softmax of the live pair rows (atc_softmax_row).  Rows past the group's pairs are
+      // not computed: they only reach output columns never stored.
       for (int pl = warp; pl < gp; pl += ATT_THREADS / 32) {
         const int i = (pg0 + pl) / a.G;
         const int lim = pos_s[i] - key0;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < ATT_CHUNK / 32; ++k) {
-          const int j = lane + 32 * k;
-          if (j <= lim && j < nvalid) mx = fmaxf(mx, S[pl * ATC_SST + j]);
-        }
-        mx = warp_max(mx);
-        float sum = 0.f;
-#pragma unroll
-        for (int k = 0; k < ATT_CHUNK / 32; ++k) {
-          const int j = lane + 32 * k;
-          float pj = 0.f;
-          if (j <= lim && j < nvalid) pj = expf(S[pl * ATC_SST + j] - mx);
-          sum += pj;
-          const uint16_t p0 = f32_to_bf16_bits(pj);
-          const float r0 = pj - bf16_bits_to_f32(p0);
-          const uint16_t p1 = f32_to_bf16_bits(r0);
-          const uint16_t p2 = f32_to_bf16_bits(r0 - bf16_bits_to_f32(p1));
-          const uint32_t off = atc_poff(pl, j);
-          *reinterpret_cast<uint16_t*>(Pp + 0 * (NP * 512) + off) = p0;
-          *reinterpret_cast<uint16_t*>(Pp + 1 * (NP * 512) + off) = p1;
-          *reinterpret_cast<uint16_t*>(Pp + 2 * (NP * 512) + off) = p2;
-        }
-        sum = warp_sum_fixed(sum);
+        float mx, sum;
+        atc_softmax_row(S + pl * ATC_SST, Pp, NP * 512, pl, lim, nvalid, lane, mx, sum);
         if (lane == 0) {
           m_s[pl] = mx;
           l_s[pl] = sum;
@@ -876,30 +902,8 @@ __global__ void __launch_bounds__(ATP_THREADS, 1)
       for (int pl = wl; pl < gp; pl += 8) {
         const int i = (pg0 + pl) / a.G;
         const int lim = pos_s[i] - key0;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < ATT_CHUNK / 32; ++k) {
-          const int j = lane + 32 * k;
-          if (j <= lim && j < nvalid) mx = fmaxf(mx, S[pl * ATC_SST + j]);
-        }
-        mx = warp_max(mx);
-        float sum = 0.f;
-#pragma unroll
-        for (int k = 0; k < ATT_CHUNK / 32; ++k) {
-          const int j = lane + 32 * k;
-          float pj = 0.f;
-          if (j <= lim && j < nvalid) pj = expf(S[pl * ATC_SST + j] - mx);
-          sum += pj;
-          const uint16_t p0 = f32_to_bf16_bits(pj);
-          const float r0 = pj - bf16_bits_to_f32(p0);
-          const uint16_t p1 = f32_to_bf16_bits(r0);
-          const uint16_t p2 = f32_to_bf16_bits(r0 - bf16_bits_to_f32(p1));
-          const uint32_t off = atc_poff(pl, j);
-          *reinterpret_cast<uint16_t*>(Pp + 0 * (NP * 512) + off) = p0;
-          *reinterpret_cast<uint16_t*>(Pp + 1 * (NP * 512) + off) = p1;
-          *reinterpret_cast<uint16_t*>(Pp + 2 * (NP * 512) + off) = p2;
-        }
-        sum = warp_sum_fixed(sum);
+        float mx, sum;
+        atc_softmax_row(S + pl * ATC_SST, Pp, NP * 512, pl, lim, nvalid, lane, mx, sum);
         if (lane == 0) {
           m_s[wg][pl] = mx;
           l_s[wg][pl] = sum;
@@ -995,7 +999,7 @@ __global__ void __launch_bounds__(ATP_THREADS, 1)
 // warps 0-3 the even 64-key sub-tiles, warps 4-7 the odd ones.  Every score, every
 // softmax and every P.V chain is the instruction sequence of attn_tc_kernel
 // (each score one warp's chain of 8 ascending k16 mma over the head; the same
-// lane-strided max and denominator; the same 3-part P split and per-part
+// softmax row function; the same 3-part P split and per-part
 // chains over ascending 16-key steps; the same record and merge), so the two
 // kernels, and prefill and decode, give the same bits.
 constexpr int ATD_SEG = 3;                   // chunks per CTA (scores of all of them are kept)
@@ -1183,32 +1187,8 @@ __global__ void __launch_bounds__(ATC_THREADS)
     const int key0 = (c_lo + cl) * a.chunk;
     const int nvalid = min(a.chunk, pmax - key0 + 1);
     const int lim = pmax - key0;  // keys j <= lim are visible to the query
-    const float* Sc = S + cl * 256;
-    float mx = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < ATT_CHUNK / 32; ++k) {
-      const int j = lane + 32 * k;
-      if (j <= lim && j < nvalid) mx = fmaxf(mx, Sc[pl * ATD_SST + j]);
-    }
-    mx = warp_max(mx);
-    float sum = 0.f;
-    uint8_t* Pc = Pp + cl * (3 * PPART);
-#pragma unroll
-    for (int k = 0; k < ATT_CHUNK / 32; ++k) {
-      const int j = lane + 32 * k;
-      float pj = 0.f;
-      if (j <= lim && j < nvalid) pj = expf(Sc[pl * ATD_SST + j] - mx);
-      sum += pj;
-      const uint16_t p0 = f32_to_bf16_bits(pj);
-      const float r0 = pj - bf16_bits_to_f32(p0);
-      const uint16_t p1 = f32_to_bf16_bits(r0);
-      const uint16_t p2 = f32_to_bf16_bits(r0 - bf16_bits_to_f32(p1));
-      const uint32_t off = atc_poff(pl, j);
-      *reinterpret_cast<uint16_t*>(Pc + 0 * PPART + off) = p0;
-      *reinterpret_cast<uint16_t*>(Pc + 1 * PPART + off) = p1;
-      *reinterpret_cast<uint16_t*>(Pc + 2 * PPART + off) = p2;
-    }
-    sum = warp_sum_fixed(sum);
+    float mx, sum;
+    atc_softmax_row(S + cl * 256 + pl * ATD_SST, Pp + cl * (3 * PPART), PPART, pl, lim, nvalid, lane, mx, sum);
     if (lane == 0) {
       m_s[cl][pl] = mx;
       l_s[cl][pl] = sum;
