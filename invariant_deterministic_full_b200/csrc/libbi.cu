@@ -535,10 +535,11 @@ int bi_gemm(const void* x, int ldx, const void* w, void* y, int ldy, int y_dtype
                   n_full);
 }
 
-int bi_rmsnorm(const void* x, const void* residual_in, void* residual_out, const void* gamma, void* y, float* y_f32,
-               int M, int H, float eps, int mode, void* stream) {
-  BI_RANGE("bi_rmsnorm");
-  clear_error();
+// early: the residual row and gamma were written before the kernel preceding
+// this launch (the decode step's norms), so the kernel loads them before its
+// dependency wait.
+static int rmsnorm_run(const void* x, const void* residual_in, void* residual_out, const void* gamma, void* y,
+                       float* y_f32, int M, int H, float eps, int mode, void* stream, bool early) {
   BI_REQUIRE(x && gamma && y, BI_ERR_INVALID_ARG, "bi_rmsnorm: NULL pointer");
   BI_REQUIRE(M >= 0 && H > 0 && H % 8 == 0 && H <= NORM_THREADS * NORM_MAX_CHUNKS * 8, BI_ERR_UNSUPPORTED,
              "bi_rmsnorm: H=%d (need H %% 8 == 0, H <= 16384)", H);
@@ -548,20 +549,27 @@ int bi_rmsnorm(const void* x, const void* residual_in, void* residual_out, const
              BI_ERR_UNSUPPORTED, "bi_rmsnorm: buffers must be 16-byte aligned");
   if (M == 0) return BI_OK;
   const uint16_t* g16 = reinterpret_cast<const uint16_t*>(gamma);
-  const int f32 = act_f32(mode);
+  const int f32 = act_f32(mode), e = early ? 1 : 0;
   cudaStream_t st = as_stream(stream);
   switch (norm_cpt(H)) {
     case 1: return launch(rmsnorm_kernel<1>, dim3(M), dim3(NORM_THREADS), 0, st, x, residual_in, residual_out, g16, y,
-                          y_f32, H, eps, f32);
+                          y_f32, H, eps, f32, e);
     case 2: return launch(rmsnorm_kernel<2>, dim3(M), dim3(NORM_THREADS), 0, st, x, residual_in, residual_out, g16, y,
-                          y_f32, H, eps, f32);
+                          y_f32, H, eps, f32, e);
     case 4: return launch(rmsnorm_kernel<4>, dim3(M), dim3(NORM_THREADS), 0, st, x, residual_in, residual_out, g16, y,
-                          y_f32, H, eps, f32);
+                          y_f32, H, eps, f32, e);
     case 8: return launch(rmsnorm_kernel<8>, dim3(M), dim3(NORM_THREADS), 0, st, x, residual_in, residual_out, g16, y,
-                          y_f32, H, eps, f32);
+                          y_f32, H, eps, f32, e);
     default: return launch(rmsnorm_kernel<16>, dim3(M), dim3(NORM_THREADS), 0, st, x, residual_in, residual_out, g16,
-                           y, y_f32, H, eps, f32);
+                           y, y_f32, H, eps, f32, e);
   }
+}
+
+int bi_rmsnorm(const void* x, const void* residual_in, void* residual_out, const void* gamma, void* y, float* y_f32,
+               int M, int H, float eps, int mode, void* stream) {
+  BI_RANGE("bi_rmsnorm");
+  clear_error();
+  return rmsnorm_run(x, residual_in, residual_out, gamma, y, y_f32, M, H, eps, mode, stream, false);
 }
 
 int bi_rope_table_fill(float* table, int max_pos, int head_dim, double theta, void* stream) {
@@ -816,7 +824,9 @@ int bi_decode_step(bi_ctx* ctx, const bi_batch* batch, const bi_step_out* out, v
   for (int l = 0; l < d.n_layers; ++l) {
     const void* g_attn = lg(w.attn_norm, l);
     const void* g_ffn = lg(w.ffn_norm, l);
-    BI_TRY(bi_rmsnorm(s.y, l == 0 ? nullptr : s.res, s.res, g_attn, s.u, nullptr, T, H, d.eps, d.mode, stream));
+    // the step's norms read the residual row written by the norm two or more kernels back (early loads)
+    BI_TRY(rmsnorm_run(s.y, l == 0 ? nullptr : s.res, s.res, g_attn, s.u, nullptr, T, H, d.eps, d.mode, stream,
+                       true));
     if (f32 || d.variant == BI_VARIANT_FAST) {  // projection, then RoPE + KV append as a kernel
       BI_TRY(gemm_run(s.u, H, lw(w.w_qkv, (size_t)QKV * H, l), s.qkv, QKV, BI_DTYPE_F32, T, QKV, H, BI_EPI_NONE,
                       nullptr, d.mode, d.variant, s.gemm, s.gemm_bytes, st));
@@ -831,13 +841,13 @@ int bi_decode_step(bi_ctx* ctx, const bi_batch* batch, const bi_step_out* out, v
                          scale, d.mode, d.variant, s.attn, s.attn_bytes, st, true));
     BI_TRY(gemm_run(s.o, QD, lw(w.w_o, (size_t)H * QD, l), s.y, H, act_dtype, T, H, QD, BI_EPI_NONE, nullptr, d.mode,
                     d.variant, s.gemm, s.gemm_bytes, st));
-    BI_TRY(bi_rmsnorm(s.y, s.res, s.res, g_ffn, s.u, nullptr, T, H, d.eps, d.mode, stream));
+    BI_TRY(rmsnorm_run(s.y, s.res, s.res, g_ffn, s.u, nullptr, T, H, d.eps, d.mode, stream, true));
     BI_TRY(gemm_run(s.u, H, lw(w.w_gu, (size_t)2 * F * H, l), s.a, F, act_dtype, T, 2 * F, H, BI_EPI_SWIGLU, nullptr, d.mode,
                     d.variant, s.gemm, s.gemm_bytes, st));
     BI_TRY(gemm_run(s.a, F, lw(w.w_down, (size_t)H * F, l), s.y, H, act_dtype, T, H, F, BI_EPI_NONE, nullptr, d.mode,
                     d.variant, s.gemm, s.gemm_bytes, st));
   }
-  BI_TRY(bi_rmsnorm(s.y, s.res, s.res, w.final_norm, s.u, s.h32, T, H, d.eps, d.mode, stream));
+  BI_TRY(rmsnorm_run(s.y, s.res, s.res, w.final_norm, s.u, s.h32, T, H, d.eps, d.mode, stream, true));
   if (n_lm == 0) return BI_OK;
   BI_TRY(launch(gather_lm_rows_kernel, dim3(T), dim3(256), 0, st, batch->lm_row, s.h32, T, H, n_lm, s.hl, out->h));
   return lmhead_run(s.hl, w.lm_head, batch->target, n_lm, H, d.vocab, d.margin_threshold, d.mode, out->logprob,

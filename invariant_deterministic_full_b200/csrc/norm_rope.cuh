@@ -45,28 +45,41 @@ __device__ __forceinline__ float as_stored(float v, bool f32) {
 // warp order (every thread repeats that same sequential sum).  r = x
 // (+ res_in, rounded as stored), written to res_out; y = (r * inv) * gamma.
 // `bar` synchronises the NORM_THREADS threads (a CTA barrier, or a named
-// barrier inside a larger CTA).
+// barrier inside a larger CTA).  The row waits for the previous kernel
+// (pdl_wait) before it reads x; with `early` the residual row and gamma, which
+// the caller guarantees were written before the previous kernel, are loaded
+// before that wait.
 template <int CPT, typename Bar>
 __device__ __forceinline__ void rmsnorm_row(const void* __restrict__ x, const void* __restrict__ res_in,
                                             void* __restrict__ res_out, const uint16_t* __restrict__ gamma,
                                             void* __restrict__ y, float* __restrict__ y32, int row, int H, float eps,
-                                            int f32, int tid, float* wsum, Bar bar) {
+                                            int f32, int tid, float* wsum, Bar bar, bool early) {
   const int nch = H / 8;
   const size_t rbase = (size_t)row * H;
-  float v[CPT][8];
+  float v[CPT][8], r[CPT][8];
   uint4 gu[CPT];
+  auto load_res_gamma = [&]() {
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+      const int ch = tid + i * NORM_THREADS;
+      if (ch < nch) {
+        if (res_in) load8(res_in, rbase + ch * 8, f32, r[i]);
+        gu[i] = *reinterpret_cast<const uint4*>(gamma + ch * 8);
+      }
+    }
+  };
+  if (early) load_res_gamma();
+  pdl_wait();
+  if (!early) load_res_gamma();
 #pragma unroll
   for (int i = 0; i < CPT; ++i) {
     const int ch = tid + i * NORM_THREADS;
     if (ch < nch) {
       load8(x, rbase + ch * 8, f32, v[i]);
       if (res_in) {
-        float r[8];
-        load8(res_in, rbase + ch * 8, f32, r);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[i][j] = as_stored(v[i][j] + r[j], f32);
+        for (int j = 0; j < 8; ++j) v[i][j] = as_stored(v[i][j] + r[i][j], f32);
       }
-      gu[i] = *reinterpret_cast<const uint4*>(gamma + ch * 8);
     }
   }
   float ss = 0.f;
@@ -107,15 +120,17 @@ __device__ __forceinline__ void rmsnorm_row(const void* __restrict__ x, const vo
   }
 }
 
-// One CTA per row (see rmsnorm_row, which also releases the next kernel once
-// the row's loads have landed); CPT: chunks per thread, the smallest of 1, 2,
-// 4, 8, 16 that covers the row.
+// One CTA per row (see rmsnorm_row, which waits for the previous kernel and
+// releases the next once the row's loads have landed); CPT: chunks per
+// thread, the smallest of 1, 2, 4, 8, 16 that covers the row.  early: see
+// rmsnorm_row (the decode step, where the residual row was written by a norm
+// at least two kernels back).
 template <int CPT>
 __global__ void __launch_bounds__(NORM_THREADS)
     rmsnorm_kernel(const void* __restrict__ x, const void* __restrict__ res_in, void* __restrict__ res_out,
                    const uint16_t* __restrict__ gamma, void* __restrict__ y, float* __restrict__ y32, int H, float eps,
-                   int f32) {
-  {
+                   int f32, int early) {
+  if (!early) {
     // Before the dependency wait, request the row's residual and gamma into
     // L2 (a prefetch returns no value, so it cannot observe data that an
     // earlier kernel is still writing): after the wait the row's loads find
@@ -128,10 +143,9 @@ __global__ void __launch_bounds__(NORM_THREADS)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(pa));
     }
   }
-  pdl_wait();
   __shared__ float wsum[NORM_THREADS / 32];
   rmsnorm_row<CPT>(x, res_in, res_out, gamma, y, y32, blockIdx.x, H, eps, f32, threadIdx.x, wsum,
-                   [] { __syncthreads(); });
+                   [] { __syncthreads(); }, early != 0);
 }
 __host__ __device__ constexpr int norm_cpt(int H) {
   return H / 8 <= NORM_THREADS ? 1 : H / 8 <= 2 * NORM_THREADS ? 2 : H / 8 <= 4 * NORM_THREADS ? 4
