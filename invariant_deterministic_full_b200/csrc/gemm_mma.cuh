@@ -81,6 +81,7 @@ __global__ void __launch_bounds__(160, CPS)
                      const RopeEpi re, int xr) {
   using C = GemmCfg<BN, MT, CPS>;
   static_assert(MT == 1 || C::KS == 1, "M-blocking needs one k-phase per warp");
+  static_assert(EPI != EPI_ROPE || MT == 1, "the RoPE epilogue takes one token tile per item");
   // Token rows per k-block slab of a stage: xr = 8 or 16 when M fits (MT = 1),
   // else 32.  Rows of the slab past M are zero-filled by the copy and never
   // read: the consumers stop at the last n8 tile holding live rows.
@@ -226,6 +227,46 @@ __global__ void __launch_bounds__(160, CPS)
     int ntvs[MT];  // n8 token tiles holding live rows, per token tile
 #pragma unroll
     for (int j = 0; j < MT; ++j) ntvs[j] = max(0, min(4, (Me - (mt0 + j) * GEMM_BM + 7) / 8));
+    // RoPE epilogue (one token tile): this thread's token positions and slots,
+    // and the cos/sin of its rotation pairs, requested before the K loop so
+    // that the epilogue waits on no load
+    int pp[4][2], ss[4][2];
+    bool ok[4][2];
+    if constexpr (EPI == EPI_ROPE) {
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int m = mt0 * GEMM_BM + nt * 8 + 2 * t4 + j;
+          ok[nt][j] = splits == 1 && nt % C::KS == kp && nt < ntvs[0] && m < Me;
+          pp[nt][j] = ok[nt][j] ? __ldg(re.pos + m) : 0;
+          ss[nt][j] = ok[nt][j] ? __ldg(re.slot + m) : 0;
+        }
+    }
+    float cs[4][2][2], sn[4][2][2];
+    if constexpr (EPI == EPI_ROPE) {
+      const int QD = re.Hq * re.d, KD = re.Hkv * re.d;
+      const int nb = g * BN + row0;
+      const bool isv = nb >= QD + KD, isq = nb < QD;
+      const int rel = isq ? nb : nb - QD;
+      const int e0 = (rel % re.d) >> 1;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int p = pp[nt][j], sl = ss[nt][j];
+          if (ok[nt][j] && (p < 0 || p >= re.cap || p >= re.table_max_pos || sl < 0 || sl >= re.n_slots)) {
+            dev_flag(DEVERR_CAPACITY);
+            ok[nt][j] = false;
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const size_t ti = (size_t)(ok[nt][j] && !isv ? p : 0) * re.d + 2 * (e0 + g8 + h * 8);
+            cs[nt][j][h] = ok[nt][j] ? __ldg(re.table + ti) : 0.f;
+            sn[nt][j][h] = ok[nt][j] ? __ldg(re.table + ti + 1) : 0.f;
+          }
+        }
+    }
     // accumulator set kp of this warp's outputs: k16 steps kk = kp, kp + KS, ... of every 64-k block
     float accm[MT][2][4][4];
 #pragma unroll
@@ -329,40 +370,11 @@ __global__ void __launch_bounds__(160, CPS)
     const int nbase = g * BN + row0;
     if constexpr (EPI == EPI_ROPE) {
       if (splits == 1) {
-        // positions, slots and cos/sin of this thread's tokens are all fetched
-        // before any store, so the dependent loads overlap
+        // positions, slots and cos/sin of this thread's tokens came in before the K loop
         const int QD = re.Hq * re.d, KD = re.Hkv * re.d, half = re.d >> 1;
         const bool isv = nbase >= QD + KD, isq = nbase < QD;
         const int rel = isq ? nbase : nbase - QD;
         const int head = rel / re.d, e0 = (rel % re.d) >> 1;  // first-half element 16b
-        int pp[4][2], ss[4][2];
-        bool ok[4][2];
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int m = mt * GEMM_BM + nt * 8 + 2 * t4 + j;
-            ok[nt][j] = nt % C::KS == kp && nt < ntv && m < Me;
-            pp[nt][j] = ok[nt][j] ? __ldg(re.pos + m) : 0;
-            ss[nt][j] = ok[nt][j] ? __ldg(re.slot + m) : 0;
-          }
-        float cs[4][2][2], sn[4][2][2];
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int p = pp[nt][j], sl = ss[nt][j];
-            if (ok[nt][j] && (p < 0 || p >= re.cap || p >= re.table_max_pos || sl < 0 || sl >= re.n_slots)) {
-              dev_flag(DEVERR_CAPACITY);
-              ok[nt][j] = false;
-            }
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const size_t ti = (size_t)(ok[nt][j] && !isv ? p : 0) * re.d + 2 * (e0 + g8 + h * 8);
-              cs[nt][j][h] = __ldg(re.table + ti);
-              sn[nt][j][h] = __ldg(re.table + ti + 1);
-            }
-          }
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
