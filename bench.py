@@ -167,8 +167,8 @@ def step_bytes(cfg, B, ctx_lens, f32_kv=False):
 # capture (dram__bytes_read.sum + dram__bytes_write.sum) of the same shapes on the 2-layer 8B-width case (the
 # weights per launch do not depend on the layer count).  Valid only for the GEMM kernel source that was captured,
 # recognised by gemm_source_digest; None until a capture of this source.
-GEMM_TRAFFIC = {"gemm_source_sha256": "c9927272f6323bbe58765e0d661abbc40114b7ee935f5118e23d3427132623eb",
-                "batch": 32, "per_layer_bytes": 444953600}
+GEMM_TRAFFIC = {"gemm_source_sha256": "f9cf186530efc55554b30d6969cc7ed6e294fefb332fce824f312bfc4cda1fbc",
+                "batch": 32, "per_layer_bytes": 448002816}
 
 CSRC = os.path.join(ROOT, "invariant_deterministic_full_b200", "csrc")
 
