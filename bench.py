@@ -167,8 +167,8 @@ def step_bytes(cfg, B, ctx_lens, f32_kv=False):
 # capture (dram__bytes_read.sum + dram__bytes_write.sum) of the same shapes on the 2-layer 8B-width case (the
 # weights per launch do not depend on the layer count).  Valid only for the GEMM kernel source that was captured,
 # recognised by gemm_source_digest; None until a capture of this source.
-GEMM_TRAFFIC = {"gemm_source_sha256": "f9cf186530efc55554b30d6969cc7ed6e294fefb332fce824f312bfc4cda1fbc",
-                "batch": 32, "per_layer_bytes": 448002816}
+GEMM_TRAFFIC = {"gemm_source_sha256": "78b8680b7f0e5605458b68383829e3543da3c923c0f7aff97d799c6585c493f3",
+                "batch": 32, "per_layer_bytes": 445704448}
 
 CSRC = os.path.join(ROOT, "invariant_deterministic_full_b200", "csrc")
 

@@ -179,8 +179,11 @@ static TcPlan tc_plan(int M, int N, int K, int variant, int ks) {
   p.ks = ks;
   p.mt = (M <= TC_TILE_M || p.ks == 4) ? 1 : 2;
   // widest weight tile the TMEM holds (one token tile: at most 128 rows, so that
-  // the launches of up to 128 tokens spread over more SMs)
-  const int cols = std::min(512 / (p.ks * p.mt), p.mt == 1 ? 128 : 256);
+  // the launches of up to 128 tokens spread over more SMs); four-set matrices
+  // take 64-row tiles when 128-row ones would leave SMs without an item (the
+  // launch is then bound by the weight stream, e.g. LayerCast's split rows)
+  int cols = std::min(512 / (p.ks * p.mt), p.mt == 1 ? 128 : 256);
+  if (p.ks == 4 && (N / 128) * ((M + TC_TILE_M - 1) / TC_TILE_M) < num_sms()) cols = 64;
   p.bn = (cols >= 256 && N % 256 == 0) ? 256 : ((cols >= 128 && N % 128 == 0) ? 128 : 64);
   p.splits = 1;
   if (variant == BI_VARIANT_FAST) {
